@@ -1,0 +1,85 @@
+"""Plant one plausible mistake at a time in a copy of the oracle (on the CPU)
+and check that the pins in tests/test_oracle.py catch every one of them."""
+from __future__ import annotations
+
+import os
+import subprocess
+
+import pytest
+
+from oracle import oracle as orc
+from tests import test_oracle as pins
+
+# (name, exact text in oracle.c, replacement)
+MUTATIONS = [
+    ("relu_dropped", "double relu = dot > 0.0 ? dot : 0.0;", "double relu = dot;"),
+    ("relu_wrong_side", "double relu = dot > 0.0 ? dot : 0.0;", "double relu = dot < 0.0 ? dot : 0.0;"),
+    ("weight_sign", "acc += wt[h] * relu;", "acc -= wt[h] * relu;"),
+    ("sigma_dropped", "*I_out = sigma * acc;", "*I_out = acc;"),
+    ("q_transposed", "double p = qd[h * ORC_DIM + d] * kd[d];",
+     "double p = qd[d * ORC_HEADS + h] * kd[d];"),
+    ("weight_index", "wt[h] = (double)weights[t * ORC_HEADS + h];",
+     "wt[h] = (double)weights[t * ORC_HEADS + (h ^ 1)];"),
+    ("first_key_dropped", "for (int64_t s = ks[t]; s < ke[t]; ++s) {",
+     "for (int64_t s = ks[t] + 1; s < ke[t]; ++s) {"),
+    ("error_scale_signed", "err += fabs(wt[h]) * absdot;", "err += wt[h] * absdot;"),
+    ("tie_to_larger_index", "return (x->i < y->i) ? -1 : (x->i > y->i) ? 1 : 0;",
+     "return (x->i > y->i) ? -1 : (x->i < y->i) ? 1 : 0;"),
+    ("ascending_order", "if (x->v > y->v)\n            return -1;", "if (x->v < y->v)\n            return -1;"),
+    ("e4m3_bias", "mag = ldexp(1.0 + (double)m / 8.0, (int)e - 7);",
+     "mag = ldexp(1.0 + (double)m / 8.0, (int)e - 8);"),
+    ("e4m3_subnormal", "mag = ldexp((double)m / 8.0, -6);", "mag = ldexp((double)m / 8.0, -7);"),
+    ("bf16_shift", "uint32_t w = (uint32_t)(bits & 0xFFFFu) << 16;",
+     "uint32_t w = (uint32_t)(bits & 0xFFFFu) << 15;"),
+    ("padding_index", "out_idx[j] = j < n ? buf[j].i : -1;", "out_idx[j] = j < n ? buf[j].i : 0;"),
+    ("short_window_loses_one", "int64_t n = L < k ? L : k;", "int64_t n = L < k ? L - 1 : k;"),
+]
+
+CHECKS = [
+    pins.check_e4m3_table,
+    pins.check_bf16_table,
+    lambda: pins.check_score_equal_heads_matmul("fp8"),
+    lambda: pins.check_score_equal_heads_matmul("bf16"),
+    lambda: pins.check_score_one_hot_heads("fp8"),
+    lambda: pins.check_score_one_hot_heads("bf16"),
+    lambda: pins.check_score_linear_in_weights("fp8"),
+    pins.check_score_homogeneity,
+    pins.check_hand_example,
+    pins.check_select_brute_force,
+    pins.check_select_all_equal,
+    pins.check_select_torch_topk_tie_free,
+    pins.check_select_signed_zero,
+    pins.check_topk_rows_brute_force,
+    pins.check_topk_rows_torch_tie_free,
+    pins.check_fused_all_equal,
+]
+
+
+def _build_mutant(tmp_path, old, new):
+    src = open(orc.SRC).read()
+    assert src.count(old) == 1, f"mutation anchor not unique: {old!r}"
+    path = tmp_path / "oracle_mutant.c"
+    path.write_text(src.replace(old, new))
+    so = tmp_path / "liboracle_mutant.so"
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
+                           "-o", str(so), str(path), "-lm"])
+    return str(so)
+
+
+def test_pins_pass_on_the_real_oracle():
+    for chk in CHECKS:
+        chk()
+
+
+@pytest.mark.parametrize("name,old,new", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_planted_mistake_is_caught(tmp_path, name, old, new):
+    so = _build_mutant(tmp_path, old, new)
+    caught = []
+    with orc.use_library(so):
+        for chk in CHECKS:
+            try:
+                chk()
+            except AssertionError:
+                caught.append(chk)
+                break
+    assert caught, f"no pin catches the planted mistake {name}"
