@@ -1,0 +1,215 @@
+/*
+ * ftk.h -- C ABI of libftk: fused lightning-indexer scoring with exact,
+ * deterministic per-query top-k, and a standalone row top-k, for NVIDIA
+ * B200 (sm_100a).
+ *
+ * Plain C: pointers, sizes, enums.  No CUDA or torch types appear here; a
+ * CUDA stream is passed as `void *` (a cudaStream_t, NULL = legacy default
+ * stream).  "device" pointers are CUDA device memory of the current device;
+ * "host" pointers are ordinary CPU memory.
+ *
+ * Conventions shared by every call
+ *  - Calls are asynchronous and stream-ordered unless stated otherwise; they
+ *    never synchronise the host with the device (except ftk_read_info).
+ *  - Argument errors that the host can see (NULL pointers, sizes, dtypes,
+ *    topk range, alignment, workspace size) return a negative ftk_status and
+ *    launch nothing.
+ *  - Errors that only the device can see (a window outside [0, S], a NaN
+ *    score, a bounded wait that gave up) never abort a kernel: they set bits
+ *    of a device status word (FTK_STATUS_*), readable after the stream
+ *    completes.
+ *  - The caller owns every buffer.  The library allocates no device memory.
+ *  - Output order: the selected keys of a row are written in ascending key
+ *    index, which makes the output bits a pure function of the inputs
+ *    (FlashTopK README, "Highlights": the same bits on every run).
+ */
+#ifndef FTK_H
+#define FTK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Indexer shape (FlashTopK README, "Support": indexers of 32 heads x 128). */
+#define FTK_HEADS 32
+#define FTK_DIM 128
+/* topk range (FlashTopK README, "Support"; DeepSelect README, "Supported
+ * Cases": topk must be <= 4096). */
+#define FTK_MAX_TOPK 4096
+
+typedef enum {
+    FTK_F8E4M3 = 1, /* float8 e4m3fn, 1 byte */
+    FTK_BF16 = 2,   /* bfloat16, 2 bytes */
+    FTK_F32 = 3     /* float32, 4 bytes */
+} ftk_dtype;
+
+typedef enum {
+    FTK_OK = 0,
+    FTK_ERR_INVALID_ARG = -1, /* NULL pointer, negative/oversized size, bad dtype */
+    FTK_ERR_UNSUPPORTED = -2, /* a valid request this build does not handle */
+    FTK_ERR_TOPK_RANGE = -3,  /* topk outside [1, FTK_MAX_TOPK] */
+    FTK_ERR_ALIGNMENT = -4,   /* pointer or row stride not 16-byte aligned */
+    FTK_ERR_WORKSPACE = -5,   /* workspace NULL, misaligned or too small */
+    FTK_ERR_CUDA = -6,        /* a CUDA runtime call failed */
+    FTK_ERR_DEVICE = -7       /* current device is not compute capability 10.0 */
+} ftk_status;
+
+/* Device status bits (ftk_info.status, and the status word of
+ * ftk_topk_rows).  A row hit by BAD_WINDOW is written as all (-1, -inf);
+ * a row hit by NAN has unspecified contents. */
+#define FTK_STATUS_BAD_WINDOW 0x1u /* ks < 0, ks > ke or ke > S in some row */
+#define FTK_STATUS_NAN 0x2u        /* a NaN score or input value was seen */
+#define FTK_STATUS_TIMEOUT 0x4u    /* a bounded device wait gave up */
+#define FTK_STATUS_BAD_SCALE 0x8u  /* a kv_scales entry was <= 0 or not finite */
+#define FTK_STATUS_INTERNAL 0x10u  /* an internal bounds check failed */
+
+/* Tuning knobs of ftk_select.  None of them changes the result (the
+ * selection is exact); they trade speed against the rate of rows that need
+ * dense recovery.  Pass NULL for the defaults. */
+typedef struct {
+    int32_t sample_keys; /* target strided-sample size per row, m (default 4096) */
+    float oversample;    /* beta: the threshold keeps ~beta*topk keys (default 1.5) */
+    int32_t capacity;    /* C: candidate slots per row (0: 2*topk) */
+    int32_t prune;       /* score-bound key pruning: -1 auto (default), 0 off, 1 on */
+    int32_t recovery_rows; /* rows rescored densely per recovery pass (0: auto) */
+    int32_t reserved[3];   /* must be 0 */
+} ftk_config;
+
+/* Per-call information (FlashTopK README, "Usage": last_info), filled on
+ * the device by ftk_select and read back with ftk_read_info. */
+typedef struct {
+    uint32_t status;          /* FTK_STATUS_* bits */
+    int32_t prune_enabled;    /* 1 if the call scanned with key pruning */
+    int64_t rows;             /* T */
+    int64_t rows_underflow;   /* rows whose threshold kept fewer than min(topk, L) keys */
+    int64_t rows_overflow;    /* rows whose candidates exceeded the capacity */
+    int64_t blocks_total;     /* (query tile, 128-key block) pairs in the windows */
+    int64_t blocks_pruned;    /* of which skipped by the score bound */
+    int64_t candidates_total; /* sum over rows of candidates kept */
+    int64_t candidates_max;   /* largest per-row candidate count */
+} ftk_info;
+
+/*
+ * ftk_select -- for every query row t, the topk keys s of its window
+ * [ks[t], ke[t]) with the largest indexer score
+ *     I[t,s] = sigma_s * sum_{h<32} w[t,h] * ReLU(q[t,h] . kv[s])
+ * (FlashTopK README, "Quick start"), exact, with ties at the k-th score
+ * resolved to the smallest key indices (FlashTopK README, "Highlights").
+ *
+ *   dtype      FTK_F8E4M3 or FTK_BF16 (q and kv share it)
+ *   q          device [T, 32, 128] of dtype, contiguous, 16-byte aligned
+ *   kv         device [S, 128] of dtype, contiguous, 16-byte aligned
+ *   kv_scales  device [S] float32 sigma_s, or NULL for all ones (BF16 keys);
+ *              values must be > 0 (checked, FTK_STATUS_BAD_SCALE)
+ *   weights    device [T, 32] float32
+ *   ks, ke     device [T] int32 windows, 0 <= ks <= ke <= S
+ *   T, S       1 <= T, S and T, S < 2^31
+ *   topk       1 .. FTK_MAX_TOPK
+ *   out_idx    device [T, topk] int32: selected key indices in ascending
+ *              order; rows whose window holds L < topk keys get the L keys
+ *              then index -1
+ *   out_val    device [T, topk] float32 scores of out_idx (-inf for padding),
+ *              or NULL to skip them
+ *   workspace  device scratch of at least ftk_select_workspace_size() bytes,
+ *              256-byte aligned; owned by the caller; one call at a time per
+ *              workspace (calls on different streams need different ones)
+ *   config     host pointer to tuning knobs, or NULL
+ *   stream     cudaStream_t
+ * Scores are computed with FP8/BF16 products and float32 accumulation; each
+ * returned score is within 1e-4 * sigma_s * sum_h |w[t,h]| *
+ * sum_d |q[t,h,d] * kv[s,d]| of the exact value.
+ */
+ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
+                      const float *kv_scales, const float *weights,
+                      const int32_t *ks, const int32_t *ke, int64_t T,
+                      int64_t S, int topk, int32_t *out_idx, float *out_val,
+                      void *workspace, size_t workspace_bytes,
+                      const ftk_config *config, void *stream);
+
+/* Bytes of workspace ftk_select needs for these sizes (FlashTopK README,
+ * "Usage": Selector.plan(max_rows, max_kv) owns the workspace).  A
+ * workspace sized for (T, S) serves any call with smaller T and S and the
+ * same topk and config.  Returns 0 for invalid sizes. */
+size_t ftk_select_workspace_size(int64_t T, int64_t S, int topk,
+                                 const ftk_config *config);
+
+/* Copies the ftk_info of the last ftk_select run on this workspace to the
+ * host struct *out.  Synchronises `stream` first.  workspace: device. */
+ftk_status ftk_read_info(const void *workspace, ftk_info *out, void *stream);
+
+/*
+ * ftk_topk_rows -- row top-k (DeepSelect README, "Supported Cases" and
+ * "Usage"): for each row r of x, the topk columns with the largest values,
+ * ties to the smaller column index, output in ascending column order.
+ *
+ *   dtype       FTK_BF16 or FTK_F32
+ *   x           device [rows, cols] of dtype; row r starts at
+ *               x + r * row_stride elements; x and row_stride * elem_size
+ *               must be 16-byte aligned (DeepSelect README, "Usage": the row
+ *               stride alignment requirement)
+ *   rows        >= 1;  cols: 1 .. 393216
+ *   topk        1 .. FTK_MAX_TOPK; rows with cols < topk are padded with
+ *               index -1 and value -inf
+ *   out_idx     device [rows, topk] int32
+ *   out_val     device [rows, topk] of dtype (x's), or NULL to skip values
+ *               (DeepSelect README, "Usage": return_value=False)
+ *   status      device uint32 word that receives FTK_STATUS_NAN bits
+ *               (OR-ed in; DeepSelect README, "NaN handling" aborts instead),
+ *               or NULL
+ *   stream      cudaStream_t
+ */
+ftk_status ftk_topk_rows(ftk_dtype dtype, const void *x, int64_t rows,
+                         int64_t cols, int64_t row_stride, int topk,
+                         int32_t *out_idx, void *out_val, uint32_t *status,
+                         void *stream);
+
+/*
+ * ftk_score_dense -- the fused scores themselves, for checking: for each
+ * listed row r (query t = rows ? rows[r] : r) writes
+ *     out[r * ld + (s - ks[t])] = I[t, s]   for s in [ks[t], ke[t])
+ * with exactly the arithmetic ftk_select uses (same kernel, same bits).
+ * Entries past a row's window are left untouched.
+ *   rows   device [nrows] int32 query indices, or NULL for 0 .. nrows-1
+ *   out    device float32 [nrows, ld], ld >= max window length, ld % 4 == 0
+ *   workspace  as for ftk_select, sized by ftk_score_dense_workspace_size
+ * Other arguments as for ftk_select.
+ */
+ftk_status ftk_score_dense(ftk_dtype dtype, const void *q, const void *kv,
+                           const float *kv_scales, const float *weights,
+                           const int32_t *ks, const int32_t *ke, int64_t T,
+                           int64_t S, const int32_t *rows, int64_t nrows,
+                           float *out, int64_t ld, void *workspace,
+                           size_t workspace_bytes, void *stream);
+
+size_t ftk_score_dense_workspace_size(int64_t nrows);
+
+/*
+ * ftk_windows_from_cu_seqlens -- causal windows of packed sequences
+ * (FlashTopK README, "Usage": windows_from_cu_seqlens).  Sequence j owns
+ * query rows [cu_q[j], cu_q[j+1]) and keys [cu_k[j], cu_k[j+1]); its
+ * queries are its last tokens, so its i-th query sees keys
+ *     [cu_k[j], cu_k[j] + (Lk_j - Lq_j) + i + 1)
+ * (FlashTopK README, "Quick start": query i sees keys [0, S - T + i + 1)),
+ * clamped to an empty window when Lk_j < Lq_j - i.
+ *   cu_q, cu_k  device [nseq + 1] int32 prefix offsets, cu_q[nseq] == T
+ *   ks, ke      device [T] int32 outputs
+ */
+ftk_status ftk_windows_from_cu_seqlens(const int32_t *cu_q,
+                                       const int32_t *cu_k, int64_t nseq,
+                                       int64_t T, int32_t *ks, int32_t *ke,
+                                       void *stream);
+
+/* Human-readable name of an ftk_status value (static string). */
+const char *ftk_status_string(int status);
+
+/* Library version as MAJOR * 10000 + MINOR * 100 + PATCH. */
+int ftk_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FTK_H */

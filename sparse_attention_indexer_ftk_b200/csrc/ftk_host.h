@@ -1,0 +1,57 @@
+// ftk_host.h -- host-side helpers shared by the libftk entry points.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/ftk.h"
+
+namespace ftk {
+
+inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// FTK_OK when the current device is compute capability 10.0 (B200, sm_100a).
+ftk_status check_device();
+
+// Maps a CUDA error to FTK_ERR_CUDA (and clears the sticky launch error
+// only for launch-configuration errors, which do not poison the context).
+inline ftk_status cuda_status(cudaError_t e)
+{
+    if (e == cudaSuccess) return FTK_OK;
+    (void)cudaGetLastError();
+    return FTK_ERR_CUDA;
+}
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Bump allocator over a caller-owned workspace (256-byte aligned pieces).
+struct Carver {
+    uint8_t *base;
+    size_t size;
+    size_t used = 0;
+    bool ok = true;
+    template <class T>
+    T *take(size_t count)
+    {
+        size_t off = align_up(used, 256);
+        size_t bytes = align_up(count * sizeof(T), 256);
+        if (base == nullptr || off + bytes > size) {
+            ok = false;
+            used = off + bytes;
+            return nullptr;
+        }
+        used = off + bytes;
+        return reinterpret_cast<T *>(base + off);
+    }
+};
+
+struct RowsArgs;
+// Launches the row top-k kernel for the given dtype (FTK_BF16 / FTK_F32)
+// with one cluster of `cluster` CTAs per grid row.
+ftk_status launch_rows_topk(int dtype, const RowsArgs &a, int cluster, cudaStream_t stream);
+// Cluster size and per-CTA chunk for rows of `cols` columns.
+void rows_plan(int64_t rows, int64_t cols, int *cluster, int *chunk);
+
+}  // namespace ftk

@@ -1,0 +1,109 @@
+// ftk_rows.cu -- host side of the row top-k (ftk_topk_rows) and the launch
+// helper the dense-recovery step reuses.
+#include <stdio.h>
+#include <stdlib.h>
+
+#include "ftk_host.h"
+#include "ftk_rows.cuh"
+
+namespace ftk {
+
+ftk_status check_device()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cuda_status(cudaErrorInvalidDevice);
+    static int cached[64];  // 0 unknown, 1 ok, 2 wrong arch
+    if (dev >= 0 && dev < 64 && cached[dev]) return cached[dev] == 1 ? FTK_OK : FTK_ERR_DEVICE;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+        return cuda_status(cudaErrorInvalidDevice);
+    const bool ok = major == 10 && minor == 0;
+    if (dev >= 0 && dev < 64) cached[dev] = ok ? 1 : 2;
+    return ok ? FTK_OK : FTK_ERR_DEVICE;
+}
+
+static int env_int(const char *name, int dflt)
+{
+    const char *v = getenv(name);
+    return v && *v ? atoi(v) : dflt;
+}
+
+void rows_plan(int64_t rows, int64_t cols, int *cluster, int *chunk)
+{
+    // Enough CTAs to keep every SM streaming (two per SM), and a chunk that
+    // fits the shared-memory budget.
+    int cs = 1;
+    while (cs < kRowsMaxCluster && (rows * cs < 2 * 148 || (cols + cs - 1) / cs > kRowsMaxChunk))
+        cs *= 2;
+    const int forced = env_int("FTK_ROWS_CLUSTER", 0);
+    if (forced == 1 || forced == 2 || forced == 4 || forced == 8) cs = forced;
+    int64_t ch = (cols + cs - 1) / cs;
+    ch = (ch + 7) / 8 * 8;
+    *cluster = cs;
+    *chunk = static_cast<int>(ch);
+}
+
+template <int DT>
+static ftk_status launch_rows_dt(const RowsArgs &a, int cluster, cudaStream_t stream)
+{
+    const size_t smem = sizeof(RowsSmem) + static_cast<size_t>(a.chunk) * 2;
+    auto kern = rows_topk_kernel<DT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return cuda_status(e);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(a.rows * cluster), 1, 1);
+    cfg.blockDim = dim3(kRowsThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cuda_status(cudaLaunchKernelEx(&cfg, kern, a));
+}
+
+ftk_status launch_rows_topk(int dtype, const RowsArgs &a, int cluster, cudaStream_t stream)
+{
+    if (a.chunk <= 0 || a.chunk > kRowsMaxChunk || a.chunk % 8) return FTK_ERR_UNSUPPORTED;
+    if (dtype == FTK_BF16) return launch_rows_dt<FTK_BF16>(a, cluster, stream);
+    if (dtype == FTK_F32) return launch_rows_dt<FTK_F32>(a, cluster, stream);
+    return FTK_ERR_UNSUPPORTED;
+}
+
+}  // namespace ftk
+
+using namespace ftk;
+
+extern "C" ftk_status ftk_topk_rows(ftk_dtype dtype, const void *x, int64_t rows, int64_t cols,
+                                    int64_t row_stride, int topk, int32_t *out_idx,
+                                    void *out_val, uint32_t *status, void *stream)
+{
+    if (dtype != FTK_BF16 && dtype != FTK_F32) return FTK_ERR_UNSUPPORTED;
+    if (!x || !out_idx) return FTK_ERR_INVALID_ARG;
+    if (rows < 1 || cols < 1 || row_stride < cols || rows > (int64_t(1) << 31) / kRowsMaxCluster)
+        return FTK_ERR_INVALID_ARG;
+    if (topk < 1 || topk > FTK_MAX_TOPK) return FTK_ERR_TOPK_RANGE;
+    if (cols > static_cast<int64_t>(kRowsMaxCluster) * kRowsMaxChunk) return FTK_ERR_UNSUPPORTED;
+    const int esz = dtype == FTK_BF16 ? 2 : 4;
+    if (!aligned16(x) || (row_stride * esz) % 16) return FTK_ERR_ALIGNMENT;
+    ftk_status st = check_device();
+    if (st != FTK_OK) return st;
+    RowsArgs a = {};
+    a.x = x;
+    a.ld = row_stride;
+    a.cols = cols;
+    a.rows = rows;
+    a.out_idx = out_idx;
+    a.out_val = out_val;
+    a.k = topk;
+    a.status = status;
+    int cluster = 1, chunk = 8;
+    rows_plan(rows, cols, &cluster, &chunk);
+    a.chunk = chunk;
+    return launch_rows_topk(dtype, a, cluster, as_stream(stream));
+}

@@ -1,0 +1,536 @@
+// ftk_score.cuh -- fused lightning-indexer scoring on the 5th-generation
+// tensor cores (tcgen05 + TMEM, operands staged by TMA).
+//
+// Score (FlashTopK README, "Quick start"):
+//     I[t,s] = sigma_s * sum_{h<32} w[t,h] * ReLU(q[t,h] . k[s])
+//
+// GEMM orientation: A = a tile of 128 keys (M = 128, K = 128 head dims),
+// B = a tile of 8 queries x 32 heads (N = 256), both K-major with the
+// 128-byte swizzle.  The fp32 accumulator tile (128 lanes x 256 columns)
+// lives in tensor memory, double-buffered (2 x 256 of the 512 columns), so
+// the MMA of key tile i+1 overlaps the epilogue of key tile i.  TMEM lane =
+// key, so each epilogue thread owns one key and reduces the 32 heads of a
+// query in registers: ReLU, the head weights and sigma are applied and the
+// T x S x 32 intermediate never leaves the SM.
+//
+// Warp roles (10 warps):
+//   warp 0      TMA producer: q tile per work item, key tiles through a
+//               multi-stage mbarrier ring;
+//   warp 1      TMEM allocator and MMA issuer (one elected thread);
+//   warps 2-9   epilogue: warp w reads TMEM lane quarter (w % 4) and the
+//               queries 4*((w-2)/4) .. +3 of the tile.
+//
+// Modes (one kernel body, so every mode produces bit-identical scores):
+//   SAMPLE   keys are a strided sample k[j*stride] (a strided TMA view of kv);
+//            scores go to a dense [row, sample] buffer (the threshold input);
+//   COLLECT  keeps the keys with I >= tau[t] (NaN kept too, so that it is
+//            seen): warp ballot + shared-memory staging, flushed to per-row
+//            candidate buffers with one global atomic per query per flush;
+//   DUMP     writes every in-window score to out[row, s - ks[t]] (dense
+//            recovery of rows the threshold missed, and score checks).
+#pragma once
+
+#include "ftk_device.cuh"
+
+namespace ftk {
+
+enum ScoreMode { MODE_SAMPLE = 0, MODE_COLLECT = 1, MODE_DUMP = 2 };
+
+constexpr int kQTile = 8;            // queries per tile -> N = 256
+constexpr int kKeyTile = 128;        // keys per tile -> M = 128
+constexpr int kChunkTiles = 128;     // key tiles per work item (16384 keys)
+constexpr int kChunkKeys = kChunkTiles * kKeyTile;
+constexpr int kScoreThreads = 320;   // 10 warps
+constexpr int kEpiThreads = 256;     // warps 2..9
+constexpr int kNumStrideMaps = 20;   // sample strides 2^0 .. 2^19
+
+template <int DT>
+struct ScoreCfg;
+
+template <>
+struct ScoreCfg<FTK_F8E4M3> {
+    static constexpr int kAtoms = 1;      // 128-byte swizzle atoms along K (128 dims x 1 B)
+    static constexpr int kQStages = 2;
+    static constexpr int kKStages = 4;
+    static constexpr int kStageCap = 1024; // staged candidates per query
+    static constexpr int kMmaK = 4;       // MMAs per tile (K = 32 each)
+    static constexpr uint32_t kIdesc = instr_desc(0, 0, 128, 256);  // e4m3 x e4m3 -> f32
+};
+
+template <>
+struct ScoreCfg<FTK_BF16> {
+    static constexpr int kAtoms = 2;      // 128 dims x 2 B = two 128-byte atoms
+    static constexpr int kQStages = 1;
+    static constexpr int kKStages = 3;
+    static constexpr int kStageCap = 512;
+    static constexpr int kMmaK = 8;       // K = 16 each
+    static constexpr uint32_t kIdesc = instr_desc(1, 1, 128, 256);  // bf16 x bf16 -> f32
+};
+
+struct ScoreArgs {
+    int64_t T, S;
+    const float *kv_scales;   // [S] or NULL (all ones)
+    const float *weights;     // [T, 32]
+    const int32_t *ks, *ke;   // [T]
+    // Row list: position p of the list is query rows[p] (identity if NULL).
+    // The list holds min(nrows, *count_dev - count_off) rows when count_dev
+    // is given (device-side counts, e.g. the rows that need recovery).
+    const int32_t *rows;
+    int64_t nrows;
+    const int32_t *count_dev;
+    int32_t count_off;
+    // Schedule.  Planned: per-tile ranges and an item prefix written by the
+    // plan kernel.  Static: item = (tile, chunk), ranges found on the fly.
+    int32_t planned;
+    const int32_t *tile_lo, *tile_hi, *tile_lg, *item_start;
+    int32_t ntiles;
+    int32_t static_chunks;
+    // COLLECT
+    const float *tau;         // [T]
+    int32_t *cnt;             // [T] running candidate counts
+    float *cand_val;          // [T, cap]
+    int32_t *cand_idx;        // [T, cap]
+    int32_t cap;
+    // SAMPLE / DUMP output rows of stride ld
+    float *out;
+    int64_t ld;
+    uint32_t *status;
+};
+
+struct KvMaps {
+    CUtensorMap m[kNumStrideMaps];  // m[i]: kv rows 0, 2^i, 2*2^i, ... (m[0] = kv itself)
+};
+
+struct Item {
+    int32_t tile;
+    int32_t key0;   // first key (SAMPLE: first sample index j)
+    int32_t kend;   // end key (SAMPLE: end sample index)
+    int32_t nkt;    // key tiles in this item
+    int32_t lg;     // SAMPLE: log2 of the stride
+};
+
+__device__ __forceinline__ int64_t list_rows(const ScoreArgs &a)
+{
+    int64_t n = a.nrows;
+    if (a.count_dev) {
+        int64_t c = static_cast<int64_t>(*a.count_dev) - a.count_off;
+        n = c < 0 ? 0 : (c < n ? c : n);
+    }
+    return n;
+}
+
+__device__ __forceinline__ bool window_ok(int64_t ks, int64_t ke, int64_t S)
+{
+    return ks >= 0 && ks <= ke && ke <= S;
+}
+
+// Query row of list position p, or -1 if the position is empty or the
+// row's window is invalid (such rows are masked out of every tile).
+__device__ __forceinline__ int32_t list_query(const ScoreArgs &a, int64_t p, int64_t nlist)
+{
+    if (p >= nlist) return -1;
+    const int64_t t = a.rows ? a.rows[p] : p;
+    if (t < 0 || t >= a.T) return -1;
+    if (!window_ok(a.ks[t], a.ke[t], a.S)) return -1;
+    return static_cast<int32_t>(t);
+}
+
+template <int MODE>
+__device__ __forceinline__ bool get_item(const ScoreArgs &a, int it, int64_t nlist, Item &m)
+{
+    if (a.planned) {
+        const int32_t nt = a.ntiles;
+        if (it >= a.item_start[nt]) return false;
+        int lo = 0, hi = nt;  // largest tile with item_start[tile] <= it
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (a.item_start[mid] <= it) lo = mid; else hi = mid;
+        }
+        m.tile = lo;
+        const int chunk = it - a.item_start[lo];
+        if (MODE == MODE_SAMPLE) {
+            m.lg = a.tile_lg[lo];
+            m.key0 = a.tile_lo[lo];
+            m.kend = a.tile_hi[lo];
+        } else {
+            m.lg = 0;
+            m.key0 = a.tile_lo[lo] + chunk * kChunkKeys;
+            m.kend = min(a.tile_hi[lo], m.key0 + kChunkKeys);
+        }
+    } else {
+        m.tile = it / a.static_chunks;
+        const int chunk = it - m.tile * a.static_chunks;
+        m.lg = 0;
+        int64_t lo = INT64_MAX, hi = -1;
+        for (int j = 0; j < kQTile; ++j) {
+            const int32_t t = list_query(a, static_cast<int64_t>(m.tile) * kQTile + j, nlist);
+            if (t < 0 || a.ks[t] == a.ke[t]) continue;
+            lo = min(lo, static_cast<int64_t>(a.ks[t]));
+            hi = max(hi, static_cast<int64_t>(a.ke[t]));
+        }
+        if (hi < 0) return false;
+        lo &= ~static_cast<int64_t>(kKeyTile - 1);
+        const int64_t k0 = lo + static_cast<int64_t>(chunk) * kChunkKeys;
+        if (k0 >= hi) return false;
+        m.key0 = static_cast<int32_t>(k0);
+        m.kend = static_cast<int32_t>(min(hi, k0 + kChunkKeys));
+    }
+    m.nkt = (m.kend - m.key0 + kKeyTile - 1) / kKeyTile;
+    return m.nkt > 0;
+}
+
+// The head reduction of one (query, key) pair: sum_h w_h * max(x_h, 0) in a
+// fixed order (four interleaved partial sums), then sigma, then +0.0 turns
+// a -0.0 into +0.0.  Every mode and every caller uses exactly this.
+__device__ __forceinline__ float head_reduce(const float (&x)[32], const float *w, float sigma)
+{
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+    for (int h = 0; h < 32; h += 4) {
+        const float4 wv = *reinterpret_cast<const float4 *>(w + h);
+        a0 = __fmaf_rn(wv.x, fmaxf(x[h + 0], 0.f), a0);
+        a1 = __fmaf_rn(wv.y, fmaxf(x[h + 1], 0.f), a1);
+        a2 = __fmaf_rn(wv.z, fmaxf(x[h + 2], 0.f), a2);
+        a3 = __fmaf_rn(wv.w, fmaxf(x[h + 3], 0.f), a3);
+    }
+    const float acc = __fadd_rn(__fadd_rn(a0, a1), __fadd_rn(a2, a3));
+    return __fmaf_rn(sigma, acc, 0.0f);
+}
+
+template <int DT>
+struct ScoreSmemLayout {
+    using C = ScoreCfg<DT>;
+    static constexpr int kQBytes = C::kAtoms * kQTile * kHeads * 128;   // 32 KB per atom
+    static constexpr int kKBytes = C::kAtoms * kKeyTile * 128;          // 16 KB per atom
+    static constexpr int kOffQ = 0;
+    static constexpr int kOffK = kOffQ + C::kQStages * kQBytes;
+    static constexpr int kOffStageVal = kOffK + C::kKStages * kKBytes;
+    static constexpr int kOffStageIdx = kOffStageVal + kQTile * C::kStageCap * 4;
+    static constexpr int kOffW = kOffStageIdx + kQTile * C::kStageCap * 4;
+    static constexpr int kOffMisc = kOffW + kQTile * kHeads * 4;
+    static constexpr int kMiscBytes = 512;  // >= sizeof(ScoreMisc), checked below
+    static constexpr int kBytes = kOffMisc + kMiscBytes + 1024;  // + alignment slack
+};
+
+struct ScoreMisc {
+    uint64_t kv_full[4], kv_empty[4];
+    uint64_t q_full[2], q_empty[2];
+    uint64_t acc_full[2], acc_empty[2];
+    uint64_t final_bar;
+    uint64_t epi_bar;          // group barrier of the epilogue warps
+    uint32_t tmem_base;
+    int32_t flush_now;
+    int32_t abort;
+    int32_t qt[kQTile];        // query of each tile slot (-1: none)
+    int32_t qks[kQTile], qke[kQTile];
+    float qtau[kQTile];
+    int32_t stage_cnt[kQTile];
+    int32_t qpos[kQTile];      // list position of each tile slot
+};
+
+static_assert(sizeof(ScoreMisc) <= ScoreSmemLayout<FTK_F8E4M3>::kMiscBytes, "misc area");
+static_assert(ScoreSmemLayout<FTK_F8E4M3>::kBytes <= 227 * 1024, "fp8 smem budget");
+static_assert(ScoreSmemLayout<FTK_BF16>::kBytes <= 227 * 1024, "bf16 smem budget");
+
+template <int DT, int MODE>
+__global__ void __launch_bounds__(kScoreThreads, 1)
+    score_kernel(const __grid_constant__ ScoreArgs a, const __grid_constant__ CUtensorMap tm_q,
+                 const __grid_constant__ KvMaps kvm)
+{
+    using C = ScoreCfg<DT>;
+    using Lay = ScoreSmemLayout<DT>;
+    extern __shared__ uint8_t smem_dyn[];
+    // 1024-byte alignment: the 128-byte swizzle pattern repeats every 8 rows.
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t *sq = smem + Lay::kOffQ;
+    uint8_t *sk = smem + Lay::kOffK;
+    float *stage_val = reinterpret_cast<float *>(smem + Lay::kOffStageVal);
+    int32_t *stage_idx = reinterpret_cast<int32_t *>(smem + Lay::kOffStageIdx);
+    float *sw = reinterpret_cast<float *>(smem + Lay::kOffW);
+    ScoreMisc &ms = *reinterpret_cast<ScoreMisc *>(smem + Lay::kOffMisc);
+    volatile int *abort = &ms.abort;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t nlist = list_rows(a);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < C::kKStages; ++i) {
+            mbar_init(&ms.kv_full[i], 1);
+            mbar_init(&ms.kv_empty[i], 1);
+        }
+        for (int i = 0; i < C::kQStages; ++i) {
+            mbar_init(&ms.q_full[i], 1);
+            mbar_init(&ms.q_empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&ms.acc_full[i], 1);
+            mbar_init(&ms.acc_empty[i], kEpiThreads / 32);
+        }
+        mbar_init(&ms.final_bar, 1);
+        mbar_init(&ms.epi_bar, kEpiThreads);
+        ms.abort = 0;
+        for (int j = 0; j < kQTile; ++j) ms.stage_cnt[j] = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) tmem_alloc(&ms.tmem_base, 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ms.tmem_base;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_q);
+            int ks_ = 0, qs = 0;
+            uint32_t kph = 0, qph = 0;
+            int k_armed[4] = {0, 0, 0, 0};  // loads issued per stage, for the abort drain
+            uint32_t k_armed_ph[4] = {0, 0, 0, 0};
+            int q_armed[2] = {0, 0};
+            uint32_t q_armed_ph[2] = {0, 0};
+            for (int it = blockIdx.x; !*abort; it += gridDim.x) {
+                Item m;
+                if (a.planned) {
+                    if (it >= a.item_start[a.ntiles]) break;
+                    if (!get_item<MODE>(a, it, nlist, m)) continue;
+                } else {
+                    if (it >= a.static_chunks * ((a.nrows + kQTile - 1) / kQTile)) break;
+                    if (!get_item<MODE>(a, it, nlist, m)) continue;
+                }
+                // q tile: the 32 head rows of each of the 8 queries.
+                if (!mbar_wait(&ms.q_empty[qs], qph ^ 1u, abort, a.status)) break;
+                mbar_arrive_expect_tx(&ms.q_full[qs], Lay::kQBytes);
+                q_armed[qs] = 1;
+                q_armed_ph[qs] = qph;
+                for (int j = 0; j < kQTile; ++j) {
+                    int32_t t = list_query(a, static_cast<int64_t>(m.tile) * kQTile + j, nlist);
+                    if (t < 0) t = 0;  // placeholder rows are masked in the epilogue
+                    for (int at = 0; at < C::kAtoms; ++at)
+                        tma_load_2d(sq + qs * Lay::kQBytes + at * (Lay::kQBytes / C::kAtoms) +
+                                        j * kHeads * 128,
+                                    &tm_q, &ms.q_full[qs], at * 64, t * kHeads);
+                }
+                if (++qs == C::kQStages) { qs = 0; qph ^= 1u; }
+                const CUtensorMap *map = &kvm.m[MODE == MODE_SAMPLE ? m.lg : 0];
+                for (int kt = 0; kt < m.nkt; ++kt) {
+                    if (!mbar_wait(&ms.kv_empty[ks_], kph ^ 1u, abort, a.status)) break;
+                    mbar_arrive_expect_tx(&ms.kv_full[ks_], Lay::kKBytes);
+                    k_armed[ks_] = 1;
+                    k_armed_ph[ks_] = kph;
+                    const int32_t y = m.key0 + kt * kKeyTile;
+                    for (int at = 0; at < C::kAtoms; ++at)
+                        tma_load_2d(sk + ks_ * Lay::kKBytes + at * (Lay::kKBytes / C::kAtoms), map,
+                                    &ms.kv_full[ks_], at * 64, y);
+                    if (++ks_ == C::kKStages) { ks_ = 0; kph ^= 1u; }
+                }
+            }
+            if (*abort) {
+                // Drain: every issued TMA load lands before the CTA exits.
+                for (int i = 0; i < C::kKStages; ++i)
+                    if (k_armed[i]) mbar_wait_drain(&ms.kv_full[i], k_armed_ph[i]);
+                for (int i = 0; i < C::kQStages; ++i)
+                    if (q_armed[i]) mbar_wait_drain(&ms.q_full[i], q_armed_ph[i]);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int ks_ = 0, qs = 0, ab = 0;
+            uint32_t kph = 0, qph = 0, aph = 0;
+            bool issued = false;
+            for (int it = blockIdx.x; !*abort; it += gridDim.x) {
+                Item m;
+                if (a.planned) {
+                    if (it >= a.item_start[a.ntiles]) break;
+                    if (!get_item<MODE>(a, it, nlist, m)) continue;
+                } else {
+                    if (it >= a.static_chunks * ((a.nrows + kQTile - 1) / kQTile)) break;
+                    if (!get_item<MODE>(a, it, nlist, m)) continue;
+                }
+                if (!mbar_wait(&ms.q_full[qs], qph, abort, a.status)) break;
+                tc_fence_after();
+                const uint32_t qaddr = smem_u32(sq + qs * Lay::kQBytes);
+                bool ok = true;
+                for (int kt = 0; kt < m.nkt; ++kt) {
+                    if (!mbar_wait(&ms.acc_empty[ab], aph ^ 1u, abort, a.status) ||
+                        !mbar_wait(&ms.kv_full[ks_], kph, abort, a.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t kaddr = smem_u32(sk + ks_ * Lay::kKBytes);
+                    const uint32_t d = tmem + static_cast<uint32_t>(ab * 256);
+#pragma unroll
+                    for (int kk = 0; kk < C::kMmaK; ++kk) {
+                        const int at = kk / 4, off = (kk % 4) * 32;
+                        const uint64_t ad = smem_desc_sw128(kaddr + at * (Lay::kKBytes / C::kAtoms) + off);
+                        const uint64_t bd = smem_desc_sw128(qaddr + at * (Lay::kQBytes / C::kAtoms) + off);
+                        if (DT == FTK_F8E4M3)
+                            mma_f8f6f4(d, ad, bd, C::kIdesc, kk > 0 ? 1u : 0u);
+                        else
+                            mma_f16(d, ad, bd, C::kIdesc, kk > 0 ? 1u : 0u);
+                    }
+                    issued = true;
+                    mma_commit(&ms.kv_empty[ks_]);
+                    mma_commit(&ms.acc_full[ab]);
+                    if (++ks_ == C::kKStages) { ks_ = 0; kph ^= 1u; }
+                    if (++ab == 2) { ab = 0; aph ^= 1u; }
+                }
+                mma_commit(&ms.q_empty[qs]);
+                if (++qs == C::kQStages) { qs = 0; qph ^= 1u; }
+                if (!ok) break;
+            }
+            // Every issued MMA completes before TMEM is released.
+            if (issued) {
+                mma_commit(&ms.final_bar);
+                mbar_wait_drain(&ms.final_bar, 0);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int ew = warp - 2;                 // 0..7
+        const int quad = warp & 3;               // TMEM lane quarter
+        const int half = ew >> 2;                // queries 4*half .. 4*half+3
+        const int et = threadIdx.x - 64;         // 0..255
+        const int key_lane = quad * 32 + lane;   // row of the 128-key tile
+        const uint32_t tlane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+        int ab = 0;
+        uint32_t aph = 0, eph = 0;
+        bool bad_scale = false;
+        for (int it = blockIdx.x; !*abort; it += gridDim.x) {
+            Item m;
+            if (a.planned) {
+                if (it >= a.item_start[a.ntiles]) break;
+                if (!get_item<MODE>(a, it, nlist, m)) continue;
+            } else {
+                if (it >= a.static_chunks * ((a.nrows + kQTile - 1) / kQTile)) break;
+                if (!get_item<MODE>(a, it, nlist, m)) continue;
+            }
+            // The previous item (and its flush) is retired before its
+            // per-query parameters are replaced.
+            if (!__all_sync(0xFFFFFFFFu, group_sync(&ms.epi_bar, eph, abort, a.status))) break;
+            {
+                const int j = et >> 5, h = et & 31;
+                const int64_t p = static_cast<int64_t>(m.tile) * kQTile + j;
+                const int32_t t = list_query(a, p, nlist);
+                sw[j * kHeads + h] = t >= 0 ? a.weights[static_cast<int64_t>(t) * kHeads + h] : 0.f;
+                if (h == 0) {
+                    ms.qt[j] = t;
+                    ms.qpos[j] = static_cast<int32_t>(p);
+                    ms.qks[j] = t >= 0 ? a.ks[t] : 0;
+                    ms.qke[j] = t >= 0 ? a.ke[t] : 0;
+                    ms.qtau[j] = (MODE == MODE_COLLECT && t >= 0) ? a.tau[t] : 0.f;
+                }
+            }
+            if (!__all_sync(0xFFFFFFFFu, group_sync(&ms.epi_bar, eph, abort, a.status))) break;
+            bool ok = true;
+            for (int kt = 0; kt < m.nkt; ++kt) {
+                const int32_t kidx = m.key0 + kt * kKeyTile + key_lane;  // key (SAMPLE: sample j)
+                int64_t s;
+                bool in_range;
+                if (MODE == MODE_SAMPLE) {
+                    s = static_cast<int64_t>(kidx) << m.lg;
+                    in_range = kidx < m.kend && s < a.S;
+                } else {
+                    s = kidx;
+                    in_range = kidx < m.kend;
+                }
+                float sigma = 1.f;
+                if (a.kv_scales && in_range) {
+                    sigma = __ldg(a.kv_scales + s);
+                    bad_scale |= !(sigma > 0.f) || isinf(sigma);
+                }
+                const bool got = mbar_wait(&ms.acc_full[ab], aph, abort, a.status);
+                if (!__all_sync(0xFFFFFFFFu, got)) {  // also reconverges the warp
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll 1
+                for (int qi = 0; qi < 4; ++qi) {
+                    const int j = half * 4 + qi;
+                    float x[32];
+                    tmem_ld32(tlane + static_cast<uint32_t>(ab * 256 + j * 32), x);
+                    const float I = head_reduce(x, sw + j * kHeads, sigma);
+                    const int32_t t = ms.qt[j];
+                    const bool valid = in_range && t >= 0 && s >= ms.qks[j] && s < ms.qke[j];
+                    if (MODE == MODE_COLLECT) {
+                        const bool take = valid && !(I < ms.qtau[j]);
+                        const uint32_t bal = __ballot_sync(0xFFFFFFFFu, take);
+                        if (bal) {
+                            const int leader = __ffs(bal) - 1;
+                            int base = 0;
+                            if (lane == leader) base = atomicAdd(&ms.stage_cnt[j], __popc(bal));
+                            base = __shfl_sync(0xFFFFFFFFu, base, leader);
+                            if (take) {
+                                const int pos = base + __popc(bal & ((1u << lane) - 1u));
+                                stage_val[j * C::kStageCap + pos] = I;
+                                stage_idx[j * C::kStageCap + pos] = static_cast<int32_t>(s);
+                            }
+                        }
+                    } else if (MODE == MODE_SAMPLE) {
+                        if (t >= 0 && kidx < m.kend)
+                            a.out[static_cast<int64_t>(t) * a.ld + (kidx - m.key0)] =
+                                valid ? I : -INFINITY;
+                    } else {
+                        if (valid)
+                            a.out[static_cast<int64_t>(ms.qpos[j]) * a.ld + (s - ms.qks[j])] = I;
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ms.acc_empty[ab]);
+                if (++ab == 2) { ab = 0; aph ^= 1u; }
+                if (MODE == MODE_COLLECT) {
+                    // Every candidate of this tile is staged; one thread decides
+                    // whether the staging buffers must be flushed before another
+                    // tile (<= 128 more per query) could overflow them.
+                    if (!__all_sync(0xFFFFFFFFu, group_sync(&ms.epi_bar, eph, abort, a.status))) { ok = false; break; }
+                    if (et == 0) {
+                        bool need = kt == m.nkt - 1;
+#pragma unroll
+                        for (int j = 0; j < kQTile; ++j)
+                            need |= ms.stage_cnt[j] > C::kStageCap - kKeyTile;
+                        ms.flush_now = need;
+                    }
+                    if (!__all_sync(0xFFFFFFFFu, group_sync(&ms.epi_bar, eph, abort, a.status))) { ok = false; break; }
+                    if (ms.flush_now) {
+                        const int j = ew;  // warp ew flushes query slot ew
+                        const int n = ms.stage_cnt[j];
+                        const int32_t t = ms.qt[j];
+                        if (n > 0 && t >= 0) {
+                            int base = 0;
+                            if (lane == 0) base = atomicAdd(a.cnt + t, n);
+                            base = __shfl_sync(0xFFFFFFFFu, base, 0);
+                            float *cv = a.cand_val + static_cast<int64_t>(t) * a.cap;
+                            int32_t *ci = a.cand_idx + static_cast<int64_t>(t) * a.cap;
+                            for (int i = lane; i < n; i += 32) {
+                                const int slot = base + i;
+                                if (slot < a.cap) {
+                                    cv[slot] = stage_val[j * C::kStageCap + i];
+                                    ci[slot] = stage_idx[j * C::kStageCap + i];
+                                }
+                            }
+                        }
+                        __syncwarp();
+                        if (lane == 0) ms.stage_cnt[j] = 0;
+                        if (!__all_sync(0xFFFFFFFFu, group_sync(&ms.epi_bar, eph, abort, a.status))) { ok = false; break; }
+                    }
+                }
+            }
+            if (!ok) break;
+        }
+        if (bad_scale) set_status(a.status, FTK_STATUS_BAD_SCALE);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace ftk

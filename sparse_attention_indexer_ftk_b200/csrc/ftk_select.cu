@@ -1,0 +1,856 @@
+// ftk_select.cu -- exact fused indexer top-k (ftk_select) and the dense
+// score dump (ftk_score_dense).
+//
+// Per call, all stream-ordered, no host synchronisation:
+//   plan       one CTA: zeroes the per-call state, checks every window and
+//              lays out the work items of the sample and scan passes;
+//   sample     score_kernel<SAMPLE>: each query tile scores a strided sample
+//              of its windows (stride a power of two, so the sample of each
+//              row is a strided sample of the row's own window -- FlashTopK
+//              README, "Highlights": CP-compatible per-row thresholds);
+//   threshold  per row: tau = the r-th largest sampled score, r chosen so
+//              that about oversample * topk keys pass; tau = -inf when the
+//              whole window fits in the candidate buffer;
+//   scan       score_kernel<COLLECT>: dense fused scoring, keeping I >= tau;
+//   refine     per row: exact radix select of the topk candidates with the
+//              (score desc, index asc) order, written in ascending index
+//              order; rows whose candidates overflowed or fell short of
+//              min(topk, L) are listed for recovery instead (triage);
+//   recovery   score_kernel<DUMP> rescores the listed rows' whole windows
+//              into scratch rows with the same arithmetic, and the row top-k
+//              kernel selects from them (FlashTopK README, "Highlights":
+//              rows the sampled threshold misses are rescored on the GPU).
+#include <cudaTypedefs.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include "ftk_host.h"
+#include "ftk_rows.cuh"
+#include "ftk_score.cuh"
+
+namespace ftk {
+
+constexpr int kPlanThreads = 1024;
+constexpr int kSelThreads = 256;
+constexpr int kBitmapWords = 2048;   // 65536-key segments for the ordered output
+
+// Device copy of ftk_info plus counters (same layout for the leading part).
+struct DevInfo {
+    ftk_info info;
+};
+
+// ---------------------------------------------------------------------------
+// plan
+// ---------------------------------------------------------------------------
+
+struct PlanArgs {
+    int64_t T, S;
+    const int32_t *ks, *ke;
+    int32_t ntiles;
+    int32_t sample_keys;
+    // sample pass
+    int32_t *s_lo, *s_hi, *s_lg, *s_start;
+    // scan pass
+    int32_t *c_lo, *c_hi, *c_start;
+    int32_t *cnt;
+    int32_t *bad_count;
+    DevInfo *info;
+};
+
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *sh, uint32_t &total)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    uint32_t inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t u = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+        if (lane >= o) inc += u;
+    }
+    if (lane == 31) sh[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+        const uint32_t x = lane < nw ? sh[lane] : 0;
+        uint32_t y = x;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t u = __shfl_up_sync(0xFFFFFFFFu, y, o);
+            if (lane >= o) y += u;
+        }
+        if (lane < nw) sh[32 + lane] = y - x;
+        if (lane == 31) sh[64] = y;
+    }
+    __syncthreads();
+    const uint32_t r = sh[32 + warp] + inc - v;
+    total = sh[64];
+    __syncthreads();
+    return r;
+}
+
+__global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanArgs p)
+{
+    __shared__ uint32_t sh[96];
+    const int tid = threadIdx.x;
+    bool bad = false;
+    for (int64_t t = tid; t < p.T; t += blockDim.x) {
+        p.cnt[t] = 0;
+        bad |= !window_ok(p.ks[t], p.ke[t], p.S);
+    }
+    if (tid == 0) {
+        *p.bad_count = 0;
+        memset(&p.info->info, 0, sizeof(ftk_info));
+        p.info->info.rows = p.T;
+    }
+    __syncthreads();
+    if (bad) atomicOr(&p.info->info.status, FTK_STATUS_BAD_WINDOW);
+    uint32_t carry_s = 0, carry_c = 0;
+    for (int32_t base = 0; base < p.ntiles; base += blockDim.x) {
+        const int32_t tile = base + tid;
+        uint32_t ns = 0, nc = 0;
+        if (tile < p.ntiles) {
+            int64_t lo = INT64_MAX, hi = -1;
+            for (int j = 0; j < kQTile; ++j) {
+                const int64_t t = static_cast<int64_t>(tile) * kQTile + j;
+                if (t >= p.T) break;
+                const int64_t a = p.ks[t], b = p.ke[t];
+                if (!window_ok(a, b, p.S) || a == b) continue;
+                lo = min(lo, a);
+                hi = max(hi, b);
+            }
+            int32_t slo = 0, shi = 0, slg = 0, clo = 0, chi = 0;
+            if (hi >= 0) {
+                const int64_t L = hi - lo;
+                const int64_t want = (L + p.sample_keys - 1) / p.sample_keys;  // >= 1
+                int lg = 0;
+                while ((int64_t(1) << lg) < want) ++lg;
+                const int64_t j0 = (lo + (int64_t(1) << lg) - 1) >> lg;
+                const int64_t j1 = (hi + (int64_t(1) << lg) - 1) >> lg;
+                slo = static_cast<int32_t>(j0);
+                shi = static_cast<int32_t>(j1);
+                slg = lg;
+                ns = j1 > j0 ? 1u : 0u;
+                const int64_t lo_al = lo & ~static_cast<int64_t>(kKeyTile - 1);
+                clo = static_cast<int32_t>(lo_al);
+                chi = static_cast<int32_t>(hi);
+                nc = static_cast<uint32_t>((hi - lo_al + kChunkKeys - 1) / kChunkKeys);
+            }
+            p.s_lo[tile] = slo;
+            p.s_hi[tile] = shi;
+            p.s_lg[tile] = slg;
+            p.c_lo[tile] = clo;
+            p.c_hi[tile] = chi;
+        }
+        uint32_t tot_s, tot_c;
+        const uint32_t es = block_excl_scan(ns, sh, tot_s);
+        const uint32_t ec = block_excl_scan(nc, sh, tot_c);
+        if (tile < p.ntiles) {
+            p.s_start[tile] = static_cast<int32_t>(carry_s + es);
+            p.c_start[tile] = static_cast<int32_t>(carry_c + ec);
+        }
+        carry_s += tot_s;
+        carry_c += tot_c;
+    }
+    if (tid == 0) {
+        p.s_start[p.ntiles] = static_cast<int32_t>(carry_s);
+        p.c_start[p.ntiles] = static_cast<int32_t>(carry_c);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// block-level radix select on 32-bit keys
+// ---------------------------------------------------------------------------
+
+struct SelShared {
+    uint32_t hist[256];
+    uint32_t bin, above;
+    uint32_t red[96];
+};
+
+// The k-th largest (1 <= k <= count of keys) of key(i), i < n, where key
+// is any functor.  *gt receives how many keys are strictly larger.
+// Block-wide; must be called by every thread of the block.
+template <class KeyFn>
+__device__ uint32_t block_kth_largest(int n, uint32_t k, KeyFn key, SelShared &ss, uint32_t *gt)
+{
+    uint32_t prefix = 0, mask = 0, above_total = 0;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int b = tid; b < 256; b += blockDim.x) ss.hist[b] = 0;
+        __syncthreads();
+        for (int i = tid; i < n; i += blockDim.x) {
+            const uint32_t u = key(i);
+            if ((u & mask) == prefix) atomicAdd(&ss.hist[(u >> shift) & 255u], 1u);
+        }
+        __syncthreads();
+        if (warp == 0) {
+            // lane l owns bins 255-8l .. 248-8l (highest first)
+            uint32_t c[8], sum = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                c[i] = ss.hist[255 - 8 * lane - i];
+                sum += c[i];
+            }
+            uint32_t inc = sum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t u = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+                if (lane >= o) inc += u;
+            }
+            uint32_t above = inc - sum;
+            if (above < k && inc >= k) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    if (above + c[i] >= k) {
+                        ss.bin = 255 - 8 * lane - i;
+                        ss.above = above;
+                        break;
+                    }
+                    above += c[i];
+                }
+            }
+        }
+        __syncthreads();
+        const uint32_t bin = ss.bin;
+        prefix |= bin << shift;
+        mask |= 255u << shift;
+        k -= ss.above;
+        above_total += ss.above;
+        __syncthreads();
+    }
+    *gt = above_total;
+    return prefix;
+}
+
+__device__ __forceinline__ uint32_t block_sum(uint32_t v, SelShared &ss)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    if (lane == 0) ss.red[warp] = v;
+    __syncthreads();
+    uint32_t s = 0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) s += ss.red[w];
+    __syncthreads();
+    return s;
+}
+
+// ---------------------------------------------------------------------------
+// threshold
+// ---------------------------------------------------------------------------
+
+struct ThreshArgs {
+    int64_t T, S;
+    const int32_t *ks, *ke;
+    const int32_t *s_lo, *s_hi, *s_lg;
+    const float *samp;
+    int64_t sld;
+    float *tau;
+    int32_t cap;
+    int32_t topk;
+    float oversample;
+};
+
+__global__ void __launch_bounds__(kSelThreads) threshold_kernel(const ThreshArgs p)
+{
+    extern __shared__ uint32_t tkeys[];
+    __shared__ SelShared ss;
+    const int64_t t = blockIdx.x;
+    const int64_t a = p.ks[t], b = p.ke[t];
+    const int64_t L = b - a;
+    if (!window_ok(a, b, p.S) || L <= p.cap) {
+        if (threadIdx.x == 0) p.tau[t] = -INFINITY;
+        return;
+    }
+    const int tile = static_cast<int>(t / kQTile);
+    const int lg = p.s_lg[tile];
+    const int64_t st = int64_t(1) << lg;
+    const int J = p.s_hi[tile] - p.s_lo[tile];
+    const int64_t mt = ((b + st - 1) >> lg) - ((a + st - 1) >> lg);  // samples in my window
+    int64_t r = static_cast<int64_t>(ceil(static_cast<double>(p.oversample) * p.topk *
+                                          static_cast<double>(mt) / static_cast<double>(L)));
+    if (r < 1) r = 1;
+    if (mt <= 0 || r > mt) {
+        if (threadIdx.x == 0) p.tau[t] = -INFINITY;
+        return;
+    }
+    const float *row = p.samp + t * p.sld;
+    for (int i = threadIdx.x; i < J; i += blockDim.x) tkeys[i] = f32_key(__float_as_uint(row[i]));
+    __syncthreads();
+    uint32_t gt;
+    const uint32_t u = block_kth_largest(J, static_cast<uint32_t>(r), [&](int i) { return tkeys[i]; }, ss, &gt);
+    if (threadIdx.x == 0) p.tau[t] = __uint_as_float(f32_from_key(u));
+}
+
+// ---------------------------------------------------------------------------
+// refine + triage
+// ---------------------------------------------------------------------------
+
+struct RefineArgs {
+    int64_t T, S;
+    const int32_t *ks, *ke;
+    const int32_t *cnt;
+    const float *cand_val;
+    const int32_t *cand_idx;
+    int32_t cap;
+    int32_t topk;
+    int32_t *out_idx;
+    float *out_val;
+    int32_t *bad_rows;
+    int32_t *bad_count;
+    DevInfo *info;
+};
+
+__device__ __forceinline__ void pad_row(int32_t *oi, float *ov, int from, int k)
+{
+    for (int j = from + threadIdx.x; j < k; j += blockDim.x) {
+        oi[j] = -1;
+        if (ov) ov[j] = -INFINITY;
+    }
+}
+
+__global__ void __launch_bounds__(kSelThreads) refine_kernel(const RefineArgs p)
+{
+    extern __shared__ __align__(16) uint32_t rsm[];
+    __shared__ SelShared ss;
+    __shared__ uint32_t bitmap[kBitmapWords];
+    __shared__ uint32_t wpre[kBitmapWords];
+    __shared__ int nan_seen;
+    const int64_t t = blockIdx.x;
+    const int k = p.topk;
+    int32_t *oi = p.out_idx + t * k;
+    float *ov = p.out_val ? p.out_val + t * k : nullptr;
+    const int64_t a = p.ks[t], b = p.ke[t];
+    if (!window_ok(a, b, p.S)) {
+        pad_row(oi, ov, 0, k);
+        return;
+    }
+    const int64_t L = b - a;
+    const int32_t c = p.cnt[t];
+    const int64_t need_min = L < k ? L : k;
+    if (c > p.cap || c < need_min) {
+        if (threadIdx.x == 0) {
+            const int pos = atomicAdd(p.bad_count, 1);
+            p.bad_rows[pos] = static_cast<int32_t>(t);
+            atomicAdd(reinterpret_cast<unsigned long long *>(
+                          c > p.cap ? &p.info->info.rows_overflow : &p.info->info.rows_underflow),
+                      1ull);
+        }
+        return;
+    }
+    const int n = c;
+    uint32_t *keys = rsm;
+    int32_t *idx = reinterpret_cast<int32_t *>(rsm + p.cap);
+    if (threadIdx.x == 0) nan_seen = 0;
+    __syncthreads();
+    const float *cv = p.cand_val + t * p.cap;
+    const int32_t *ci = p.cand_idx + t * p.cap;
+    bool nan = false;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const uint32_t bits = __float_as_uint(cv[i]);
+        nan |= f32_bits_isnan(bits);
+        keys[i] = f32_key(bits);
+        idx[i] = ci[i];
+    }
+    if (nan) nan_seen = 1;
+    if (threadIdx.x == 0) {
+        atomicAdd(reinterpret_cast<unsigned long long *>(&p.info->info.candidates_total),
+                  static_cast<unsigned long long>(n));
+        atomicMax(reinterpret_cast<unsigned long long *>(&p.info->info.candidates_max),
+                  static_cast<unsigned long long>(n));
+    }
+    __syncthreads();
+    if (nan_seen && threadIdx.x == 0) atomicOr(&p.info->info.status, FTK_STATUS_NAN);
+
+    // Threshold key u* and the tie cut idx*: selected = key > u*, or
+    // key == u* and index <= idx* (the smallest indices among the ties).
+    uint32_t ustar = 0, idxcut = 0xFFFFFFFFu;
+    if (n > k) {
+        uint32_t gt;
+        ustar = block_kth_largest(n, static_cast<uint32_t>(k), [&](int i) { return keys[i]; }, ss, &gt);
+        const uint32_t need = static_cast<uint32_t>(k) - gt;
+        uint32_t eq = 0;
+        for (int i = threadIdx.x; i < n; i += blockDim.x) eq += keys[i] == ustar;
+        eq = block_sum(eq, ss);
+        if (eq > need) {
+            // need-th smallest index among the ties = need-th largest of ~index.
+            uint32_t g2;
+            const uint32_t inv = block_kth_largest(
+                n, need,
+                [&](int i) { return keys[i] == ustar ? ~static_cast<uint32_t>(idx[i]) : 0u; }, ss, &g2);
+            idxcut = ~inv;
+        }
+    }
+    auto selected = [&](int i) {
+        const uint32_t u = keys[i];
+        return u > ustar || (u == ustar && static_cast<uint32_t>(idx[i]) <= idxcut);
+    };
+
+    // Ordered output: rank of a selected key = number of selected keys with
+    // a smaller index, from a bitmap over the window (65536-key segments).
+    uint32_t out_base = 0;
+    for (int64_t seg0 = a; seg0 < b; seg0 += 32 * kBitmapWords) {
+        const int64_t seg1 = min(b, seg0 + 32 * kBitmapWords);
+        const int words = static_cast<int>((seg1 - seg0 + 31) >> 5);
+        for (int w = threadIdx.x; w < words; w += blockDim.x) bitmap[w] = 0;
+        __syncthreads();
+        for (int i = threadIdx.x; i < n; i += blockDim.x) {
+            const int64_t s = idx[i];
+            if (s >= seg0 && s < seg1 && selected(i)) {
+                const uint32_t off = static_cast<uint32_t>(s - seg0);
+                atomicOr(&bitmap[off >> 5], 1u << (off & 31u));
+            }
+        }
+        __syncthreads();
+        constexpr int per = kBitmapWords / kSelThreads;
+        uint32_t cnt = 0;
+        const int w0 = threadIdx.x * per;
+#pragma unroll
+        for (int i = 0; i < per; ++i) cnt += w0 + i < words ? __popc(bitmap[w0 + i]) : 0u;
+        uint32_t total;
+        uint32_t run = block_excl_scan(cnt, ss.red, total);
+#pragma unroll
+        for (int i = 0; i < per; ++i) {
+            if (w0 + i < words) {
+                wpre[w0 + i] = run;
+                run += __popc(bitmap[w0 + i]);
+            }
+        }
+        __syncthreads();
+        for (int i = threadIdx.x; i < n; i += blockDim.x) {
+            const int64_t s = idx[i];
+            if (s >= seg0 && s < seg1 && selected(i)) {
+                const uint32_t off = static_cast<uint32_t>(s - seg0);
+                const uint32_t w = off >> 5;
+                const uint32_t rank =
+                    out_base + wpre[w] + __popc(bitmap[w] & ((1u << (off & 31u)) - 1u));
+                if (rank < static_cast<uint32_t>(k)) {
+                    oi[rank] = static_cast<int32_t>(s);
+                    if (ov) ov[rank] = __uint_as_float(f32_from_key(keys[i]));
+                } else {
+                    atomicOr(&p.info->info.status, FTK_STATUS_INTERNAL);
+                }
+            }
+        }
+        out_base += total;
+        __syncthreads();
+    }
+    pad_row(oi, ov, static_cast<int>(out_base), k);
+}
+
+// ---------------------------------------------------------------------------
+// host helpers
+// ---------------------------------------------------------------------------
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// 2-D map over rows of 128 elements (row stride `stride_bytes`), box of
+// (128 bytes, box_rows) with the 128-byte swizzle; out-of-range rows read 0.
+static bool make_map(CUtensorMap *m, int dtype, const void *base, uint64_t rows,
+                     uint64_t stride_bytes, uint32_t box_rows)
+{
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const bool f8 = dtype == FTK_F8E4M3;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(kDim), rows};
+    cuuint64_t strides[1] = {stride_bytes};
+    cuuint32_t box[2] = {f8 ? 128u : 64u, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                    const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+static int num_sms()
+{
+    int dev = 0, n = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+struct SelectCfg {
+    int m;          // sample keys
+    float beta;
+    int cap;
+    int prune;
+    int rec_rows;
+};
+
+static SelectCfg resolve_cfg(int64_t T, int64_t S, int topk, const ftk_config *c)
+{
+    SelectCfg r;
+    r.m = c && c->sample_keys > 0 ? c->sample_keys : 4096;
+    r.beta = c && c->oversample > 0.f ? c->oversample : 1.5f;
+    r.cap = c && c->capacity > 0 ? c->capacity : 2 * topk;
+    if (r.cap > 2 * FTK_MAX_TOPK) r.cap = 2 * FTK_MAX_TOPK;
+    r.prune = c ? c->prune : -1;
+    // Strides are powers of two up to 2^(kNumStrideMaps - 1).
+    const int64_t min_m = (S + (int64_t(1) << (kNumStrideMaps - 1)) - 1) >> (kNumStrideMaps - 1);
+    if (r.m < min_m) r.m = static_cast<int>(min_m);
+    if (r.m < 32) r.m = 32;
+    if (r.m > 32768) r.m = 32768;
+    int64_t rr = c && c->recovery_rows > 0 ? c->recovery_rows : 0;
+    if (rr == 0) {
+        // ~512 MB of recovery scratch, at least 64 rows.
+        rr = (int64_t(1) << 27) / (S > 0 ? S : 1);
+        if (rr < 64) rr = 64;
+    }
+    if (rr > T) rr = T;
+    rr = (rr + kQTile - 1) / kQTile * kQTile;
+    r.rec_rows = static_cast<int>(rr);
+    return r;
+}
+
+struct SelectWs {
+    DevInfo *info;
+    int32_t *s_lo, *s_hi, *s_lg, *s_start, *c_lo, *c_hi, *c_start;
+    float *samp;
+    int64_t sld;
+    float *tau;
+    int32_t *cnt;
+    float *cand_val;
+    int32_t *cand_idx;
+    int32_t *bad_rows;
+    int32_t *bad_count;
+    float *scratch;
+    int64_t scratch_ld;
+};
+
+static bool carve_select(Carver &cv, int64_t T, int64_t S, const SelectCfg &c, SelectWs &w)
+{
+    const int64_t ntiles = (T + kQTile - 1) / kQTile;
+    w.info = cv.take<DevInfo>(1);
+    w.s_lo = cv.take<int32_t>(ntiles);
+    w.s_hi = cv.take<int32_t>(ntiles);
+    w.s_lg = cv.take<int32_t>(ntiles);
+    w.s_start = cv.take<int32_t>(ntiles + 1);
+    w.c_lo = cv.take<int32_t>(ntiles);
+    w.c_hi = cv.take<int32_t>(ntiles);
+    w.c_start = cv.take<int32_t>(ntiles + 1);
+    w.sld = (c.m + 3) / 4 * 4;
+    w.samp = cv.take<float>(T * w.sld);
+    w.tau = cv.take<float>(T);
+    w.cnt = cv.take<int32_t>(T);
+    w.cand_val = cv.take<float>(T * static_cast<int64_t>(c.cap));
+    w.cand_idx = cv.take<int32_t>(T * static_cast<int64_t>(c.cap));
+    w.bad_rows = cv.take<int32_t>(T);
+    w.bad_count = cv.take<int32_t>(1);
+    w.scratch_ld = (S + 7) / 8 * 8;
+    w.scratch = cv.take<float>(static_cast<int64_t>(c.rec_rows) * w.scratch_ld);
+    return cv.ok;
+}
+
+template <int DT, int MODE>
+static ftk_status launch_score(const ScoreArgs &a, const CUtensorMap &tq, const KvMaps &kvm,
+                               int grid, cudaStream_t st)
+{
+    const int smem = ScoreSmemLayout<DT>::kBytes;
+    auto kern = score_kernel<DT, MODE>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_status(e);
+    kern<<<grid, kScoreThreads, smem, st>>>(a, tq, kvm);
+    return cuda_status(cudaGetLastError());
+}
+
+template <int MODE>
+static ftk_status launch_score_dt(int dtype, const ScoreArgs &a, const CUtensorMap &tq,
+                                  const KvMaps &kvm, int grid, cudaStream_t st)
+{
+    if (dtype == FTK_F8E4M3) return launch_score<FTK_F8E4M3, MODE>(a, tq, kvm, grid, st);
+    return launch_score<FTK_BF16, MODE>(a, tq, kvm, grid, st);
+}
+
+static bool build_maps(int dtype, const void *q, const void *kv, int64_t T, int64_t S, int max_lg,
+                       CUtensorMap *tq, KvMaps *kvm)
+{
+    const uint64_t esz = dtype == FTK_F8E4M3 ? 1 : 2;
+    if (!make_map(tq, dtype, q, static_cast<uint64_t>(T) * kHeads, kDim * esz, kHeads)) return false;
+    for (int i = 0; i < kNumStrideMaps; ++i) {
+        if (i > max_lg) {
+            kvm->m[i] = kvm->m[0];
+            continue;
+        }
+        const uint64_t st = uint64_t(1) << i;
+        const uint64_t rows = (static_cast<uint64_t>(S) + st - 1) / st;
+        if (!make_map(&kvm->m[i], dtype, kv, rows, kDim * esz * st, kKeyTile)) return false;
+    }
+    return true;
+}
+
+static ftk_status check_select_args(int dtype, const void *q, const void *kv, const float *w,
+                                    const int32_t *ks, const int32_t *ke, int64_t T, int64_t S,
+                                    int topk, const int32_t *out_idx)
+{
+    if (dtype != FTK_F8E4M3 && dtype != FTK_BF16) return FTK_ERR_UNSUPPORTED;
+    if (!q || !kv || !w || !ks || !ke || !out_idx) return FTK_ERR_INVALID_ARG;
+    if (T < 1 || S < 1 || T >= (int64_t(1) << 31) / kHeads || S >= (int64_t(1) << 31) - kChunkKeys)
+        return FTK_ERR_INVALID_ARG;
+    if (topk < 1 || topk > FTK_MAX_TOPK) return FTK_ERR_TOPK_RANGE;
+    if (!aligned16(q) || !aligned16(kv) || !aligned16(w)) return FTK_ERR_ALIGNMENT;
+    return FTK_OK;
+}
+
+}  // namespace ftk
+
+using namespace ftk;
+
+extern "C" size_t ftk_select_workspace_size(int64_t T, int64_t S, int topk, const ftk_config *config)
+{
+    if (T < 1 || S < 1 || topk < 1 || topk > FTK_MAX_TOPK) return 0;
+    const SelectCfg c = resolve_cfg(T, S, topk, config);
+    Carver cv{nullptr, 0};
+    SelectWs w;
+    carve_select(cv, T, S, c, w);
+    return cv.used;
+}
+
+extern "C" ftk_status ftk_read_info(const void *workspace, ftk_info *out, void *stream)
+{
+    if (!workspace || !out) return FTK_ERR_INVALID_ARG;
+    cudaStream_t st = as_stream(stream);
+    cudaError_t e = cudaMemcpyAsync(out, workspace, sizeof(ftk_info), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    return cuda_status(e);
+}
+
+extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
+                                 const float *kv_scales, const float *weights, const int32_t *ks,
+                                 const int32_t *ke, int64_t T, int64_t S, int topk,
+                                 int32_t *out_idx, float *out_val, void *workspace,
+                                 size_t workspace_bytes, const ftk_config *config, void *stream)
+{
+    ftk_status st = check_select_args(dtype, q, kv, weights, ks, ke, T, S, topk, out_idx);
+    if (st != FTK_OK) return st;
+    if (config && (config->reserved[0] || config->reserved[1] || config->reserved[2]))
+        return FTK_ERR_INVALID_ARG;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return FTK_ERR_WORKSPACE;
+    const SelectCfg c = resolve_cfg(T, S, topk, config);
+    if (c.cap < topk) return FTK_ERR_INVALID_ARG;
+    Carver cv{static_cast<uint8_t *>(workspace), workspace_bytes};
+    SelectWs w;
+    if (!carve_select(cv, T, S, c, w)) return FTK_ERR_WORKSPACE;
+    st = check_device();
+    if (st != FTK_OK) return st;
+    cudaStream_t s = as_stream(stream);
+
+    const int64_t want = (S + c.m - 1) / c.m;
+    int max_lg = 0;
+    while ((int64_t(1) << max_lg) < want) ++max_lg;
+    if (max_lg >= kNumStrideMaps) return FTK_ERR_UNSUPPORTED;
+    CUtensorMap tq;
+    KvMaps kvm;
+    if (!build_maps(dtype, q, kv, T, S, max_lg, &tq, &kvm)) return FTK_ERR_CUDA;
+
+    const int32_t ntiles = static_cast<int32_t>((T + kQTile - 1) / kQTile);
+    const int sms = num_sms();
+    uint32_t *status = &w.info->info.status;
+
+    PlanArgs pa;
+    pa.T = T;
+    pa.S = S;
+    pa.ks = ks;
+    pa.ke = ke;
+    pa.ntiles = ntiles;
+    pa.sample_keys = c.m;
+    pa.s_lo = w.s_lo;
+    pa.s_hi = w.s_hi;
+    pa.s_lg = w.s_lg;
+    pa.s_start = w.s_start;
+    pa.c_lo = w.c_lo;
+    pa.c_hi = w.c_hi;
+    pa.c_start = w.c_start;
+    pa.cnt = w.cnt;
+    pa.bad_count = w.bad_count;
+    pa.info = w.info;
+    plan_kernel<<<1, kPlanThreads, 0, s>>>(pa);
+    if ((st = cuda_status(cudaGetLastError())) != FTK_OK) return st;
+
+    ScoreArgs sa = {};
+    sa.T = T;
+    sa.S = S;
+    sa.kv_scales = kv_scales;
+    sa.weights = weights;
+    sa.ks = ks;
+    sa.ke = ke;
+    sa.rows = nullptr;
+    sa.nrows = T;
+    sa.planned = 1;
+    sa.ntiles = ntiles;
+    sa.status = status;
+    // sample pass
+    sa.tile_lo = w.s_lo;
+    sa.tile_hi = w.s_hi;
+    sa.tile_lg = w.s_lg;
+    sa.item_start = w.s_start;
+    sa.out = w.samp;
+    sa.ld = w.sld;
+    st = launch_score_dt<MODE_SAMPLE>(dtype, sa, tq, kvm, sms < ntiles ? sms : ntiles, s);
+    if (st != FTK_OK) return st;
+
+    ThreshArgs ta;
+    ta.T = T;
+    ta.S = S;
+    ta.ks = ks;
+    ta.ke = ke;
+    ta.s_lo = w.s_lo;
+    ta.s_hi = w.s_hi;
+    ta.s_lg = w.s_lg;
+    ta.samp = w.samp;
+    ta.sld = w.sld;
+    ta.tau = w.tau;
+    ta.cap = c.cap;
+    ta.topk = topk;
+    ta.oversample = c.beta;
+    {
+        const size_t smem = static_cast<size_t>(w.sld) * 4;
+        cudaError_t e = cudaFuncSetAttribute(threshold_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem));
+        if (e != cudaSuccess) return cuda_status(e);
+        threshold_kernel<<<static_cast<unsigned>(T), kSelThreads, smem, s>>>(ta);
+        if ((st = cuda_status(cudaGetLastError())) != FTK_OK) return st;
+    }
+
+    // dense scan
+    sa.tile_lo = w.c_lo;
+    sa.tile_hi = w.c_hi;
+    sa.tile_lg = nullptr;
+    sa.item_start = w.c_start;
+    sa.tau = w.tau;
+    sa.cnt = w.cnt;
+    sa.cand_val = w.cand_val;
+    sa.cand_idx = w.cand_idx;
+    sa.cap = c.cap;
+    sa.out = nullptr;
+    st = launch_score_dt<MODE_COLLECT>(dtype, sa, tq, kvm, sms, s);
+    if (st != FTK_OK) return st;
+
+    RefineArgs ra;
+    ra.T = T;
+    ra.S = S;
+    ra.ks = ks;
+    ra.ke = ke;
+    ra.cnt = w.cnt;
+    ra.cand_val = w.cand_val;
+    ra.cand_idx = w.cand_idx;
+    ra.cap = c.cap;
+    ra.topk = topk;
+    ra.out_idx = out_idx;
+    ra.out_val = out_val;
+    ra.bad_rows = w.bad_rows;
+    ra.bad_count = w.bad_count;
+    ra.info = w.info;
+    {
+        const size_t smem = static_cast<size_t>(c.cap) * 8;
+        cudaError_t e = cudaFuncSetAttribute(refine_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem));
+        if (e != cudaSuccess) return cuda_status(e);
+        refine_kernel<<<static_cast<unsigned>(T), kSelThreads, smem, s>>>(ra);
+        if ((st = cuda_status(cudaGetLastError())) != FTK_OK) return st;
+    }
+
+    // dense recovery of the listed rows, rec_rows at a time
+    int rcluster = 1, rchunk = 8;
+    rows_plan(c.rec_rows, S, &rcluster, &rchunk);
+    const int32_t chunks = static_cast<int32_t>((S + kKeyTile - 1 + kChunkKeys - 1) / kChunkKeys);
+    for (int64_t b0 = 0; b0 < T; b0 += c.rec_rows) {
+        ScoreArgs da = {};
+        da.T = T;
+        da.S = S;
+        da.kv_scales = kv_scales;
+        da.weights = weights;
+        da.ks = ks;
+        da.ke = ke;
+        da.rows = w.bad_rows + b0;
+        da.nrows = c.rec_rows;
+        da.count_dev = w.bad_count;
+        da.count_off = static_cast<int32_t>(b0);
+        da.planned = 0;
+        da.static_chunks = chunks;
+        da.out = w.scratch;
+        da.ld = w.scratch_ld;
+        da.status = status;
+        const int64_t items = static_cast<int64_t>(chunks) * (c.rec_rows / kQTile);
+        st = launch_score_dt<MODE_DUMP>(dtype, da, tq, kvm,
+                                        static_cast<int>(items < sms ? items : sms), s);
+        if (st != FTK_OK) return st;
+        RowsArgs ra2 = {};
+        ra2.x = w.scratch;
+        ra2.ld = w.scratch_ld;
+        ra2.cols = S;
+        ra2.rows = c.rec_rows;
+        ra2.nrows_dev = w.bad_count;
+        ra2.nrows_off = static_cast<int32_t>(b0);
+        ra2.row_map = w.bad_rows + b0;
+        ra2.win_ks = ks;
+        ra2.win_ke = ke;
+        ra2.out_idx = out_idx;
+        ra2.out_val = out_val;
+        ra2.k = topk;
+        ra2.chunk = rchunk;
+        ra2.status = status;
+        st = launch_rows_topk(FTK_F32, ra2, rcluster, s);
+        if (st != FTK_OK) return st;
+    }
+    return FTK_OK;
+}
+
+extern "C" size_t ftk_score_dense_workspace_size(int64_t nrows)
+{
+    (void)nrows;
+    return 256;
+}
+
+extern "C" ftk_status ftk_score_dense(ftk_dtype dtype, const void *q, const void *kv,
+                                      const float *kv_scales, const float *weights,
+                                      const int32_t *ks, const int32_t *ke, int64_t T, int64_t S,
+                                      const int32_t *rows, int64_t nrows, float *out, int64_t ld,
+                                      void *workspace, size_t workspace_bytes, void *stream)
+{
+    ftk_status st = check_select_args(dtype, q, kv, weights, ks, ke, T, S, 1, rows ? rows : ks);
+    if (st != FTK_OK) return st;
+    if (!out || nrows < 1 || nrows > T * 64 || ld < 1 || (ld & 3)) return FTK_ERR_INVALID_ARG;
+    if (!rows && nrows > T) return FTK_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < 256 || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return FTK_ERR_WORKSPACE;
+    st = check_device();
+    if (st != FTK_OK) return st;
+    CUtensorMap tq;
+    KvMaps kvm;
+    if (!build_maps(dtype, q, kv, T, S, 0, &tq, &kvm)) return FTK_ERR_CUDA;
+    ScoreArgs da = {};
+    da.T = T;
+    da.S = S;
+    da.kv_scales = kv_scales;
+    da.weights = weights;
+    da.ks = ks;
+    da.ke = ke;
+    da.rows = rows;
+    da.nrows = nrows;
+    da.planned = 0;
+    da.static_chunks = static_cast<int32_t>((S + kKeyTile - 1 + kChunkKeys - 1) / kChunkKeys);
+    da.out = out;
+    da.ld = ld;
+    da.status = static_cast<uint32_t *>(workspace);
+    cudaStream_t s = as_stream(stream);
+    cudaError_t e = cudaMemsetAsync(workspace, 0, 4, s);
+    if (e != cudaSuccess) return cuda_status(e);
+    const int64_t items = static_cast<int64_t>(da.static_chunks) * ((nrows + kQTile - 1) / kQTile);
+    const int sms = num_sms();
+    return launch_score_dt<MODE_DUMP>(dtype, da, tq, kvm,
+                                      static_cast<int>(items < sms ? items : sms), s);
+}

@@ -1,0 +1,280 @@
+"""Python binding of libftk (argument marshalling only).
+
+Every step of the computation runs in the library's CUDA kernels; this
+module checks shapes and dtypes, allocates outputs with torch, and passes
+raw device pointers plus the current CUDA stream through the C ABI declared
+in include/ftk.h.  If libftk.so is missing the calls raise: there is no CPU
+fallback.
+
+API (names after the pages' own):
+  select(q, kv, weights, ks, ke, kv_scales=None, topk=2048, return_scores=False)
+      FlashTopK README, "Usage": flashtopk.select
+  Selector(topk, dtype).plan(max_rows, max_kv).run(...)
+      FlashTopK README, "Usage": Selector (owns the workspace)
+  windows_from_cu_seqlens(cu_seqlens_q, cu_seqlens_k)
+      FlashTopK README, "Usage"
+  topk_rows(x, topk, return_value=True)
+      DeepSelect README, "Usage": deep_select.topk (unsorted values, int32
+      indices; ours come in ascending index order)
+  score_dense(q, kv, weights, ks, ke, kv_scales=None, rows=None)
+      the fused scores themselves, for checking
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libftk.so")
+
+F8E4M3, BF16, F32 = 1, 2, 3
+STATUS_BAD_WINDOW, STATUS_NAN, STATUS_TIMEOUT, STATUS_BAD_SCALE, STATUS_INTERNAL = 1, 2, 4, 8, 16
+HEADS, DIM, MAX_TOPK = 32, 128, 4096
+
+# Every symbol include/ftk.h declares.
+EXPORTS = (
+    "ftk_select", "ftk_select_workspace_size", "ftk_read_info", "ftk_topk_rows",
+    "ftk_score_dense", "ftk_score_dense_workspace_size", "ftk_windows_from_cu_seqlens",
+    "ftk_status_string", "ftk_version",
+)
+
+
+class FtkError(RuntimeError):
+    pass
+
+
+class FtkConfig(ctypes.Structure):
+    _fields_ = [("sample_keys", ctypes.c_int32), ("oversample", ctypes.c_float),
+                ("capacity", ctypes.c_int32), ("prune", ctypes.c_int32),
+                ("recovery_rows", ctypes.c_int32), ("reserved", ctypes.c_int32 * 3)]
+
+
+class FtkInfo(ctypes.Structure):
+    _fields_ = [("status", ctypes.c_uint32), ("prune_enabled", ctypes.c_int32),
+                ("rows", ctypes.c_int64), ("rows_underflow", ctypes.c_int64),
+                ("rows_overflow", ctypes.c_int64), ("blocks_total", ctypes.c_int64),
+                ("blocks_pruned", ctypes.c_int64), ("candidates_total", ctypes.c_int64),
+                ("candidates_max", ctypes.c_int64)]
+
+    def as_dict(self) -> dict:
+        return {name: getattr(self, name) for name, _ in self._fields_}
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Opens libftk.so and declares the C signatures."""
+    if not os.path.exists(path):
+        raise FtkError(f"{path} is not built: run `python -m sparse_attention_indexer_ftk_b200.build`")
+    L = ctypes.CDLL(path)
+    P, I64, I32, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+    L.ftk_select.restype = I32
+    L.ftk_select.argtypes = [I32, P, P, P, P, P, P, I64, I64, I32, P, P, P, SZ, P, P]
+    L.ftk_select_workspace_size.restype = SZ
+    L.ftk_select_workspace_size.argtypes = [I64, I64, I32, P]
+    L.ftk_read_info.restype = I32
+    L.ftk_read_info.argtypes = [P, P, P]
+    L.ftk_topk_rows.restype = I32
+    L.ftk_topk_rows.argtypes = [I32, P, I64, I64, I64, I32, P, P, P, P]
+    L.ftk_score_dense.restype = I32
+    L.ftk_score_dense.argtypes = [I32, P, P, P, P, P, P, I64, I64, P, I64, P, I64, P, SZ, P]
+    L.ftk_score_dense_workspace_size.restype = SZ
+    L.ftk_score_dense_workspace_size.argtypes = [I64]
+    L.ftk_windows_from_cu_seqlens.restype = I32
+    L.ftk_windows_from_cu_seqlens.argtypes = [P, P, I64, I64, P, P, P]
+    L.ftk_status_string.restype = ctypes.c_char_p
+    L.ftk_status_string.argtypes = [I32]
+    L.ftk_version.restype = I32
+    L.ftk_version.argtypes = []
+    return L
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        _lib = load_library()
+    return _lib
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        msg = lib().ftk_status_string(status).decode()
+        raise FtkError(f"{what} failed: {msg} ({status})")
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    codes = {torch.float8_e4m3fn: F8E4M3, torch.bfloat16: BF16, torch.float32: F32}
+    if t.dtype not in codes:
+        raise FtkError(f"unsupported dtype {t.dtype}")
+    return codes[t.dtype]
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise FtkError("inputs must be CUDA tensors")
+
+
+def _config(cfg: dict | None):
+    if not cfg:
+        return None
+    c = FtkConfig()
+    c.prune = -1
+    for k, v in cfg.items():
+        setattr(c, k, v)
+    return c
+
+
+def _check_select_inputs(q, kv, weights, ks, ke, kv_scales):
+    _need_cuda(q, kv, weights, ks, ke, kv_scales)
+    if q.dim() != 3 or q.shape[1:] != (HEADS, DIM) or not q.is_contiguous():
+        raise FtkError("q must be a contiguous [T, 32, 128] tensor")
+    if kv.dim() != 2 or kv.shape[1] != DIM or not kv.is_contiguous() or kv.dtype != q.dtype:
+        raise FtkError("kv must be a contiguous [S, 128] tensor of q's dtype")
+    T = q.shape[0]
+    if weights.shape != (T, HEADS) or weights.dtype != torch.float32 or not weights.is_contiguous():
+        raise FtkError("weights must be a contiguous float32 [T, 32] tensor")
+    for name, w in (("ks", ks), ("ke", ke)):
+        if w.shape != (T,) or w.dtype != torch.int32 or not w.is_contiguous():
+            raise FtkError(f"{name} must be a contiguous int32 [T] tensor")
+    if kv_scales is not None and (kv_scales.shape != (kv.shape[0],) or kv_scales.dtype != torch.float32
+                                  or not kv_scales.is_contiguous()):
+        raise FtkError("kv_scales must be a contiguous float32 [S] tensor")
+
+
+def select_workspace_size(T: int, S: int, topk: int, config: dict | None = None) -> int:
+    c = _config(config)
+    return int(lib().ftk_select_workspace_size(T, S, topk, ctypes.byref(c) if c else None))
+
+
+def select(q, kv, weights, ks, ke, kv_scales=None, topk: int = 2048, return_scores: bool = False,
+           workspace: torch.Tensor | None = None, config: dict | None = None,
+           out_idx: torch.Tensor | None = None, out_val: torch.Tensor | None = None):
+    """Exact top-k keys per query of I[t,s] = sigma_s sum_h w[t,h] ReLU(q[t,h].k[s]).
+
+    Returns int32 indices [T, topk] in ascending key order (padding -1), and
+    with return_scores=True also their float32 scores (padding -inf).
+    """
+    _check_select_inputs(q, kv, weights, ks, ke, kv_scales)
+    T, S = q.shape[0], kv.shape[0]
+    dev = q.device
+    if workspace is None:
+        workspace = torch.empty(select_workspace_size(T, S, topk, config), dtype=torch.uint8, device=dev)
+    if out_idx is None:
+        out_idx = torch.empty((T, topk), dtype=torch.int32, device=dev)
+    if return_scores and out_val is None:
+        out_val = torch.empty((T, topk), dtype=torch.float32, device=dev)
+    c = _config(config)
+    st = lib().ftk_select(_dtype_code(q), _ptr(q), _ptr(kv), _ptr(kv_scales), _ptr(weights), _ptr(ks),
+                          _ptr(ke), T, S, topk, _ptr(out_idx), _ptr(out_val) if return_scores else None,
+                          _ptr(workspace), workspace.numel(), ctypes.byref(c) if c else None,
+                          _stream(dev))
+    _check(st, "ftk_select")
+    return (out_idx, out_val) if return_scores else out_idx
+
+
+def read_info(workspace: torch.Tensor) -> dict:
+    """The last_info of the last select() that used this workspace (syncs)."""
+    info = FtkInfo()
+    _check(lib().ftk_read_info(_ptr(workspace), ctypes.byref(info), _stream(workspace.device)),
+           "ftk_read_info")
+    return info.as_dict()
+
+
+@dataclass
+class Selector:
+    """Owns a workspace sized by plan(max_rows, max_kv) (FlashTopK README, "Usage")."""
+    topk: int = 2048
+    dtype: torch.dtype = torch.float8_e4m3fn
+    config: dict | None = None
+    workspace: torch.Tensor | None = None
+    max_rows: int = 0
+    max_kv: int = 0
+
+    def plan(self, max_rows: int, max_kv: int, device="cuda") -> "Selector":
+        self.max_rows, self.max_kv = max_rows, max_kv
+        nbytes = select_workspace_size(max_rows, max_kv, self.topk, self.config)
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        return self
+
+    def run(self, q, kv, weights, ks, ke, kv_scales=None, return_scores=False, out_idx=None, out_val=None):
+        if self.workspace is None:
+            self.plan(q.shape[0], kv.shape[0], q.device)
+        if q.shape[0] > self.max_rows or kv.shape[0] > self.max_kv:
+            raise FtkError("inputs exceed the planned sizes")
+        return select(q, kv, weights, ks, ke, kv_scales, self.topk, return_scores,
+                      workspace=self.workspace, config=self.config, out_idx=out_idx, out_val=out_val)
+
+    @property
+    def last_info(self) -> dict:
+        return read_info(self.workspace)
+
+
+def windows_from_cu_seqlens(cu_seqlens_q: torch.Tensor, cu_seqlens_k: torch.Tensor):
+    """Causal (ks, ke) of packed sequences whose queries are their last tokens."""
+    _need_cuda(cu_seqlens_q, cu_seqlens_k)
+    cq = cu_seqlens_q.to(torch.int32).contiguous()
+    ck = cu_seqlens_k.to(torch.int32).contiguous()
+    nseq = cq.numel() - 1
+    T = int(cq[-1].item())
+    ks = torch.empty(T, dtype=torch.int32, device=cq.device)
+    ke = torch.empty(T, dtype=torch.int32, device=cq.device)
+    _check(lib().ftk_windows_from_cu_seqlens(_ptr(cq), _ptr(ck), nseq, T, _ptr(ks), _ptr(ke),
+                                             _stream(cq.device)), "ftk_windows_from_cu_seqlens")
+    return ks, ke
+
+
+def topk_rows(x: torch.Tensor, topk: int, return_value: bool = True, status: torch.Tensor | None = None,
+              out_idx: torch.Tensor | None = None, out_val: torch.Tensor | None = None):
+    """Row top-k of a [rows, cols] bf16/fp32 CUDA tensor (ties to smaller columns).
+
+    Returns (values, indices) like deep_select.topk, or indices alone when
+    return_value=False.  Indices are int32 in ascending column order.
+    """
+    _need_cuda(x, status)
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise FtkError("x must be 2-D with a contiguous last dimension")
+    rows, cols = x.shape
+    if out_idx is None:
+        out_idx = torch.empty((rows, topk), dtype=torch.int32, device=x.device)
+    if return_value and out_val is None:
+        out_val = torch.empty((rows, topk), dtype=x.dtype, device=x.device)
+    st = lib().ftk_topk_rows(_dtype_code(x), _ptr(x), rows, cols, x.stride(0), topk, _ptr(out_idx),
+                             _ptr(out_val) if return_value else None, _ptr(status), _stream(x.device))
+    _check(st, "ftk_topk_rows")
+    return (out_val, out_idx) if return_value else out_idx
+
+
+def score_dense(q, kv, weights, ks, ke, kv_scales=None, rows: torch.Tensor | None = None,
+                ld: int | None = None) -> torch.Tensor:
+    """Fused scores of the listed rows: out[r, s - ks[t]] = I[t, s] (float32).
+
+    Entries past a row's window are NaN.  Same kernel and bits as select().
+    """
+    _check_select_inputs(q, kv, weights, ks, ke, kv_scales)
+    T, S = q.shape[0], kv.shape[0]
+    dev = q.device
+    if rows is not None:
+        rows = rows.to(device=dev, dtype=torch.int32).contiguous()
+    nrows = T if rows is None else rows.numel()
+    if ld is None:
+        ld = (S + 3) // 4 * 4
+    out = torch.full((nrows, ld), float("nan"), dtype=torch.float32, device=dev)
+    ws = torch.empty(int(lib().ftk_score_dense_workspace_size(nrows)), dtype=torch.uint8, device=dev)
+    st = lib().ftk_score_dense(_dtype_code(q), _ptr(q), _ptr(kv), _ptr(kv_scales), _ptr(weights), _ptr(ks),
+                               _ptr(ke), T, S, _ptr(rows), nrows, _ptr(out), ld, _ptr(ws), ws.numel(),
+                               _stream(dev))
+    _check(st, "ftk_score_dense")
+    return out

@@ -1,0 +1,137 @@
+"""The C-ABI library loads, exports every symbol include/ftk.h declares, and
+rejects bad arguments on the host before touching a GPU."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from sparse_attention_indexer_ftk_b200 import build as ftk_build
+from sparse_attention_indexer_ftk_b200 import ftk
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ftk.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    ftk_build.build()
+    return ftk.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ftk_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_matches_binding_list():
+    assert declared_functions() == sorted(ftk.EXPORTS)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    out = subprocess.check_output(["nm", "-D", "--defined-only", ftk.LIB_PATH], text=True)
+    exported = set(re.findall(r"\bT (ftk_[a-z0-9_]+)$", out, flags=re.M))
+    missing = [f for f in declared_functions() if f not in exported]
+    assert not missing, missing
+    for f in declared_functions():
+        assert hasattr(lib, f)
+
+
+def test_version_and_strings(lib):
+    assert lib.ftk_version() == 100
+    assert lib.ftk_status_string(0) == b"ok"
+    assert b"topk" in lib.ftk_status_string(-3)
+    assert lib.ftk_status_string(12345) == b"unknown status"
+
+
+def test_structs_match_header_sizes():
+    assert ctypes.sizeof(ftk.FtkConfig) == 32
+    assert ctypes.sizeof(ftk.FtkInfo) == 8 + 7 * 8
+
+
+def test_workspace_size(lib):
+    n1 = lib.ftk_select_workspace_size(4096, 131072, 2048, None)
+    n2 = lib.ftk_select_workspace_size(128, 2048, 256, None)
+    assert n1 > n2 > 0
+    assert lib.ftk_select_workspace_size(0, 10, 5, None) == 0
+    assert lib.ftk_select_workspace_size(10, 10, 5000, None) == 0
+    cfg = ftk.FtkConfig(capacity=4096 * 2)
+    assert lib.ftk_select_workspace_size(4096, 131072, 2048, ctypes.byref(cfg)) >= n1
+
+
+A = 0x10000  # a 16-byte aligned stand-in pointer (never dereferenced on the host)
+
+
+def test_topk_rows_host_validation(lib):
+    P = ctypes.c_void_p
+    assert lib.ftk_topk_rows(2, P(A), 4, 100, 104, 0, P(A), None, None, None) == -3
+    assert lib.ftk_topk_rows(2, P(A), 4, 100, 104, 4097, P(A), None, None, None) == -3
+    assert lib.ftk_topk_rows(2, None, 4, 100, 104, 8, P(A), None, None, None) == -1
+    assert lib.ftk_topk_rows(1, P(A), 4, 100, 104, 8, P(A), None, None, None) == -2
+    assert lib.ftk_topk_rows(2, P(A + 2), 4, 100, 104, 8, P(A), None, None, None) == -4
+    assert lib.ftk_topk_rows(2, P(A), 4, 100, 101, 8, P(A), None, None, None) == -4
+    assert lib.ftk_topk_rows(3, P(A), 4, 100, 99, 8, P(A), None, None, None) == -1
+    assert lib.ftk_topk_rows(3, P(A), 4, 10 ** 7, 10 ** 7, 8, P(A), None, None, None) == -2
+
+
+def test_select_host_validation(lib):
+    P = ctypes.c_void_p
+    args = lambda **kw: dict(dict(dtype=1, q=P(A), kv=P(A), sc=None, w=P(A), ks=P(A), ke=P(A), T=16,
+                                  S=1000, k=8, oi=P(A), ov=None, ws=P(A), wsb=1 << 30, cfg=None,
+                                  st=None), **kw)
+
+    def call(**kw):
+        a = args(**kw)
+        return lib.ftk_select(a["dtype"], a["q"], a["kv"], a["sc"], a["w"], a["ks"], a["ke"], a["T"],
+                              a["S"], a["k"], a["oi"], a["ov"], a["ws"], a["wsb"], a["cfg"], a["st"])
+
+    assert call(k=0) == -3
+    assert call(k=4097) == -3
+    assert call(dtype=3) == -2
+    assert call(q=None) == -1
+    assert call(T=0) == -1
+    assert call(q=P(A + 8)) == -4
+    assert call(ws=None) == -5
+    assert call(ws=P(A + 16)) == -5
+    assert call(wsb=1000) == -5
+    bad = ftk.FtkConfig()
+    bad.reserved[0] = 1
+    assert call(cfg=ctypes.byref(bad)) == -1
+
+
+def test_score_dense_host_validation(lib):
+    P = ctypes.c_void_p
+    r = lib.ftk_score_dense(1, P(A), P(A), None, P(A), P(A), P(A), 16, 1000, None, 16, P(A), 1002,
+                            P(A), 256, None)
+    assert r == -1  # ld not a multiple of 4
+    r = lib.ftk_score_dense(1, P(A), P(A), None, P(A), P(A), P(A), 16, 1000, None, 17, P(A), 1000,
+                            P(A), 256, None)
+    assert r == -1  # more rows than T without a row list
+
+
+def test_windows_host_validation(lib):
+    P = ctypes.c_void_p
+    assert lib.ftk_windows_from_cu_seqlens(None, P(A), 2, 10, P(A), P(A), None) == -1
+    assert lib.ftk_windows_from_cu_seqlens(P(A), P(A), 0, 10, P(A), P(A), None) == -1
+    assert lib.ftk_windows_from_cu_seqlens(P(A), P(A), 2, 0, P(A), P(A), None) == 0
+
+
+def test_product_has_no_cpu_fallback(tmp_path, monkeypatch):
+    """Without libftk.so the binding raises instead of computing on the CPU."""
+    monkeypatch.setattr(ftk, "_lib", None)
+    monkeypatch.setattr(ftk, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(ftk.FtkError):
+        ftk.load_library(str(tmp_path / "missing.so"))
+
+
+def test_package_does_not_import_the_oracle():
+    pkg = os.path.join(ROOT, "sparse_attention_indexer_ftk_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"(from|import)\s+oracle|liboracle|orc_", text), f

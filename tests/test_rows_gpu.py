@@ -1,0 +1,99 @@
+"""ftk_topk_rows against the oracle: bit-exact index sets and values."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as orc
+from sparse_attention_indexer_ftk_b200 import ftk
+from sparse_attention_indexer_ftk_b200 import workloads as wl
+from tests.parity import check_row_invariants, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+def run_and_compare(x_cpu: torch.Tensor, k: int, return_value=True, rows_subset=None):
+    x = x_cpu.cuda()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    res = ftk.topk_rows(x, k, return_value=return_value, status=status)
+    torch.cuda.synchronize()
+    if return_value:
+        val, idx = res
+    else:
+        val, idx = None, res
+    idx = to_np(idx)
+    rows = range(x_cpu.shape[0]) if rows_subset is None else rows_subset
+    xs = x_cpu[list(rows)]
+    oidx, oval, flags = orc.topk_rows(xs, k)
+    for r_out, r in enumerate(rows):
+        check_row_invariants(idx[r], 0, x_cpu.shape[1], k)
+        n = min(k, x_cpu.shape[1])
+        want = np.sort(oidx[r_out, :n])
+        assert np.array_equal(idx[r, :n], want), f"row {r}: index set differs"
+        if val is not None:
+            got = val[r, :n].float().cpu().numpy().astype(np.float64)
+            # values in column order = x at those columns (bit-exact)
+            ref = x_cpu[r, idx[r, :n]]
+            assert torch.equal(val[r, :n].cpu().view(torch.int16 if x.dtype == torch.bfloat16 else torch.int32),
+                               ref.view(torch.int16 if x.dtype == torch.bfloat16 else torch.int32))
+            assert np.array_equal(np.sort(got), np.sort(oval[r_out, :n]))
+    return int(status.item())
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("rows,cols,k", [(1, 1, 1), (3, 7, 5), (5, 100, 100), (4, 1000, 37),
+                                         (2, 5000, 4096), (9, 33333, 512), (300, 2048, 64),
+                                         (1, 393216, 4096), (2, 131072, 1)])
+def test_random_rows(dtype, rows, cols, k):
+    g = torch.Generator().manual_seed(rows * 1000 + cols + k)
+    x = torch.randn((rows, cols), generator=g).to(dtype)
+    assert run_and_compare(x, k) == 0
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_heavy_ties_and_signed_zero(dtype):
+    g = torch.Generator().manual_seed(5)
+    x = torch.randint(-2, 3, (8, 20000), generator=g).float() * 0.5
+    x[1] = 0.0
+    x[2, ::2] = -0.0
+    x[3] = 1.0
+    x[4, :] = torch.tensor(float("-inf"))
+    x[4, 100:110] = 3.0
+    x = x.to(dtype)
+    for k in (1, 7, 511, 512, 4096):
+        assert run_and_compare(x, k) == 0
+
+
+def test_return_value_false_and_determinism():
+    x = torch.randn((16, 50000), generator=torch.Generator().manual_seed(6)).to(torch.bfloat16)
+    run_and_compare(x, 512, return_value=False)
+    xg = x.cuda()
+    a = ftk.topk_rows(xg, 512)
+    b = ftk.topk_rows(xg, 512)
+    assert torch.equal(a[1], b[1]) and torch.equal(a[0].view(torch.int16), b[0].view(torch.int16))
+
+
+def test_row_stride_padding():
+    base = torch.randn((6, 1032), generator=torch.Generator().manual_seed(7))
+    x = base[:, :1000]  # row stride 1032 floats (16-byte multiple), last dim contiguous
+    val, idx = ftk.topk_rows(x.cuda(), 50)
+    oidx, _, _ = orc.topk_rows(x.contiguous(), 50)
+    for r in range(6):
+        assert np.array_equal(to_np(idx[r]), np.sort(oidx[r]))
+
+
+def test_nan_is_flagged_not_trapped():
+    x = torch.randn((4, 3000), generator=torch.Generator().manual_seed(8))
+    x[2, 17] = float("nan")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ftk.topk_rows(x.cuda(), 16, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) & ftk.STATUS_NAN
+
+
+@pytest.mark.parametrize("name", ["rows_bf16", "rows_f32"])
+def test_full_size_workload(name):
+    """The row top-k workload at full size (64 rows), every row bit-exact."""
+    c = wl.get(name)
+    assert run_and_compare(c.x, c.topk) == 0
