@@ -13,8 +13,19 @@ from tests.parity import check_row_invariants, to_np
 pytestmark = pytest.mark.gpu
 
 
+def aligned_rows(x_cpu: torch.Tensor) -> torch.Tensor:
+    """x on the GPU with its row stride padded to a 16-byte multiple (the
+    row-alignment requirement; DeepSelect README, "Usage")."""
+    rows, cols = x_cpu.shape
+    per = 16 // x_cpu.element_size()
+    ld = (cols + per - 1) // per * per
+    buf = torch.zeros((rows, ld), dtype=x_cpu.dtype, device="cuda")
+    buf[:, :cols] = x_cpu.cuda()
+    return buf[:, :cols]
+
+
 def run_and_compare(x_cpu: torch.Tensor, k: int, return_value=True, rows_subset=None):
-    x = x_cpu.cuda()
+    x = aligned_rows(x_cpu)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     res = ftk.topk_rows(x, k, return_value=return_value, status=status)
     torch.cuda.synchronize()
@@ -68,7 +79,7 @@ def test_heavy_ties_and_signed_zero(dtype):
 def test_return_value_false_and_determinism():
     x = torch.randn((16, 50000), generator=torch.Generator().manual_seed(6)).to(torch.bfloat16)
     run_and_compare(x, 512, return_value=False)
-    xg = x.cuda()
+    xg = aligned_rows(x)
     a = ftk.topk_rows(xg, 512)
     b = ftk.topk_rows(xg, 512)
     assert torch.equal(a[1], b[1]) and torch.equal(a[0].view(torch.int16), b[0].view(torch.int16))
@@ -87,7 +98,7 @@ def test_nan_is_flagged_not_trapped():
     x = torch.randn((4, 3000), generator=torch.Generator().manual_seed(8))
     x[2, 17] = float("nan")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    ftk.topk_rows(x.cuda(), 16, status=status)
+    ftk.topk_rows(aligned_rows(x), 16, status=status)
     torch.cuda.synchronize()
     assert int(status.item()) & ftk.STATUS_NAN
 
