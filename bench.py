@@ -1,0 +1,376 @@
+#!/usr/bin/env python
+"""Throughput of the fused indexer score + exact top-k (ftk_select).
+
+Workload: the FP8 prefill chunk of the FlashTopK README "Quick start" --
+q [4096, 32, 128] and kv [131072, 128] FP8-e4m3 from N(0,1), kv_scales in
+(0.5, 1], weights N(0,1)/sqrt(32), causal windows ke[t] = 126976 + t + 1,
+topk 2048 -- seeded and synthetic (sparse_attention_indexer_ftk_b200.workloads).
+
+One step = one ftk_select call over the whole 4096-query batch (sample pass,
+thresholds, dense scan, refine, recovery).  Inputs are resident in HBM; the
+L2 is flushed (a 256 MB write) between timed steps, outside the timed events.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (launched with torch.distributed.run): every rank runs its own
+independent batch of the same shape (weak scaling; no data-path collective);
+the step time is the max over ranks.
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fused score+top-k queries/s & dense-eq TFLOP/s (4096q×128K FP8, k=2048)"
+WORKLOAD = "fp8_prefill"
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "scan_kernel_fp8_prefill.md")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def profiled_traffic():
+    """DRAM bytes per scan-kernel launch from the committed ncu summary."""
+    try:
+        text = open(PROFILE_TRAFFIC).read()
+    except OSError:
+        return None
+    import re
+    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    s = re.search(r"kernel_source_hash:\s*([0-9a-f]+)", text)
+    if not m:
+        return None
+    if s and s.group(1) != scan_kernel_hash():
+        return None  # the kernel changed since the counters were taken
+    return float(m.group(1))
+
+
+def scan_kernel_hash() -> str:
+    import hashlib
+    h = hashlib.sha1()
+    for f in ("ftk_score.cuh", "ftk_device.cuh"):
+        with open(os.path.join(ROOT, "sparse_attention_indexer_ftk_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:12]
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.idx), "-lms", "50", "-f", self.path],
+                stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                p = [x.strip() for x in line.split(",")]
+                if len(p) >= 9 and p[1].isdigit():
+                    rows.append(p)
+        except OSError:
+            pass
+        finally:
+            if self.path:
+                try:
+                    os.unlink(self.path)
+                except OSError:
+                    pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [int(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": int(rows[0][2]), "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows if r[3] not in ("", "[N/A]"))}
+
+
+def gpu_index(local_rank: int) -> int:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v for v in vis.split(",") if v.strip()]
+        if local_rank < len(ids) and ids[local_rank].strip().isdigit():
+            return int(ids[local_rank])
+    return local_rank
+
+
+def cpu_baseline(c, seconds: float):
+    """The oracle as it stands, on a bounded row sample of the same workload."""
+    from oracle import oracle as orc
+    from sparse_attention_indexer_ftk_b200 import workloads as wl
+
+    threads = orc.num_threads()
+    n = max(2, threads)
+    done, t_total, rows_total = 0, 0.0, 0
+    seed = 0
+    while t_total < seconds and rows_total < c.T:
+        rows = wl.sample_rows(c.T, min(n, c.T), seed=seed)
+        t0 = time.perf_counter()
+        orc.fused_select(c.q, c.kv, c.kv_scales, c.weights, c.ks, c.ke, c.topk, rows=rows)
+        t_total += time.perf_counter() - t0
+        rows_total += len(rows)
+        seed += 1
+        done += 1
+    return {"value": rows_total / t_total, "unit": "queries/s", "cores": threads, "kind": "oracle",
+            "sample": f"{rows_total} seeded query rows of the {c.T}-row batch (first and last "
+                      f"included), fp64 score + full sort per row, {t_total:.1f} s on {threads} threads"}
+
+
+def run_reference(args):
+    """--impl reference: the oracle, timed on the host cores (rank 0 only)."""
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return
+    from oracle import oracle as orc
+    from sparse_attention_indexer_ftk_b200 import workloads as wl
+
+    c = wl.get(WORKLOAD)
+    threads = orc.num_threads()
+    per_step = max(1, threads // 4)
+    seed = 0
+
+    def step():
+        nonlocal seed
+        rows = wl.sample_rows(c.T, per_step, seed=seed)
+        seed += 1
+        orc.fused_select(c.q, c.kv, c.kv_scales, c.weights, c.ks, c.ke, c.topk, rows=rows)
+        return len(rows)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    rows = sum(step() for _ in range(args.steps))
+    dt = time.perf_counter() - t0
+    value = rows / dt
+    pairs_per_row = c.pairs() / c.T
+    out = {
+        "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": WORKLOAD, "T": c.T, "S": c.S, "topk": c.topk, "dtype_in": "fp8_e4m3",
+                   "rows_per_step": per_step, "l2": "host"},
+        "dense_eq_tflops": value * pairs_per_row * 2 * 32 * 128 / 1e12,
+        "cpu_baseline": {"value": value, "unit": "queries/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{per_step} seeded rows per step"},
+        "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def run_ours(args):
+    import torch
+
+    world, rank, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+
+    from sparse_attention_indexer_ftk_b200 import ftk
+    from sparse_attention_indexer_ftk_b200 import workloads as wl
+
+    c = wl.get(WORKLOAD)
+    g = c.to(dev)
+    T, S, k = c.T, c.S, c.topk
+    pairs = c.pairs()
+    ws = torch.empty(ftk.select_workspace_size(T, S, k), dtype=torch.uint8, device=dev)
+    out_idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    out_val = torch.empty((T, k), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ftk.select(g.q, g.kv, g.weights, g.ks, g.ke, g.kv_scales, k, return_scores=True,
+                   workspace=ws, out_idx=out_idx, out_val=out_val)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    info = ftk.read_info(ws)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    stage_evs = [ftk.stage_events() for _ in range(K)]
+    with ClockSampler(gpu_index(local)) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        for i in range(K):
+            flush.zero_()  # evict the L2 between timed steps (outside the events)
+            with stage_evs[i]:
+                ev[i][0].record(stream)
+                step()
+                ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    clocks = clk.summary()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    mean_ms = sum(step_ms) / K
+    stages = [s.times_ms() for s in stage_evs]
+    stage_mean = {name: sum(s[name] for s in stages) / K for name in stages[0]}
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([mean_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        mean_ms = float(t.item())
+
+    # end to end through the public API: inputs from pinned host memory,
+    # results back to pinned host memory, every step.
+    host = {name: getattr(c, name).pin_memory() for name in ("q", "kv", "kv_scales", "weights", "ks", "ke")}
+    dev_in = {name: torch.empty_like(getattr(g, name)) for name in host}
+    h_idx = torch.empty((T, k), dtype=torch.int32).pin_memory()
+    h_val = torch.empty((T, k), dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = h_idx.numel() * 4 + h_val.numel() * 4
+    E = args.e2e_steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(E):
+        for name, t in host.items():
+            dev_in[name].copy_(t, non_blocking=True)
+        ftk.select(dev_in["q"], dev_in["kv"], dev_in["weights"], dev_in["ks"], dev_in["ke"],
+                   dev_in["kv_scales"], k, return_scores=True, workspace=ws, out_idx=out_idx,
+                   out_val=out_val)
+        h_idx.copy_(out_idx, non_blocking=True)
+        h_val.copy_(out_val, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / E
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
+    peaks, peak_src = measured_peaks()
+    fp8_peak = 2.0 * peaks["bf16_tflops"]   # FP8 dense = 2 x BF16 dense (nominal ratio)
+    scan_ms = stage_mean["scan"]
+    scan_flops = 2.0 * 32 * 128 * pairs
+    achieved = scan_flops / (scan_ms * 1e-3) / 1e12
+    traffic = profiled_traffic()
+    value = world * T / (mean_ms * 1e-3)
+    out = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "queries/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": mean_ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "fp8_e4m3 x fp8_e4m3 -> f32",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "T": T, "S": S, "topk": k, "pairs": pairs,
+                   "l2": "flushed between steps (256 MB write)", "parallelism": f"dp{world} (independent batches)"},
+        "dense_eq_tflops": world * scan_flops / (mean_ms * 1e-3) / 1e12,
+        "stage_ms": stage_mean,
+        "info": info,
+        "roofline": {"kernel": "score_kernel<fp8, COLLECT> (dense scan)", "bound": "tensor",
+                     "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
+                     "frac": achieved / fp8_peak, "traffic": traffic,
+                     "peak_source": f"2 x bf16_tflops ({peak_src}, burst) -- FP8 dense = 2 x BF16",
+                     "frac_of_sustained": achieved / (2.0 * peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))},
+        "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": "queries/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": int(info["kernel_launches"]) * K,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(c, args.cpu_seconds)
+    print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -90,6 +90,7 @@ typedef struct {
     int64_t blocks_pruned;    /* of which skipped by the score bound */
     int64_t candidates_total; /* sum over rows of candidates kept */
     int64_t candidates_max;   /* largest per-row candidate count */
+    int64_t kernel_launches;  /* kernels the call launched */
 } ftk_info;
 
 /*
@@ -201,6 +202,14 @@ ftk_status ftk_windows_from_cu_seqlens(const int32_t *cu_q,
                                        const int32_t *cu_k, int64_t nseq,
                                        int64_t T, int32_t *ks, int32_t *ke,
                                        void *stream);
+
+/* Diagnostic timing hook.  While set, every ftk_select call made from the
+ * calling host thread records events[i] (cudaEvent_t values created by the
+ * caller, passed as void *) on the call's stream at its stage boundaries:
+ * 0 start, 1 plan done, 2 sample pass done, 3 thresholds done, 4 dense scan
+ * done, 5 refine done, 6 recovery done.  n must be 0 (or events NULL) to
+ * stop, else >= 7.  The library does not own the events. */
+ftk_status ftk_set_stage_events(void *const *events, int n);
 
 /* Human-readable name of an ftk_status value (static string). */
 const char *ftk_status_string(int status);

@@ -55,6 +55,7 @@ struct PlanArgs {
     int32_t *cnt;
     int32_t *bad_count;
     DevInfo *info;
+    int64_t launches;
 };
 
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *sh, uint32_t &total)
@@ -99,6 +100,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanArgs p)
         *p.bad_count = 0;
         memset(&p.info->info, 0, sizeof(ftk_info));
         p.info->info.rows = p.T;
+        p.info->info.kernel_launches = p.launches;
     }
     __syncthreads();
     if (bad) atomicOr(&p.info->info.status, FTK_STATUS_BAD_WINDOW);
@@ -504,12 +506,15 @@ static SelectCfg resolve_cfg(int64_t T, int64_t S, int topk, const ftk_config *c
     if (r.m > 32768) r.m = 32768;
     int64_t rr = c && c->recovery_rows > 0 ? c->recovery_rows : 0;
     if (rr == 0) {
-        // ~512 MB of recovery scratch, at least 64 rows.
-        rr = (int64_t(1) << 27) / (S > 0 ? S : 1);
+        // At most 2^27 floats (512 MB) of recovery scratch, at least 64 rows;
+        // non-increasing in S so that a larger plan serves smaller calls.
+        const int64_t ld = (S + 7) / 8 * 8;
+        rr = ((int64_t(1) << 27) / ld) & ~static_cast<int64_t>(kQTile - 1);
         if (rr < 64) rr = 64;
     }
-    if (rr > T) rr = T;
     rr = (rr + kQTile - 1) / kQTile * kQTile;
+    const int64_t tcap = (T + kQTile - 1) / kQTile * kQTile;
+    if (rr > tcap) rr = tcap;
     r.rec_rows = static_cast<int>(rr);
     return r;
 }
@@ -603,9 +608,27 @@ static ftk_status check_select_args(int dtype, const void *q, const void *kv, co
     return FTK_OK;
 }
 
+thread_local void *const *g_stage_events = nullptr;
+
+static void stage_mark(int i, cudaStream_t s)
+{
+    if (g_stage_events) cudaEventRecord(static_cast<cudaEvent_t>(g_stage_events[i]), s);
+}
+
 }  // namespace ftk
 
 using namespace ftk;
+
+extern "C" ftk_status ftk_set_stage_events(void *const *events, int n)
+{
+    if (events == nullptr || n == 0) {
+        g_stage_events = nullptr;
+        return FTK_OK;
+    }
+    if (n < 7) return FTK_ERR_INVALID_ARG;
+    g_stage_events = events;
+    return FTK_OK;
+}
 
 extern "C" size_t ftk_select_workspace_size(int64_t T, int64_t S, int topk, const ftk_config *config)
 {
@@ -658,6 +681,7 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
     const int sms = num_sms();
     uint32_t *status = &w.info->info.status;
 
+    stage_mark(0, s);
     PlanArgs pa;
     pa.T = T;
     pa.S = S;
@@ -675,8 +699,10 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
     pa.cnt = w.cnt;
     pa.bad_count = w.bad_count;
     pa.info = w.info;
+    pa.launches = 5 + 2 * ((T + c.rec_rows - 1) / c.rec_rows);
     plan_kernel<<<1, kPlanThreads, 0, s>>>(pa);
     if ((st = cuda_status(cudaGetLastError())) != FTK_OK) return st;
+    stage_mark(1, s);
 
     ScoreArgs sa = {};
     sa.T = T;
@@ -699,6 +725,7 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
     sa.ld = w.sld;
     st = launch_score_dt<MODE_SAMPLE>(dtype, sa, tq, kvm, sms < ntiles ? sms : ntiles, s);
     if (st != FTK_OK) return st;
+    stage_mark(2, s);
 
     ThreshArgs ta;
     ta.T = T;
@@ -723,6 +750,7 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
         threshold_kernel<<<static_cast<unsigned>(T), kSelThreads, smem, s>>>(ta);
         if ((st = cuda_status(cudaGetLastError())) != FTK_OK) return st;
     }
+    stage_mark(3, s);
 
     // dense scan
     sa.tile_lo = w.c_lo;
@@ -737,6 +765,7 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
     sa.out = nullptr;
     st = launch_score_dt<MODE_COLLECT>(dtype, sa, tq, kvm, sms, s);
     if (st != FTK_OK) return st;
+    stage_mark(4, s);
 
     RefineArgs ra;
     ra.T = T;
@@ -762,6 +791,7 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
         refine_kernel<<<static_cast<unsigned>(T), kSelThreads, smem, s>>>(ra);
         if ((st = cuda_status(cudaGetLastError())) != FTK_OK) return st;
     }
+    stage_mark(5, s);
 
     // dense recovery of the listed rows, rec_rows at a time
     int rcluster = 1, rchunk = 8;
@@ -806,6 +836,7 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
         st = launch_rows_topk(FTK_F32, ra2, rcluster, s);
         if (st != FTK_OK) return st;
     }
+    stage_mark(6, s);
     return FTK_OK;
 }
 

@@ -38,7 +38,7 @@ HEADS, DIM, MAX_TOPK = 32, 128, 4096
 EXPORTS = (
     "ftk_select", "ftk_select_workspace_size", "ftk_read_info", "ftk_topk_rows",
     "ftk_score_dense", "ftk_score_dense_workspace_size", "ftk_windows_from_cu_seqlens",
-    "ftk_status_string", "ftk_version",
+    "ftk_set_stage_events", "ftk_status_string", "ftk_version",
 )
 
 
@@ -57,7 +57,7 @@ class FtkInfo(ctypes.Structure):
                 ("rows", ctypes.c_int64), ("rows_underflow", ctypes.c_int64),
                 ("rows_overflow", ctypes.c_int64), ("blocks_total", ctypes.c_int64),
                 ("blocks_pruned", ctypes.c_int64), ("candidates_total", ctypes.c_int64),
-                ("candidates_max", ctypes.c_int64)]
+                ("candidates_max", ctypes.c_int64), ("kernel_launches", ctypes.c_int64)]
 
     def as_dict(self) -> dict:
         return {name: getattr(self, name) for name, _ in self._fields_}
@@ -86,6 +86,8 @@ def load_library(path: str = LIB_PATH):
     L.ftk_score_dense_workspace_size.argtypes = [I64]
     L.ftk_windows_from_cu_seqlens.restype = I32
     L.ftk_windows_from_cu_seqlens.argtypes = [P, P, I64, I64, P, P, P]
+    L.ftk_set_stage_events.restype = I32
+    L.ftk_set_stage_events.argtypes = [P, I32]
     L.ftk_status_string.restype = ctypes.c_char_p
     L.ftk_status_string.argtypes = [I32]
     L.ftk_version.restype = I32
@@ -183,6 +185,30 @@ def select(q, kv, weights, ks, ke, kv_scales=None, topk: int = 2048, return_scor
                           _stream(dev))
     _check(st, "ftk_select")
     return (out_idx, out_val) if return_scores else out_idx
+
+
+STAGES = ("plan", "sample", "threshold", "scan", "refine", "recovery")
+
+
+class stage_events:
+    """Context manager: records CUDA events at ftk_select's stage boundaries
+    (diagnostic; see ftk_set_stage_events).  After synchronising, .times_ms()
+    gives the duration of each stage of the last recorded call."""
+
+    def __init__(self):
+        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)]
+        self._arr = (ctypes.c_void_p * len(self.events))(*[ctypes.c_void_p(e.cuda_event) for e in self.events])
+
+    def __enter__(self):
+        _check(lib().ftk_set_stage_events(self._arr, len(self.events)), "ftk_set_stage_events")
+        return self
+
+    def __exit__(self, *exc):
+        lib().ftk_set_stage_events(None, 0)
+        return False
+
+    def times_ms(self) -> dict:
+        return {name: self.events[i].elapsed_time(self.events[i + 1]) for i, name in enumerate(STAGES)}
 
 
 def read_info(workspace: torch.Tensor) -> dict:

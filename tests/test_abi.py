@@ -50,7 +50,7 @@ def test_version_and_strings(lib):
 
 def test_structs_match_header_sizes():
     assert ctypes.sizeof(ftk.FtkConfig) == 32
-    assert ctypes.sizeof(ftk.FtkInfo) == 8 + 7 * 8
+    assert ctypes.sizeof(ftk.FtkInfo) == 8 + 8 * 8
 
 
 def test_workspace_size(lib):

@@ -193,3 +193,18 @@ def test_selector_and_last_info():
     assert info["candidates_total"] >= 16 * 64
     ref, _, _ = run_select(g)
     assert np.array_equal(to_np(idx), ref)
+
+
+@pytest.mark.parametrize("name,nrows,nfp64", [("fp8_prefill", 64, 16), ("fp8_packed", 64, 16),
+                                              ("fp8_large", 64, 8)])
+def test_full_size_workloads(name, nrows, nfp64):
+    """Full-size FP8 workloads: every row checked against the invariants,
+    64 seeded rows bit-exact against the oracle's selection of the GPU's own
+    scores, and a subset against the fp64 oracle (scores and sets)."""
+    c = wl.get(name)
+    rows = wl.sample_rows(c.T, nrows, seed=1)
+    fp64_rows = rows[:: max(1, len(rows) // nfp64)][:nfp64] + [rows[-1]]
+    _, _, info, worst, overlaps = check_case(c, rows=rows, fp64_rows=fp64_rows)
+    assert worst < 1e-4
+    assert min(overlaps) >= 0.99
+    print(f"{name}: worst |dI|/E {worst:.2e}, info {info}")
