@@ -47,6 +47,8 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--rows", type=int, default=0,
+                    help="use only the first ROWS queries of the batch (profiling captures)")
     return ap.parse_args()
 
 
@@ -240,6 +242,10 @@ def run_ours(args):
     from sparse_attention_indexer_ftk_b200 import workloads as wl
 
     c = wl.get(WORKLOAD)
+    if args.rows and args.rows < c.T:
+        c = wl.SelectInputs(c.name, c.q[:args.rows].contiguous(), c.kv, c.kv_scales,
+                            c.weights[:args.rows].contiguous(), c.ks[:args.rows].contiguous(),
+                            c.ke[:args.rows].contiguous(), c.topk)
     g = c.to(dev)
     T, S, k = c.T, c.S, c.topk
     pairs = c.pairs()

@@ -208,7 +208,9 @@ ftk_status ftk_windows_from_cu_seqlens(const int32_t *cu_q,
  * caller, passed as void *) on the call's stream at its stage boundaries:
  * 0 start, 1 plan done, 2 sample pass done, 3 thresholds done, 4 dense scan
  * done, 5 refine done, 6 recovery done.  n must be 0 (or events NULL) to
- * stop, else >= 7.  The library does not own the events. */
+ * stop, else >= 7 with non-NULL events (FTK_ERR_INVALID_ARG otherwise).  If
+ * recording fails the hook switches itself off.  The library does not own
+ * the events. */
 ftk_status ftk_set_stage_events(void *const *events, int n);
 
 /* Human-readable name of an ftk_status value (static string). */

@@ -52,7 +52,7 @@ struct ScoreCfg<FTK_F8E4M3> {
     static constexpr int kAtoms = 1;      // 128-byte swizzle atoms along K (128 dims x 1 B)
     static constexpr int kQStages = 2;
     static constexpr int kKStages = 4;
-    static constexpr int kStageCap = 1024; // staged candidates per query
+    static constexpr int kWarpStage = 256; // staged candidates per (epilogue warp, query)
     static constexpr int kMmaK = 4;       // MMAs per tile (K = 32 each)
     static constexpr uint32_t kIdesc = instr_desc(0, 0, 128, 256);  // e4m3 x e4m3 -> f32
 };
@@ -62,7 +62,7 @@ struct ScoreCfg<FTK_BF16> {
     static constexpr int kAtoms = 2;      // 128 dims x 2 B = two 128-byte atoms
     static constexpr int kQStages = 1;
     static constexpr int kKStages = 3;
-    static constexpr int kStageCap = 512;
+    static constexpr int kWarpStage = 128;
     static constexpr int kMmaK = 8;       // K = 16 each
     static constexpr uint32_t kIdesc = instr_desc(1, 1, 128, 256);  // bf16 x bf16 -> f32
 };
@@ -179,20 +179,35 @@ __device__ __forceinline__ bool get_item(const ScoreArgs &a, int it, int64_t nli
     return m.nkt > 0;
 }
 
-// The head reduction of one (query, key) pair: sum_h w_h * max(x_h, 0) in a
-// fixed order (four interleaved partial sums), then sigma, then +0.0 turns
-// a -0.0 into +0.0.  Every mode and every caller uses exactly this.
+__device__ __forceinline__ uint64_t pack2(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ void ffma2(uint64_t &acc, uint64_t a, uint64_t b)
+{
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
+}
+
+// The head reduction of one (query, key) pair: sum_h w_h * max(x_h, 0) as
+// four partial sums over h = 0, 1, 2, 3 (mod 4), each a chain of
+// correctly rounded fmas (two packed lanes per instruction), combined as
+// (p0 + p1) + (p2 + p3); then sigma, with +0.0 added so that a -0.0 becomes
+// +0.0.  Every mode and every caller uses exactly this arithmetic.
 __device__ __forceinline__ float head_reduce(const float (&x)[32], const float *w, float sigma)
 {
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    uint64_t p01 = 0, p23 = 0;  // (+0.0, +0.0)
 #pragma unroll
     for (int h = 0; h < 32; h += 4) {
-        const float4 wv = *reinterpret_cast<const float4 *>(w + h);
-        a0 = __fmaf_rn(wv.x, fmaxf(x[h + 0], 0.f), a0);
-        a1 = __fmaf_rn(wv.y, fmaxf(x[h + 1], 0.f), a1);
-        a2 = __fmaf_rn(wv.z, fmaxf(x[h + 2], 0.f), a2);
-        a3 = __fmaf_rn(wv.w, fmaxf(x[h + 3], 0.f), a3);
+        const ulonglong2 wv = *reinterpret_cast<const ulonglong2 *>(w + h);
+        ffma2(p01, wv.x, pack2(fmaxf(x[h + 0], 0.f), fmaxf(x[h + 1], 0.f)));
+        ffma2(p23, wv.y, pack2(fmaxf(x[h + 2], 0.f), fmaxf(x[h + 3], 0.f)));
     }
+    float a0, a1, a2, a3;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(p01));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a2), "=f"(a3) : "l"(p23));
     const float acc = __fadd_rn(__fadd_rn(a0, a1), __fadd_rn(a2, a3));
     return __fmaf_rn(sigma, acc, 0.0f);
 }
@@ -204,10 +219,11 @@ struct ScoreSmemLayout {
     static constexpr int kKBytes = C::kAtoms * kKeyTile * 128;          // 16 KB per atom
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + C::kQStages * kQBytes;
+    static constexpr int kStageEntries = (kEpiThreads / 32) * 4 * C::kWarpStage;
     static constexpr int kOffStageVal = kOffK + C::kKStages * kKBytes;
-    static constexpr int kOffStageIdx = kOffStageVal + kQTile * C::kStageCap * 4;
-    static constexpr int kOffW = kOffStageIdx + kQTile * C::kStageCap * 4;
-    static constexpr int kOffMisc = kOffW + kQTile * kHeads * 4;
+    static constexpr int kOffStageIdx = kOffStageVal + kStageEntries * 4;
+    static constexpr int kOffW = kOffStageIdx + kStageEntries * 4;
+    static constexpr int kOffMisc = kOffW + (kEpiThreads / 32) * 4 * kHeads * 4;
     static constexpr int kMiscBytes = 512;  // >= sizeof(ScoreMisc), checked below
     static constexpr int kBytes = kOffMisc + kMiscBytes + 1024;  // + alignment slack
 };
@@ -217,15 +233,8 @@ struct ScoreMisc {
     uint64_t q_full[2], q_empty[2];
     uint64_t acc_full[2], acc_empty[2];
     uint64_t final_bar;
-    uint64_t epi_bar;          // group barrier of the epilogue warps
     uint32_t tmem_base;
-    int32_t flush_now;
     int32_t abort;
-    int32_t qt[kQTile];        // query of each tile slot (-1: none)
-    int32_t qks[kQTile], qke[kQTile];
-    float qtau[kQTile];
-    int32_t stage_cnt[kQTile];
-    int32_t qpos[kQTile];      // list position of each tile slot
 };
 
 static_assert(sizeof(ScoreMisc) <= ScoreSmemLayout<FTK_F8E4M3>::kMiscBytes, "misc area");
@@ -268,9 +277,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             mbar_init(&ms.acc_empty[i], kEpiThreads / 32);
         }
         mbar_init(&ms.final_bar, 1);
-        mbar_init(&ms.epi_bar, kEpiThreads);
         ms.abort = 0;
-        for (int j = 0; j < kQTile; ++j) ms.stage_cnt[j] = 0;
         fence_barrier_init();
     }
     if (warp == 1) tmem_alloc(&ms.tmem_base, 512);
@@ -389,14 +396,20 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         }
     } else {
         // ------------------------------------------------------------ epilogue
+        // Each epilogue warp works on its own: its 4 queries' parameters and
+        // weights, and its own candidate staging, so the tile loop has no
+        // cross-warp synchronisation besides releasing the accumulator.
         const int ew = warp - 2;                 // 0..7
         const int quad = warp & 3;               // TMEM lane quarter
-        const int half = ew >> 2;                // queries 4*half .. 4*half+3
-        const int et = threadIdx.x - 64;         // 0..255
+        const int half = ew >> 2;                // tile queries 4*half .. 4*half+3
         const int key_lane = quad * 32 + lane;   // row of the 128-key tile
         const uint32_t tlane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+        const uint32_t lt_mask = (1u << lane) - 1u;
+        float *my_w = sw + ew * 4 * kHeads;
+        float *my_sv = stage_val + ew * 4 * C::kWarpStage;
+        int32_t *my_si = stage_idx + ew * 4 * C::kWarpStage;
         int ab = 0;
-        uint32_t aph = 0, eph = 0;
+        uint32_t aph = 0;
         bool bad_scale = false;
         for (int it = blockIdx.x; !*abort; it += gridDim.x) {
             Item m;
@@ -407,23 +420,34 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                 if (it >= a.static_chunks * ((a.nrows + kQTile - 1) / kQTile)) break;
                 if (!get_item<MODE>(a, it, nlist, m)) continue;
             }
-            // The previous item (and its flush) is retired before its
-            // per-query parameters are replaced.
-            if (!__all_sync(0xFFFFFFFFu, group_sync(&ms.epi_bar, eph, abort, a.status))) break;
+            // Per-item parameters of this warp's 4 queries (warp-uniform).
+            int32_t qt[4], qks[4], qke[4], qpos[4];
+            float qtau[4];
             {
-                const int j = et >> 5, h = et & 31;
-                const int64_t p = static_cast<int64_t>(m.tile) * kQTile + j;
-                const int32_t t = list_query(a, p, nlist);
-                sw[j * kHeads + h] = t >= 0 ? a.weights[static_cast<int64_t>(t) * kHeads + h] : 0.f;
-                if (h == 0) {
-                    ms.qt[j] = t;
-                    ms.qpos[j] = static_cast<int32_t>(p);
-                    ms.qks[j] = t >= 0 ? a.ks[t] : 0;
-                    ms.qke[j] = t >= 0 ? a.ke[t] : 0;
-                    ms.qtau[j] = (MODE == MODE_COLLECT && t >= 0) ? a.tau[t] : 0.f;
+                const int64_t p = static_cast<int64_t>(m.tile) * kQTile + half * 4 + (lane & 3);
+                int32_t t_l = -1, ks_l = 0, ke_l = 0;
+                float tau_l = 0.f;
+                if (lane < 4) {
+                    t_l = list_query(a, p, nlist);
+                    if (t_l >= 0) {
+                        ks_l = a.ks[t_l];
+                        ke_l = a.ke[t_l];
+                        if (MODE == MODE_COLLECT) tau_l = a.tau[t_l];
+                    }
                 }
+#pragma unroll
+                for (int qi = 0; qi < 4; ++qi) {
+                    qt[qi] = __shfl_sync(0xFFFFFFFFu, t_l, qi);
+                    qks[qi] = __shfl_sync(0xFFFFFFFFu, ks_l, qi);
+                    qke[qi] = __shfl_sync(0xFFFFFFFFu, ke_l, qi);
+                    qtau[qi] = __shfl_sync(0xFFFFFFFFu, tau_l, qi);
+                    qpos[qi] = m.tile * kQTile + half * 4 + qi;
+                    my_w[qi * kHeads + lane] =
+                        qt[qi] >= 0 ? a.weights[static_cast<int64_t>(qt[qi]) * kHeads + lane] : 0.f;
+                }
+                __syncwarp();
             }
-            if (!__all_sync(0xFFFFFFFFu, group_sync(&ms.epi_bar, eph, abort, a.status))) break;
+            int cnt[4] = {0, 0, 0, 0};  // staged candidates per query (warp-uniform)
             bool ok = true;
             for (int kt = 0; kt < m.nkt; ++kt) {
                 const int32_t kidx = m.key0 + kt * kKeyTile + key_lane;  // key (SAMPLE: sample j)
@@ -447,75 +471,82 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                     break;
                 }
                 tc_fence_after();
-#pragma unroll 1
+                const uint32_t tcol = tlane + static_cast<uint32_t>(ab * 256 + half * 4 * 32);
+                float xa[32], xb[32];
+                tmem_ld32_async(tcol, xa);
+                tmem_wait_ld(xa);
+#pragma unroll
                 for (int qi = 0; qi < 4; ++qi) {
-                    const int j = half * 4 + qi;
-                    float x[32];
-                    tmem_ld32(tlane + static_cast<uint32_t>(ab * 256 + j * 32), x);
-                    const float I = head_reduce(x, sw + j * kHeads, sigma);
-                    const int32_t t = ms.qt[j];
-                    const bool valid = in_range && t >= 0 && s >= ms.qks[j] && s < ms.qke[j];
+                    float (&cur)[32] = (qi & 1) ? xb : xa;
+                    float (&nxt)[32] = (qi & 1) ? xa : xb;
+                    if (qi < 3) {
+                        tmem_ld32_async(tcol + static_cast<uint32_t>((qi + 1) * 32), nxt);
+                    } else {
+                        // Every column of this tile is in registers: hand the
+                        // accumulator back to the MMA warp.
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&ms.acc_empty[ab]);
+                    }
+                    const float I = head_reduce(cur, my_w + qi * kHeads, sigma);
+                    if (qi < 3) tmem_wait_ld(nxt);
+                    const bool valid = in_range && qt[qi] >= 0 && s >= qks[qi] && s < qke[qi];
                     if (MODE == MODE_COLLECT) {
-                        const bool take = valid && !(I < ms.qtau[j]);
+                        const bool take = valid && !(I < qtau[qi]);  // NaN is kept, to be seen
                         const uint32_t bal = __ballot_sync(0xFFFFFFFFu, take);
                         if (bal) {
-                            const int leader = __ffs(bal) - 1;
-                            int base = 0;
-                            if (lane == leader) base = atomicAdd(&ms.stage_cnt[j], __popc(bal));
-                            base = __shfl_sync(0xFFFFFFFFu, base, leader);
                             if (take) {
-                                const int pos = base + __popc(bal & ((1u << lane) - 1u));
-                                stage_val[j * C::kStageCap + pos] = I;
-                                stage_idx[j * C::kStageCap + pos] = static_cast<int32_t>(s);
+                                const int pos = cnt[qi] + __popc(bal & lt_mask);
+                                my_sv[qi * C::kWarpStage + pos] = I;
+                                my_si[qi * C::kWarpStage + pos] = static_cast<int32_t>(s);
                             }
+                            cnt[qi] += __popc(bal);
                         }
                     } else if (MODE == MODE_SAMPLE) {
-                        if (t >= 0 && kidx < m.kend)
-                            a.out[static_cast<int64_t>(t) * a.ld + (kidx - m.key0)] =
+                        if (qt[qi] >= 0 && kidx < m.kend)
+                            a.out[static_cast<int64_t>(qt[qi]) * a.ld + (kidx - m.key0)] =
                                 valid ? I : -INFINITY;
                     } else {
-                        if (valid)
-                            a.out[static_cast<int64_t>(ms.qpos[j]) * a.ld + (s - ms.qks[j])] = I;
+                        if (valid) a.out[static_cast<int64_t>(qpos[qi]) * a.ld + (s - qks[qi])] = I;
                     }
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&ms.acc_empty[ab]);
                 if (++ab == 2) { ab = 0; aph ^= 1u; }
                 if (MODE == MODE_COLLECT) {
-                    // Every candidate of this tile is staged; one thread decides
-                    // whether the staging buffers must be flushed before another
-                    // tile (<= 128 more per query) could overflow them.
-                    if (!__all_sync(0xFFFFFFFFu, group_sync(&ms.epi_bar, eph, abort, a.status))) { ok = false; break; }
-                    if (et == 0) {
-                        bool need = kt == m.nkt - 1;
+                    // Flush a query's staging before one more tile (<= 32 per
+                    // warp and query) could overflow it, and at the item's end.
+                    const bool last = kt == m.nkt - 1;
+                    bool need[4], any = false;
 #pragma unroll
-                        for (int j = 0; j < kQTile; ++j)
-                            need |= ms.stage_cnt[j] > C::kStageCap - kKeyTile;
-                        ms.flush_now = need;
+                    for (int qi = 0; qi < 4; ++qi) {
+                        need[qi] = cnt[qi] > 0 && (last || cnt[qi] > C::kWarpStage - 32);
+                        any |= need[qi];
                     }
-                    if (!__all_sync(0xFFFFFFFFu, group_sync(&ms.epi_bar, eph, abort, a.status))) { ok = false; break; }
-                    if (ms.flush_now) {
-                        const int j = ew;  // warp ew flushes query slot ew
-                        const int n = ms.stage_cnt[j];
-                        const int32_t t = ms.qt[j];
-                        if (n > 0 && t >= 0) {
-                            int base = 0;
-                            if (lane == 0) base = atomicAdd(a.cnt + t, n);
-                            base = __shfl_sync(0xFFFFFFFFu, base, 0);
-                            float *cv = a.cand_val + static_cast<int64_t>(t) * a.cap;
-                            int32_t *ci = a.cand_idx + static_cast<int64_t>(t) * a.cap;
-                            for (int i = lane; i < n; i += 32) {
-                                const int slot = base + i;
-                                if (slot < a.cap) {
-                                    cv[slot] = stage_val[j * C::kStageCap + i];
-                                    ci[slot] = stage_idx[j * C::kStageCap + i];
+                    if (any) {
+                        __syncwarp();  // staged entries visible to every lane
+                        int base[4] = {0, 0, 0, 0};
+                        if (lane == 0) {
+#pragma unroll
+                            for (int qi = 0; qi < 4; ++qi)  // independent atomics, latencies overlap
+                                if (need[qi] && qt[qi] >= 0) base[qi] = atomicAdd(a.cnt + qt[qi], cnt[qi]);
+                        }
+#pragma unroll
+                        for (int qi = 0; qi < 4; ++qi) {
+                            if (!need[qi]) continue;
+                            const int b = __shfl_sync(0xFFFFFFFFu, base[qi], 0);
+                            if (qt[qi] >= 0) {
+                                float *cv = a.cand_val + static_cast<int64_t>(qt[qi]) * a.cap;
+                                int32_t *ci = a.cand_idx + static_cast<int64_t>(qt[qi]) * a.cap;
+                                for (int i = lane; i < cnt[qi]; i += 32) {
+                                    const int slot = b + i;
+                                    if (slot < a.cap) {
+                                        cv[slot] = my_sv[qi * C::kWarpStage + i];
+                                        ci[slot] = my_si[qi * C::kWarpStage + i];
+                                    }
                                 }
                             }
+                            cnt[qi] = 0;
                         }
                         __syncwarp();
-                        if (lane == 0) ms.stage_cnt[j] = 0;
-                        if (!__all_sync(0xFFFFFFFFu, group_sync(&ms.epi_bar, eph, abort, a.status))) { ok = false; break; }
                     }
                 }
             }

@@ -612,7 +612,10 @@ thread_local void *const *g_stage_events = nullptr;
 
 static void stage_mark(int i, cudaStream_t s)
 {
-    if (g_stage_events) cudaEventRecord(static_cast<cudaEvent_t>(g_stage_events[i]), s);
+    if (g_stage_events && cudaEventRecord(static_cast<cudaEvent_t>(g_stage_events[i]), s) != cudaSuccess) {
+        (void)cudaGetLastError();  // a bad event must not poison the launch checks
+        g_stage_events = nullptr;
+    }
 }
 
 }  // namespace ftk
@@ -626,6 +629,8 @@ extern "C" ftk_status ftk_set_stage_events(void *const *events, int n)
         return FTK_OK;
     }
     if (n < 7) return FTK_ERR_INVALID_ARG;
+    for (int i = 0; i < 7; ++i)
+        if (events[i] == nullptr) return FTK_ERR_INVALID_ARG;
     g_stage_events = events;
     return FTK_OK;
 }

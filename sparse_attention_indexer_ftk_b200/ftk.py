@@ -197,6 +197,8 @@ class stage_events:
 
     def __init__(self):
         self.events = [torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)]
+        for e in self.events:  # torch creates the CUDA event on first record
+            e.record()
         self._arr = (ctypes.c_void_p * len(self.events))(*[ctypes.c_void_p(e.cuda_event) for e in self.events])
 
     def __enter__(self):
