@@ -13,12 +13,13 @@
 // query in registers: ReLU, the head weights and sigma are applied and the
 // T x S x 32 intermediate never leaves the SM.
 //
-// Warp roles (10 warps):
+// Warp roles (18 warps):
 //   warp 0      TMA producer: q tile per work item, key tiles through a
 //               multi-stage mbarrier ring;
 //   warp 1      TMEM allocator and MMA issuer (one elected thread);
-//   warps 2-9   epilogue: warp w reads TMEM lane quarter (w % 4) and the
-//               queries 4*((w-2)/4) .. +3 of the tile.
+//   warps 2-17  epilogue: warp w reads TMEM lane quarter (w % 4) and the
+//               queries 2*((w-2)/4), 2*((w-2)/4)+1 of the tile, four warps
+//               per scheduler so that their dependency chains interleave.
 //
 // Modes (one kernel body, so every mode produces bit-identical scores):
 //   SAMPLE   keys are a strided sample k[j*stride] (a strided TMA view of kv);
@@ -40,8 +41,10 @@ constexpr int kQTile = 8;            // queries per tile -> N = 256
 constexpr int kKeyTile = 128;        // keys per tile -> M = 128
 constexpr int kChunkTiles = 128;     // key tiles per work item (16384 keys)
 constexpr int kChunkKeys = kChunkTiles * kKeyTile;
-constexpr int kScoreThreads = 320;   // 10 warps
-constexpr int kEpiThreads = 256;     // warps 2..9
+constexpr int kEpiWarps = 16;        // warps 2..17
+constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kScoreThreads = 64 + kEpiThreads;  // + producer and MMA warps
+constexpr int kEpiQueries = kQTile * 4 / kEpiWarps;  // queries per epilogue warp (2)
 constexpr int kNumStrideMaps = 20;   // sample strides 2^0 .. 2^19
 
 template <int DT>
@@ -212,6 +215,35 @@ __device__ __forceinline__ float head_reduce(const float (&x)[32], const float *
     return __fmaf_rn(sigma, acc, 0.0f);
 }
 
+// One step of the head reduction of two queries over heads h0 .. h0+15:
+// xa / xb hold those 16 columns of query 0 / 1, w0 / w1 point at the
+// queries' 32 weights.  Four fma chains (query 0 heads = 0,1 | 2,3 mod 4,
+// query 1 likewise) advance in head order, so after both halves each
+// query's arithmetic is exactly head_reduce's.
+__device__ __forceinline__ void head_step2(const float (&xa)[16], const float (&xb)[16],
+                                           const float *w0, const float *w1, int h0,
+                                           uint64_t &p01, uint64_t &p23, uint64_t &q01,
+                                           uint64_t &q23)
+{
+#pragma unroll
+    for (int h = 0; h < 16; h += 4) {
+        const ulonglong2 wv = *reinterpret_cast<const ulonglong2 *>(w0 + h0 + h);
+        const ulonglong2 wu = *reinterpret_cast<const ulonglong2 *>(w1 + h0 + h);
+        ffma2(p01, wv.x, pack2(fmaxf(xa[h + 0], 0.f), fmaxf(xa[h + 1], 0.f)));
+        ffma2(q01, wu.x, pack2(fmaxf(xb[h + 0], 0.f), fmaxf(xb[h + 1], 0.f)));
+        ffma2(p23, wv.y, pack2(fmaxf(xa[h + 2], 0.f), fmaxf(xa[h + 3], 0.f)));
+        ffma2(q23, wu.y, pack2(fmaxf(xb[h + 2], 0.f), fmaxf(xb[h + 3], 0.f)));
+    }
+}
+
+__device__ __forceinline__ float head_finish(uint64_t p01, uint64_t p23, float sigma)
+{
+    float a0, a1, a2, a3;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(p01));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a2), "=f"(a3) : "l"(p23));
+    return __fmaf_rn(sigma, __fadd_rn(__fadd_rn(a0, a1), __fadd_rn(a2, a3)), 0.0f);
+}
+
 template <int DT>
 struct ScoreSmemLayout {
     using C = ScoreCfg<DT>;
@@ -219,11 +251,11 @@ struct ScoreSmemLayout {
     static constexpr int kKBytes = C::kAtoms * kKeyTile * 128;          // 16 KB per atom
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + C::kQStages * kQBytes;
-    static constexpr int kStageEntries = (kEpiThreads / 32) * 4 * C::kWarpStage;
+    static constexpr int kStageEntries = kEpiWarps * kEpiQueries * C::kWarpStage;
     static constexpr int kOffStageVal = kOffK + C::kKStages * kKBytes;
     static constexpr int kOffStageIdx = kOffStageVal + kStageEntries * 4;
     static constexpr int kOffW = kOffStageIdx + kStageEntries * 4;
-    static constexpr int kOffMisc = kOffW + (kEpiThreads / 32) * 4 * kHeads * 4;
+    static constexpr int kOffMisc = kOffW + kEpiWarps * kEpiQueries * kHeads * 4;
     static constexpr int kMiscBytes = 512;  // >= sizeof(ScoreMisc), checked below
     static constexpr int kBytes = kOffMisc + kMiscBytes + 1024;  // + alignment slack
 };
@@ -274,7 +306,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&ms.acc_full[i], 1);
-            mbar_init(&ms.acc_empty[i], kEpiThreads / 32);
+            mbar_init(&ms.acc_empty[i], kEpiWarps);
         }
         mbar_init(&ms.final_bar, 1);
         ms.abort = 0;
@@ -396,18 +428,19 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        // Each epilogue warp works on its own: its 4 queries' parameters and
+        // Each epilogue warp works on its own: its 2 queries' parameters and
         // weights, and its own candidate staging, so the tile loop has no
         // cross-warp synchronisation besides releasing the accumulator.
-        const int ew = warp - 2;                 // 0..7
+        constexpr int NQ = kEpiQueries;
+        const int ew = warp - 2;                 // 0..15
         const int quad = warp & 3;               // TMEM lane quarter
-        const int half = ew >> 2;                // tile queries 4*half .. 4*half+3
+        const int qg = ew >> 2;                  // tile queries NQ*qg .. NQ*qg+NQ-1
         const int key_lane = quad * 32 + lane;   // row of the 128-key tile
         const uint32_t tlane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
         const uint32_t lt_mask = (1u << lane) - 1u;
-        float *my_w = sw + ew * 4 * kHeads;
-        float *my_sv = stage_val + ew * 4 * C::kWarpStage;
-        int32_t *my_si = stage_idx + ew * 4 * C::kWarpStage;
+        float *my_w = sw + ew * NQ * kHeads;
+        float *my_sv = stage_val + ew * NQ * C::kWarpStage;
+        int32_t *my_si = stage_idx + ew * NQ * C::kWarpStage;
         int ab = 0;
         uint32_t aph = 0;
         bool bad_scale = false;
@@ -420,14 +453,14 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                 if (it >= a.static_chunks * ((a.nrows + kQTile - 1) / kQTile)) break;
                 if (!get_item<MODE>(a, it, nlist, m)) continue;
             }
-            // Per-item parameters of this warp's 4 queries (warp-uniform).
-            int32_t qt[4], qks[4], qke[4], qpos[4];
-            float qtau[4];
+            // Per-item parameters of this warp's queries (warp-uniform).
+            int32_t qt[NQ], qks[NQ], qke[NQ], qpos[NQ];
+            float qtau[NQ];
             {
-                const int64_t p = static_cast<int64_t>(m.tile) * kQTile + half * 4 + (lane & 3);
+                const int64_t p = static_cast<int64_t>(m.tile) * kQTile + qg * NQ + (lane % NQ);
                 int32_t t_l = -1, ks_l = 0, ke_l = 0;
                 float tau_l = 0.f;
-                if (lane < 4) {
+                if (lane < NQ) {
                     t_l = list_query(a, p, nlist);
                     if (t_l >= 0) {
                         ks_l = a.ks[t_l];
@@ -436,117 +469,134 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                     }
                 }
 #pragma unroll
-                for (int qi = 0; qi < 4; ++qi) {
+                for (int qi = 0; qi < NQ; ++qi) {
                     qt[qi] = __shfl_sync(0xFFFFFFFFu, t_l, qi);
                     qks[qi] = __shfl_sync(0xFFFFFFFFu, ks_l, qi);
                     qke[qi] = __shfl_sync(0xFFFFFFFFu, ke_l, qi);
                     qtau[qi] = __shfl_sync(0xFFFFFFFFu, tau_l, qi);
-                    qpos[qi] = m.tile * kQTile + half * 4 + qi;
+                    qpos[qi] = m.tile * kQTile + qg * NQ + qi;
                     my_w[qi * kHeads + lane] =
                         qt[qi] >= 0 ? a.weights[static_cast<int64_t>(qt[qi]) * kHeads + lane] : 0.f;
                 }
                 __syncwarp();
             }
-            int cnt[4] = {0, 0, 0, 0};  // staged candidates per query (warp-uniform)
+            int cnt[NQ];  // staged candidates per query (warp-uniform)
+#pragma unroll
+            for (int qi = 0; qi < NQ; ++qi) cnt[qi] = 0;
+            // Keys are int32 (S < 2^31).  A query outside the list has the
+            // empty window [0, 0).  In SAMPLE mode key j of the tile is
+            // sample j, at kv row j << lg.
+            int32_t wlo[NQ], wlen[NQ];
+#pragma unroll
+            for (int qi = 0; qi < NQ; ++qi) {
+                wlo[qi] = qt[qi] >= 0 ? qks[qi] : 0;
+                wlen[qi] = qt[qi] >= 0 ? qke[qi] - qks[qi] : 0;
+            }
+            const float *scales = a.kv_scales;
+            int32_t kidx_next = m.key0 + key_lane;
+            float sig_next = 1.f;
+            if (scales) {
+                const int64_t s0 = static_cast<int64_t>(kidx_next) << m.lg;
+                if (kidx_next < m.kend && s0 < a.S) sig_next = __ldg(scales + s0);
+            }
             bool ok = true;
             for (int kt = 0; kt < m.nkt; ++kt) {
-                const int32_t kidx = m.key0 + kt * kKeyTile + key_lane;  // key (SAMPLE: sample j)
-                int64_t s;
-                bool in_range;
-                if (MODE == MODE_SAMPLE) {
-                    s = static_cast<int64_t>(kidx) << m.lg;
-                    in_range = kidx < m.kend && s < a.S;
-                } else {
-                    s = kidx;
-                    in_range = kidx < m.kend;
+                const int32_t kidx = kidx_next;
+                const float sigma = sig_next;
+                kidx_next += kKeyTile;
+                if (scales && kt + 1 < m.nkt) {  // sigma one tile ahead
+                    const int64_t s1 = static_cast<int64_t>(kidx_next) << m.lg;
+                    sig_next = (kidx_next < m.kend && s1 < a.S) ? __ldg(scales + s1) : 1.f;
                 }
-                float sigma = 1.f;
-                if (a.kv_scales && in_range) {
-                    sigma = __ldg(a.kv_scales + s);
-                    bad_scale |= !(sigma > 0.f) || isinf(sigma);
-                }
+                bad_scale |= scales && kidx < m.kend && (!(sigma > 0.f) || isinf(sigma));
+                const int32_t s = MODE == MODE_SAMPLE ? (kidx << m.lg) : kidx;
                 const bool got = mbar_wait(&ms.acc_full[ab], aph, abort, a.status);
                 if (!__all_sync(0xFFFFFFFFu, got)) {  // also reconverges the warp
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t tcol = tlane + static_cast<uint32_t>(ab * 256 + half * 4 * 32);
-                float xa[32], xb[32];
-                tmem_ld32_async(tcol, xa);
-                tmem_wait_ld(xa);
+                const uint32_t c0 = tlane + static_cast<uint32_t>(ab * 256 + qg * NQ * 32);
+                uint64_t p01 = 0, p23 = 0, q01 = 0, q23 = 0;
 #pragma unroll
-                for (int qi = 0; qi < 4; ++qi) {
-                    float (&cur)[32] = (qi & 1) ? xb : xa;
-                    float (&nxt)[32] = (qi & 1) ? xa : xb;
-                    if (qi < 3) {
-                        tmem_ld32_async(tcol + static_cast<uint32_t>((qi + 1) * 32), nxt);
-                    } else {
+                for (int hh = 0; hh < 2; ++hh) {
+                    float xa[16], xb[16];
+                    tmem_ld16x2(c0 + hh * 16, c0 + 32 + hh * 16, xa, xb);
+                    if (hh == 1) {
                         // Every column of this tile is in registers: hand the
                         // accumulator back to the MMA warp.
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&ms.acc_empty[ab]);
                     }
-                    const float I = head_reduce(cur, my_w + qi * kHeads, sigma);
-                    if (qi < 3) tmem_wait_ld(nxt);
-                    const bool valid = in_range && qt[qi] >= 0 && s >= qks[qi] && s < qke[qi];
+                    head_step2(xa, xb, my_w, my_w + kHeads, hh * 16, p01, p23, q01, q23);
+                }
+                if (++ab == 2) { ab = 0; aph ^= 1u; }
+                float I[NQ];
+                I[0] = head_finish(p01, p23, sigma);
+                I[1] = head_finish(q01, q23, sigma);
+#pragma unroll
+                for (int qi = 0; qi < NQ; ++qi) {
+                    // s in [wlo, wlo + wlen) as one unsigned compare
+                    const bool valid = static_cast<uint32_t>(s - wlo[qi]) < static_cast<uint32_t>(wlen[qi]);
                     if (MODE == MODE_COLLECT) {
-                        const bool take = valid && !(I < qtau[qi]);  // NaN is kept, to be seen
+                        const bool take = valid && !(I[qi] < qtau[qi]);  // NaN is kept, to be seen
                         const uint32_t bal = __ballot_sync(0xFFFFFFFFu, take);
-                        if (bal) {
-                            if (take) {
-                                const int pos = cnt[qi] + __popc(bal & lt_mask);
-                                my_sv[qi * C::kWarpStage + pos] = I;
-                                my_si[qi * C::kWarpStage + pos] = static_cast<int32_t>(s);
-                            }
-                            cnt[qi] += __popc(bal);
+                        const int pos = cnt[qi] + __popc(bal & lt_mask);
+                        if (take) {
+                            my_sv[qi * C::kWarpStage + pos] = I[qi];
+                            my_si[qi * C::kWarpStage + pos] = s;
                         }
+                        cnt[qi] += __popc(bal);
                     } else if (MODE == MODE_SAMPLE) {
                         if (qt[qi] >= 0 && kidx < m.kend)
                             a.out[static_cast<int64_t>(qt[qi]) * a.ld + (kidx - m.key0)] =
-                                valid ? I : -INFINITY;
+                                valid ? I[qi] : -INFINITY;
                     } else {
-                        if (valid) a.out[static_cast<int64_t>(qpos[qi]) * a.ld + (s - qks[qi])] = I;
+                        if (valid) a.out[static_cast<int64_t>(qpos[qi]) * a.ld + (s - wlo[qi])] = I[qi];
                     }
                 }
-                if (++ab == 2) { ab = 0; aph ^= 1u; }
                 if (MODE == MODE_COLLECT) {
-                    // Flush a query's staging before one more tile (<= 32 per
-                    // warp and query) could overflow it, and at the item's end.
+                    // Every 4 tiles (<= 4 * 32 new entries per warp and query)
+                    // and at the item's end, flush the queries whose staging
+                    // could otherwise overflow.
                     const bool last = kt == m.nkt - 1;
-                    bool need[4], any = false;
+                    if (last || (kt & 3) == 3) {
+                        bool need[NQ], any = false;
 #pragma unroll
-                    for (int qi = 0; qi < 4; ++qi) {
-                        need[qi] = cnt[qi] > 0 && (last || cnt[qi] > C::kWarpStage - 32);
-                        any |= need[qi];
-                    }
-                    if (any) {
-                        __syncwarp();  // staged entries visible to every lane
-                        int base[4] = {0, 0, 0, 0};
-                        if (lane == 0) {
-#pragma unroll
-                            for (int qi = 0; qi < 4; ++qi)  // independent atomics, latencies overlap
-                                if (need[qi] && qt[qi] >= 0) base[qi] = atomicAdd(a.cnt + qt[qi], cnt[qi]);
+                        for (int qi = 0; qi < NQ; ++qi) {
+                            need[qi] = cnt[qi] > 0 && (last || cnt[qi] > C::kWarpStage - 4 * 32);
+                            any |= need[qi];
                         }
+                        if (any) {
+                            __syncwarp();  // staged entries visible to every lane
+                            int base[NQ];
 #pragma unroll
-                        for (int qi = 0; qi < 4; ++qi) {
-                            if (!need[qi]) continue;
-                            const int b = __shfl_sync(0xFFFFFFFFu, base[qi], 0);
-                            if (qt[qi] >= 0) {
-                                float *cv = a.cand_val + static_cast<int64_t>(qt[qi]) * a.cap;
-                                int32_t *ci = a.cand_idx + static_cast<int64_t>(qt[qi]) * a.cap;
-                                for (int i = lane; i < cnt[qi]; i += 32) {
-                                    const int slot = b + i;
-                                    if (slot < a.cap) {
-                                        cv[slot] = my_sv[qi * C::kWarpStage + i];
-                                        ci[slot] = my_si[qi * C::kWarpStage + i];
+                            for (int qi = 0; qi < NQ; ++qi) base[qi] = 0;
+                            if (lane == 0) {
+#pragma unroll
+                                for (int qi = 0; qi < NQ; ++qi)  // independent atomics, latencies overlap
+                                    if (need[qi] && qt[qi] >= 0) base[qi] = atomicAdd(a.cnt + qt[qi], cnt[qi]);
+                            }
+#pragma unroll
+                            for (int qi = 0; qi < NQ; ++qi) {
+                                if (!need[qi]) continue;
+                                const int b = __shfl_sync(0xFFFFFFFFu, base[qi], 0);
+                                if (qt[qi] >= 0) {
+                                    float *cv = a.cand_val + static_cast<int64_t>(qt[qi]) * a.cap;
+                                    int32_t *ci = a.cand_idx + static_cast<int64_t>(qt[qi]) * a.cap;
+                                    for (int i = lane; i < cnt[qi]; i += 32) {
+                                        const int slot = b + i;
+                                        if (slot < a.cap) {
+                                            cv[slot] = my_sv[qi * C::kWarpStage + i];
+                                            ci[slot] = my_si[qi * C::kWarpStage + i];
+                                        }
                                     }
                                 }
+                                cnt[qi] = 0;
                             }
-                            cnt[qi] = 0;
+                            __syncwarp();
                         }
-                        __syncwarp();
                     }
                 }
             }
