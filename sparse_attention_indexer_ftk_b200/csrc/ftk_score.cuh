@@ -6,20 +6,31 @@
 //
 // GEMM orientation: A = a tile of 128 keys (M = 128, K = 128 head dims),
 // B = a tile of 8 queries x 32 heads (N = 256), both K-major with the
-// 128-byte swizzle.  The fp32 accumulator tile (128 lanes x 256 columns)
-// lives in tensor memory, double-buffered (2 x 256 of the 512 columns), so
-// the MMA of key tile i+1 overlaps the epilogue of key tile i.  TMEM lane =
-// key, so each epilogue thread owns one key and reduces the 32 heads of a
-// query in registers: ReLU, the head weights and sigma are applied and the
-// T x S x 32 intermediate never leaves the SM.
+// 128-byte swizzle.  A work item holds a group of QG such query tiles
+// resident in shared memory (QG = 2 for FP8) and streams key tiles through
+// a TMA ring; each key tile feeds QG MMAs, one per query tile, which halves
+// the key traffic from L2 per FLOP.  The fp32 accumulator (128 lanes x 256
+// columns) alternates between two tensor-memory buffers (2 x 256 of the 512
+// columns), so the MMA of the next (key tile, query tile) overlaps the
+// epilogue of the current one.  TMEM lane = key, so each epilogue thread
+// owns one key and reduces the 32 heads of a query in registers: ReLU, the
+// head weights and sigma are applied and the T x S x 32 intermediate never
+// leaves the SM.
 //
 // Warp roles (18 warps):
-//   warp 0      TMA producer: q tile per work item, key tiles through a
-//               multi-stage mbarrier ring;
+//   warp 0      TMA producer: the query group per work item, key tiles
+//               through a multi-stage mbarrier ring;
 //   warp 1      TMEM allocator and MMA issuer (one elected thread);
 //   warps 2-17  epilogue: warp w reads TMEM lane quarter (w % 4) and the
-//               queries 2*((w-2)/4), 2*((w-2)/4)+1 of the tile, four warps
-//               per scheduler so that their dependency chains interleave.
+//               queries 2*((w-2)/4), 2*((w-2)/4)+1 of every query tile, four
+//               warps per scheduler so that their dependency chains
+//               interleave.
+//
+// Head reduction: for each (query, key), four partial sums over the heads
+// h = 0, 1, 2, 3 (mod 4), each a chain of correctly rounded fmas in head
+// order, combined as (p0 + p1) + (p2 + p3), times sigma, plus +0.0 (which
+// turns -0.0 into +0.0).  ReLU propagates NaN, so a NaN dot product makes the
+// score NaN, which the candidate test keeps and the refine step reports.
 //
 // Modes (one kernel body, so every mode produces bit-identical scores):
 //   SAMPLE   keys are a strided sample k[j*stride] (a strided TMA view of kv);
@@ -37,14 +48,14 @@ namespace ftk {
 
 enum ScoreMode { MODE_SAMPLE = 0, MODE_COLLECT = 1, MODE_DUMP = 2 };
 
-constexpr int kQTile = 8;            // queries per tile -> N = 256
+constexpr int kQTile = 8;            // queries per MMA tile -> N = 256
 constexpr int kKeyTile = 128;        // keys per tile -> M = 128
 constexpr int kChunkTiles = 128;     // key tiles per work item (16384 keys)
 constexpr int kChunkKeys = kChunkTiles * kKeyTile;
 constexpr int kEpiWarps = 16;        // warps 2..17
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kScoreThreads = 64 + kEpiThreads;  // + producer and MMA warps
-constexpr int kEpiQueries = kQTile * 4 / kEpiWarps;  // queries per epilogue warp (2)
+constexpr int kEpiQueries = kQTile * 4 / kEpiWarps;  // queries per epilogue warp per query tile (2)
 constexpr int kNumStrideMaps = 20;   // sample strides 2^0 .. 2^19
 
 template <int DT>
@@ -52,23 +63,29 @@ struct ScoreCfg;
 
 template <>
 struct ScoreCfg<FTK_F8E4M3> {
-    static constexpr int kAtoms = 1;      // 128-byte swizzle atoms along K (128 dims x 1 B)
-    static constexpr int kQStages = 2;
+    static constexpr int kAtoms = 1;       // 128-byte swizzle atoms along K (128 dims x 1 B)
+    static constexpr int kQG = 2;          // query tiles per work item (rows per item: 16)
     static constexpr int kKStages = 4;
-    static constexpr int kWarpStage = 256; // staged candidates per (epilogue warp, query)
-    static constexpr int kMmaK = 4;       // MMAs per tile (K = 32 each)
+    static constexpr int kWarpStage = 128; // staged candidates per (epilogue warp, query)
+    static constexpr int kMmaK = 4;        // MMAs per tile (K = 32 each)
     static constexpr uint32_t kIdesc = instr_desc(0, 0, 128, 256);  // e4m3 x e4m3 -> f32
 };
 
 template <>
 struct ScoreCfg<FTK_BF16> {
-    static constexpr int kAtoms = 2;      // 128 dims x 2 B = two 128-byte atoms
-    static constexpr int kQStages = 1;
+    static constexpr int kAtoms = 2;       // 128 dims x 2 B = two 128-byte atoms
+    static constexpr int kQG = 1;          // rows per item: 8
     static constexpr int kKStages = 3;
     static constexpr int kWarpStage = 128;
-    static constexpr int kMmaK = 8;       // K = 16 each
+    static constexpr int kMmaK = 8;        // K = 16 each
     static constexpr uint32_t kIdesc = instr_desc(1, 1, 128, 256);  // bf16 x bf16 -> f32
 };
+
+// Rows of the row list per work item (the planning granularity).
+__host__ __device__ constexpr int row_tile_of(int dtype)
+{
+    return dtype == FTK_F8E4M3 ? ScoreCfg<FTK_F8E4M3>::kQG * kQTile : ScoreCfg<FTK_BF16>::kQG * kQTile;
+}
 
 struct ScoreArgs {
     int64_t T, S;
@@ -82,8 +99,9 @@ struct ScoreArgs {
     int64_t nrows;
     const int32_t *count_dev;
     int32_t count_off;
-    // Schedule.  Planned: per-tile ranges and an item prefix written by the
-    // plan kernel.  Static: item = (tile, chunk), ranges found on the fly.
+    // Schedule over row tiles of row_tile_of(dtype) rows.  Planned: per-tile
+    // ranges and an item prefix written by the plan kernel.  Static: item =
+    // (tile, chunk), ranges found on the fly.
     int32_t planned;
     const int32_t *tile_lo, *tile_hi, *tile_lg, *item_start;
     int32_t ntiles;
@@ -138,7 +156,7 @@ __device__ __forceinline__ int32_t list_query(const ScoreArgs &a, int64_t p, int
     return static_cast<int32_t>(t);
 }
 
-template <int MODE>
+template <int MODE, int RT>
 __device__ __forceinline__ bool get_item(const ScoreArgs &a, int it, int64_t nlist, Item &m)
 {
     if (a.planned) {
@@ -165,8 +183,8 @@ __device__ __forceinline__ bool get_item(const ScoreArgs &a, int it, int64_t nli
         const int chunk = it - m.tile * a.static_chunks;
         m.lg = 0;
         int64_t lo = INT64_MAX, hi = -1;
-        for (int j = 0; j < kQTile; ++j) {
-            const int32_t t = list_query(a, static_cast<int64_t>(m.tile) * kQTile + j, nlist);
+        for (int j = 0; j < RT; ++j) {
+            const int32_t t = list_query(a, static_cast<int64_t>(m.tile) * RT + j, nlist);
             if (t < 0 || a.ks[t] == a.ke[t]) continue;
             lo = min(lo, static_cast<int64_t>(a.ks[t]));
             hi = max(hi, static_cast<int64_t>(a.ke[t]));
@@ -180,6 +198,21 @@ __device__ __forceinline__ bool get_item(const ScoreArgs &a, int it, int64_t nli
     }
     m.nkt = (m.kend - m.key0 + kKeyTile - 1) / kKeyTile;
     return m.nkt > 0;
+}
+
+// Next work item of this CTA (static round-robin over the item space), or
+// false when there are no more.  Every role walks the same sequence.
+template <int MODE, int RT>
+__device__ __forceinline__ bool next_item(const ScoreArgs &a, int &it, int64_t nlist, Item &m)
+{
+    for (;; it += gridDim.x) {
+        if (a.planned) {
+            if (it >= a.item_start[a.ntiles]) return false;
+        } else {
+            if (it >= a.static_chunks * ((a.nrows + RT - 1) / RT)) return false;
+        }
+        if (get_item<MODE, RT>(a, it, nlist, m)) return true;
+    }
 }
 
 __device__ __forceinline__ uint64_t pack2(float lo, float hi)
@@ -215,11 +248,25 @@ __device__ __forceinline__ float head_reduce(const float (&x)[32], const float *
     return __fmaf_rn(sigma, acc, 0.0f);
 }
 
+// ReLU on the ALU pipe: max(x, 0), NaN propagating.
+__device__ __forceinline__ float relu_alu(float x)
+{
+    float r;
+    asm("max.NaN.f32 %0, %1, 0f00000000;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+// Twice the ReLU on the FMA pipe: x + |x| (= 2x or +0; NaN propagates).  Its
+// weight is pre-halved, so (w/2) * (x + |x|) is bit for bit w * ReLU(x).
+__device__ __forceinline__ float relu2_fma(float x) { return __fadd_rn(x, fabsf(x)); }
+
 // One step of the head reduction of two queries over heads h0 .. h0+15:
 // xa / xb hold those 16 columns of query 0 / 1, w0 / w1 point at the
-// queries' 32 weights.  Four fma chains (query 0 heads = 0,1 | 2,3 mod 4,
-// query 1 likewise) advance in head order, so after both halves each
-// query's arithmetic is exactly head_reduce's.
+// queries' 32 weights as stored (heads = 2, 3 mod 4 pre-halved).  Four fma
+// chains (query 0 heads = 0,1 | 2,3 mod 4, query 1 likewise) advance in
+// head order, so after both halves each query's value is exactly
+//   sum over chains c of (sum_{h = c mod 4, in order} w_h * ReLU(x_h)).
+// Half of the ReLUs run on the ALU pipe and half on the FMA pipe.
 __device__ __forceinline__ void head_step2(const float (&xa)[16], const float (&xb)[16],
                                            const float *w0, const float *w1, int h0,
                                            uint64_t &p01, uint64_t &p23, uint64_t &q01,
@@ -229,12 +276,15 @@ __device__ __forceinline__ void head_step2(const float (&xa)[16], const float (&
     for (int h = 0; h < 16; h += 4) {
         const ulonglong2 wv = *reinterpret_cast<const ulonglong2 *>(w0 + h0 + h);
         const ulonglong2 wu = *reinterpret_cast<const ulonglong2 *>(w1 + h0 + h);
-        ffma2(p01, wv.x, pack2(fmaxf(xa[h + 0], 0.f), fmaxf(xa[h + 1], 0.f)));
-        ffma2(q01, wu.x, pack2(fmaxf(xb[h + 0], 0.f), fmaxf(xb[h + 1], 0.f)));
-        ffma2(p23, wv.y, pack2(fmaxf(xa[h + 2], 0.f), fmaxf(xa[h + 3], 0.f)));
-        ffma2(q23, wu.y, pack2(fmaxf(xb[h + 2], 0.f), fmaxf(xb[h + 3], 0.f)));
+        ffma2(p01, wv.x, pack2(relu_alu(xa[h + 0]), relu_alu(xa[h + 1])));
+        ffma2(q01, wu.x, pack2(relu_alu(xb[h + 0]), relu_alu(xb[h + 1])));
+        ffma2(p23, wv.y, pack2(relu2_fma(xa[h + 2]), relu2_fma(xa[h + 3])));
+        ffma2(q23, wu.y, pack2(relu2_fma(xb[h + 2]), relu2_fma(xb[h + 3])));
     }
 }
+
+// Stored weight of head h: heads = 2, 3 (mod 4) are halved (see head_step2).
+__device__ __forceinline__ float stored_weight(float w, int h) { return (h & 2) ? 0.5f * w : w; }
 
 __device__ __forceinline__ float head_finish(uint64_t p01, uint64_t p23, float sigma)
 {
@@ -247,22 +297,24 @@ __device__ __forceinline__ float head_finish(uint64_t p01, uint64_t p23, float s
 template <int DT>
 struct ScoreSmemLayout {
     using C = ScoreCfg<DT>;
-    static constexpr int kQBytes = C::kAtoms * kQTile * kHeads * 128;   // 32 KB per atom
-    static constexpr int kKBytes = C::kAtoms * kKeyTile * 128;          // 16 KB per atom
+    static constexpr int kQTileBytes = C::kAtoms * kQTile * kHeads * 128;  // 32 KB per atom
+    static constexpr int kQBytes = C::kQG * kQTileBytes;
+    static constexpr int kKBytes = C::kAtoms * kKeyTile * 128;             // 16 KB per atom
+    static constexpr int kWarpQueries = C::kQG * kEpiQueries;              // queries per epilogue warp
     static constexpr int kOffQ = 0;
-    static constexpr int kOffK = kOffQ + C::kQStages * kQBytes;
-    static constexpr int kStageEntries = kEpiWarps * kEpiQueries * C::kWarpStage;
+    static constexpr int kOffK = kOffQ + kQBytes;
+    static constexpr int kStageEntries = kEpiWarps * kWarpQueries * C::kWarpStage;
     static constexpr int kOffStageVal = kOffK + C::kKStages * kKBytes;
     static constexpr int kOffStageIdx = kOffStageVal + kStageEntries * 4;
     static constexpr int kOffW = kOffStageIdx + kStageEntries * 4;
-    static constexpr int kOffMisc = kOffW + kEpiWarps * kEpiQueries * kHeads * 4;
+    static constexpr int kOffMisc = kOffW + kEpiWarps * kWarpQueries * kHeads * 4;
     static constexpr int kMiscBytes = 512;  // >= sizeof(ScoreMisc), checked below
     static constexpr int kBytes = kOffMisc + kMiscBytes + 1024;  // + alignment slack
 };
 
 struct ScoreMisc {
     uint64_t kv_full[4], kv_empty[4];
-    uint64_t q_full[2], q_empty[2];
+    uint64_t q_full, q_empty;
     uint64_t acc_full[2], acc_empty[2];
     uint64_t final_bar;
     uint32_t tmem_base;
@@ -272,6 +324,7 @@ struct ScoreMisc {
 static_assert(sizeof(ScoreMisc) <= ScoreSmemLayout<FTK_F8E4M3>::kMiscBytes, "misc area");
 static_assert(ScoreSmemLayout<FTK_F8E4M3>::kBytes <= 227 * 1024, "fp8 smem budget");
 static_assert(ScoreSmemLayout<FTK_BF16>::kBytes <= 227 * 1024, "bf16 smem budget");
+static_assert(ScoreCfg<FTK_F8E4M3>::kKStages <= 4 && ScoreCfg<FTK_BF16>::kKStages <= 4, "barriers");
 
 template <int DT, int MODE>
 __global__ void __launch_bounds__(kScoreThreads, 1)
@@ -280,6 +333,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 {
     using C = ScoreCfg<DT>;
     using Lay = ScoreSmemLayout<DT>;
+    constexpr int QG = C::kQG;
+    constexpr int RT = QG * kQTile;  // rows per work item
     extern __shared__ uint8_t smem_dyn[];
     // 1024-byte alignment: the 128-byte swizzle pattern repeats every 8 rows.
     uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -300,10 +355,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             mbar_init(&ms.kv_full[i], 1);
             mbar_init(&ms.kv_empty[i], 1);
         }
-        for (int i = 0; i < C::kQStages; ++i) {
-            mbar_init(&ms.q_full[i], 1);
-            mbar_init(&ms.q_empty[i], 1);
-        }
+        mbar_init(&ms.q_full, 1);
+        mbar_init(&ms.q_empty, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&ms.acc_full[i], 1);
             mbar_init(&ms.acc_empty[i], kEpiWarps);
@@ -322,35 +375,30 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
-            int ks_ = 0, qs = 0;
+            int ks_ = 0;
             uint32_t kph = 0, qph = 0;
             int k_armed[4] = {0, 0, 0, 0};  // loads issued per stage, for the abort drain
             uint32_t k_armed_ph[4] = {0, 0, 0, 0};
-            int q_armed[2] = {0, 0};
-            uint32_t q_armed_ph[2] = {0, 0};
-            for (int it = blockIdx.x; !*abort; it += gridDim.x) {
-                Item m;
-                if (a.planned) {
-                    if (it >= a.item_start[a.ntiles]) break;
-                    if (!get_item<MODE>(a, it, nlist, m)) continue;
-                } else {
-                    if (it >= a.static_chunks * ((a.nrows + kQTile - 1) / kQTile)) break;
-                    if (!get_item<MODE>(a, it, nlist, m)) continue;
+            int q_armed = 0;
+            uint32_t q_armed_ph = 0;
+            Item m;
+            for (int it = blockIdx.x; !*abort && next_item<MODE, RT>(a, it, nlist, m); it += gridDim.x) {
+                // The query group: the 32 head rows of each of RT queries.
+                if (!mbar_wait(&ms.q_empty, qph ^ 1u, abort, a.status)) break;
+                mbar_arrive_expect_tx(&ms.q_full, Lay::kQBytes);
+                q_armed = 1;
+                q_armed_ph = qph;
+                for (int vt = 0; vt < QG; ++vt) {
+                    for (int j = 0; j < kQTile; ++j) {
+                        int32_t t = list_query(a, static_cast<int64_t>(m.tile) * RT + vt * kQTile + j, nlist);
+                        if (t < 0) t = 0;  // placeholder rows are masked in the epilogue
+                        for (int at = 0; at < C::kAtoms; ++at)
+                            tma_load_2d(sq + vt * Lay::kQTileBytes + at * (Lay::kQTileBytes / C::kAtoms) +
+                                            j * kHeads * 128,
+                                        &tm_q, &ms.q_full, at * 64, t * kHeads);
+                    }
                 }
-                // q tile: the 32 head rows of each of the 8 queries.
-                if (!mbar_wait(&ms.q_empty[qs], qph ^ 1u, abort, a.status)) break;
-                mbar_arrive_expect_tx(&ms.q_full[qs], Lay::kQBytes);
-                q_armed[qs] = 1;
-                q_armed_ph[qs] = qph;
-                for (int j = 0; j < kQTile; ++j) {
-                    int32_t t = list_query(a, static_cast<int64_t>(m.tile) * kQTile + j, nlist);
-                    if (t < 0) t = 0;  // placeholder rows are masked in the epilogue
-                    for (int at = 0; at < C::kAtoms; ++at)
-                        tma_load_2d(sq + qs * Lay::kQBytes + at * (Lay::kQBytes / C::kAtoms) +
-                                        j * kHeads * 128,
-                                    &tm_q, &ms.q_full[qs], at * 64, t * kHeads);
-                }
-                if (++qs == C::kQStages) { qs = 0; qph ^= 1u; }
+                qph ^= 1u;
                 const CUtensorMap *map = &kvm.m[MODE == MODE_SAMPLE ? m.lg : 0];
                 for (int kt = 0; kt < m.nkt; ++kt) {
                     if (!mbar_wait(&ms.kv_empty[ks_], kph ^ 1u, abort, a.status)) break;
@@ -368,57 +416,54 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                 // Drain: every issued TMA load lands before the CTA exits.
                 for (int i = 0; i < C::kKStages; ++i)
                     if (k_armed[i]) mbar_wait_drain(&ms.kv_full[i], k_armed_ph[i]);
-                for (int i = 0; i < C::kQStages; ++i)
-                    if (q_armed[i]) mbar_wait_drain(&ms.q_full[i], q_armed_ph[i]);
+                if (q_armed) mbar_wait_drain(&ms.q_full, q_armed_ph);
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            int ks_ = 0, qs = 0, ab = 0;
+            int ks_ = 0, ab = 0;
             uint32_t kph = 0, qph = 0, aph = 0;
-            bool issued = false;
-            for (int it = blockIdx.x; !*abort; it += gridDim.x) {
-                Item m;
-                if (a.planned) {
-                    if (it >= a.item_start[a.ntiles]) break;
-                    if (!get_item<MODE>(a, it, nlist, m)) continue;
-                } else {
-                    if (it >= a.static_chunks * ((a.nrows + kQTile - 1) / kQTile)) break;
-                    if (!get_item<MODE>(a, it, nlist, m)) continue;
-                }
-                if (!mbar_wait(&ms.q_full[qs], qph, abort, a.status)) break;
+            bool issued = false, ok = true;
+            Item m;
+            for (int it = blockIdx.x; ok && !*abort && next_item<MODE, RT>(a, it, nlist, m); it += gridDim.x) {
+                if (!mbar_wait(&ms.q_full, qph, abort, a.status)) break;
+                qph ^= 1u;
                 tc_fence_after();
-                const uint32_t qaddr = smem_u32(sq + qs * Lay::kQBytes);
-                bool ok = true;
-                for (int kt = 0; kt < m.nkt; ++kt) {
-                    if (!mbar_wait(&ms.acc_empty[ab], aph ^ 1u, abort, a.status) ||
-                        !mbar_wait(&ms.kv_full[ks_], kph, abort, a.status)) {
+                const uint32_t qaddr = smem_u32(sq);
+                for (int kt = 0; kt < m.nkt && ok; ++kt) {
+                    if (!mbar_wait(&ms.kv_full[ks_], kph, abort, a.status)) {
                         ok = false;
                         break;
                     }
-                    tc_fence_after();
                     const uint32_t kaddr = smem_u32(sk + ks_ * Lay::kKBytes);
-                    const uint32_t d = tmem + static_cast<uint32_t>(ab * 256);
 #pragma unroll
-                    for (int kk = 0; kk < C::kMmaK; ++kk) {
-                        const int at = kk / 4, off = (kk % 4) * 32;
-                        const uint64_t ad = smem_desc_sw128(kaddr + at * (Lay::kKBytes / C::kAtoms) + off);
-                        const uint64_t bd = smem_desc_sw128(qaddr + at * (Lay::kQBytes / C::kAtoms) + off);
-                        if (DT == FTK_F8E4M3)
-                            mma_f8f6f4(d, ad, bd, C::kIdesc, kk > 0 ? 1u : 0u);
-                        else
-                            mma_f16(d, ad, bd, C::kIdesc, kk > 0 ? 1u : 0u);
+                    for (int vt = 0; vt < QG; ++vt) {
+                        if (!mbar_wait(&ms.acc_empty[ab], aph ^ 1u, abort, a.status)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t d = tmem + static_cast<uint32_t>(ab * 256);
+                        const uint32_t baddr = qaddr + vt * Lay::kQTileBytes;
+#pragma unroll
+                        for (int kk = 0; kk < C::kMmaK; ++kk) {
+                            const int at = kk / 4, off = (kk % 4) * 32;
+                            const uint64_t ad = smem_desc_sw128(kaddr + at * (Lay::kKBytes / C::kAtoms) + off);
+                            const uint64_t bd = smem_desc_sw128(baddr + at * (Lay::kQTileBytes / C::kAtoms) + off);
+                            if (DT == FTK_F8E4M3)
+                                mma_f8f6f4(d, ad, bd, C::kIdesc, kk > 0 ? 1u : 0u);
+                            else
+                                mma_f16(d, ad, bd, C::kIdesc, kk > 0 ? 1u : 0u);
+                        }
+                        issued = true;
+                        mma_commit(&ms.acc_full[ab]);
+                        if (++ab == 2) { ab = 0; aph ^= 1u; }
                     }
-                    issued = true;
-                    mma_commit(&ms.kv_empty[ks_]);
-                    mma_commit(&ms.acc_full[ab]);
+                    mma_commit(&ms.kv_empty[ks_]);  // key tile free once its MMAs are done
                     if (++ks_ == C::kKStages) { ks_ = 0; kph ^= 1u; }
-                    if (++ab == 2) { ab = 0; aph ^= 1u; }
                 }
-                mma_commit(&ms.q_empty[qs]);
-                if (++qs == C::kQStages) { qs = 0; qph ^= 1u; }
-                if (!ok) break;
+                mma_commit(&ms.q_empty);
             }
             // Every issued MMA completes before TMEM is released.
             if (issued) {
@@ -428,39 +473,35 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        // Each epilogue warp works on its own: its 2 queries' parameters and
+        // Each epilogue warp works on its own: its queries' parameters and
         // weights, and its own candidate staging, so the tile loop has no
         // cross-warp synchronisation besides releasing the accumulator.
-        constexpr int NQ = kEpiQueries;
+        constexpr int NQ = kEpiQueries;          // queries per warp per query tile
+        constexpr int WQ = QG * NQ;              // queries per warp
         const int ew = warp - 2;                 // 0..15
         const int quad = warp & 3;               // TMEM lane quarter
-        const int qg = ew >> 2;                  // tile queries NQ*qg .. NQ*qg+NQ-1
+        const int qg = ew >> 2;                  // query pair within each query tile
         const int key_lane = quad * 32 + lane;   // row of the 128-key tile
         const uint32_t tlane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
         const uint32_t lt_mask = (1u << lane) - 1u;
-        float *my_w = sw + ew * NQ * kHeads;
-        float *my_sv = stage_val + ew * NQ * C::kWarpStage;
-        int32_t *my_si = stage_idx + ew * NQ * C::kWarpStage;
+        float *my_w = sw + ew * WQ * kHeads;
+        float *my_sv = stage_val + ew * WQ * C::kWarpStage;
+        int32_t *my_si = stage_idx + ew * WQ * C::kWarpStage;
         int ab = 0;
         uint32_t aph = 0;
         bool bad_scale = false;
-        for (int it = blockIdx.x; !*abort; it += gridDim.x) {
-            Item m;
-            if (a.planned) {
-                if (it >= a.item_start[a.ntiles]) break;
-                if (!get_item<MODE>(a, it, nlist, m)) continue;
-            } else {
-                if (it >= a.static_chunks * ((a.nrows + kQTile - 1) / kQTile)) break;
-                if (!get_item<MODE>(a, it, nlist, m)) continue;
-            }
-            // Per-item parameters of this warp's queries (warp-uniform).
-            int32_t qt[NQ], qks[NQ], qke[NQ], qpos[NQ];
-            float qtau[NQ];
+        Item m;
+        for (int it = blockIdx.x; !*abort && next_item<MODE, RT>(a, it, nlist, m); it += gridDim.x) {
+            // Per-item parameters of this warp's queries (warp-uniform).  Slot
+            // qq = vt * NQ + qi is query qg * NQ + qi of query tile vt.
+            int32_t qt[WQ], qpos[WQ], wlo[WQ], wlen[WQ];
+            float qtau[WQ];
             {
-                const int64_t p = static_cast<int64_t>(m.tile) * kQTile + qg * NQ + (lane % NQ);
+                const int sl = lane % WQ;
+                const int64_t p = static_cast<int64_t>(m.tile) * RT + (sl / NQ) * kQTile + qg * NQ + (sl % NQ);
                 int32_t t_l = -1, ks_l = 0, ke_l = 0;
                 float tau_l = 0.f;
-                if (lane < NQ) {
+                if (lane < WQ) {
                     t_l = list_query(a, p, nlist);
                     if (t_l >= 0) {
                         ks_l = a.ks[t_l];
@@ -469,29 +510,24 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                     }
                 }
 #pragma unroll
-                for (int qi = 0; qi < NQ; ++qi) {
-                    qt[qi] = __shfl_sync(0xFFFFFFFFu, t_l, qi);
-                    qks[qi] = __shfl_sync(0xFFFFFFFFu, ks_l, qi);
-                    qke[qi] = __shfl_sync(0xFFFFFFFFu, ke_l, qi);
-                    qtau[qi] = __shfl_sync(0xFFFFFFFFu, tau_l, qi);
-                    qpos[qi] = m.tile * kQTile + qg * NQ + qi;
-                    my_w[qi * kHeads + lane] =
-                        qt[qi] >= 0 ? a.weights[static_cast<int64_t>(qt[qi]) * kHeads + lane] : 0.f;
+                for (int qq = 0; qq < WQ; ++qq) {
+                    qt[qq] = __shfl_sync(0xFFFFFFFFu, t_l, qq);
+                    wlo[qq] = __shfl_sync(0xFFFFFFFFu, ks_l, qq);
+                    wlen[qq] = __shfl_sync(0xFFFFFFFFu, ke_l, qq) - wlo[qq];
+                    qtau[qq] = __shfl_sync(0xFFFFFFFFu, tau_l, qq);
+                    qpos[qq] = m.tile * RT + (qq / NQ) * kQTile + qg * NQ + (qq % NQ);
+                    my_w[qq * kHeads + lane] =
+                        qt[qq] >= 0 ? stored_weight(a.weights[static_cast<int64_t>(qt[qq]) * kHeads + lane], lane)
+                                    : 0.f;
                 }
                 __syncwarp();
             }
-            int cnt[NQ];  // staged candidates per query (warp-uniform)
+            int cnt[WQ];  // staged candidates per query (warp-uniform)
 #pragma unroll
-            for (int qi = 0; qi < NQ; ++qi) cnt[qi] = 0;
+            for (int qq = 0; qq < WQ; ++qq) cnt[qq] = 0;
             // Keys are int32 (S < 2^31).  A query outside the list has the
             // empty window [0, 0).  In SAMPLE mode key j of the tile is
             // sample j, at kv row j << lg.
-            int32_t wlo[NQ], wlen[NQ];
-#pragma unroll
-            for (int qi = 0; qi < NQ; ++qi) {
-                wlo[qi] = qt[qi] >= 0 ? qks[qi] : 0;
-                wlen[qi] = qt[qi] >= 0 ? qke[qi] - qks[qi] : 0;
-            }
             const float *scales = a.kv_scales;
             int32_t kidx_next = m.key0 + key_lane;
             float sig_next = 1.f;
@@ -500,7 +536,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                 if (kidx_next < m.kend && s0 < a.S) sig_next = __ldg(scales + s0);
             }
             bool ok = true;
-            for (int kt = 0; kt < m.nkt; ++kt) {
+            for (int kt = 0; kt < m.nkt && ok; ++kt) {
                 const int32_t kidx = kidx_next;
                 const float sigma = sig_next;
                 kidx_next += kKeyTile;
@@ -510,90 +546,97 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                 }
                 bad_scale |= scales && kidx < m.kend && (!(sigma > 0.f) || isinf(sigma));
                 const int32_t s = MODE == MODE_SAMPLE ? (kidx << m.lg) : kidx;
-                const bool got = mbar_wait(&ms.acc_full[ab], aph, abort, a.status);
-                if (!__all_sync(0xFFFFFFFFu, got)) {  // also reconverges the warp
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const uint32_t c0 = tlane + static_cast<uint32_t>(ab * 256 + qg * NQ * 32);
-                uint64_t p01 = 0, p23 = 0, q01 = 0, q23 = 0;
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    float xa[16], xb[16];
-                    tmem_ld16x2(c0 + hh * 16, c0 + 32 + hh * 16, xa, xb);
-                    if (hh == 1) {
-                        // Every column of this tile is in registers: hand the
-                        // accumulator back to the MMA warp.
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&ms.acc_empty[ab]);
+                for (int vt = 0; vt < QG; ++vt) {
+                    const bool got = mbar_wait(&ms.acc_full[ab], aph, abort, a.status);
+                    if (!__all_sync(0xFFFFFFFFu, got)) {  // also reconverges the warp
+                        ok = false;
+                        break;
                     }
-                    head_step2(xa, xb, my_w, my_w + kHeads, hh * 16, p01, p23, q01, q23);
-                }
-                if (++ab == 2) { ab = 0; aph ^= 1u; }
-                float I[NQ];
-                I[0] = head_finish(p01, p23, sigma);
-                I[1] = head_finish(q01, q23, sigma);
+                    tc_fence_after();
+                    const uint32_t c0 = tlane + static_cast<uint32_t>(ab * 256 + qg * NQ * 32);
+                    const float *w0 = my_w + (vt * NQ) * kHeads;
+                    uint64_t p01 = 0, p23 = 0, q01 = 0, q23 = 0;
 #pragma unroll
-                for (int qi = 0; qi < NQ; ++qi) {
-                    // s in [wlo, wlo + wlen) as one unsigned compare
-                    const bool valid = static_cast<uint32_t>(s - wlo[qi]) < static_cast<uint32_t>(wlen[qi]);
-                    if (MODE == MODE_COLLECT) {
-                        const bool take = valid && !(I[qi] < qtau[qi]);  // NaN is kept, to be seen
-                        const uint32_t bal = __ballot_sync(0xFFFFFFFFu, take);
-                        const int pos = cnt[qi] + __popc(bal & lt_mask);
-                        if (take) {
-                            my_sv[qi * C::kWarpStage + pos] = I[qi];
-                            my_si[qi * C::kWarpStage + pos] = s;
+                    for (int hh = 0; hh < 2; ++hh) {
+                        float xa[16], xb[16];
+                        tmem_ld16x2(c0 + hh * 16, c0 + 32 + hh * 16, xa, xb);
+                        if (hh == 1) {
+                            // Every column of this tile is in registers: hand the
+                            // accumulator back to the MMA warp.
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&ms.acc_empty[ab]);
                         }
-                        cnt[qi] += __popc(bal);
-                    } else if (MODE == MODE_SAMPLE) {
-                        if (qt[qi] >= 0 && kidx < m.kend)
-                            a.out[static_cast<int64_t>(qt[qi]) * a.ld + (kidx - m.key0)] =
-                                valid ? I[qi] : -INFINITY;
-                    } else {
-                        if (valid) a.out[static_cast<int64_t>(qpos[qi]) * a.ld + (s - wlo[qi])] = I[qi];
+                        head_step2(xa, xb, w0, w0 + kHeads, hh * 16, p01, p23, q01, q23);
+                    }
+                    if (++ab == 2) { ab = 0; aph ^= 1u; }
+                    float I[NQ];
+                    I[0] = head_finish(p01, p23, sigma);
+                    I[1] = head_finish(q01, q23, sigma);
+#pragma unroll
+                    for (int qi = 0; qi < NQ; ++qi) {
+                        const int qq = vt * NQ + qi;
+                        // s in [wlo, wlo + wlen) as one unsigned compare
+                        const bool valid = static_cast<uint32_t>(s - wlo[qq]) < static_cast<uint32_t>(wlen[qq]);
+                        if (MODE == MODE_COLLECT) {
+                            const bool take = valid && !(I[qi] < qtau[qq]);  // NaN is kept, to be seen
+                            const uint32_t bal = __ballot_sync(0xFFFFFFFFu, take);
+                            if (bal) {
+                                const int pos = cnt[qq] + __popc(bal & lt_mask);
+                                if (take) {
+                                    my_sv[qq * C::kWarpStage + pos] = I[qi];
+                                    my_si[qq * C::kWarpStage + pos] = s;
+                                }
+                                cnt[qq] += __popc(bal);
+                            }
+                        } else if (MODE == MODE_SAMPLE) {
+                            if (qt[qq] >= 0 && kidx < m.kend)
+                                a.out[static_cast<int64_t>(qt[qq]) * a.ld + (kidx - m.key0)] =
+                                    valid ? I[qi] : -INFINITY;
+                        } else {
+                            if (valid) a.out[static_cast<int64_t>(qpos[qq]) * a.ld + (s - wlo[qq])] = I[qi];
+                        }
                     }
                 }
-                if (MODE == MODE_COLLECT) {
-                    // Every 4 tiles (<= 4 * 32 new entries per warp and query)
-                    // and at the item's end, flush the queries whose staging
-                    // could otherwise overflow.
+                if (MODE == MODE_COLLECT && ok) {
+                    // Every 2 key tiles (<= 2 * 32 new entries per warp and
+                    // query) and at the item's end, flush the queries whose
+                    // staging could otherwise overflow.
                     const bool last = kt == m.nkt - 1;
-                    if (last || (kt & 3) == 3) {
-                        bool need[NQ], any = false;
+                    if (last || (kt & 1) == 1) {
+                        bool need[WQ], any = false;
 #pragma unroll
-                        for (int qi = 0; qi < NQ; ++qi) {
-                            need[qi] = cnt[qi] > 0 && (last || cnt[qi] > C::kWarpStage - 4 * 32);
-                            any |= need[qi];
+                        for (int qq = 0; qq < WQ; ++qq) {
+                            need[qq] = cnt[qq] > 0 && (last || cnt[qq] > C::kWarpStage - 2 * 32);
+                            any |= need[qq];
                         }
                         if (any) {
                             __syncwarp();  // staged entries visible to every lane
-                            int base[NQ];
+                            int base[WQ];
 #pragma unroll
-                            for (int qi = 0; qi < NQ; ++qi) base[qi] = 0;
+                            for (int qq = 0; qq < WQ; ++qq) base[qq] = 0;
                             if (lane == 0) {
 #pragma unroll
-                                for (int qi = 0; qi < NQ; ++qi)  // independent atomics, latencies overlap
-                                    if (need[qi] && qt[qi] >= 0) base[qi] = atomicAdd(a.cnt + qt[qi], cnt[qi]);
+                                for (int qq = 0; qq < WQ; ++qq)  // independent atomics, latencies overlap
+                                    if (need[qq] && qt[qq] >= 0) base[qq] = atomicAdd(a.cnt + qt[qq], cnt[qq]);
                             }
 #pragma unroll
-                            for (int qi = 0; qi < NQ; ++qi) {
-                                if (!need[qi]) continue;
-                                const int b = __shfl_sync(0xFFFFFFFFu, base[qi], 0);
-                                if (qt[qi] >= 0) {
-                                    float *cv = a.cand_val + static_cast<int64_t>(qt[qi]) * a.cap;
-                                    int32_t *ci = a.cand_idx + static_cast<int64_t>(qt[qi]) * a.cap;
-                                    for (int i = lane; i < cnt[qi]; i += 32) {
+                            for (int qq = 0; qq < WQ; ++qq) {
+                                if (!need[qq]) continue;
+                                const int b = __shfl_sync(0xFFFFFFFFu, base[qq], 0);
+                                if (qt[qq] >= 0) {
+                                    float *cv = a.cand_val + static_cast<int64_t>(qt[qq]) * a.cap;
+                                    int32_t *ci = a.cand_idx + static_cast<int64_t>(qt[qq]) * a.cap;
+                                    for (int i = lane; i < cnt[qq]; i += 32) {
                                         const int slot = b + i;
                                         if (slot < a.cap) {
-                                            cv[slot] = my_sv[qi * C::kWarpStage + i];
-                                            ci[slot] = my_si[qi * C::kWarpStage + i];
+                                            cv[slot] = my_sv[qq * C::kWarpStage + i];
+                                            ci[slot] = my_si[qq * C::kWarpStage + i];
                                         }
                                     }
                                 }
-                                cnt[qi] = 0;
+                                cnt[qq] = 0;
                             }
                             __syncwarp();
                         }

@@ -33,6 +33,7 @@ namespace ftk {
 constexpr int kPlanThreads = 1024;
 constexpr int kSelThreads = 256;
 constexpr int kBitmapWords = 2048;   // 65536-key segments for the ordered output
+constexpr int kMaxRowTile = 16;      // largest row_tile_of(dtype)
 
 // Device copy of ftk_info plus counters (same layout for the leading part).
 struct DevInfo {
@@ -47,6 +48,7 @@ struct PlanArgs {
     int64_t T, S;
     const int32_t *ks, *ke;
     int32_t ntiles;
+    int32_t rt;               // rows per tile
     int32_t sample_keys;
     // sample pass
     int32_t *s_lo, *s_hi, *s_lg, *s_start;
@@ -110,8 +112,8 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanArgs p)
         uint32_t ns = 0, nc = 0;
         if (tile < p.ntiles) {
             int64_t lo = INT64_MAX, hi = -1;
-            for (int j = 0; j < kQTile; ++j) {
-                const int64_t t = static_cast<int64_t>(tile) * kQTile + j;
+            for (int j = 0; j < p.rt; ++j) {
+                const int64_t t = static_cast<int64_t>(tile) * p.rt + j;
                 if (t >= p.T) break;
                 const int64_t a = p.ks[t], b = p.ke[t];
                 if (!window_ok(a, b, p.S) || a == b) continue;
@@ -248,6 +250,7 @@ struct ThreshArgs {
     float *tau;
     int32_t cap;
     int32_t topk;
+    int32_t rt;
     float oversample;
 };
 
@@ -262,7 +265,7 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const ThreshArgs
         if (threadIdx.x == 0) p.tau[t] = -INFINITY;
         return;
     }
-    const int tile = static_cast<int>(t / kQTile);
+    const int tile = static_cast<int>(t / p.rt);
     const int lg = p.s_lg[tile];
     const int64_t st = int64_t(1) << lg;
     const int J = p.s_hi[tile] - p.s_lo[tile];
@@ -509,11 +512,11 @@ static SelectCfg resolve_cfg(int64_t T, int64_t S, int topk, const ftk_config *c
         // At most 2^27 floats (512 MB) of recovery scratch, at least 64 rows;
         // non-increasing in S so that a larger plan serves smaller calls.
         const int64_t ld = (S + 7) / 8 * 8;
-        rr = ((int64_t(1) << 27) / ld) & ~static_cast<int64_t>(kQTile - 1);
+        rr = ((int64_t(1) << 27) / ld) & ~static_cast<int64_t>(kMaxRowTile - 1);
         if (rr < 64) rr = 64;
     }
-    rr = (rr + kQTile - 1) / kQTile * kQTile;
-    const int64_t tcap = (T + kQTile - 1) / kQTile * kQTile;
+    rr = (rr + kMaxRowTile - 1) / kMaxRowTile * kMaxRowTile;
+    const int64_t tcap = (T + kMaxRowTile - 1) / kMaxRowTile * kMaxRowTile;
     if (rr > tcap) rr = tcap;
     r.rec_rows = static_cast<int>(rr);
     return r;
@@ -682,7 +685,8 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
     KvMaps kvm;
     if (!build_maps(dtype, q, kv, T, S, max_lg, &tq, &kvm)) return FTK_ERR_CUDA;
 
-    const int32_t ntiles = static_cast<int32_t>((T + kQTile - 1) / kQTile);
+    const int rt = row_tile_of(dtype);
+    const int32_t ntiles = static_cast<int32_t>((T + rt - 1) / rt);
     const int sms = num_sms();
     uint32_t *status = &w.info->info.status;
 
@@ -693,6 +697,7 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
     pa.ks = ks;
     pa.ke = ke;
     pa.ntiles = ntiles;
+    pa.rt = rt;
     pa.sample_keys = c.m;
     pa.s_lo = w.s_lo;
     pa.s_hi = w.s_hi;
@@ -745,6 +750,7 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
     ta.tau = w.tau;
     ta.cap = c.cap;
     ta.topk = topk;
+    ta.rt = rt;
     ta.oversample = c.beta;
     {
         const size_t smem = static_cast<size_t>(w.sld) * 4;
@@ -819,7 +825,7 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
         da.out = w.scratch;
         da.ld = w.scratch_ld;
         da.status = status;
-        const int64_t items = static_cast<int64_t>(chunks) * (c.rec_rows / kQTile);
+        const int64_t items = static_cast<int64_t>(chunks) * ((c.rec_rows + rt - 1) / rt);
         st = launch_score_dt<MODE_DUMP>(dtype, da, tq, kvm,
                                         static_cast<int>(items < sms ? items : sms), s);
         if (st != FTK_OK) return st;
@@ -885,7 +891,8 @@ extern "C" ftk_status ftk_score_dense(ftk_dtype dtype, const void *q, const void
     cudaStream_t s = as_stream(stream);
     cudaError_t e = cudaMemsetAsync(workspace, 0, 4, s);
     if (e != cudaSuccess) return cuda_status(e);
-    const int64_t items = static_cast<int64_t>(da.static_chunks) * ((nrows + kQTile - 1) / kQTile);
+    const int rt = row_tile_of(dtype);
+    const int64_t items = static_cast<int64_t>(da.static_chunks) * ((nrows + rt - 1) / rt);
     const int sms = num_sms();
     return launch_score_dt<MODE_DUMP>(dtype, da, tq, kvm,
                                       static_cast<int>(items < sms ? items : sms), s);

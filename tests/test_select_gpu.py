@@ -208,3 +208,13 @@ def test_full_size_workloads(name, nrows, nfp64):
     assert worst < 1e-4
     assert min(overlaps) >= 0.99
     print(f"{name}: worst |dI|/E {worst:.2e}, info {info}")
+
+
+def test_nan_key_is_flagged():
+    """A NaN in kv makes the dot products NaN; ReLU propagates it and the
+    status reports it (the row's result is unspecified, nothing traps)."""
+    c = wl.small_case(seed=16, dtype="fp8", T=8, S=3000, topk=32, windows="causal")
+    c.kv.view(torch.uint8)[1234, 7] = 0x7F  # e4m3fn NaN
+    g = gpu_inputs(c)
+    _, _, info = run_select(g)
+    assert info["status"] & ftk.STATUS_NAN
