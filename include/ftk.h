@@ -203,6 +203,36 @@ ftk_status ftk_windows_from_cu_seqlens(const int32_t *cu_q,
                                        int64_t T, int32_t *ks, int32_t *ke,
                                        void *stream);
 
+/*
+ * ftk_select_noalloc -- ftk_select without a caller-supplied workspace, for
+ * callers that cannot allocate device memory (code inside another
+ * allocator's arena or under a memory cap, code that must not fail with an
+ * out-of-memory error at call time, plain C hosts with no allocator).  It
+ * allocates nothing: its scratch is a fixed __device__ array of
+ * FTK_NOALLOC_SCRATCH_BYTES inside the library, held by every GPU that
+ * loads the library until the process exits.  The pages describe no such
+ * call; it has no counterpart there.
+ *
+ * Arguments and results are those of ftk_select (same kernels, same bits),
+ * minus the workspace.  If config->recovery_rows is 0 (or config is NULL),
+ * the recovery batch is the largest that fits the array.
+ * Returns FTK_ERR_WORKSPACE when the problem needs more scratch than
+ * FTK_NOALLOC_SCRATCH_BYTES (smaller T, S or topk fit).
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * All calls share the one array and leave their state in it (each call
+ * clears what it needs): calls that overlap on the same GPU, for example
+ * on two streams, race on it, so serialise them.  There is no
+ * ftk_read_info for this entry point.
+ */
+#define FTK_NOALLOC_SCRATCH_BYTES (64u << 20)
+ftk_status ftk_select_noalloc(ftk_dtype dtype, const void *q, const void *kv,
+                              const float *kv_scales, const float *weights,
+                              const int32_t *ks, const int32_t *ke, int64_t T,
+                              int64_t S, int topk, int32_t *out_idx,
+                              float *out_val, const ftk_config *config,
+                              void *stream);
+
 /* Diagnostic timing hook.  While set, every ftk_select call made from the
  * calling host thread records events[i] (cudaEvent_t values created by the
  * caller, passed as void *) on the call's stream at its stage boundaries:

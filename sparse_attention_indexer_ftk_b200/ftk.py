@@ -38,7 +38,7 @@ HEADS, DIM, MAX_TOPK = 32, 128, 4096
 EXPORTS = (
     "ftk_select", "ftk_select_workspace_size", "ftk_read_info", "ftk_topk_rows",
     "ftk_score_dense", "ftk_score_dense_workspace_size", "ftk_windows_from_cu_seqlens",
-    "ftk_set_stage_events", "ftk_status_string", "ftk_version",
+    "ftk_set_stage_events", "ftk_status_string", "ftk_version", "ftk_select_noalloc",
 )
 
 
@@ -86,6 +86,8 @@ def load_library(path: str = LIB_PATH):
     L.ftk_score_dense_workspace_size.argtypes = [I64]
     L.ftk_windows_from_cu_seqlens.restype = I32
     L.ftk_windows_from_cu_seqlens.argtypes = [P, P, I64, I64, P, P, P]
+    L.ftk_select_noalloc.restype = I32
+    L.ftk_select_noalloc.argtypes = [I32, P, P, P, P, P, P, I64, I64, I32, P, P, P, P]
     L.ftk_set_stage_events.restype = I32
     L.ftk_set_stage_events.argtypes = [P, I32]
     L.ftk_status_string.restype = ctypes.c_char_p
