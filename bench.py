@@ -46,6 +46,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-rows", action="store_true", help="skip the row top-k section")
+    ap.add_argument("--only-rows", action="store_true", help="run only the row top-k section")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--rows", type=int, default=0,
                     help="use only the first ROWS queries of the batch (profiling captures)")
@@ -225,6 +227,45 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
+def bench_rows(name: str, dev, reps: int = 64):
+    """Row top-k (ftk_topk_rows) on a row workload, HBM-bound.  Rotates over
+    enough input copies that each launch reads data not in the L2."""
+    import torch
+    from sparse_attention_indexer_ftk_b200 import ftk
+    from sparse_attention_indexer_ftk_b200 import workloads as wl
+
+    c = wl.get(name)
+    x = c.x.to(dev)
+    rows, cols = x.shape
+    esz = x.element_size()
+    in_bytes = rows * cols * esz
+    out_bytes = rows * c.topk * (4 + esz)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    ncopy = max(2, -(-3 * l2 // in_bytes))
+    xs = [x.clone() for _ in range(ncopy)]
+    oi = torch.empty((rows, c.topk), dtype=torch.int32, device=dev)
+    ov = torch.empty((rows, c.topk), dtype=x.dtype, device=dev)
+    for i in range(3):
+        ftk.topk_rows(xs[i % ncopy], c.topk, out_idx=oi, out_val=ov)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for i in range(reps):
+        evs[i][0].record()
+        ftk.topk_rows(xs[i % ncopy], c.topk, out_idx=oi, out_val=ov)
+        evs[i][1].record()
+    torch.cuda.synchronize()
+    ms = sorted(a.elapsed_time(b) for a, b in evs)
+    mean = sum(ms) / reps
+    peaks, src = measured_peaks()
+    gbs = (in_bytes + out_bytes) / (mean * 1e-3) / 1e9
+    return {"workload": name, "rows": rows, "cols": cols, "topk": c.topk, "dtype": str(x.dtype),
+            "us_per_call": mean * 1e3, "us_min": ms[0] * 1e3, "rows_per_s": rows / (mean * 1e-3),
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "bytes_per_call": in_bytes + out_bytes,
+                         "peak_source": src},
+            "inputs": f"{ncopy} rotating copies (> L2) so every call reads from HBM"}
+
+
 def run_ours(args):
     import torch
 
@@ -363,6 +404,8 @@ def run_ours(args):
         "gpu_launches": int(info["kernel_launches"]) * K,
         "clocks": clocks,
     }
+    if world == 1 and not args.no_rows:
+        out["row_topk"] = [bench_rows("rows_bf16", dev), bench_rows("rows_f32", dev)]
     if world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(c, args.cpu_seconds)
     print(json.dumps(out), flush=True)
@@ -372,6 +415,11 @@ def run_ours(args):
 
 def main():
     args = parse_args()
+    if args.only_rows:
+        import torch
+        print(json.dumps({"row_topk": [bench_rows("rows_bf16", torch.device("cuda")),
+                                       bench_rows("rows_f32", torch.device("cuda"))]}), flush=True)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

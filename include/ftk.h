@@ -151,7 +151,7 @@ ftk_status ftk_read_info(const void *workspace, ftk_info *out, void *stream);
  *               x + r * row_stride elements; x and row_stride * elem_size
  *               must be 16-byte aligned (DeepSelect README, "Usage": the row
  *               stride alignment requirement)
- *   rows        >= 1;  cols: 1 .. 393216
+ *   rows        >= 1;  cols: 1 .. 2^30
  *   topk        1 .. FTK_MAX_TOPK; rows with cols < topk are padded with
  *               index -1 and value -inf
  *   out_idx     device [rows, topk] int32

@@ -52,6 +52,6 @@ struct RowsArgs;
 // with one cluster of `cluster` CTAs per grid row.
 ftk_status launch_rows_topk(int dtype, const RowsArgs &a, int cluster, cudaStream_t stream);
 // Cluster size and per-CTA chunk for rows of `cols` columns.
-void rows_plan(int64_t rows, int64_t cols, int *cluster, int *chunk);
+void rows_plan(int64_t rows, int64_t cols, int k, int *cluster, int *chunk);
 
 }  // namespace ftk

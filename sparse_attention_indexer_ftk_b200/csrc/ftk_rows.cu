@@ -29,12 +29,13 @@ static int env_int(const char *name, int dflt)
     return v && *v ? atoi(v) : dflt;
 }
 
-void rows_plan(int64_t rows, int64_t cols, int *cluster, int *chunk)
+void rows_plan(int64_t rows, int64_t cols, int k, int *cluster, int *chunk)
 {
-    // Enough CTAs to keep every SM streaming (two per SM), and a chunk that
-    // fits the shared-memory budget.
+    // At least one CTA per SM (148), and few enough expected candidates per
+    // warp (~4 * k over the row) to stay well inside a warp's candidate list.
     int cs = 1;
-    while (cs < kRowsMaxCluster && (rows * cs < 2 * 148 || (cols + cs - 1) / cs > kRowsMaxChunk))
+    while (cs < kRowsMaxCluster &&
+           (rows * cs < 148 || 4 * static_cast<int64_t>(k) > static_cast<int64_t>(cs) * kRowsWarps * (kRowsCapWarp / 2)))
         cs *= 2;
     const int forced = env_int("FTK_ROWS_CLUSTER", 0);
     if (forced == 1 || forced == 2 || forced == 4 || forced == 8) cs = forced;
@@ -47,7 +48,7 @@ void rows_plan(int64_t rows, int64_t cols, int *cluster, int *chunk)
 template <int DT>
 static ftk_status launch_rows_dt(const RowsArgs &a, int cluster, cudaStream_t stream)
 {
-    const size_t smem = sizeof(RowsSmem) + static_cast<size_t>(a.chunk) * 2;
+    const size_t smem = sizeof(RowsSmem);
     auto kern = rows_topk_kernel<DT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
@@ -69,7 +70,7 @@ static ftk_status launch_rows_dt(const RowsArgs &a, int cluster, cudaStream_t st
 
 ftk_status launch_rows_topk(int dtype, const RowsArgs &a, int cluster, cudaStream_t stream)
 {
-    if (a.chunk <= 0 || a.chunk > kRowsMaxChunk || a.chunk % 8) return FTK_ERR_UNSUPPORTED;
+    if (a.chunk <= 0 || a.chunk % 8) return FTK_ERR_UNSUPPORTED;
     if (dtype == FTK_BF16) return launch_rows_dt<FTK_BF16>(a, cluster, stream);
     if (dtype == FTK_F32) return launch_rows_dt<FTK_F32>(a, cluster, stream);
     return FTK_ERR_UNSUPPORTED;
@@ -88,7 +89,7 @@ extern "C" ftk_status ftk_topk_rows(ftk_dtype dtype, const void *x, int64_t rows
     if (rows < 1 || cols < 1 || row_stride < cols || rows > (int64_t(1) << 31) / kRowsMaxCluster)
         return FTK_ERR_INVALID_ARG;
     if (topk < 1 || topk > FTK_MAX_TOPK) return FTK_ERR_TOPK_RANGE;
-    if (cols > static_cast<int64_t>(kRowsMaxCluster) * kRowsMaxChunk) return FTK_ERR_UNSUPPORTED;
+    if (cols > kRowsMaxCols) return FTK_ERR_UNSUPPORTED;
     const int esz = dtype == FTK_BF16 ? 2 : 4;
     if (!aligned16(x) || (row_stride * esz) % 16) return FTK_ERR_ALIGNMENT;
     ftk_status st = check_device();
@@ -103,7 +104,7 @@ extern "C" ftk_status ftk_topk_rows(ftk_dtype dtype, const void *x, int64_t rows
     a.k = topk;
     a.status = status;
     int cluster = 1, chunk = 8;
-    rows_plan(rows, cols, &cluster, &chunk);
+    rows_plan(rows, cols, topk, &cluster, &chunk);
     a.chunk = chunk;
     return launch_rows_topk(dtype, a, cluster, as_stream(stream));
 }

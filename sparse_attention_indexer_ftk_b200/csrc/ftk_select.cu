@@ -806,7 +806,7 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
 
     // dense recovery of the listed rows, rec_rows at a time
     int rcluster = 1, rchunk = 8;
-    rows_plan(c.rec_rows, S, &rcluster, &rchunk);
+    rows_plan(c.rec_rows, S, topk, &rcluster, &rchunk);
     const int32_t chunks = static_cast<int32_t>((S + kKeyTile - 1 + kChunkKeys - 1) / kChunkKeys);
     for (int64_t b0 = 0; b0 < T; b0 += c.rec_rows) {
         ScoreArgs da = {};

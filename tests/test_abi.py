@@ -75,7 +75,7 @@ def test_topk_rows_host_validation(lib):
     assert lib.ftk_topk_rows(2, P(A + 2), 4, 100, 104, 8, P(A), None, None, None) == -4
     assert lib.ftk_topk_rows(2, P(A), 4, 100, 101, 8, P(A), None, None, None) == -4
     assert lib.ftk_topk_rows(3, P(A), 4, 100, 99, 8, P(A), None, None, None) == -1
-    assert lib.ftk_topk_rows(3, P(A), 4, 10 ** 7, 10 ** 7, 8, P(A), None, None, None) == -2
+    assert lib.ftk_topk_rows(3, P(A), 4, 1 << 31, 1 << 31, 8, P(A), None, None, None) == -2
 
 
 def test_select_host_validation(lib):
