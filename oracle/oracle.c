@@ -25,7 +25,7 @@
  *             short rows padded with fill values.
  *   [DS-NAN]  DeepSelect README, "NaN handling".
  *
- * Readings where the pages are silent (each also listed in the design doc):
+ * Readings where the pages are silent:
  *   - padding of a window shorter than topk: index -1, value -inf;
  *   - -0.0 and +0.0 are the same score (compared by value);
  *   - a NaN anywhere in a row's scores makes that row's result unspecified
@@ -176,6 +176,81 @@ int64_t orc_index_scores(int dtype, const void *q, const void *kv,
         }
     }
     return bad;
+}
+
+/* ---------------------------------------------------------------------- */
+/* Score bound of a key block  [FTK-HL]                                     */
+/* ---------------------------------------------------------------------- */
+
+/*
+ * Upper bound on the score of row t over a block of keys [FTK-HL: adaptive
+ * key pruning skips keys by a score bound.  The pages give the bound no
+ * formula; this is the plain per-dimension box bound].
+ * For the keys s of block b, i.e. [b*block, min((b+1)*block, S)):
+ *   hi[d] = max_s sigma_s * k[s,d],  lo[d] = min_s sigma_s * k[s,d]
+ *   U_h = sum_d max(q[t,h,d] * hi[d], q[t,h,d] * lo[d])   (>= q_h . sigma_s k_s)
+ *   L_h = sum_d min(q[t,h,d] * hi[d], q[t,h,d] * lo[d])   (<= q_h . sigma_s k_s)
+ *   UB  = sum_h (w[t,h] >= 0 ? w[t,h] * ReLU(U_h) : w[t,h] * ReLU(L_h))
+ * For sigma_s > 0, sigma_s * sum_h w_h ReLU(x_h) = sum_h w_h ReLU(sigma_s x_h),
+ * so UB >= I[t,s] for every key of the block.
+ *   out_ub    [nrows, nblocks]: UB of (rows[r], b)
+ *   out_scale [nrows, nblocks] or NULL: sum_h |w| sum_d |q| max(|hi|, |lo|),
+ *             the size of the terms UB is summed from
+ */
+void orc_block_bound(int dtype, const void *q, const void *kv, const float *kv_scales,
+                     const float *weights, int64_t T, int64_t S, int64_t block,
+                     const int64_t *rows, int64_t nrows, double *out_ub, double *out_scale)
+{
+    int64_t nb = (S + block - 1) / block;
+    double *hi = malloc(sizeof(double) * nb * ORC_DIM);
+    double *lo = malloc(sizeof(double) * nb * ORC_DIM);
+    for (int64_t b = 0; b < nb; ++b) {
+        for (int d = 0; d < ORC_DIM; ++d) {
+            hi[b * ORC_DIM + d] = -INFINITY;
+            lo[b * ORC_DIM + d] = INFINITY;
+        }
+        for (int64_t s = b * block; s < S && s < (b + 1) * block; ++s) {
+            double sigma = kv_scales ? (double)kv_scales[s] : 1.0;
+            for (int d = 0; d < ORC_DIM; ++d) {
+                double v = sigma * element(dtype, kv, s * ORC_DIM + d);
+                if (v > hi[b * ORC_DIM + d]) hi[b * ORC_DIM + d] = v;
+                if (v < lo[b * ORC_DIM + d]) lo[b * ORC_DIM + d] = v;
+            }
+        }
+    }
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < nrows; ++r) {
+        int64_t t = rows[r];
+        double qd[ORC_HEADS * ORC_DIM], wt[ORC_HEADS];
+        for (int i = 0; i < ORC_HEADS * ORC_DIM; ++i)
+            qd[i] = element(dtype, q, t * ORC_HEADS * ORC_DIM + i);
+        for (int h = 0; h < ORC_HEADS; ++h)
+            wt[h] = weights[(int64_t)t * ORC_HEADS + h];
+        for (int64_t b = 0; b < nb; ++b) {
+            const double *bh = hi + b * ORC_DIM, *bl = lo + b * ORC_DIM;
+            double ub = 0.0, scale = 0.0;
+            for (int h = 0; h < ORC_HEADS; ++h) {
+                double U = 0.0, L = 0.0, mag = 0.0;
+                for (int d = 0; d < ORC_DIM; ++d) {
+                    double x = qd[h * ORC_DIM + d] * bh[d];
+                    double y = qd[h * ORC_DIM + d] * bl[d];
+                    U += x > y ? x : y;
+                    L += x < y ? x : y;
+                    mag += fabs(qd[h * ORC_DIM + d]) * (fabs(bh[d]) > fabs(bl[d]) ? fabs(bh[d]) : fabs(bl[d]));
+                }
+                if (wt[h] >= 0.0)
+                    ub += wt[h] * (U > 0.0 ? U : 0.0);
+                else
+                    ub += wt[h] * (L > 0.0 ? L : 0.0);
+                scale += fabs(wt[h]) * mag;
+            }
+            out_ub[r * nb + b] = ub;
+            if (out_scale)
+                out_scale[r * nb + b] = scale;
+        }
+    }
+    free(hi);
+    free(lo);
 }
 
 /* ---------------------------------------------------------------------- */

@@ -65,6 +65,8 @@ def load(path: str):
     L.orc_topk_rows.restype = I64
     L.orc_topk_rows.argtypes = [I32, P, I64, I64, I64, I32, P, P, P]
     L.orc_num_threads.restype = I32
+    L.orc_block_bound.argtypes = [I32, P, P, P, P, I64, I64, I64, P, I64, P, P]
+    L.orc_block_bound.restype = None
     L.orc_num_threads.argtypes = []
     return L
 
@@ -172,6 +174,25 @@ def index_scores(q, kv, kv_scales, weights, ks, ke, rows=None, ld=None):
     lib().orc_index_scores(dtype_code(q), _ptr(qr), _ptr(kr), _ptr(sc), _ptr(w), T, S,
                            _ptr(ks_), _ptr(ke_), _ptr(rows), rows.size, ld, _ptr(I), _ptr(E))
     return I, E
+
+
+def block_bound(q, kv, kv_scales, weights, block: int = 128, rows=None):
+    """Score upper bound of every listed row over every key block of `block`
+    keys (the box bound of orc_block_bound).
+
+    Returns (UB, scale), each [len(rows), ceil(S / block)] float64.
+    """
+    T, S = q.shape[0], kv.shape[0]
+    qr, kr = _raw(q), _raw(kv)
+    sc = None if kv_scales is None else np.ascontiguousarray(_raw(kv_scales), dtype=np.float32)
+    w = np.ascontiguousarray(_raw(weights), dtype=np.float32)
+    rows = _rows_arg(rows, T)
+    nb = (S + block - 1) // block
+    ub = np.empty((rows.size, nb))
+    scale = np.empty((rows.size, nb))
+    lib().orc_block_bound(dtype_code(q), _ptr(qr), _ptr(kr), _ptr(sc), _ptr(w), T, S, block,
+                          _ptr(rows), rows.size, _ptr(ub), _ptr(scale))
+    return ub, scale
 
 
 def select_f64(vals: np.ndarray, first_index: int, k: int):

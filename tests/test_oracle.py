@@ -15,7 +15,10 @@ What pins what:
 * the selection: brute-force enumeration of all subsets on tiny windows,
   the all-equal row, windows shorter than topk, torch.topk on tie-free rows,
   signed zeros;
-* fused select: the all-equal workload's closed form and window locality.
+* fused select: the all-equal workload's closed form and window locality;
+* the block score bound: it dominates every score of its block (checked
+  against the score oracle, which the pins above tie down), it equals the
+  score for one-key blocks (closed form), and a hand-worked case.
 """
 from __future__ import annotations
 
@@ -435,3 +438,75 @@ def test_fused_window_locality():
     b = orc.fused_select(q, kv2, sc, w, ks, ke, 8)
     for t in (0, 1, 3):
         assert np.array_equal(a[0][t], b[0][t])
+
+
+# ---------------------------------------------------------------------------
+# block score bound
+# ---------------------------------------------------------------------------
+
+def _bound_case(dtype, seed=21, T=3, S=300):
+    q, kv, sc = _case(seed, dtype, T, S)
+    w = torch.randn((T, 32), generator=torch.Generator().manual_seed(seed + 1)) / math.sqrt(32)
+    return q, kv, sc, w
+
+
+def check_bound_dominates_scores(dtype):
+    """UB(t, b) >= I(t, s) for every key s of block b (blocks of 128 and a
+    ragged last block of 44 keys), with weights of both signs."""
+    q, kv, sc, w = _bound_case(dtype)
+    T, S = q.shape[0], kv.shape[0]
+    ks, ke = _full_windows(T, S)
+    I, _ = orc.index_scores(q, kv, sc, w, ks, ke)
+    ub, scale = orc.block_bound(q, kv, sc, w, block=128)
+    assert ub.shape == (T, 3)
+    for b in range(3):
+        blk = I[:, b * 128:min(S, (b + 1) * 128)]
+        assert np.all(ub[:, b] >= blk.max(axis=1) - 1e-12 * scale[:, b]), (b, ub[:, b], blk.max(axis=1))
+    # the bound is not vacuous: it stays within the size of its own terms
+    assert np.all(np.abs(ub) <= scale * (1 + 1e-12))
+
+
+def check_bound_one_key_blocks(dtype):
+    """A block of one key is a point box: UB(t, s) = I(t, s)."""
+    q, kv, sc, w = _bound_case(dtype, seed=22, T=2, S=40)
+    ks, ke = _full_windows(2, 40)
+    I, E = orc.index_scores(q, kv, sc, w, ks, ke)
+    ub, scale = orc.block_bound(q, kv, sc, w, block=1)
+    np.testing.assert_allclose(ub, I, rtol=0, atol=1e-12 * E.max())
+    np.testing.assert_allclose(scale, E, rtol=1e-12, atol=0)
+
+
+def check_bound_hand_example():
+    """Worked by hand from the definition.  Row 0: q[0,0,0] = 2,
+    q[0,1,0] = -1, q[0,2,1] = 1; w = (0.5, -2, -1, 0, ...); two keys with
+    k0 = (-1, 2, 0...), k1 = (3, 5, 0...), sigma = 1.  Box: hi = (3, 5),
+    lo = (-1, 2).  Head 0: U = max(6, -2) = 6.  Head 1: U = max(-3, 1) = 1,
+    L = -3.  Head 2: U = 5, L = 2.  UB = 0.5*6 + (-2)*ReLU(-3) + (-1)*ReLU(2)
+    = 1.  Term sizes: 0.5*2*3 + 2*1*3 + 1*1*5 = 14.  The scores are
+    I(k0) = 0 - 2 - 2 = -4 and I(k1) = 3 + 0 - 5 = -2."""
+    q = torch.zeros((1, 32, 128))
+    q[0, 0, 0], q[0, 1, 0], q[0, 2, 1] = 2.0, -1.0, 1.0
+    w = torch.zeros((1, 32))
+    w[0, 0], w[0, 1], w[0, 2] = 0.5, -2.0, -1.0
+    kv = torch.zeros((2, 128))
+    kv[0, 0], kv[0, 1], kv[1, 0], kv[1, 1] = -1.0, 2.0, 3.0, 5.0
+    qb, kb = q.to(torch.bfloat16), kv.to(torch.bfloat16)
+    ub, scale = orc.block_bound(qb, kb, None, w, block=128)
+    assert ub.tolist() == [[1.0]] and scale.tolist() == [[14.0]], (ub, scale)
+    ks, ke = _full_windows(1, 2)
+    I, _ = orc.index_scores(qb, kb, None, w, ks, ke)
+    assert I[0].tolist() == [-4.0, -2.0]
+
+
+@pytest.mark.parametrize("dtype", ["fp8", "bf16"])
+def test_bound_dominates_scores(dtype):
+    check_bound_dominates_scores(dtype)
+
+
+@pytest.mark.parametrize("dtype", ["fp8", "bf16"])
+def test_bound_one_key_blocks(dtype):
+    check_bound_one_key_blocks(dtype)
+
+
+def test_bound_hand_example():
+    check_bound_hand_example()

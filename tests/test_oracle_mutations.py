@@ -33,6 +33,16 @@ MUTATIONS = [
      "uint32_t w = (uint32_t)(bits & 0xFFFFu) << 15;"),
     ("padding_index", "out_idx[j] = j < n ? buf[j].i : -1;", "out_idx[j] = j < n ? buf[j].i : 0;"),
     ("short_window_loses_one", "int64_t n = L < k ? L : k;", "int64_t n = L < k ? L - 1 : k;"),
+    ("bound_negative_weight_uses_upper", "ub += wt[h] * (L > 0.0 ? L : 0.0);",
+     "ub += wt[h] * (U > 0.0 ? U : 0.0);"),
+    ("bound_upper_takes_min", "U += x > y ? x : y;", "U += x < y ? x : y;"),
+    ("bound_sigma_dropped", "double v = sigma * element(dtype, kv, s * ORC_DIM + d);",
+     "double v = element(dtype, kv, s * ORC_DIM + d);"),
+    ("bound_last_key_dropped", "for (int64_t s = b * block; s < S && s < (b + 1) * block; ++s) {",
+     "for (int64_t s = b * block; s < S && s < (b + 1) * block - 1; ++s) {"),
+    ("bound_scale_smaller_side",
+     "(fabs(bh[d]) > fabs(bl[d]) ? fabs(bh[d]) : fabs(bl[d]))",
+     "(fabs(bh[d]) < fabs(bl[d]) ? fabs(bh[d]) : fabs(bl[d]))"),
 ]
 
 CHECKS = [
@@ -52,6 +62,9 @@ CHECKS = [
     pins.check_topk_rows_brute_force,
     pins.check_topk_rows_torch_tie_free,
     pins.check_fused_all_equal,
+    lambda: pins.check_bound_dominates_scores("fp8"),
+    lambda: pins.check_bound_one_key_blocks("bf16"),
+    pins.check_bound_hand_example,
 ]
 
 
