@@ -73,7 +73,10 @@ typedef struct {
     int32_t sample_keys; /* target strided-sample size per row, m (default 4096) */
     float oversample;    /* beta: the threshold keeps ~beta*topk keys (default 1.5) */
     int32_t capacity;    /* C: candidate slots per row (0: 2*topk) */
-    int32_t prune;       /* score-bound key pruning: -1 auto (default), 0 off, 1 on */
+    int32_t prune;       /* score-bound key pruning (FlashTopK README, "Highlights":
+                          * adaptive key pruning by a score bound): 0 auto, the
+                          * default (estimate the skippable share of key blocks on
+                          * a sample and prune if it is >= 25%), 1 always, -1 off */
     int32_t recovery_rows; /* rows rescored densely per recovery pass (0: auto) */
     int32_t reserved[3];   /* must be 0 */
 } ftk_config;
@@ -188,6 +191,31 @@ ftk_status ftk_score_dense(ftk_dtype dtype, const void *q, const void *kv,
 size_t ftk_score_dense_workspace_size(int64_t nrows);
 
 /*
+ * ftk_block_bound -- the score bound that ftk_select's key pruning uses
+ * (FlashTopK README, "Highlights": keys are skipped by a score bound; the
+ * pages give no formula, this is the per-dimension box bound).  For every
+ * query row t < T and key block b (keys [128 b, min(128 b + 128, S)))
+ * writes out[t * ld + b] = UB[t, b] >= I[t, s] for every key s of block b:
+ *     hi[d] = max_s sigma_s kv[s,d],  lo[d] = min_s sigma_s kv[s,d]
+ *     U_h = sum_d max(q[t,h,d] hi[d], q[t,h,d] lo[d]),  L_h = same with min
+ *     UB  = sum_{w[t,h] >= 0} w[t,h] ReLU(U_h) + sum_{w[t,h] < 0} w[t,h] ReLU(L_h)
+ * computed in float32 (within about 1e-5 * sum_h |w| sum_d |q| max(|hi|,
+ * |lo|) of the exact value).  A block holding a NaN key, a kv_scales entry
+ * that is not finite and > 0, or a product that overflows gets +inf.
+ *   out        device float32 [T, ld], ld >= ceil(S / 128)
+ *   workspace  device, >= ftk_block_bound_workspace_size(S) bytes,
+ *              256-byte aligned
+ * Other arguments as for ftk_select (no windows: every block of every row).
+ */
+ftk_status ftk_block_bound(ftk_dtype dtype, const void *q, const void *kv,
+                           const float *kv_scales, const float *weights,
+                           int64_t T, int64_t S, float *out, int64_t ld,
+                           void *workspace, size_t workspace_bytes,
+                           void *stream);
+
+size_t ftk_block_bound_workspace_size(int64_t S);
+
+/*
  * ftk_windows_from_cu_seqlens -- causal windows of packed sequences
  * (FlashTopK README, "Usage": windows_from_cu_seqlens).  Sequence j owns
  * query rows [cu_q[j], cu_q[j+1]) and keys [cu_k[j], cu_k[j+1]); its
@@ -236,11 +264,13 @@ ftk_status ftk_select_noalloc(ftk_dtype dtype, const void *q, const void *kv,
 /* Diagnostic timing hook.  While set, every ftk_select call made from the
  * calling host thread records events[i] (cudaEvent_t values created by the
  * caller, passed as void *) on the call's stream at its stage boundaries:
- * 0 start, 1 plan done, 2 sample pass done, 3 thresholds done, 4 dense scan
- * done, 5 refine done, 6 recovery done.  n must be 0 (or events NULL) to
- * stop, else >= 7 with non-NULL events (FTK_ERR_INVALID_ARG otherwise).  If
- * recording fails the hook switches itself off.  The library does not own
- * the events. */
+ * 0 start, 1 plan done, 2 sample pass done, 3 thresholds done, 4 scan done,
+ * 5 refine done, 6 recovery done, and, when n >= 8, 7 pruning done (after
+ * the score-bound kernels, before the scan; right after 3 when pruning is
+ * off).  n must be 0 (or events NULL) to stop, else >= 7 with non-NULL
+ * events (the first min(n, 8) are used; FTK_ERR_INVALID_ARG otherwise).
+ * If recording fails the hook switches itself off.  The library does not
+ * own the events. */
 ftk_status ftk_set_stage_events(void *const *events, int n);
 
 /* Human-readable name of an ftk_status value (static string). */

@@ -53,8 +53,16 @@ static ftk_status launch_rows_dt(const RowsArgs &a, int cluster, cudaStream_t st
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return cuda_status(e);
+    // Clusters stride over the rows: at most as many as fit at once (two
+    // CTAs per SM).
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int64_t nclusters = 2 * static_cast<int64_t>(sms) / cluster;
+    if (nclusters < 1) nclusters = 1;
+    if (a.rows < nclusters) nclusters = a.rows;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(a.rows * cluster), 1, 1);
+    cfg.gridDim = dim3(static_cast<unsigned>(nclusters * cluster), 1, 1);
     cfg.blockDim = dim3(kRowsThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;

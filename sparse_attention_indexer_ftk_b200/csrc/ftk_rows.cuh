@@ -231,25 +231,18 @@ __device__ __forceinline__ void cluster_sum256(cg::cluster_group &cluster, RowsS
 __device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 
+// Top-k of grid row r by the whole cluster.  Returns with every cp.async
+// of this CTA complete and, for rows that used distributed shared memory,
+// with every CTA of the cluster done reading this CTA's shared memory.
 template <int DT>
-__global__ void __launch_bounds__(kRowsThreads, 2) rows_topk_kernel(const RowsArgs a)
+__device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, cg::cluster_group &cluster,
+                                              unsigned cs, unsigned rank, int64_t r)
 {
     using Tr = RowsTraits<DT>;
     using elem = typename Tr::elem;
     constexpr int VEC = Tr::kVec;
-    extern __shared__ __align__(16) uint8_t smem_raw[];
-    RowsSmem &sm = *reinterpret_cast<RowsSmem *>(smem_raw);
-
-    cg::cluster_group cluster = cg::this_cluster();
-    const unsigned cs = cluster.num_blocks();
-    const unsigned rank = cluster.block_rank();
-    const int64_t r = blockIdx.x / cs;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint32_t lt_mask = (1u << lane) - 1u;
-
-    // Row selection is uniform over the cluster, so whole clusters exit together.
-    if (r >= a.rows) return;
-    if (a.nrows_dev && r >= static_cast<int64_t>(*a.nrows_dev) - a.nrows_off) return;
     const int64_t orow = a.row_map ? a.row_map[r] : r;
     int64_t len = a.cols, base_index = 0;
     if (a.win_ks) {
@@ -681,6 +674,29 @@ __global__ void __launch_bounds__(kRowsThreads, 2) rows_topk_kernel(const RowsAr
     if (tid == 0 && sm.nan_seen) set_status(a.status, FTK_STATUS_NAN);
     __syncwarp();
     cluster_wait();  // keep my shared memory alive until every CTA is done with it
+}
+
+// One cluster per row at a time; clusters stride over the rows (the count
+// may be on the device), so a grid sized for the SMs serves any row count.
+template <int DT>
+__global__ void __launch_bounds__(kRowsThreads, 2) rows_topk_kernel(const RowsArgs a)
+{
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    RowsSmem &sm = *reinterpret_cast<RowsSmem *>(smem_raw);
+    cg::cluster_group cluster = cg::this_cluster();
+    const unsigned cs = cluster.num_blocks();
+    const unsigned rank = cluster.block_rank();
+    int64_t nrows = a.rows;
+    if (a.nrows_dev) {
+        const int64_t c = static_cast<int64_t>(*a.nrows_dev) - a.nrows_off;
+        nrows = c < nrows ? c : nrows;
+    }
+    // Row selection is uniform over the cluster: its CTAs walk the same rows.
+    for (int64_t r = blockIdx.x / cs; r < nrows; r += gridDim.x / cs) {
+        rows_topk_row<DT>(a, sm, cluster, cs, rank, r);
+        cp_async_wait<0>();
+        __syncthreads();  // shared memory is free for the next row
+    }
 }
 
 }  // namespace ftk

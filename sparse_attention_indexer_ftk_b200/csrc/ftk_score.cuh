@@ -101,17 +101,23 @@ struct ScoreArgs {
     int32_t count_off;
     // Schedule over row tiles of row_tile_of(dtype) rows.  Planned: per-tile
     // ranges and an item prefix written by the plan kernel.  Static: item =
-    // (tile, chunk), ranges found on the fly.
-    int32_t planned;
+    // (tile, chunk of keys), ranges found on the fly, chunk size chosen at
+    // kernel start from the rows in the list (make_sched).
     const int32_t *tile_lo, *tile_hi, *tile_lg, *item_start;
     int32_t ntiles;
-    int32_t static_chunks;
     // COLLECT
     const float *tau;         // [T]
     int32_t *cnt;             // [T] running candidate counts
     float *cand_val;          // [T, cap]
     int32_t *cand_idx;        // [T, cap]
     int32_t cap;
+    // COLLECT with key pruning: bit b of word prune_bits[tile * prune_words
+    // + b / 32] set means key block b (keys 128 b .. 128 b + 127) holds no
+    // candidate of any row of the tile.  Read only if prune_bits is set
+    // and *prune_on != 0 (both decided on the device before the scan).
+    const uint32_t *prune_bits;
+    int32_t prune_words;
+    const int32_t *prune_on;
     // SAMPLE / DUMP output rows of stride ld
     float *out;
     int64_t ld;
@@ -156,10 +162,53 @@ __device__ __forceinline__ int32_t list_query(const ScoreArgs &a, int64_t p, int
     return static_cast<int32_t>(t);
 }
 
-template <int MODE, int RT>
-__device__ __forceinline__ bool get_item(const ScoreArgs &a, int it, int64_t nlist, Item &m)
+// True if the scan skips key tile kt of item m (its key block was pruned
+// for the item's row tile).  Collect items start on a key-tile boundary.
+__device__ __forceinline__ bool tile_pruned(const ScoreArgs &a, const Item &m, int kt)
 {
-    if (a.planned) {
+    const int32_t blk = (m.key0 / kKeyTile) + kt;
+    const uint32_t w = __ldg(a.prune_bits + static_cast<int64_t>(m.tile) * a.prune_words + (blk >> 5));
+    return (w >> (blk & 31)) & 1u;
+}
+
+// Static schedules: a few rows (dense recovery of the rows a threshold
+// missed) must still spread over every SM, so the key chunk of an item
+// shrinks until the row tiles in use give about two items per CTA.
+constexpr int kMinChunkTiles = 8;
+
+struct Sched {
+    int32_t chunk_keys;  // keys per item (static)
+    int32_t chunks;      // items per row tile (static)
+    int64_t tiles;       // row tiles in use (static)
+};
+
+// SAMPLE and COLLECT run planned schedules, DUMP a static one.
+template <int MODE>
+__device__ __forceinline__ constexpr bool planned_mode() { return MODE != MODE_DUMP; }
+
+template <int MODE, int RT>
+__device__ __forceinline__ Sched make_sched(const ScoreArgs &a, int64_t nlist)
+{
+    Sched sc;
+    sc.tiles = (nlist + RT - 1) / RT;
+    sc.chunk_keys = kChunkKeys;
+    sc.chunks = 0;
+    if (!planned_mode<MODE>()) {
+        const int64_t kt = (a.S + kKeyTile - 1) / kKeyTile + 1;  // + 1: the aligned start
+        const int64_t want = 2 * static_cast<int64_t>(gridDim.x);
+        int64_t ct = (sc.tiles * kt + want - 1) / want;
+        ct = ct < kMinChunkTiles ? kMinChunkTiles : (ct > kChunkTiles ? kChunkTiles : ct);
+        sc.chunk_keys = static_cast<int32_t>(ct * kKeyTile);
+        sc.chunks = static_cast<int32_t>((kt + ct - 1) / ct);
+    }
+    return sc;
+}
+
+template <int MODE, int RT>
+__device__ __forceinline__ bool get_item(const ScoreArgs &a, const Sched &sc, int it, int64_t nlist,
+                                         Item &m)
+{
+    if (planned_mode<MODE>()) {
         const int32_t nt = a.ntiles;
         if (it >= a.item_start[nt]) return false;
         int lo = 0, hi = nt;  // largest tile with item_start[tile] <= it
@@ -179,8 +228,8 @@ __device__ __forceinline__ bool get_item(const ScoreArgs &a, int it, int64_t nli
             m.kend = min(a.tile_hi[lo], m.key0 + kChunkKeys);
         }
     } else {
-        m.tile = it / a.static_chunks;
-        const int chunk = it - m.tile * a.static_chunks;
+        m.tile = it / sc.chunks;
+        const int chunk = it - m.tile * sc.chunks;
         m.lg = 0;
         int64_t lo = INT64_MAX, hi = -1;
         for (int j = 0; j < RT; ++j) {
@@ -191,10 +240,10 @@ __device__ __forceinline__ bool get_item(const ScoreArgs &a, int it, int64_t nli
         }
         if (hi < 0) return false;
         lo &= ~static_cast<int64_t>(kKeyTile - 1);
-        const int64_t k0 = lo + static_cast<int64_t>(chunk) * kChunkKeys;
+        const int64_t k0 = lo + static_cast<int64_t>(chunk) * sc.chunk_keys;
         if (k0 >= hi) return false;
         m.key0 = static_cast<int32_t>(k0);
-        m.kend = static_cast<int32_t>(min(hi, k0 + kChunkKeys));
+        m.kend = static_cast<int32_t>(min(hi, k0 + sc.chunk_keys));
     }
     m.nkt = (m.kend - m.key0 + kKeyTile - 1) / kKeyTile;
     return m.nkt > 0;
@@ -203,15 +252,16 @@ __device__ __forceinline__ bool get_item(const ScoreArgs &a, int it, int64_t nli
 // Next work item of this CTA (static round-robin over the item space), or
 // false when there are no more.  Every role walks the same sequence.
 template <int MODE, int RT>
-__device__ __forceinline__ bool next_item(const ScoreArgs &a, int &it, int64_t nlist, Item &m)
+__device__ __forceinline__ bool next_item(const ScoreArgs &a, const Sched &sc, int &it, int64_t nlist,
+                                          Item &m)
 {
     for (;; it += gridDim.x) {
-        if (a.planned) {
+        if (planned_mode<MODE>()) {
             if (it >= a.item_start[a.ntiles]) return false;
         } else {
-            if (it >= a.static_chunks * ((a.nrows + RT - 1) / RT)) return false;
+            if (it >= static_cast<int64_t>(sc.chunks) * sc.tiles) return false;
         }
-        if (get_item<MODE, RT>(a, it, nlist, m)) return true;
+        if (get_item<MODE, RT>(a, sc, it, nlist, m)) return true;
     }
 }
 
@@ -349,6 +399,9 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t nlist = list_rows(a);
+    const Sched sc = make_sched<MODE, RT>(a, nlist);
+    // Key pruning on (the same value in every thread: set by an earlier kernel).
+    const bool pruned = MODE == MODE_COLLECT && a.prune_bits != nullptr && *a.prune_on != 0;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::kKStages; ++i) {
@@ -382,7 +435,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             int q_armed = 0;
             uint32_t q_armed_ph = 0;
             Item m;
-            for (int it = blockIdx.x; !*abort && next_item<MODE, RT>(a, it, nlist, m); it += gridDim.x) {
+            for (int it = blockIdx.x; !*abort && next_item<MODE, RT>(a, sc, it, nlist, m); it += gridDim.x) {
                 // The query group: the 32 head rows of each of RT queries.
                 if (!mbar_wait(&ms.q_empty, qph ^ 1u, abort, a.status)) break;
                 mbar_arrive_expect_tx(&ms.q_full, Lay::kQBytes);
@@ -401,6 +454,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                 qph ^= 1u;
                 const CUtensorMap *map = &kvm.m[MODE == MODE_SAMPLE ? m.lg : 0];
                 for (int kt = 0; kt < m.nkt; ++kt) {
+                    if (pruned && tile_pruned(a, m, kt)) continue;
                     if (!mbar_wait(&ms.kv_empty[ks_], kph ^ 1u, abort, a.status)) break;
                     mbar_arrive_expect_tx(&ms.kv_full[ks_], Lay::kKBytes);
                     k_armed[ks_] = 1;
@@ -426,12 +480,13 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             uint32_t kph = 0, qph = 0, aph = 0;
             bool issued = false, ok = true;
             Item m;
-            for (int it = blockIdx.x; ok && !*abort && next_item<MODE, RT>(a, it, nlist, m); it += gridDim.x) {
+            for (int it = blockIdx.x; ok && !*abort && next_item<MODE, RT>(a, sc, it, nlist, m); it += gridDim.x) {
                 if (!mbar_wait(&ms.q_full, qph, abort, a.status)) break;
                 qph ^= 1u;
                 tc_fence_after();
                 const uint32_t qaddr = smem_u32(sq);
                 for (int kt = 0; kt < m.nkt && ok; ++kt) {
+                    if (pruned && tile_pruned(a, m, kt)) continue;
                     if (!mbar_wait(&ms.kv_full[ks_], kph, abort, a.status)) {
                         ok = false;
                         break;
@@ -491,7 +546,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         uint32_t aph = 0;
         bool bad_scale = false;
         Item m;
-        for (int it = blockIdx.x; !*abort && next_item<MODE, RT>(a, it, nlist, m); it += gridDim.x) {
+        for (int it = blockIdx.x; !*abort && next_item<MODE, RT>(a, sc, it, nlist, m); it += gridDim.x) {
             // Per-item parameters of this warp's queries (warp-uniform).  Slot
             // qq = vt * NQ + qi is query qg * NQ + qi of query tile vt.
             int32_t qt[WQ], qpos[WQ], wlo[WQ], wlen[WQ];
@@ -544,8 +599,10 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                     const int64_t s1 = static_cast<int64_t>(kidx_next) << m.lg;
                     sig_next = (kidx_next < m.kend && s1 < a.S) ? __ldg(scales + s1) : 1.f;
                 }
-                bad_scale |= scales && kidx < m.kend && (!(sigma > 0.f) || isinf(sigma));
+                const bool skip = pruned && tile_pruned(a, m, kt);  // warp-uniform
+                bad_scale |= !skip && scales && kidx < m.kend && (!(sigma > 0.f) || isinf(sigma));
                 const int32_t s = MODE == MODE_SAMPLE ? (kidx << m.lg) : kidx;
+                if (!skip) {
 #pragma unroll
                 for (int vt = 0; vt < QG; ++vt) {
                     const bool got = mbar_wait(&ms.acc_full[ab], aph, abort, a.status);
@@ -598,6 +655,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                             if (valid) a.out[static_cast<int64_t>(qpos[qq]) * a.ld + (s - wlo[qq])] = I[qi];
                         }
                     }
+                }
                 }
                 if (MODE == MODE_COLLECT && ok) {
                     // Every 2 key tiles (<= 2 * 32 new entries per warp and

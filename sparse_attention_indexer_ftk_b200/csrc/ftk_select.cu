@@ -11,7 +11,12 @@
 //   threshold  per row: tau = the r-th largest sampled score, r chosen so
 //              that about oversample * topk keys pass; tau = -inf when the
 //              whole window fits in the candidate buffer;
-//   scan       score_kernel<COLLECT>: dense fused scoring, keeping I >= tau;
+//   prune      (unless switched off) the score bound of every 128-key block:
+//              box of the keys, a sampled estimate of the skippable
+//              fraction, and, when it pays, the skip bitmap of (row tile,
+//              block) pairs that cannot hold a candidate (ftk_prune.cuh);
+//   scan       score_kernel<COLLECT>: fused scoring of every key tile not
+//              skipped, keeping I >= tau;
 //   refine     per row: exact radix select of the topk candidates with the
 //              (score desc, index asc) order, written in ascending index
 //              order; rows whose candidates overflowed or fell short of
@@ -25,6 +30,7 @@
 #include <string.h>
 
 #include "ftk_host.h"
+#include "ftk_prune.cuh"
 #include "ftk_rows.cuh"
 #include "ftk_score.cuh"
 
@@ -38,6 +44,7 @@ constexpr int kMaxRowTile = 16;      // largest row_tile_of(dtype)
 // Device copy of ftk_info plus counters (same layout for the leading part).
 struct DevInfo {
     ftk_info info;
+    uint32_t est_total, est_pruned;  // sampled (tile, block) pairs of the prune estimate
 };
 
 // ---------------------------------------------------------------------------
@@ -103,8 +110,11 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanArgs p)
         memset(&p.info->info, 0, sizeof(ftk_info));
         p.info->info.rows = p.T;
         p.info->info.kernel_launches = p.launches;
+        p.info->est_total = 0;
+        p.info->est_pruned = 0;
     }
     __syncthreads();
+    unsigned long long nblocks = 0;  // (row tile, key block) pairs of the scan
     if (bad) atomicOr(&p.info->info.status, FTK_STATUS_BAD_WINDOW);
     uint32_t carry_s = 0, carry_c = 0;
     for (int32_t base = 0; base < p.ntiles; base += blockDim.x) {
@@ -136,6 +146,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanArgs p)
                 clo = static_cast<int32_t>(lo_al);
                 chi = static_cast<int32_t>(hi);
                 nc = static_cast<uint32_t>((hi - lo_al + kChunkKeys - 1) / kChunkKeys);
+                nblocks += static_cast<unsigned long long>((hi - lo_al + kKeyTile - 1) / kKeyTile);
             }
             p.s_lo[tile] = slo;
             p.s_hi[tile] = shi;
@@ -157,6 +168,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanArgs p)
         p.s_start[p.ntiles] = static_cast<int32_t>(carry_s);
         p.c_start[p.ntiles] = static_cast<int32_t>(carry_c);
     }
+    if (nblocks) atomicAdd(reinterpret_cast<unsigned long long *>(&p.info->info.blocks_total), nblocks);
 }
 
 // ---------------------------------------------------------------------------
@@ -486,11 +498,13 @@ static int num_sms()
     return n > 0 ? n : 148;
 }
 
+enum PruneMode { PRUNE_AUTO = 0, PRUNE_ON = 1, PRUNE_OFF = 2 };
+
 struct SelectCfg {
     int m;          // sample keys
     float beta;
     int cap;
-    int prune;
+    PruneMode prune;
     int rec_rows;
 };
 
@@ -501,7 +515,8 @@ static SelectCfg resolve_cfg(int64_t T, int64_t S, int topk, const ftk_config *c
     r.beta = c && c->oversample > 0.f ? c->oversample : 1.5f;
     r.cap = c && c->capacity > 0 ? c->capacity : 2 * topk;
     if (r.cap > 2 * FTK_MAX_TOPK) r.cap = 2 * FTK_MAX_TOPK;
-    r.prune = c ? c->prune : -1;
+    const int pr = c ? c->prune : 0;
+    r.prune = pr == 0 ? PRUNE_AUTO : pr > 0 ? PRUNE_ON : PRUNE_OFF;
     // Strides are powers of two up to 2^(kNumStrideMaps - 1).
     const int64_t min_m = (S + (int64_t(1) << (kNumStrideMaps - 1)) - 1) >> (kNumStrideMaps - 1);
     if (r.m < min_m) r.m = static_cast<int>(min_m);
@@ -535,6 +550,10 @@ struct SelectWs {
     int32_t *bad_count;
     float *scratch;
     int64_t scratch_ld;
+    float *box;       // [nblocks][2][128] score-bound box of each key block
+    float *mb;        // [nblocks]
+    uint32_t *prune_bits;  // [ntiles][nwords]
+    int32_t nblocks, nwords;
 };
 
 static bool carve_select(Carver &cv, int64_t T, int64_t S, const SelectCfg &c, SelectWs &w)
@@ -558,6 +577,17 @@ static bool carve_select(Carver &cv, int64_t T, int64_t S, const SelectCfg &c, S
     w.bad_count = cv.take<int32_t>(1);
     w.scratch_ld = (S + 7) / 8 * 8;
     w.scratch = cv.take<float>(static_cast<int64_t>(c.rec_rows) * w.scratch_ld);
+    w.nblocks = static_cast<int32_t>((S + kBlockKeys - 1) / kBlockKeys);
+    w.nwords = (w.nblocks + kBoundWordBlocks - 1) / kBoundWordBlocks;
+    if (c.prune != PRUNE_OFF) {
+        w.box = cv.take<float>(static_cast<int64_t>(w.nblocks) * 2 * kDim);
+        w.mb = cv.take<float>(w.nblocks);
+        w.prune_bits = cv.take<uint32_t>(ntiles * w.nwords);
+    } else {
+        w.box = nullptr;
+        w.mb = nullptr;
+        w.prune_bits = nullptr;
+    }
     return cv.ok;
 }
 
@@ -612,10 +642,11 @@ static ftk_status check_select_args(int dtype, const void *q, const void *kv, co
 }
 
 thread_local void *const *g_stage_events = nullptr;
+thread_local int g_stage_count = 0;
 
 static void stage_mark(int i, cudaStream_t s)
 {
-    if (g_stage_events && cudaEventRecord(static_cast<cudaEvent_t>(g_stage_events[i]), s) != cudaSuccess) {
+    if (g_stage_events && i < g_stage_count && cudaEventRecord(static_cast<cudaEvent_t>(g_stage_events[i]), s) != cudaSuccess) {
         (void)cudaGetLastError();  // a bad event must not poison the launch checks
         g_stage_events = nullptr;
     }
@@ -629,12 +660,15 @@ extern "C" ftk_status ftk_set_stage_events(void *const *events, int n)
 {
     if (events == nullptr || n == 0) {
         g_stage_events = nullptr;
+        g_stage_count = 0;
         return FTK_OK;
     }
     if (n < 7) return FTK_ERR_INVALID_ARG;
-    for (int i = 0; i < 7; ++i)
+    const int used = n < 8 ? n : 8;
+    for (int i = 0; i < used; ++i)
         if (events[i] == nullptr) return FTK_ERR_INVALID_ARG;
     g_stage_events = events;
+    g_stage_count = used;
     return FTK_OK;
 }
 
@@ -709,7 +743,7 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
     pa.cnt = w.cnt;
     pa.bad_count = w.bad_count;
     pa.info = w.info;
-    pa.launches = 5 + 2 * ((T + c.rec_rows - 1) / c.rec_rows);
+    pa.launches = 5 + 2 * ((T + c.rec_rows - 1) / c.rec_rows) + (c.prune == PRUNE_OFF ? 0 : c.prune == PRUNE_AUTO ? 3 : 2);
     plan_kernel<<<1, kPlanThreads, 0, s>>>(pa);
     if ((st = cuda_status(cudaGetLastError())) != FTK_OK) return st;
     stage_mark(1, s);
@@ -723,7 +757,6 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
     sa.ke = ke;
     sa.rows = nullptr;
     sa.nrows = T;
-    sa.planned = 1;
     sa.ntiles = ntiles;
     sa.status = status;
     // sample pass
@@ -763,7 +796,50 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
     }
     stage_mark(3, s);
 
-    // dense scan
+    if (c.prune != PRUNE_OFF) {
+        BoxArgs xa;
+        xa.kv = kv;
+        xa.kv_scales = kv_scales;
+        xa.S = S;
+        xa.nblocks = w.nblocks;
+        xa.box = w.box;
+        xa.mb = w.mb;
+        if ((st = launch_box(dtype, xa, s)) != FTK_OK) return st;
+        BoundArgs ba = {};
+        ba.q = q;
+        ba.weights = weights;
+        ba.ks = ks;
+        ba.ke = ke;
+        ba.T = T;
+        ba.S = S;
+        ba.rt = rt;
+        ba.ntiles = ntiles;
+        ba.nblocks = w.nblocks;
+        ba.nwords = w.nwords;
+        ba.box = w.box;
+        ba.mb = w.mb;
+        ba.tau = w.tau;
+        ba.c_lo = w.c_lo;
+        ba.c_hi = w.c_hi;
+        ba.est_tiles = ntiles < kEstTiles ? ntiles : kEstTiles;
+        ba.bits = w.prune_bits;
+        ba.est_total = &w.info->est_total;
+        ba.est_pruned = &w.info->est_pruned;
+        ba.mode = c.prune == PRUNE_AUTO ? 0 : 1;
+        ba.prune_enabled = &w.info->info.prune_enabled;
+        ba.blocks_pruned = reinterpret_cast<unsigned long long *>(&w.info->info.blocks_pruned);
+        if (c.prune == PRUNE_AUTO) {
+            st = launch_bound(dtype, BOUND_EST, ba, ba.est_tiles * (kEstBlocks / kEstChunk), s);
+            if (st != FTK_OK) return st;
+        }
+        const int64_t items = static_cast<int64_t>(ntiles) * w.nwords;
+        const int64_t cap = static_cast<int64_t>(sms) * 2;
+        st = launch_bound(dtype, BOUND_FULL, ba, static_cast<int>(items < cap ? items : cap), s);
+        if (st != FTK_OK) return st;
+    }
+    stage_mark(7, s);
+
+    // scan
     sa.tile_lo = w.c_lo;
     sa.tile_hi = w.c_hi;
     sa.tile_lg = nullptr;
@@ -774,6 +850,9 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
     sa.cand_idx = w.cand_idx;
     sa.cap = c.cap;
     sa.out = nullptr;
+    sa.prune_bits = w.prune_bits;
+    sa.prune_words = w.nwords;
+    sa.prune_on = &w.info->info.prune_enabled;
     st = launch_score_dt<MODE_COLLECT>(dtype, sa, tq, kvm, sms, s);
     if (st != FTK_OK) return st;
     stage_mark(4, s);
@@ -804,10 +883,11 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
     }
     stage_mark(5, s);
 
-    // dense recovery of the listed rows, rec_rows at a time
+    // dense recovery of the listed rows, rec_rows at a time; the row count
+    // is on the device and usually small, so plan the row top-k for few
+    // rows (widest clusters) and let its clusters stride over the rest
     int rcluster = 1, rchunk = 8;
-    rows_plan(c.rec_rows, S, topk, &rcluster, &rchunk);
-    const int32_t chunks = static_cast<int32_t>((S + kKeyTile - 1 + kChunkKeys - 1) / kChunkKeys);
+    rows_plan(c.rec_rows < 16 ? c.rec_rows : 16, S, topk, &rcluster, &rchunk);
     for (int64_t b0 = 0; b0 < T; b0 += c.rec_rows) {
         ScoreArgs da = {};
         da.T = T;
@@ -820,14 +900,10 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
         da.nrows = c.rec_rows;
         da.count_dev = w.bad_count;
         da.count_off = static_cast<int32_t>(b0);
-        da.planned = 0;
-        da.static_chunks = chunks;
         da.out = w.scratch;
         da.ld = w.scratch_ld;
         da.status = status;
-        const int64_t items = static_cast<int64_t>(chunks) * ((c.rec_rows + rt - 1) / rt);
-        st = launch_score_dt<MODE_DUMP>(dtype, da, tq, kvm,
-                                        static_cast<int>(items < sms ? items : sms), s);
+        st = launch_score_dt<MODE_DUMP>(dtype, da, tq, kvm, sms, s);
         if (st != FTK_OK) return st;
         RowsArgs ra2 = {};
         ra2.x = w.scratch;
@@ -883,17 +959,11 @@ extern "C" ftk_status ftk_score_dense(ftk_dtype dtype, const void *q, const void
     da.ke = ke;
     da.rows = rows;
     da.nrows = nrows;
-    da.planned = 0;
-    da.static_chunks = static_cast<int32_t>((S + kKeyTile - 1 + kChunkKeys - 1) / kChunkKeys);
     da.out = out;
     da.ld = ld;
     da.status = static_cast<uint32_t *>(workspace);
     cudaStream_t s = as_stream(stream);
     cudaError_t e = cudaMemsetAsync(workspace, 0, 4, s);
     if (e != cudaSuccess) return cuda_status(e);
-    const int rt = row_tile_of(dtype);
-    const int64_t items = static_cast<int64_t>(da.static_chunks) * ((nrows + rt - 1) / rt);
-    const int sms = num_sms();
-    return launch_score_dt<MODE_DUMP>(dtype, da, tq, kvm,
-                                      static_cast<int>(items < sms ? items : sms), s);
+    return launch_score_dt<MODE_DUMP>(dtype, da, tq, kvm, num_sms(), s);
 }

@@ -39,6 +39,7 @@ EXPORTS = (
     "ftk_select", "ftk_select_workspace_size", "ftk_read_info", "ftk_topk_rows",
     "ftk_score_dense", "ftk_score_dense_workspace_size", "ftk_windows_from_cu_seqlens",
     "ftk_set_stage_events", "ftk_status_string", "ftk_version", "ftk_select_noalloc",
+    "ftk_block_bound", "ftk_block_bound_workspace_size",
 )
 
 
@@ -90,6 +91,10 @@ def load_library(path: str = LIB_PATH):
     L.ftk_select_noalloc.argtypes = [I32, P, P, P, P, P, P, I64, I64, I32, P, P, P, P]
     L.ftk_set_stage_events.restype = I32
     L.ftk_set_stage_events.argtypes = [P, I32]
+    L.ftk_block_bound.restype = I32
+    L.ftk_block_bound.argtypes = [I32, P, P, P, P, I64, I64, P, I64, P, SZ, P]
+    L.ftk_block_bound_workspace_size.restype = SZ
+    L.ftk_block_bound_workspace_size.argtypes = [I64]
     L.ftk_status_string.restype = ctypes.c_char_p
     L.ftk_status_string.argtypes = [I32]
     L.ftk_version.restype = I32
@@ -135,7 +140,6 @@ def _config(cfg: dict | None):
     if not cfg:
         return None
     c = FtkConfig()
-    c.prune = -1
     for k, v in cfg.items():
         setattr(c, k, v)
     return c
@@ -189,7 +193,10 @@ def select(q, kv, weights, ks, ke, kv_scales=None, topk: int = 2048, return_scor
     return (out_idx, out_val) if return_scores else out_idx
 
 
-STAGES = ("plan", "sample", "threshold", "scan", "refine", "recovery")
+# Stage name -> (start event, end event), in the numbering of
+# ftk_set_stage_events (event 7 marks the end of the pruning kernels).
+STAGES = {"plan": (0, 1), "sample": (1, 2), "threshold": (2, 3), "prune": (3, 7), "scan": (7, 4),
+          "refine": (4, 5), "recovery": (5, 6)}
 
 
 class stage_events:
@@ -198,7 +205,7 @@ class stage_events:
     gives the duration of each stage of the last recorded call."""
 
     def __init__(self):
-        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(len(STAGES) + 1)]
+        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(8)]
         for e in self.events:  # torch creates the CUDA event on first record
             e.record()
         self._arr = (ctypes.c_void_p * len(self.events))(*[ctypes.c_void_p(e.cuda_event) for e in self.events])
@@ -212,7 +219,7 @@ class stage_events:
         return False
 
     def times_ms(self) -> dict:
-        return {name: self.events[i].elapsed_time(self.events[i + 1]) for i, name in enumerate(STAGES)}
+        return {name: self.events[a].elapsed_time(self.events[b]) for name, (a, b) in STAGES.items()}
 
 
 def read_info(workspace: torch.Tensor) -> dict:
@@ -307,4 +314,20 @@ def score_dense(q, kv, weights, ks, ke, kv_scales=None, rows: torch.Tensor | Non
                                _ptr(ke), T, S, _ptr(rows), nrows, _ptr(out), ld, _ptr(ws), ws.numel(),
                                _stream(dev))
     _check(st, "ftk_score_dense")
+    return out
+
+
+def block_bound(q, kv, weights, kv_scales=None) -> torch.Tensor:
+    """Score upper bound of every row over every 128-key block:
+    out[t, b] >= I[t, s] for all keys s of block b (float32, +inf for
+    blocks that can never be skipped).  The bound select() prunes with."""
+    _need_cuda(q, kv, weights, kv_scales)
+    T, S = q.shape[0], kv.shape[0]
+    dev = q.device
+    nb = (S + 127) // 128
+    out = torch.empty((T, nb), dtype=torch.float32, device=dev)
+    ws = torch.empty(int(lib().ftk_block_bound_workspace_size(S)), dtype=torch.uint8, device=dev)
+    st = lib().ftk_block_bound(_dtype_code(q), _ptr(q), _ptr(kv), _ptr(kv_scales), _ptr(weights), T, S,
+                               _ptr(out), nb, _ptr(ws), ws.numel(), _stream(dev))
+    _check(st, "ftk_block_bound")
     return out

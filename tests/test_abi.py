@@ -66,6 +66,22 @@ def test_workspace_size(lib):
 A = 0x10000  # a 16-byte aligned stand-in pointer (never dereferenced on the host)
 
 
+def test_block_bound_host_validation(lib):
+    P = ctypes.c_void_p
+    need = lib.ftk_block_bound_workspace_size(1000)
+    assert need >= 8 * 257 * 4 and lib.ftk_block_bound_workspace_size(0) == 0
+
+    def call(dtype=1, q=A, kv=A, w=A, T=4, S=1000, out=A, ld=8, ws=A, wsz=None):
+        return lib.ftk_block_bound(dtype, P(q), P(kv), None, P(w), T, S, P(out), ld, P(ws),
+                                   need if wsz is None else wsz, None)
+    assert call(dtype=3) == -2
+    assert call(q=0) == -1 and call(out=0) == -1
+    assert call(T=0) == -1 and call(S=0) == -1
+    assert call(ld=7) == -1                  # ld < ceil(S / 128)
+    assert call(kv=A + 8) == -4
+    assert call(ws=0) == -5 and call(ws=A + 16) == -5 and call(wsz=need - 1) == -5
+
+
 def test_topk_rows_host_validation(lib):
     P = ctypes.c_void_p
     assert lib.ftk_topk_rows(2, P(A), 4, 100, 104, 0, P(A), None, None, None) == -3

@@ -55,7 +55,8 @@ def run_and_compare(x_cpu: torch.Tensor, k: int, return_value=True, rows_subset=
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("rows,cols,k", [(1, 1, 1), (3, 7, 5), (5, 100, 100), (4, 1000, 37),
                                          (2, 5000, 4096), (9, 33333, 512), (300, 2048, 64),
-                                         (1, 393216, 4096), (2, 131072, 1)])
+                                         (1, 393216, 4096), (2, 131072, 1),
+                                         (1000, 3000, 64)])  # more rows than resident clusters
 def test_random_rows(dtype, rows, cols, k):
     g = torch.Generator().manual_seed(rows * 1000 + cols + k)
     x = torch.randn((rows, cols), generator=g).to(dtype)

@@ -123,7 +123,8 @@ def test_all_equal_workload_closed_form():
     dict(oversample=0.05),             # thresholds too high -> underflow -> recovery
     dict(sample_keys=64),              # coarse samples
     dict(recovery_rows=8, capacity=64),  # many recovery passes
-    dict(prune=0),
+    dict(prune=-1),
+    dict(prune=1),
 ])
 def test_config_does_not_change_the_result(config):
     c = wl.small_case(seed=11, dtype="fp8", T=29, S=9000, topk=64, windows="random")
