@@ -75,21 +75,43 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
+// try_wait that may suspend the thread in hardware (up to kSuspendNs) until
+// the phase completes, instead of returning at once: a waiting warp issues
+// almost nothing while it waits.
+constexpr uint32_t kSuspendNs = 100000;  // 100 us per try
+
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
+        : "memory");
+    return ok != 0;
+}
+
 // Waits for the phase with the given parity to complete.  Gives up (returns
 // false) when *abort becomes non-zero or after kWaitNs; a timeout sets
 // *abort and FTK_STATUS_TIMEOUT so that every other role bails out too.
+// The abort flag and the clock are looked at every 32 tries (each try is
+// itself bounded by kSuspendNs).
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
                                           uint32_t *status)
 {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity)) return true;
     const unsigned long long t0 = global_ns();
-    for (;;) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if (*abort) return false;
-        if (global_ns() - t0 > kWaitNs) {
-            *abort = 1;
-            set_status(status, FTK_STATUS_TIMEOUT);
-            return false;
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait_sleep(bar, parity)) return true;
+        if ((i & 31u) == 0) {
+            if (*abort) return false;
+            if (global_ns() - t0 > kWaitNs) {
+                *abort = 1;
+                set_status(status, FTK_STATUS_TIMEOUT);
+                return false;
+            }
         }
     }
 }

@@ -48,19 +48,20 @@ void rows_plan(int64_t rows, int64_t cols, int k, int *cluster, int *chunk)
 template <int DT>
 static ftk_status launch_rows_dt(const RowsArgs &a, int cluster, cudaStream_t stream)
 {
-    const size_t smem = sizeof(RowsSmem);
-    auto kern = rows_topk_kernel<DT>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return cuda_status(e);
-    // Clusters stride over the rows: at most as many as fit at once (two
-    // CTAs per SM).
+    // One cluster per row if they all fit at once (two CTAs per SM) and the
+    // row count is known here; else as many clusters as fit, striding.
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    int64_t nclusters = 2 * static_cast<int64_t>(sms) / cluster;
-    if (nclusters < 1) nclusters = 1;
-    if (a.rows < nclusters) nclusters = a.rows;
+    int64_t fit = 2 * static_cast<int64_t>(sms) / cluster;
+    if (fit < 1) fit = 1;
+    const bool loop = a.nrows_dev != nullptr || a.rows > fit;
+    const int64_t nclusters = loop ? (a.rows < fit ? a.rows : fit) : a.rows;
+    const size_t smem = sizeof(RowsSmem);
+    auto kern = loop ? rows_topk_kernel<DT, true> : rows_topk_kernel<DT, false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return cuda_status(e);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(nclusters * cluster), 1, 1);
     cfg.blockDim = dim3(kRowsThreads, 1, 1);

@@ -676,9 +676,10 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
     cluster_wait();  // keep my shared memory alive until every CTA is done with it
 }
 
-// One cluster per row at a time; clusters stride over the rows (the count
-// may be on the device), so a grid sized for the SMs serves any row count.
-template <int DT>
+// One cluster per row.  LOOP: clusters stride over the rows (the count may
+// be on the device), so a grid sized for the SMs serves any row count;
+// otherwise the grid holds one cluster per row.
+template <int DT, bool LOOP>
 __global__ void __launch_bounds__(kRowsThreads, 2) rows_topk_kernel(const RowsArgs a)
 {
     extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -692,10 +693,15 @@ __global__ void __launch_bounds__(kRowsThreads, 2) rows_topk_kernel(const RowsAr
         nrows = c < nrows ? c : nrows;
     }
     // Row selection is uniform over the cluster: its CTAs walk the same rows.
-    for (int64_t r = blockIdx.x / cs; r < nrows; r += gridDim.x / cs) {
-        rows_topk_row<DT>(a, sm, cluster, cs, rank, r);
-        cp_async_wait<0>();
-        __syncthreads();  // shared memory is free for the next row
+    if constexpr (!LOOP) {
+        const int64_t r = blockIdx.x / cs;
+        if (r < nrows) rows_topk_row<DT>(a, sm, cluster, cs, rank, r);
+    } else {
+        for (int64_t r = blockIdx.x / cs; r < nrows; r += gridDim.x / cs) {
+            rows_topk_row<DT>(a, sm, cluster, cs, rank, r);
+            cp_async_wait<0>();
+            __syncthreads();  // shared memory is free for the next row
+        }
     }
 }
 

@@ -102,7 +102,9 @@ struct ScoreArgs {
     // Schedule over row tiles of row_tile_of(dtype) rows.  Planned: per-tile
     // ranges and an item prefix written by the plan kernel.  Static: item =
     // (tile, chunk of keys), ranges found on the fly, chunk size chosen at
-    // kernel start from the rows in the list (make_sched).
+    // kernel start from the rows in the list (make_sched).  SAMPLE and
+    // COLLECT run planned, DUMP static.
+    int32_t planned;
     const int32_t *tile_lo, *tile_hi, *tile_lg, *item_start;
     int32_t ntiles;
     // COLLECT
@@ -182,10 +184,6 @@ struct Sched {
     int64_t tiles;       // row tiles in use (static)
 };
 
-// SAMPLE and COLLECT run planned schedules, DUMP a static one.
-template <int MODE>
-__device__ __forceinline__ constexpr bool planned_mode() { return MODE != MODE_DUMP; }
-
 template <int MODE, int RT>
 __device__ __forceinline__ Sched make_sched(const ScoreArgs &a, int64_t nlist)
 {
@@ -193,7 +191,7 @@ __device__ __forceinline__ Sched make_sched(const ScoreArgs &a, int64_t nlist)
     sc.tiles = (nlist + RT - 1) / RT;
     sc.chunk_keys = kChunkKeys;
     sc.chunks = 0;
-    if (!planned_mode<MODE>()) {
+    if (MODE == MODE_DUMP) {  // the one static-schedule mode
         const int64_t kt = (a.S + kKeyTile - 1) / kKeyTile + 1;  // + 1: the aligned start
         const int64_t want = 2 * static_cast<int64_t>(gridDim.x);
         int64_t ct = (sc.tiles * kt + want - 1) / want;
@@ -208,7 +206,7 @@ template <int MODE, int RT>
 __device__ __forceinline__ bool get_item(const ScoreArgs &a, const Sched &sc, int it, int64_t nlist,
                                          Item &m)
 {
-    if (planned_mode<MODE>()) {
+    if (a.planned) {
         const int32_t nt = a.ntiles;
         if (it >= a.item_start[nt]) return false;
         int lo = 0, hi = nt;  // largest tile with item_start[tile] <= it
@@ -256,7 +254,7 @@ __device__ __forceinline__ bool next_item(const ScoreArgs &a, const Sched &sc, i
                                           Item &m)
 {
     for (;; it += gridDim.x) {
-        if (planned_mode<MODE>()) {
+        if (a.planned) {
             if (it >= a.item_start[a.ntiles]) return false;
         } else {
             if (it >= static_cast<int64_t>(sc.chunks) * sc.tiles) return false;
@@ -376,19 +374,25 @@ static_assert(ScoreSmemLayout<FTK_F8E4M3>::kBytes <= 227 * 1024, "fp8 smem budge
 static_assert(ScoreSmemLayout<FTK_BF16>::kBytes <= 227 * 1024, "bf16 smem budget");
 static_assert(ScoreCfg<FTK_F8E4M3>::kKStages <= 4 && ScoreCfg<FTK_BF16>::kKStages <= 4, "barriers");
 
-template <int DT, int MODE>
+// PR: the scan skips pruned key tiles.  With pruning possible, both
+// COLLECT variants are launched and the one that does not match the
+// device-side decision (*prune_on) returns at once, so an unpruned scan runs
+// exactly the plain tile loop.
+template <int DT, int MODE, bool PR>
 __global__ void __launch_bounds__(kScoreThreads, 1)
     score_kernel(const __grid_constant__ ScoreArgs a, const __grid_constant__ CUtensorMap tm_q,
                  const __grid_constant__ KvMaps kvm)
 {
+    if (MODE == MODE_COLLECT && a.prune_bits != nullptr && ((*a.prune_on != 0) != PR)) return;
     using C = ScoreCfg<DT>;
     using Lay = ScoreSmemLayout<DT>;
     constexpr int QG = C::kQG;
     constexpr int RT = QG * kQTile;  // rows per work item
     extern __shared__ uint8_t smem_dyn[];
     // 1024-byte alignment: the 128-byte swizzle pattern repeats every 8 rows.
-    uint8_t *smem = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~static_cast<uintptr_t>(1023));
+    // (Offsetting the __shared__ array itself keeps every derived pointer
+    // visibly in shared memory, so its loads and stores stay shared-space.)
+    uint8_t *smem = smem_dyn + ((1024u - (smem_u32(smem_dyn) & 1023u)) & 1023u);
     uint8_t *sq = smem + Lay::kOffQ;
     uint8_t *sk = smem + Lay::kOffK;
     float *stage_val = reinterpret_cast<float *>(smem + Lay::kOffStageVal);
@@ -400,8 +404,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t nlist = list_rows(a);
     const Sched sc = make_sched<MODE, RT>(a, nlist);
-    // Key pruning on (the same value in every thread: set by an earlier kernel).
-    const bool pruned = MODE == MODE_COLLECT && a.prune_bits != nullptr && *a.prune_on != 0;
+    constexpr bool pruned = MODE == MODE_COLLECT && PR;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < C::kKStages; ++i) {

@@ -591,24 +591,24 @@ static bool carve_select(Carver &cv, int64_t T, int64_t S, const SelectCfg &c, S
     return cv.ok;
 }
 
-template <int DT, int MODE>
+template <int DT, int MODE, bool PR>
 static ftk_status launch_score(const ScoreArgs &a, const CUtensorMap &tq, const KvMaps &kvm,
                                int grid, cudaStream_t st)
 {
     const int smem = ScoreSmemLayout<DT>::kBytes;
-    auto kern = score_kernel<DT, MODE>;
+    auto kern = score_kernel<DT, MODE, PR>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_status(e);
     kern<<<grid, kScoreThreads, smem, st>>>(a, tq, kvm);
     return cuda_status(cudaGetLastError());
 }
 
-template <int MODE>
+template <int MODE, bool PR = false>
 static ftk_status launch_score_dt(int dtype, const ScoreArgs &a, const CUtensorMap &tq,
                                   const KvMaps &kvm, int grid, cudaStream_t st)
 {
-    if (dtype == FTK_F8E4M3) return launch_score<FTK_F8E4M3, MODE>(a, tq, kvm, grid, st);
-    return launch_score<FTK_BF16, MODE>(a, tq, kvm, grid, st);
+    if (dtype == FTK_F8E4M3) return launch_score<FTK_F8E4M3, MODE, PR>(a, tq, kvm, grid, st);
+    return launch_score<FTK_BF16, MODE, PR>(a, tq, kvm, grid, st);
 }
 
 static bool build_maps(int dtype, const void *q, const void *kv, int64_t T, int64_t S, int max_lg,
@@ -743,7 +743,7 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
     pa.cnt = w.cnt;
     pa.bad_count = w.bad_count;
     pa.info = w.info;
-    pa.launches = 5 + 2 * ((T + c.rec_rows - 1) / c.rec_rows) + (c.prune == PRUNE_OFF ? 0 : c.prune == PRUNE_AUTO ? 3 : 2);
+    pa.launches = 5 + 2 * ((T + c.rec_rows - 1) / c.rec_rows) + (c.prune == PRUNE_OFF ? 0 : c.prune == PRUNE_AUTO ? 4 : 2);
     plan_kernel<<<1, kPlanThreads, 0, s>>>(pa);
     if ((st = cuda_status(cudaGetLastError())) != FTK_OK) return st;
     stage_mark(1, s);
@@ -757,6 +757,7 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
     sa.ke = ke;
     sa.rows = nullptr;
     sa.nrows = T;
+    sa.planned = 1;
     sa.ntiles = ntiles;
     sa.status = status;
     // sample pass
@@ -853,8 +854,16 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
     sa.prune_bits = w.prune_bits;
     sa.prune_words = w.nwords;
     sa.prune_on = &w.info->info.prune_enabled;
-    st = launch_score_dt<MODE_COLLECT>(dtype, sa, tq, kvm, sms, s);
-    if (st != FTK_OK) return st;
+    // auto: both variants, the device-side decision picks one (the other
+    // returns at once); always: the pruned one; off: the plain one
+    if (c.prune != PRUNE_ON) {
+        st = launch_score_dt<MODE_COLLECT, false>(dtype, sa, tq, kvm, sms, s);
+        if (st != FTK_OK) return st;
+    }
+    if (c.prune != PRUNE_OFF) {
+        st = launch_score_dt<MODE_COLLECT, true>(dtype, sa, tq, kvm, sms, s);
+        if (st != FTK_OK) return st;
+    }
     stage_mark(4, s);
 
     RefineArgs ra;
