@@ -583,6 +583,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             int cnt[WQ];  // staged candidates per query (warp-uniform)
 #pragma unroll
             for (int qq = 0; qq < WQ; ++qq) cnt[qq] = 0;
+            bool flush_due = false;  // some staging could overflow within one more key tile
             // Keys are int32 (S < 2^31).  A query outside the list has the
             // empty window [0, 0).  In SAMPLE mode key j of the tile is
             // sample j, at kv row j << lg.
@@ -608,13 +609,16 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                 if (!skip) {
 #pragma unroll
                 for (int vt = 0; vt < QG; ++vt) {
-                    const bool got = mbar_wait(&ms.acc_full[ab], aph, abort, a.status);
+                    // With two query tiles per key tile, tile vt always uses
+                    // accumulator vt (every key tile consumes both).
+                    const int abx = QG == 2 ? vt : ab;
+                    const bool got = mbar_wait(&ms.acc_full[abx], aph, abort, a.status);
                     if (!__all_sync(0xFFFFFFFFu, got)) {  // also reconverges the warp
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t c0 = tlane + static_cast<uint32_t>(ab * 256 + qg * NQ * 32);
+                    const uint32_t c0 = tlane + static_cast<uint32_t>(abx * 256 + qg * NQ * 32);
                     const float *w0 = my_w + (vt * NQ) * kHeads;
                     uint64_t p01 = 0, p23 = 0, q01 = 0, q23 = 0;
 #pragma unroll
@@ -626,31 +630,52 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                             // accumulator back to the MMA warp.
                             tc_fence_before();
                             __syncwarp();
-                            if (lane == 0) mbar_arrive(&ms.acc_empty[ab]);
+                            if (lane == 0) mbar_arrive(&ms.acc_empty[abx]);
                         }
                         head_step2(xa, xb, w0, w0 + kHeads, hh * 16, p01, p23, q01, q23);
                     }
-                    if (++ab == 2) { ab = 0; aph ^= 1u; }
+                    if (QG == 2) {
+                        if (vt == 1) aph ^= 1u;
+                    } else if (++ab == 2) {
+                        ab = 0;
+                        aph ^= 1u;
+                    }
                     float I[NQ];
                     I[0] = head_finish(p01, p23, sigma);
                     I[1] = head_finish(q01, q23, sigma);
+                    if (MODE == MODE_COLLECT) {
+                        // Candidates are rare: one vote for both queries, the
+                        // staging only when some lane has one.
+                        bool take[NQ];
+                        bool anyt = false;
 #pragma unroll
-                    for (int qi = 0; qi < NQ; ++qi) {
-                        const int qq = vt * NQ + qi;
-                        // s in [wlo, wlo + wlen) as one unsigned compare
-                        const bool valid = static_cast<uint32_t>(s - wlo[qq]) < static_cast<uint32_t>(wlen[qq]);
-                        if (MODE == MODE_COLLECT) {
-                            const bool take = valid && !(I[qi] < qtau[qq]);  // NaN is kept, to be seen
-                            const uint32_t bal = __ballot_sync(0xFFFFFFFFu, take);
-                            if (bal) {
+                        for (int qi = 0; qi < NQ; ++qi) {
+                            const int qq = vt * NQ + qi;
+                            // s in [wlo, wlo + wlen) as one unsigned compare
+                            const bool valid = static_cast<uint32_t>(s - wlo[qq]) < static_cast<uint32_t>(wlen[qq]);
+                            take[qi] = valid && !(I[qi] < qtau[qq]);  // NaN is kept, to be seen
+                            anyt |= take[qi];
+                        }
+                        if (__any_sync(0xFFFFFFFFu, anyt)) {
+#pragma unroll
+                            for (int qi = 0; qi < NQ; ++qi) {
+                                const int qq = vt * NQ + qi;
+                                const uint32_t bal = __ballot_sync(0xFFFFFFFFu, take[qi]);
                                 const int pos = cnt[qq] + __popc(bal & lt_mask);
-                                if (take) {
+                                if (take[qi]) {
                                     my_sv[qq * C::kWarpStage + pos] = I[qi];
                                     my_si[qq * C::kWarpStage + pos] = s;
                                 }
                                 cnt[qq] += __popc(bal);
+                                flush_due |= cnt[qq] > C::kWarpStage - 32;
                             }
-                        } else if (MODE == MODE_SAMPLE) {
+                        }
+                    }
+#pragma unroll
+                    for (int qi = 0; qi < (MODE == MODE_COLLECT ? 0 : NQ); ++qi) {
+                        const int qq = vt * NQ + qi;
+                        const bool valid = static_cast<uint32_t>(s - wlo[qq]) < static_cast<uint32_t>(wlen[qq]);
+                        if (MODE == MODE_SAMPLE) {
                             if (qt[qq] >= 0 && kidx < m.kend)
                                 a.out[static_cast<int64_t>(qt[qq]) * a.ld + (kidx - m.key0)] =
                                     valid ? I[qi] : -INFINITY;
@@ -661,15 +686,16 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                 }
                 }
                 if (MODE == MODE_COLLECT && ok) {
-                    // Every 2 key tiles (<= 2 * 32 new entries per warp and
-                    // query) and at the item's end, flush the queries whose
-                    // staging could otherwise overflow.
+                    // A key tile adds <= 32 entries per warp and query: flush
+                    // the queries whose staging could overflow in the next
+                    // tile, and everything at the item's end.
                     const bool last = kt == m.nkt - 1;
-                    if (last || (kt & 1) == 1) {
+                    if (last || flush_due) {
+                        flush_due = false;
                         bool need[WQ], any = false;
 #pragma unroll
                         for (int qq = 0; qq < WQ; ++qq) {
-                            need[qq] = cnt[qq] > 0 && (last || cnt[qq] > C::kWarpStage - 2 * 32);
+                            need[qq] = cnt[qq] > 0 && (last || cnt[qq] > C::kWarpStage - 32);
                             any |= need[qq];
                         }
                         if (any) {
