@@ -275,27 +275,6 @@ __device__ __forceinline__ void ffma2(uint64_t &acc, uint64_t a, uint64_t b)
     asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
 }
 
-// The head reduction of one (query, key) pair: sum_h w_h * max(x_h, 0) as
-// four partial sums over h = 0, 1, 2, 3 (mod 4), each a chain of
-// correctly rounded fmas (two packed lanes per instruction), combined as
-// (p0 + p1) + (p2 + p3); then sigma, with +0.0 added so that a -0.0 becomes
-// +0.0.  Every mode and every caller uses exactly this arithmetic.
-__device__ __forceinline__ float head_reduce(const float (&x)[32], const float *w, float sigma)
-{
-    uint64_t p01 = 0, p23 = 0;  // (+0.0, +0.0)
-#pragma unroll
-    for (int h = 0; h < 32; h += 4) {
-        const ulonglong2 wv = *reinterpret_cast<const ulonglong2 *>(w + h);
-        ffma2(p01, wv.x, pack2(fmaxf(x[h + 0], 0.f), fmaxf(x[h + 1], 0.f)));
-        ffma2(p23, wv.y, pack2(fmaxf(x[h + 2], 0.f), fmaxf(x[h + 3], 0.f)));
-    }
-    float a0, a1, a2, a3;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(p01));
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(a2), "=f"(a3) : "l"(p23));
-    const float acc = __fadd_rn(__fadd_rn(a0, a1), __fadd_rn(a2, a3));
-    return __fmaf_rn(sigma, acc, 0.0f);
-}
-
 // ReLU on the ALU pipe: max(x, 0), NaN propagating.
 __device__ __forceinline__ float relu_alu(float x)
 {
@@ -308,38 +287,40 @@ __device__ __forceinline__ float relu_alu(float x)
 // weight is pre-halved, so (w/2) * (x + |x|) is bit for bit w * ReLU(x).
 __device__ __forceinline__ float relu2_fma(float x) { return __fadd_rn(x, fabsf(x)); }
 
-// One step of the head reduction of two queries over heads h0 .. h0+15:
-// xa / xb hold those 16 columns of query 0 / 1, w0 / w1 point at the
-// queries' 32 weights as stored (heads = 2, 3 mod 4 pre-halved).  Four fma
-// chains (query 0 heads = 0,1 | 2,3 mod 4, query 1 likewise) advance in
-// head order, so after both halves each query's value is exactly
-//   sum over chains c of (sum_{h = c mod 4, in order} w_h * ReLU(x_h)).
-// Half of the ReLUs run on the ALU pipe and half on the FMA pipe.
+// The head reduction of a (query, key) pair, sum_h w_h * max(x_h, 0): one
+// packed fma chain per query whose two lanes hold the even and the odd
+// heads, each advancing in head order with correctly rounded fmas, so that
+//   I = sigma * (sum_{h even} w_h ReLU(x_h) + sum_{h odd} w_h ReLU(x_h)) + 0.0
+// (the +0.0 turns a -0.0 into +0.0).  Every mode (sample, scan, dump) runs
+// exactly this arithmetic, so the three see the same bits.
+//
+// One step covers two queries and heads h0 .. h0+15: xa / xb hold those 16
+// columns of query 0 / 1, w0 / w1 point at the queries' 32 weights as
+// stored (heads = 2, 3 mod 4 pre-halved).  Half of the ReLUs run on the ALU
+// pipe and half on the FMA pipe.
 __device__ __forceinline__ void head_step2(const float (&xa)[16], const float (&xb)[16],
                                            const float *w0, const float *w1, int h0,
-                                           uint64_t &p01, uint64_t &p23, uint64_t &q01,
-                                           uint64_t &q23)
+                                           uint64_t &p, uint64_t &q)
 {
 #pragma unroll
     for (int h = 0; h < 16; h += 4) {
         const ulonglong2 wv = *reinterpret_cast<const ulonglong2 *>(w0 + h0 + h);
         const ulonglong2 wu = *reinterpret_cast<const ulonglong2 *>(w1 + h0 + h);
-        ffma2(p01, wv.x, pack2(relu_alu(xa[h + 0]), relu_alu(xa[h + 1])));
-        ffma2(q01, wu.x, pack2(relu_alu(xb[h + 0]), relu_alu(xb[h + 1])));
-        ffma2(p23, wv.y, pack2(relu2_fma(xa[h + 2]), relu2_fma(xa[h + 3])));
-        ffma2(q23, wu.y, pack2(relu2_fma(xb[h + 2]), relu2_fma(xb[h + 3])));
+        ffma2(p, wv.x, pack2(relu_alu(xa[h + 0]), relu_alu(xa[h + 1])));
+        ffma2(q, wu.x, pack2(relu_alu(xb[h + 0]), relu_alu(xb[h + 1])));
+        ffma2(p, wv.y, pack2(relu2_fma(xa[h + 2]), relu2_fma(xa[h + 3])));
+        ffma2(q, wu.y, pack2(relu2_fma(xb[h + 2]), relu2_fma(xb[h + 3])));
     }
 }
 
 // Stored weight of head h: heads = 2, 3 (mod 4) are halved (see head_step2).
 __device__ __forceinline__ float stored_weight(float w, int h) { return (h & 2) ? 0.5f * w : w; }
 
-__device__ __forceinline__ float head_finish(uint64_t p01, uint64_t p23, float sigma)
+__device__ __forceinline__ float head_finish(uint64_t p, float sigma)
 {
-    float a0, a1, a2, a3;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(p01));
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(a2), "=f"(a3) : "l"(p23));
-    return __fmaf_rn(sigma, __fadd_rn(__fadd_rn(a0, a1), __fadd_rn(a2, a3)), 0.0f);
+    float even, odd;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(even), "=f"(odd) : "l"(p));
+    return __fmaf_rn(sigma, __fadd_rn(even, odd), 0.0f);
 }
 
 template <int DT>
@@ -600,8 +581,12 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                 const float sigma = sig_next;
                 kidx_next += kKeyTile;
                 if (scales && kt + 1 < m.nkt) {  // sigma one tile ahead
-                    const int64_t s1 = static_cast<int64_t>(kidx_next) << m.lg;
-                    sig_next = (kidx_next < m.kend && s1 < a.S) ? __ldg(scales + s1) : 1.f;
+                    if (MODE == MODE_SAMPLE) {
+                        const int64_t s1 = static_cast<int64_t>(kidx_next) << m.lg;
+                        sig_next = (kidx_next < m.kend && s1 < a.S) ? __ldg(scales + s1) : 1.f;
+                    } else {  // unit stride, kend <= S
+                        sig_next = kidx_next < m.kend ? __ldg(scales + kidx_next) : 1.f;
+                    }
                 }
                 const bool skip = pruned && tile_pruned(a, m, kt);  // warp-uniform
                 bad_scale |= !skip && scales && kidx < m.kend && (!(sigma > 0.f) || isinf(sigma));
@@ -620,7 +605,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                     tc_fence_after();
                     const uint32_t c0 = tlane + static_cast<uint32_t>(abx * 256 + qg * NQ * 32);
                     const float *w0 = my_w + (vt * NQ) * kHeads;
-                    uint64_t p01 = 0, p23 = 0, q01 = 0, q23 = 0;
+                    uint64_t p = 0, q = 0;  // (+0.0, +0.0)
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
                         float xa[16], xb[16];
@@ -632,7 +617,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                             __syncwarp();
                             if (lane == 0) mbar_arrive(&ms.acc_empty[abx]);
                         }
-                        head_step2(xa, xb, w0, w0 + kHeads, hh * 16, p01, p23, q01, q23);
+                        head_step2(xa, xb, w0, w0 + kHeads, hh * 16, p, q);
                     }
                     if (QG == 2) {
                         if (vt == 1) aph ^= 1u;
@@ -641,8 +626,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                         aph ^= 1u;
                     }
                     float I[NQ];
-                    I[0] = head_finish(p01, p23, sigma);
-                    I[1] = head_finish(q01, q23, sigma);
+                    I[0] = head_finish(p, sigma);
+                    I[1] = head_finish(q, sigma);
                     if (MODE == MODE_COLLECT) {
                         // Candidates are rare: one vote for both queries, the
                         // staging only when some lane has one.
