@@ -279,7 +279,7 @@ def run_ours(args):
     dev = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(dev)
 
-    from sparse_attention_indexer_ftk_b200 import ftk
+    from sparse_attention_indexer_ftk_b200 import ftk, shard
     from sparse_attention_indexer_ftk_b200 import workloads as wl
 
     c = wl.get(WORKLOAD)
@@ -329,11 +329,7 @@ def run_ours(args):
     mean_ms = sum(step_ms) / K
     stages = [s.times_ms() for s in stage_evs]
     stage_mean = {name: sum(s[name] for s in stages) / K for name in stages[0]}
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([mean_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        mean_ms = float(t.item())
+    mean_ms = shard.max_over_ranks(mean_ms, dev)  # the step time is the slowest rank's
 
     # end to end through the public API: inputs from pinned host memory,
     # results back to pinned host memory, every step.
@@ -359,10 +355,7 @@ def run_ours(args):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / E
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = shard.max_over_ranks(e2e_ms, dev)
 
     if rank != 0:
         if world > 1:
