@@ -290,7 +290,20 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const ThreshArgs
         return;
     }
     const float *row = p.samp + t * p.sld;
-    for (int i = threadIdx.x; i < J; i += blockDim.x) tkeys[i] = f32_key(__float_as_uint(row[i]));
+    // Eight loads in flight per thread, then the conversions.
+    for (int i0 = 0; i0 < J; i0 += 8 * kSelThreads) {
+        uint32_t v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int i = i0 + j * kSelThreads + threadIdx.x;
+            v[j] = i < J ? __float_as_uint(__ldg(row + i)) : 0u;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int i = i0 + j * kSelThreads + threadIdx.x;
+            if (i < J) tkeys[i] = f32_key(v[j]);
+        }
+    }
     __syncthreads();
     uint32_t gt;
     const uint32_t u = block_kth_largest(J, static_cast<uint32_t>(r), [&](int i) { return tkeys[i]; }, ss, &gt);
@@ -361,11 +374,25 @@ __global__ void __launch_bounds__(kSelThreads) refine_kernel(const RefineArgs p)
     const float *cv = p.cand_val + t * p.cap;
     const int32_t *ci = p.cand_idx + t * p.cap;
     bool nan = false;
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-        const uint32_t bits = __float_as_uint(cv[i]);
-        nan |= f32_bits_isnan(bits);
-        keys[i] = f32_key(bits);
-        idx[i] = ci[i];
+    // Eight (value, index) loads in flight per thread, then the stores.
+    for (int i0 = 0; i0 < n; i0 += 8 * kSelThreads) {
+        uint32_t v[8];
+        int32_t x[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int i = i0 + j * kSelThreads + threadIdx.x;
+            v[j] = i < n ? __float_as_uint(__ldg(cv + i)) : 0u;
+            x[j] = i < n ? __ldg(ci + i) : 0;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int i = i0 + j * kSelThreads + threadIdx.x;
+            if (i < n) {
+                nan |= f32_bits_isnan(v[j]);
+                keys[i] = f32_key(v[j]);
+                idx[i] = x[j];
+            }
+        }
     }
     if (nan) nan_seen = 1;
     if (threadIdx.x == 0) {
