@@ -463,32 +463,58 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
         // into its own shared memory once and selects locally (identical
         // result in every CTA, no cluster barrier between passes).
         uint32_t off = 0;  // start of list (rr, warp) in gath
+        uint32_t kmn = 0xFFFFFFFFu, kmx = 0u;  // bounds of the gathered keys
         for (unsigned rr = 0; rr < cs; ++rr) {
             const RowsSmem *o = cluster.map_shared_rank(&sm, rr);
             uint32_t before = 0;
             for (int ww = 0; ww < warp; ++ww) before += o->warp_cnt[ww];
             const uint32_t cnt = o->warp_cnt[warp];
             const uint32_t *cb = o->cand_bits + warp * kRowsCapWarp;
-            for (uint32_t i = lane; i < cnt; i += 32) gath[off + before + i] = Tr::key(cb[i]);
+            for (uint32_t i = lane; i < cnt; i += 32) {
+                const uint32_t u = Tr::key(cb[i]);
+                gath[off + before + i] = u;
+                kmn = min(kmn, u);
+                kmx = max(kmx, u);
+            }
             off += o->cta_cnt;
         }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            kmn = min(kmn, __shfl_xor_sync(0xFFFFFFFFu, kmn, o));
+            kmx = max(kmx, __shfl_xor_sync(0xFFFFFFFFu, kmx, o));
+        }
+        if (lane == 0) {
+            sm.tot[warp] = kmn;
+            sm.tot[kRowsWarps + warp] = kmx;
+        }
         __syncthreads();
-        uint32_t prefix = 0, mask = 0, krem = static_cast<uint32_t>(k);
-        for (int p = 0; p < passes; ++p) {
-            const int shift = 24 - 8 * p;
+        for (int ww = 0; ww < kRowsWarps; ++ww) {
+            kmn = min(kmn, sm.tot[ww]);
+            kmx = max(kmx, sm.tot[kRowsWarps + ww]);
+        }
+        // Bits above the highest one where the keys differ are common to
+        // all of them: the 8-bit radix digits start below those.
+        const int lo_bit = 32 - 8 * passes;  // bf16 keys sit in the upper half
+        const uint32_t diff = kmn ^ kmx;
+        const int top = diff ? 31 - __clz(diff) : -1;
+        uint32_t mask = top < 0 ? 0xFFFFFFFFu : (top == 31 ? 0u : ~((2u << top) - 1u));
+        uint32_t prefix = kmx & mask, krem = static_cast<uint32_t>(k);
+        for (int hi = top; hi >= lo_bit; hi -= 8) {
+            const int shift = hi - 7 >= lo_bit ? hi - 7 : lo_bit;
+            const uint32_t dmask = (2u << (hi - shift)) - 1u;
             for (int b = tid; b < 256; b += blockDim.x) sm.hist[b] = 0;
             __syncthreads();
             for (uint32_t i0 = 0; i0 < total; i0 += blockDim.x) {
                 const uint32_t i = i0 + tid;
                 const uint32_t u = i < total ? gath[i] : 0u;
-                hist_add(sm.hist, (u >> shift) & 255u, i < total && (u & mask) == prefix);
+                hist_add(sm.hist, (u >> shift) & dmask, i < total && (u & mask) == prefix);
             }
             __syncthreads();
             for (int b = tid; b < 256; b += blockDim.x) sm.tot[b] = sm.hist[b];
             __syncthreads();
             find_kth_bin256(sm, krem);
             prefix |= sm.sel_bin << shift;
-            mask |= 255u << shift;
+            mask |= dmask << shift;
             krem -= sm.sel_above;
             above += sm.sel_above;
             __syncthreads();

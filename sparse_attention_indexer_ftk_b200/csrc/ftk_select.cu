@@ -183,18 +183,26 @@ struct SelShared {
 
 // The k-th largest (1 <= k <= count of keys) of key(i), i < n, where key
 // is any functor.  *gt receives how many keys are strictly larger.
-// Block-wide; must be called by every thread of the block.
+// kmin / kmax, if given, bound every key: the bits above the highest bit
+// where they differ are common to all keys, and the radix passes (8-bit
+// digits) start below them.  Block-wide; every thread of the block calls it.
 template <class KeyFn>
-__device__ uint32_t block_kth_largest(int n, uint32_t k, KeyFn key, SelShared &ss, uint32_t *gt)
+__device__ uint32_t block_kth_largest(int n, uint32_t k, KeyFn key, SelShared &ss, uint32_t *gt,
+                                      uint32_t kmin = 0u, uint32_t kmax = 0xFFFFFFFFu)
 {
-    uint32_t prefix = 0, mask = 0, above_total = 0;
+    const uint32_t diff = kmin ^ kmax;
+    const int top = diff ? 31 - __clz(diff) : -1;  // highest bit where keys may differ
+    uint32_t mask = top < 0 ? 0xFFFFFFFFu : (top == 31 ? 0u : ~((2u << top) - 1u));
+    uint32_t prefix = kmax & mask, above_total = 0;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int hi = top; hi >= 0; hi -= 8) {
+        const int shift = hi >= 7 ? hi - 7 : 0;
+        const uint32_t dmask = (2u << (hi - shift)) - 1u;  // digit of hi - shift + 1 <= 8 bits
         for (int b = tid; b < 256; b += blockDim.x) ss.hist[b] = 0;
         __syncthreads();
         for (int i = tid; i < n; i += blockDim.x) {
             const uint32_t u = key(i);
-            if ((u & mask) == prefix) atomicAdd(&ss.hist[(u >> shift) & 255u], 1u);
+            if ((u & mask) == prefix) atomicAdd(&ss.hist[(u >> shift) & dmask], 1u);
         }
         __syncthreads();
         if (warp == 0) {
@@ -227,7 +235,7 @@ __device__ uint32_t block_kth_largest(int n, uint32_t k, KeyFn key, SelShared &s
         __syncthreads();
         const uint32_t bin = ss.bin;
         prefix |= bin << shift;
-        mask |= 255u << shift;
+        mask |= dmask << shift;
         k -= ss.above;
         above_total += ss.above;
         __syncthreads();
@@ -374,6 +382,7 @@ __global__ void __launch_bounds__(kSelThreads) refine_kernel(const RefineArgs p)
     const float *cv = p.cand_val + t * p.cap;
     const int32_t *ci = p.cand_idx + t * p.cap;
     bool nan = false;
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;  // bounds of the keys, for the radix select
     // Eight (value, index) loads in flight per thread, then the stores.
     for (int i0 = 0; i0 < n; i0 += 8 * kSelThreads) {
         uint32_t v[8];
@@ -389,8 +398,11 @@ __global__ void __launch_bounds__(kSelThreads) refine_kernel(const RefineArgs p)
             const int i = i0 + j * kSelThreads + threadIdx.x;
             if (i < n) {
                 nan |= f32_bits_isnan(v[j]);
-                keys[i] = f32_key(v[j]);
+                const uint32_t u = f32_key(v[j]);
+                keys[i] = u;
                 idx[i] = x[j];
+                kmin = min(kmin, u);
+                kmax = max(kmax, u);
             }
         }
     }
@@ -401,15 +413,30 @@ __global__ void __launch_bounds__(kSelThreads) refine_kernel(const RefineArgs p)
         atomicMax(reinterpret_cast<unsigned long long *>(&p.info->info.candidates_max),
                   static_cast<unsigned long long>(n));
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        kmin = min(kmin, __shfl_xor_sync(0xFFFFFFFFu, kmin, o));
+        kmax = max(kmax, __shfl_xor_sync(0xFFFFFFFFu, kmax, o));
+    }
+    if ((threadIdx.x & 31) == 0) {
+        ss.red[threadIdx.x >> 5] = kmin;
+        ss.red[32 + (threadIdx.x >> 5)] = kmax;
+    }
     __syncthreads();
     if (nan_seen && threadIdx.x == 0) atomicOr(&p.info->info.status, FTK_STATUS_NAN);
+    for (int w = 0; w < kSelThreads / 32; ++w) {
+        kmin = min(kmin, ss.red[w]);
+        kmax = max(kmax, ss.red[32 + w]);
+    }
+    __syncthreads();  // ss.red is free again
 
     // Threshold key u* and the tie cut idx*: selected = key > u*, or
     // key == u* and index <= idx* (the smallest indices among the ties).
     uint32_t ustar = 0, idxcut = 0xFFFFFFFFu;
     if (n > k) {
         uint32_t gt;
-        ustar = block_kth_largest(n, static_cast<uint32_t>(k), [&](int i) { return keys[i]; }, ss, &gt);
+        ustar = block_kth_largest(n, static_cast<uint32_t>(k), [&](int i) { return keys[i]; }, ss, &gt,
+                                  kmin, kmax);
         const uint32_t need = static_cast<uint32_t>(k) - gt;
         uint32_t eq = 0;
         for (int i = threadIdx.x; i < n; i += blockDim.x) eq += keys[i] == ustar;
