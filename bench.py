@@ -256,6 +256,25 @@ def bench_rows(name: str, dev, reps: int = 64):
     torch.cuda.synchronize()
     ms = sorted(a.elapsed_time(b) for a, b in evs)
     mean = sum(ms) / reps
+
+    def timed(fn, rotate: bool) -> float:
+        """Mean ms per call of fn(input) over `reps` calls (rotating copies or one)."""
+        for i in range(3):
+            fn(xs[i % ncopy] if rotate else xs[0])
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for i in range(reps):
+            ev[i][0].record()
+            fn(xs[i % ncopy] if rotate else xs[0])
+            ev[i][1].record()
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in ev) / reps
+
+    # The same call with its input resident in L2 (labelled as such), and the
+    # bandwidth a trivial read-reduce reaches over the same bytes from HBM
+    # (torch.amax: a reference measurement only, not part of the product).
+    warm = timed(lambda t: ftk.topk_rows(t, c.topk, out_idx=oi, out_val=ov), rotate=False)
+    rr = timed(lambda t: torch.amax(t), rotate=True)
     peaks, src = measured_peaks()
     gbs = (in_bytes + out_bytes) / (mean * 1e-3) / 1e9
     return {"workload": name, "rows": rows, "cols": cols, "topk": c.topk, "dtype": str(x.dtype),
@@ -263,6 +282,11 @@ def bench_rows(name: str, dev, reps: int = 64):
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / peaks["hbm_gbs"], "bytes_per_call": in_bytes + out_bytes,
                          "peak_source": src},
+            "us_per_call_warm_l2": warm * 1e3,
+            "read_reduce_baseline": {"op": "torch.amax over the same rotating inputs",
+                                     "us_per_call": rr * 1e3,
+                                     "gbs": in_bytes / (rr * 1e-3) / 1e9,
+                                     "frac": in_bytes / (rr * 1e-3) / 1e9 / peaks["hbm_gbs"]},
             "inputs": f"{ncopy} rotating copies (> L2) so every call reads from HBM"}
 
 
@@ -398,7 +422,8 @@ def run_ours(args):
         "clocks": clocks,
     }
     if world == 1 and not args.no_rows:
-        out["row_topk"] = [bench_rows("rows_bf16", dev), bench_rows("rows_f32", dev)]
+        out["row_topk"] = [bench_rows("rows_bf16", dev), bench_rows("rows_f32", dev),
+                           bench_rows("rows_bf16_1024", dev, reps=16)]
     if world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(c, args.cpu_seconds)
     print(json.dumps(out), flush=True)
@@ -410,8 +435,9 @@ def main():
     args = parse_args()
     if args.only_rows:
         import torch
-        print(json.dumps({"row_topk": [bench_rows("rows_bf16", torch.device("cuda")),
-                                       bench_rows("rows_f32", torch.device("cuda"))]}), flush=True)
+        dev = torch.device("cuda")
+        print(json.dumps({"row_topk": [bench_rows("rows_bf16", dev), bench_rows("rows_f32", dev),
+                                       bench_rows("rows_bf16_1024", dev, reps=16)]}), flush=True)
         return
     if args.impl == "reference":
         run_reference(args)

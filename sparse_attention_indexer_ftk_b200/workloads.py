@@ -176,6 +176,15 @@ def rows_bf16() -> RowsInputs:
     return RowsInputs("rows_bf16", x, 512)
 
 
+def rows_bf16_1024() -> RowsInputs:
+    """A scaled-up copy of rows_bf16 (1024 rows, 268 MB): not one of the
+    pages' configurations; it shows the row kernel where HBM bandwidth, not
+    launch and phase latency, decides."""
+    g = _gen(12)
+    x = _normal(g, (1024, 131072)).to(torch.bfloat16)
+    return RowsInputs("rows_bf16_1024", x, 512)
+
+
 def rows_f32() -> RowsInputs:
     g = _gen(2)
     torch.randn((1,), generator=g)
@@ -305,7 +314,7 @@ def get(name: str):
     """Workload by name."""
     table = {
         "bf16_small": bf16_small, "bf16_ties": bf16_ties, "bf16_all_equal": bf16_all_equal,
-        "rows_bf16": rows_bf16, "rows_f32": rows_f32,
+        "rows_bf16": rows_bf16, "rows_f32": rows_f32, "rows_bf16_1024": rows_bf16_1024,
         "fp8_prefill": fp8_prefill, "fp8_packed": fp8_packed, "fp8_large": fp8_large,
     }
     return table[name]()
