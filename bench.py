@@ -290,6 +290,38 @@ def bench_rows(name: str, dev, reps: int = 64):
             "inputs": f"{ncopy} rotating copies (> L2) so every call reads from HBM"}
 
 
+def bench_decode(c, dev, rows: int = 64, reps: int = 50):
+    """A decode-shaped call: the first `rows` query rows of the batch (each
+    with its long causal window) through the same ftk_select, inputs in
+    HBM, L2 flushed between calls.  Reported beside the metric, not as it."""
+    import torch
+    from sparse_attention_indexer_ftk_b200 import ftk
+    from sparse_attention_indexer_ftk_b200 import workloads as wl
+
+    d = wl.SelectInputs(c.name + f"[:{rows}]", c.q[:rows].contiguous(), c.kv, c.kv_scales,
+                        c.weights[:rows].contiguous(), c.ks[:rows].contiguous(),
+                        c.ke[:rows].contiguous(), c.topk).to(dev)
+    ws = torch.empty(ftk.select_workspace_size(d.T, d.S, d.topk), dtype=torch.uint8, device=dev)
+    oi = torch.empty((d.T, d.topk), dtype=torch.int32, device=dev)
+    ov = torch.empty((d.T, d.topk), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    step = lambda: ftk.select(d.q, d.kv, d.weights, d.ks, d.ke, d.kv_scales, d.topk, return_scores=True,
+                              workspace=ws, out_idx=oi, out_val=ov)
+    for _ in range(3):
+        step()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for i in range(reps):
+        flush.zero_()
+        ev[i][0].record()
+        step()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / reps
+    pairs = d.pairs()
+    return {"workload": d.name, "T": d.T, "S": d.S, "topk": d.topk, "ms_per_call": ms,
+            "queries_per_s": d.T / (ms * 1e-3), "dense_eq_tflops": 2.0 * 32 * 128 * pairs / (ms * 1e-3) / 1e12}
+
+
 def run_ours(args):
     import torch
 
@@ -421,6 +453,8 @@ def run_ours(args):
         "gpu_launches": int(info["kernel_launches"]) * K,
         "clocks": clocks,
     }
+    if world == 1:
+        out["decode_64q"] = bench_decode(c, dev)
     if world == 1 and not args.no_rows:
         out["row_topk"] = [bench_rows("rows_bf16", dev), bench_rows("rows_f32", dev),
                            bench_rows("rows_bf16_1024", dev, reps=16)]

@@ -105,6 +105,7 @@ struct ScoreArgs {
     // kernel start from the rows in the list (make_sched).  SAMPLE and
     // COLLECT run planned, DUMP static.
     int32_t planned;
+    int32_t chunk_keys;       // planned: keys (SAMPLE: samples) per work item, a multiple of 128
     const int32_t *tile_lo, *tile_hi, *tile_lg, *item_start;
     int32_t ntiles;
     // COLLECT
@@ -136,6 +137,7 @@ struct Item {
     int32_t kend;   // end key (SAMPLE: end sample index)
     int32_t nkt;    // key tiles in this item
     int32_t lg;     // SAMPLE: log2 of the stride
+    int32_t base;   // SAMPLE: first sample index of the tile (output column 0)
 };
 
 __device__ __forceinline__ int64_t list_rows(const ScoreArgs &a)
@@ -218,12 +220,13 @@ __device__ __forceinline__ bool get_item(const ScoreArgs &a, const Sched &sc, in
         const int chunk = it - a.item_start[lo];
         if (MODE == MODE_SAMPLE) {
             m.lg = a.tile_lg[lo];
-            m.key0 = a.tile_lo[lo];
-            m.kend = a.tile_hi[lo];
+            m.base = a.tile_lo[lo];
+            m.key0 = m.base + chunk * a.chunk_keys;
+            m.kend = min(a.tile_hi[lo], m.key0 + a.chunk_keys);
         } else {
             m.lg = 0;
-            m.key0 = a.tile_lo[lo] + chunk * kChunkKeys;
-            m.kend = min(a.tile_hi[lo], m.key0 + kChunkKeys);
+            m.key0 = a.tile_lo[lo] + chunk * a.chunk_keys;
+            m.kend = min(a.tile_hi[lo], m.key0 + a.chunk_keys);
         }
     } else {
         m.tile = it / sc.chunks;
@@ -662,7 +665,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                         const bool valid = static_cast<uint32_t>(s - wlo[qq]) < static_cast<uint32_t>(wlen[qq]);
                         if (MODE == MODE_SAMPLE) {
                             if (qt[qq] >= 0 && kidx < m.kend)
-                                a.out[static_cast<int64_t>(qt[qq]) * a.ld + (kidx - m.key0)] =
+                                a.out[static_cast<int64_t>(qt[qq]) * a.ld + (kidx - m.base)] =
                                     valid ? I[qi] : -INFINITY;
                         } else {
                             if (valid) a.out[static_cast<int64_t>(qpos[qq]) * a.ld + (s - wlo[qq])] = I[qi];

@@ -57,6 +57,8 @@ struct PlanArgs {
     int32_t ntiles;
     int32_t rt;               // rows per tile
     int32_t sample_keys;
+    int32_t chunk_keys;       // keys per scan work item
+    int32_t sample_chunk;     // samples per sample-pass work item
     // sample pass
     int32_t *s_lo, *s_hi, *s_lg, *s_start;
     // scan pass
@@ -141,11 +143,11 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanArgs p)
                 slo = static_cast<int32_t>(j0);
                 shi = static_cast<int32_t>(j1);
                 slg = lg;
-                ns = j1 > j0 ? 1u : 0u;
+                ns = j1 > j0 ? static_cast<uint32_t>((j1 - j0 + p.sample_chunk - 1) / p.sample_chunk) : 0u;
                 const int64_t lo_al = lo & ~static_cast<int64_t>(kKeyTile - 1);
                 clo = static_cast<int32_t>(lo_al);
                 chi = static_cast<int32_t>(hi);
-                nc = static_cast<uint32_t>((hi - lo_al + kChunkKeys - 1) / kChunkKeys);
+                nc = static_cast<uint32_t>((hi - lo_al + p.chunk_keys - 1) / p.chunk_keys);
                 nblocks += static_cast<unsigned long long>((hi - lo_al + kKeyTile - 1) / kKeyTile);
             }
             p.s_lo[tile] = slo;
@@ -787,6 +789,25 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
     pa.ntiles = ntiles;
     pa.rt = rt;
     pa.sample_keys = c.m;
+    // Scan work items: up to 128 key tiles each, fewer when the call is
+    // small (few query rows, decode-like) so that the items still cover
+    // every SM about twice.
+    {
+        const int64_t pairs = static_cast<int64_t>(ntiles) * ((S + kKeyTile - 1) / kKeyTile);
+        int64_t ct = pairs / (2 * static_cast<int64_t>(sms));
+        ct = ct < kMinChunkTiles ? kMinChunkTiles : (ct > kChunkTiles ? kChunkTiles : ct);
+        pa.chunk_keys = static_cast<int32_t>(ct * kKeyTile);
+        // The sample pass has one item per row tile; with fewer row tiles
+        // than SMs, its samples are split so the items cover the SMs twice.
+        int64_t sc = int64_t(1) << 30;
+        if (ntiles < sms) {
+            const int64_t pieces = (2 * static_cast<int64_t>(sms) + ntiles - 1) / ntiles;
+            sc = (c.m + pieces - 1) / pieces;
+            sc = (sc + kKeyTile - 1) / kKeyTile * kKeyTile;
+            if (sc < 4 * kKeyTile) sc = 4 * kKeyTile;
+        }
+        pa.sample_chunk = static_cast<int32_t>(sc);
+    }
     pa.s_lo = w.s_lo;
     pa.s_hi = w.s_hi;
     pa.s_lg = w.s_lg;
@@ -812,6 +833,7 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
     sa.rows = nullptr;
     sa.nrows = T;
     sa.planned = 1;
+    sa.chunk_keys = pa.sample_chunk;
     sa.ntiles = ntiles;
     sa.status = status;
     // sample pass
@@ -821,7 +843,7 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
     sa.item_start = w.s_start;
     sa.out = w.samp;
     sa.ld = w.sld;
-    st = launch_score_dt<MODE_SAMPLE>(dtype, sa, tq, kvm, sms < ntiles ? sms : ntiles, s);
+    st = launch_score_dt<MODE_SAMPLE>(dtype, sa, tq, kvm, sms, s);  // CTAs without an item exit
     if (st != FTK_OK) return st;
     stage_mark(2, s);
 
@@ -895,6 +917,7 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
     stage_mark(7, s);
 
     // scan
+    sa.chunk_keys = pa.chunk_keys;
     sa.tile_lo = w.c_lo;
     sa.tile_hi = w.c_hi;
     sa.tile_lg = nullptr;

@@ -83,6 +83,10 @@ SMALL = [
     dict(seed=7, dtype="fp8", T=8, S=40000, topk=2048, windows="causal"),
     dict(seed=8, dtype="bf16", T=3, S=129, topk=1, windows="causal", scales=False),
     dict(seed=9, dtype="fp8", T=12, S=20000, topk=4096, windows="random"),
+    # decode-shaped: a few query rows over long windows (split into many
+    # sample and scan work items, candidates merged across items)
+    dict(seed=11, dtype="fp8", T=3, S=100000, topk=2048, windows="causal"),
+    dict(seed=12, dtype="bf16", T=5, S=40000, topk=512, windows="random"),
 ]
 
 
