@@ -171,6 +171,20 @@ ftk_status ftk_topk_rows(ftk_dtype dtype, const void *x, int64_t rows,
                          void *stream);
 
 /*
+ * ftk_topk_rows_end -- ftk_topk_rows over variable-length rows (DeepSelect
+ * README, "Variable-length rows": a per-row exclusive end): row r holds
+ * only its columns [0, row_end[r]), row_end[r] clamped to [0, cols]; rows
+ * that end up shorter than topk are padded with index -1 and value -inf.
+ *   row_end   device [rows] int32 (must not be NULL)
+ * Other arguments, layout and errors as for ftk_topk_rows.
+ */
+ftk_status ftk_topk_rows_end(ftk_dtype dtype, const void *x, int64_t rows,
+                             int64_t cols, int64_t row_stride,
+                             const int32_t *row_end, int topk,
+                             int32_t *out_idx, void *out_val,
+                             uint32_t *status, void *stream);
+
+/*
  * ftk_score_dense -- the fused scores themselves, for checking: for each
  * listed row r (query t = rows ? rows[r] : r) writes
  *     out[r * ld + (s - ks[t])] = I[t, s]   for s in [ks[t], ke[t])

@@ -85,13 +85,9 @@ ftk_status launch_rows_topk(int dtype, const RowsArgs &a, int cluster, cudaStrea
     return FTK_ERR_UNSUPPORTED;
 }
 
-}  // namespace ftk
-
-using namespace ftk;
-
-extern "C" ftk_status ftk_topk_rows(ftk_dtype dtype, const void *x, int64_t rows, int64_t cols,
-                                    int64_t row_stride, int topk, int32_t *out_idx,
-                                    void *out_val, uint32_t *status, void *stream)
+static ftk_status topk_rows_impl(ftk_dtype dtype, const void *x, int64_t rows, int64_t cols,
+                                 int64_t row_stride, const int32_t *row_end, int topk,
+                                 int32_t *out_idx, void *out_val, uint32_t *status, void *stream)
 {
     if (dtype != FTK_BF16 && dtype != FTK_F32) return FTK_ERR_UNSUPPORTED;
     if (!x || !out_idx) return FTK_ERR_INVALID_ARG;
@@ -108,6 +104,7 @@ extern "C" ftk_status ftk_topk_rows(ftk_dtype dtype, const void *x, int64_t rows
     a.ld = row_stride;
     a.cols = cols;
     a.rows = rows;
+    a.row_end = row_end;
     a.out_idx = out_idx;
     a.out_val = out_val;
     a.k = topk;
@@ -116,4 +113,26 @@ extern "C" ftk_status ftk_topk_rows(ftk_dtype dtype, const void *x, int64_t rows
     rows_plan(rows, cols, topk, &cluster, &chunk);
     a.chunk = chunk;
     return launch_rows_topk(dtype, a, cluster, as_stream(stream));
+}
+
+}  // namespace ftk
+
+using namespace ftk;
+
+extern "C" ftk_status ftk_topk_rows(ftk_dtype dtype, const void *x, int64_t rows, int64_t cols,
+                                    int64_t row_stride, int topk, int32_t *out_idx,
+                                    void *out_val, uint32_t *status, void *stream)
+{
+    return topk_rows_impl(dtype, x, rows, cols, row_stride, nullptr, topk, out_idx, out_val, status,
+                          stream);
+}
+
+extern "C" ftk_status ftk_topk_rows_end(ftk_dtype dtype, const void *x, int64_t rows, int64_t cols,
+                                        int64_t row_stride, const int32_t *row_end, int topk,
+                                        int32_t *out_idx, void *out_val, uint32_t *status,
+                                        void *stream)
+{
+    if (!row_end) return FTK_ERR_INVALID_ARG;
+    return topk_rows_impl(dtype, x, rows, cols, row_stride, row_end, topk, out_idx, out_val, status,
+                          stream);
 }

@@ -50,6 +50,7 @@ struct RowsArgs {
     const int32_t *row_map;     // optional: output row of grid row r (also indexes win_*)
     const int32_t *win_ks;      // optional windows: row length ke - ks,
     const int32_t *win_ke;      //   reported index = ks + column
+    const int32_t *row_end;     // optional: row r holds columns [0, row_end[r]) (clamped to [0, cols])
     int32_t *out_idx;           // [*, k]
     void *out_val;              // [*, k] of the input dtype (or NULL)
     int k;
@@ -249,6 +250,10 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
         base_index = a.win_ks[orow];
         len = static_cast<int64_t>(a.win_ke[orow]) - base_index;
         if (len < 0) len = 0;
+    }
+    if (a.row_end) {
+        const int64_t e = a.row_end[orow];
+        len = e < 0 ? 0 : (e < len ? e : len);
     }
     const int k = a.k;
     const elem *row = reinterpret_cast<const elem *>(a.x) + r * a.ld;

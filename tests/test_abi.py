@@ -66,6 +66,14 @@ def test_workspace_size(lib):
 A = 0x10000  # a 16-byte aligned stand-in pointer (never dereferenced on the host)
 
 
+def test_topk_rows_end_host_validation(lib):
+    P = ctypes.c_void_p
+    assert lib.ftk_topk_rows_end(2, P(A), 4, 100, 104, None, 8, P(A), None, None, None) == -1
+    assert lib.ftk_topk_rows_end(2, P(A), 4, 100, 104, P(A), 0, P(A), None, None, None) == -3
+    assert lib.ftk_topk_rows_end(1, P(A), 4, 100, 104, P(A), 8, P(A), None, None, None) == -2
+    assert lib.ftk_topk_rows_end(2, P(A + 2), 4, 100, 104, P(A), 8, P(A), None, None, None) == -4
+
+
 def test_block_bound_host_validation(lib):
     P = ctypes.c_void_p
     need = lib.ftk_block_bound_workspace_size(1000)

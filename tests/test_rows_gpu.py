@@ -109,3 +109,35 @@ def test_full_size_workload(name):
     """The row top-k workload at full size (64 rows), every row bit-exact."""
     c = wl.get(name)
     assert run_and_compare(c.x, c.topk) == 0
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_variable_length_rows_end(dtype):
+    """ftk_topk_rows_end: row r is x[r, :end[r]] (end clamped to [0, cols]),
+    short rows padded with (-1, -inf) (DeepSelect README, "Variable-length
+    rows"); compared row by row with the oracle on the truncated rows."""
+    rows, cols, k = 40, 20000, 300
+    g = torch.Generator().manual_seed(77)
+    x_cpu = torch.randn((rows, cols), generator=g).to(dtype)
+    ends = torch.randint(0, cols + 1, (rows,), generator=g).to(torch.int32)
+    ends[:6] = torch.tensor([0, 1, k - 1, k, k + 1, cols], dtype=torch.int32)
+    ends[6] = cols + 500   # beyond the row: clamped to cols
+    ends[7] = -3           # negative: an empty row
+    x = aligned_rows(x_cpu)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    val, idx = ftk.topk_rows(x, k, status=status, end=ends.cuda())
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    idx, val = to_np(idx), val.cpu()
+    for r in range(rows):
+        e = max(0, min(int(ends[r]), cols))
+        check_row_invariants(idx[r], 0, e, k)
+        n = min(k, e)
+        if n:
+            oidx, _, _ = orc.topk_rows(x_cpu[r:r + 1, :e].contiguous(), k)
+            assert np.array_equal(idx[r, :n], np.sort(oidx[0, :n])), f"row {r}"
+            ref = x_cpu[r, idx[r, :n]]
+            bits = torch.int16 if dtype == torch.bfloat16 else torch.int32
+            assert torch.equal(val[r, :n].view(bits), ref.view(bits))
+        assert np.all(idx[r, n:] == -1)
+        assert torch.all(torch.isneginf(val[r, n:].float()))
