@@ -48,6 +48,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rows", action="store_true", help="skip the row top-k section")
     ap.add_argument("--only-rows", action="store_true", help="run only the row top-k section")
+    ap.add_argument("--no-decode", action="store_true", help="skip the 64-query (decode-shaped) section")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--rows", type=int, default=0,
                     help="use only the first ROWS queries of the batch (profiling captures)")
@@ -453,7 +454,7 @@ def run_ours(args):
         "gpu_launches": int(info["kernel_launches"]) * K,
         "clocks": clocks,
     }
-    if world == 1:
+    if world == 1 and not args.no_decode:
         out["decode_64q"] = bench_decode(c, dev)
     if world == 1 and not args.no_rows:
         out["row_topk"] = [bench_rows("rows_bf16", dev), bench_rows("rows_f32", dev),
