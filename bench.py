@@ -7,10 +7,17 @@ q [4096, 32, 128] and kv [131072, 128] FP8-e4m3 from N(0,1), kv_scales in
 topk 2048 -- seeded and synthetic (sparse_attention_indexer_ftk_b200.workloads).
 
 One step = one ftk_select call over the whole 4096-query batch (sample pass,
-thresholds, dense scan, refine, recovery).  Inputs are resident in HBM; the
-L2 is flushed (a 256 MB write) between timed steps, outside the timed events.
+thresholds, pruning decision, scan, refine, recovery).  Inputs are resident
+in HBM; the L2 is flushed (a 256 MB write) between timed steps, outside the
+timed events.  Beside the metric, on one GPU: per-stage times, the scan's
+roofline (with the DRAM traffic of the committed ncu summary while the
+kernel source is unchanged), an end-to-end figure through host buffers, a
+64-query (decode-shaped) call, the row top-k (ftk_topk_rows) on the 64-row
+bf16 / fp32 batches and a 1024-row bf16 batch with a warm-L2 time and a
+trivial read-reduce over the same bytes, and the CPU oracle's rate.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--no-rows] [--only-rows] [--no-decode] [--no-cpu-baseline]
 
 Multi-GPU (launched with torch.distributed.run): every rank runs its own
 independent batch of the same shape (weak scaling; no data-path collective);
@@ -22,7 +29,6 @@ from __future__ import annotations
 
 import argparse
 import json
-import math
 import os
 import statistics
 import subprocess
@@ -196,7 +202,7 @@ def run_reference(args):
 
     c = wl.get(WORKLOAD)
     threads = orc.num_threads()
-    per_step = max(1, threads // 4)
+    per_step = threads  # one query row per host thread: every core busy, a step ~ one row's time
     seed = 0
 
     def step():
@@ -221,8 +227,9 @@ def run_reference(args):
         "config": {"workload": WORKLOAD, "T": c.T, "S": c.S, "topk": c.topk, "dtype_in": "fp8_e4m3",
                    "rows_per_step": per_step, "l2": "host"},
         "dense_eq_tflops": value * pairs_per_row * 2 * 32 * 128 / 1e12,
-        "cpu_baseline": {"value": value, "unit": "queries/s", "cores": threads, "kind": "oracle",
-                         "sample": f"{per_step} seeded rows per step"},
+        "cpu_baseline": {"value": value, "unit": "queries/s", "cores": min(threads, per_step), "kind": "oracle",
+                         "sample": f"{per_step} seeded query rows per step (one per host thread), "
+                                   f"{rows} rows in {dt:.1f} s"},
         "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(out), flush=True)
