@@ -330,6 +330,66 @@ def bench_decode(c, dev, rows: int = 64, reps: int = 50):
             "queries_per_s": d.T / (ms * 1e-3), "dense_eq_tflops": 2.0 * 32 * 128 * pairs / (ms * 1e-3) / 1e12}
 
 
+def fp8_gemm_peak(dev, n: int = 8192, reps: int = 10):
+    """Dense FP8-e4m3 GEMM throughput of the vendor library on this GPU
+    (torch._scaled_mm, n x n x n, best of `reps`): a measured FP8
+    denominator reported beside the roofline's 2 x BF16 one.  A reference
+    measurement only; no part of the product calls it."""
+    import torch
+    try:
+        g = torch.Generator(device="cpu").manual_seed(1)
+        a = torch.randn((n, n), generator=g).to(dev).to(torch.float8_e4m3fn)
+        b = torch.randn((n, n), generator=g).to(dev).to(torch.float8_e4m3fn).t()
+        one = torch.ones((), dtype=torch.float32, device=dev)
+        mm = lambda: torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        for _ in range(3):
+            mm()
+        best = float("inf")
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            mm()
+            e1.record()
+            torch.cuda.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        return {"op": f"torch._scaled_mm e4m3 {n}^3, best of {reps}", "tflops": 2.0 * n ** 3 / (best * 1e-3) / 1e12}
+    except Exception as e:  # the library may not offer FP8 GEMMs here
+        return {"op": "torch._scaled_mm e4m3", "unavailable": str(e)[:200]}
+
+
+def bench_config(name: str, dev, reps: int = 10):
+    """One other workload through the same call: time per call, and the
+    pruning decision and pruned share of (row tile, key block) pairs."""
+    import torch
+    from sparse_attention_indexer_ftk_b200 import ftk
+    from sparse_attention_indexer_ftk_b200 import workloads as wl
+
+    d = wl.get(name).to(dev)
+    ws = torch.empty(ftk.select_workspace_size(d.T, d.S, d.topk), dtype=torch.uint8, device=dev)
+    oi = torch.empty((d.T, d.topk), dtype=torch.int32, device=dev)
+    ov = torch.empty((d.T, d.topk), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    step = lambda: ftk.select(d.q, d.kv, d.weights, d.ks, d.ke, d.kv_scales, d.topk, return_scores=True,
+                              workspace=ws, out_idx=oi, out_val=ov)
+    for _ in range(3):
+        step()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for i in range(reps):
+        flush.zero_()
+        ev[i][0].record()
+        step()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / reps
+    info = ftk.read_info(ws)
+    return {"workload": name, "T": d.T, "S": d.S, "topk": d.topk, "ms_per_call": ms,
+            "queries_per_s": d.T / (ms * 1e-3),
+            "dense_eq_tflops": 2.0 * 32 * 128 * d.pairs() / (ms * 1e-3) / 1e12,
+            "prune_enabled": info["prune_enabled"], "blocks_total": info["blocks_total"],
+            "blocks_pruned": info["blocks_pruned"],
+            "rows_recovered": info["rows_overflow"] + info["rows_underflow"]}
+
+
 def run_ours(args):
     import torch
 
@@ -433,6 +493,11 @@ def run_ours(args):
     achieved = scan_flops / (scan_ms * 1e-3) / 1e12
     traffic = profiled_traffic()
     value = world * T / (mean_ms * 1e-3)
+    # Executed work: every (16-row tile, 128-key block) pair the scan ran
+    # (in-window or not), i.e. minus the pruned ones.
+    rt = 16 if c.q.dtype == torch.float8_e4m3fn else 8
+    exec_pairs = (int(info["blocks_total"]) - int(info["blocks_pruned"])) * rt * 128
+    fp8_direct = fp8_gemm_peak(dev) if world == 1 else None
     out = {
         "metric": METRIC,
         "value": value,
@@ -455,7 +520,11 @@ def run_ours(args):
                      "achieved": achieved, "peak": fp8_peak, "unit": "TFLOP/s",
                      "frac": achieved / fp8_peak, "traffic": traffic,
                      "peak_source": f"2 x bf16_tflops ({peak_src}, burst) -- FP8 dense = 2 x BF16",
-                     "frac_of_sustained": achieved / (2.0 * peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))},
+                     "frac_of_sustained": achieved / (2.0 * peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])),
+                     "executed_tflops": 2.0 * 32 * 128 * exec_pairs / (scan_ms * 1e-3) / 1e12,
+                     "fp8_gemm_measured": fp8_direct,
+                     "frac_of_fp8_gemm_measured": (achieved / fp8_direct["tflops"])
+                     if fp8_direct and "tflops" in fp8_direct else None},
         "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": "queries/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": int(info["kernel_launches"]) * K,
@@ -463,6 +532,7 @@ def run_ours(args):
     }
     if world == 1 and not args.no_decode:
         out["decode_64q"] = bench_decode(c, dev)
+        out["fp8_packed"] = bench_config("fp8_packed", dev)
     if world == 1 and not args.no_rows:
         out["row_topk"] = [bench_rows("rows_bf16", dev), bench_rows("rows_f32", dev),
                            bench_rows("rows_bf16_1024", dev, reps=16)]
