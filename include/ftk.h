@@ -185,6 +185,21 @@ ftk_status ftk_topk_rows_end(ftk_dtype dtype, const void *x, int64_t rows,
                              uint32_t *status, void *stream);
 
 /*
+ * ftk_topk_rows_sorted -- ftk_topk_rows (or ftk_topk_rows_end when row_end
+ * is not NULL) with each row's output ordered by value descending, ties by
+ * column ascending, padding last (DeepSelect README, "Usage": sorted=True;
+ * the unsorted calls return ascending columns, i.e. sorted_index=True).
+ *   row_end   device [rows] int32 per-row exclusive end, or NULL
+ *   out_val   required (not NULL): the sort needs the values
+ * Other arguments, layout and errors as for ftk_topk_rows.
+ */
+ftk_status ftk_topk_rows_sorted(ftk_dtype dtype, const void *x, int64_t rows,
+                                int64_t cols, int64_t row_stride,
+                                const int32_t *row_end, int topk,
+                                int32_t *out_idx, void *out_val,
+                                uint32_t *status, void *stream);
+
+/*
  * ftk_score_dense -- the fused scores themselves, for checking: for each
  * listed row r (query t = rows ? rows[r] : r) writes
  *     out[r * ld + (s - ks[t])] = I[t, s]   for s in [ks[t], ke[t])

@@ -85,6 +85,88 @@ ftk_status launch_rows_topk(int dtype, const RowsArgs &a, int cluster, cudaStrea
     return FTK_ERR_UNSUPPORTED;
 }
 
+// ---------------------------------------------------------------------------
+// sorted output: each row's k (value, column) pairs by value descending,
+// column ascending (DeepSelect README, "Usage": sorted=True)
+// ---------------------------------------------------------------------------
+
+constexpr int kSortThreads = 512;
+
+// One CTA per row: a bitonic sort of 64-bit keys (~value key, position) in
+// shared memory, padded to kp = the power of two >= k with keys that sort
+// last.  The unsorted output is in ascending column order, so ordering
+// equal values by position orders them by column; the values and columns
+// are then moved by position, bit for bit (-0.0 stays -0.0).  Padding
+// entries (-inf, -1) of short rows stay at the end.
+template <int DT>
+__global__ void __launch_bounds__(kSortThreads) sort_rows_kernel(void *vals, int32_t *idx, int k, int kp)
+{
+    using Tr = RowsTraits<DT>;
+    using elem = typename Tr::elem;
+    extern __shared__ unsigned long long skey[];
+    const int64_t r = blockIdx.x;
+    elem *v = static_cast<elem *>(vals) + r * k;
+    int32_t *ix = idx + r * k;
+    for (int i = threadIdx.x; i < kp; i += blockDim.x) {
+        unsigned long long c = ~0ull;
+        if (i < k) {
+            const uint32_t key = Tr::key(static_cast<uint32_t>(v[i]));
+            c = (static_cast<unsigned long long>(~key) << 32) | static_cast<uint32_t>(i);
+        }
+        skey[i] = c;
+    }
+    __syncthreads();
+    for (int size = 2; size <= kp; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int i = threadIdx.x; i < kp / 2; i += blockDim.x) {
+                const int lo = 2 * i - (i & (stride - 1));
+                const int hi = lo + stride;
+                const bool up = (lo & size) == 0;
+                const unsigned long long a = skey[lo], b = skey[hi];
+                if ((a > b) == up) {
+                    skey[lo] = b;
+                    skey[hi] = a;
+                }
+            }
+            __syncthreads();
+        }
+    }
+    constexpr int kPer = FTK_MAX_TOPK / kSortThreads;  // outputs per thread (k <= FTK_MAX_TOPK)
+    elem mv[kPer];
+    int32_t mi[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+        const int i = threadIdx.x + j * kSortThreads;
+        if (i < k) {
+            const int pos = static_cast<int>(static_cast<uint32_t>(skey[i]));
+            mv[j] = v[pos];
+            mi[j] = ix[pos];
+        }
+    }
+    __syncthreads();  // every read of the unsorted row precedes the writes (in place)
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+        const int i = threadIdx.x + j * kSortThreads;
+        if (i < k) {
+            v[i] = mv[j];
+            ix[i] = mi[j];
+        }
+    }
+}
+
+static ftk_status launch_sort_rows(int dtype, void *vals, int32_t *idx, int64_t rows, int k,
+                                   cudaStream_t stream)
+{
+    int kp = 1;
+    while (kp < k) kp <<= 1;
+    const size_t smem = static_cast<size_t>(kp) * sizeof(unsigned long long);
+    if (dtype == FTK_BF16)
+        sort_rows_kernel<FTK_BF16><<<static_cast<unsigned>(rows), kSortThreads, smem, stream>>>(vals, idx, k, kp);
+    else
+        sort_rows_kernel<FTK_F32><<<static_cast<unsigned>(rows), kSortThreads, smem, stream>>>(vals, idx, k, kp);
+    return cuda_status(cudaGetLastError());
+}
+
 static ftk_status topk_rows_impl(ftk_dtype dtype, const void *x, int64_t rows, int64_t cols,
                                  int64_t row_stride, const int32_t *row_end, int topk,
                                  int32_t *out_idx, void *out_val, uint32_t *status, void *stream)
@@ -135,4 +217,16 @@ extern "C" ftk_status ftk_topk_rows_end(ftk_dtype dtype, const void *x, int64_t 
     if (!row_end) return FTK_ERR_INVALID_ARG;
     return topk_rows_impl(dtype, x, rows, cols, row_stride, row_end, topk, out_idx, out_val, status,
                           stream);
+}
+
+extern "C" ftk_status ftk_topk_rows_sorted(ftk_dtype dtype, const void *x, int64_t rows, int64_t cols,
+                                           int64_t row_stride, const int32_t *row_end, int topk,
+                                           int32_t *out_idx, void *out_val, uint32_t *status,
+                                           void *stream)
+{
+    if (!out_val) return FTK_ERR_INVALID_ARG;
+    ftk_status st = topk_rows_impl(dtype, x, rows, cols, row_stride, row_end, topk, out_idx, out_val,
+                                   status, stream);
+    if (st != FTK_OK) return st;
+    return launch_sort_rows(dtype, out_val, out_idx, rows, topk, as_stream(stream));
 }

@@ -39,7 +39,7 @@ EXPORTS = (
     "ftk_select", "ftk_select_workspace_size", "ftk_read_info", "ftk_topk_rows",
     "ftk_score_dense", "ftk_score_dense_workspace_size", "ftk_windows_from_cu_seqlens",
     "ftk_set_stage_events", "ftk_status_string", "ftk_version", "ftk_select_noalloc",
-    "ftk_block_bound", "ftk_block_bound_workspace_size", "ftk_topk_rows_end",
+    "ftk_block_bound", "ftk_block_bound_workspace_size", "ftk_topk_rows_end", "ftk_topk_rows_sorted",
 )
 
 
@@ -91,6 +91,8 @@ def load_library(path: str = LIB_PATH):
     L.ftk_select_noalloc.argtypes = [I32, P, P, P, P, P, P, I64, I64, I32, P, P, P, P]
     L.ftk_set_stage_events.restype = I32
     L.ftk_set_stage_events.argtypes = [P, I32]
+    L.ftk_topk_rows_sorted.restype = I32
+    L.ftk_topk_rows_sorted.argtypes = [I32, P, I64, I64, I64, P, I32, P, P, P, P]
     L.ftk_topk_rows_end.restype = I32
     L.ftk_topk_rows_end.argtypes = [I32, P, I64, I64, I64, P, I32, P, P, P, P]
     L.ftk_block_bound.restype = I32
@@ -277,11 +279,12 @@ def windows_from_cu_seqlens(cu_seqlens_q: torch.Tensor, cu_seqlens_k: torch.Tens
 
 def topk_rows(x: torch.Tensor, topk: int, return_value: bool = True, status: torch.Tensor | None = None,
               out_idx: torch.Tensor | None = None, out_val: torch.Tensor | None = None,
-              end: torch.Tensor | None = None):
+              end: torch.Tensor | None = None, sorted: bool = False):
     """Row top-k of a [rows, cols] bf16/fp32 CUDA tensor (ties to smaller columns).
 
     Returns (values, indices) like deep_select.topk, or indices alone when
-    return_value=False.  Indices are int32 in ascending column order.
+    return_value=False.  Indices are int32 in ascending column order, or,
+    with sorted=True, by value descending (ties by column ascending).
     end: optional int32 [rows] per-row exclusive end (ftk_topk_rows_end).
     """
     _need_cuda(x, status, end)
@@ -292,13 +295,19 @@ def topk_rows(x: torch.Tensor, topk: int, return_value: bool = True, status: tor
         out_idx = torch.empty((rows, topk), dtype=torch.int32, device=x.device)
     if return_value and out_val is None:
         out_val = torch.empty((rows, topk), dtype=x.dtype, device=x.device)
-    if end is None:
+    if end is not None and (end.shape != (rows,) or end.dtype != torch.int32 or not end.is_contiguous()):
+        raise FtkError("end must be a contiguous int32 [rows] tensor")
+    if sorted:
+        if out_val is None:
+            out_val = torch.empty((rows, topk), dtype=x.dtype, device=x.device)
+        st = lib().ftk_topk_rows_sorted(_dtype_code(x), _ptr(x), rows, cols, x.stride(0), _ptr(end), topk,
+                                        _ptr(out_idx), _ptr(out_val), _ptr(status), _stream(x.device))
+        _check(st, "ftk_topk_rows_sorted")
+    elif end is None:
         st = lib().ftk_topk_rows(_dtype_code(x), _ptr(x), rows, cols, x.stride(0), topk, _ptr(out_idx),
                                  _ptr(out_val) if return_value else None, _ptr(status), _stream(x.device))
         _check(st, "ftk_topk_rows")
     else:
-        if end.shape != (rows,) or end.dtype != torch.int32 or not end.is_contiguous():
-            raise FtkError("end must be a contiguous int32 [rows] tensor")
         st = lib().ftk_topk_rows_end(_dtype_code(x), _ptr(x), rows, cols, x.stride(0), _ptr(end), topk,
                                      _ptr(out_idx), _ptr(out_val) if return_value else None, _ptr(status),
                                      _stream(x.device))

@@ -74,6 +74,13 @@ def test_topk_rows_end_host_validation(lib):
     assert lib.ftk_topk_rows_end(2, P(A + 2), 4, 100, 104, P(A), 8, P(A), None, None, None) == -4
 
 
+def test_topk_rows_sorted_host_validation(lib):
+    P = ctypes.c_void_p
+    # out_val is required: the sort needs the values
+    assert lib.ftk_topk_rows_sorted(2, P(A), 4, 100, 104, None, 8, P(A), None, None, None) == -1
+    assert lib.ftk_topk_rows_sorted(2, P(A), 4, 100, 104, None, 0, P(A), P(A), None, None) == -3
+
+
 def test_block_bound_host_validation(lib):
     P = ctypes.c_void_p
     need = lib.ftk_block_bound_workspace_size(1000)

@@ -141,3 +141,35 @@ def test_variable_length_rows_end(dtype):
             assert torch.equal(val[r, :n].view(bits), ref.view(bits))
         assert np.all(idx[r, n:] == -1)
         assert torch.all(torch.isneginf(val[r, n:].float()))
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_sorted_output(dtype):
+    """sorted=True (DeepSelect README, "Usage"): each row's topk by value
+    descending, ties by column ascending, padding last -- element by element
+    the oracle's order, values bit-exact (signed zeros kept)."""
+    rows, cols, k = 24, 9000, 700
+    g = torch.Generator().manual_seed(91)
+    x_cpu = torch.randn((rows, cols), generator=g).to(dtype)
+    x_cpu[3] = torch.randint(0, 4, (cols,), generator=g).to(dtype) - 1.5  # 4 values: heavy ties
+    x_cpu[4] = 0.0
+    x_cpu[4, ::3] = -0.0                                                 # signed zeros only
+    ends = torch.full((rows,), cols, dtype=torch.int32)
+    ends[5], ends[6] = 100, 0                                            # short and empty rows
+    x = aligned_rows(x_cpu)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    val, idx = ftk.topk_rows(x, k, status=status, end=ends.cuda(), sorted=True)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    idx, val = to_np(idx), val.cpu()
+    bits = torch.int16 if dtype == torch.bfloat16 else torch.int32
+    for r in range(rows):
+        e = int(ends[r])
+        n = min(k, e)
+        if n:
+            oidx, _, _ = orc.topk_rows(x_cpu[r:r + 1, :e].contiguous(), k)
+            assert np.array_equal(idx[r, :n], oidx[0, :n]), f"row {r}: order differs"
+            ref = x_cpu[r, idx[r, :n]]
+            assert torch.equal(val[r, :n].view(bits), ref.view(bits)), f"row {r}: value bits"
+        assert np.all(idx[r, n:] == -1)
+        assert torch.all(torch.isneginf(val[r, n:].float()))
