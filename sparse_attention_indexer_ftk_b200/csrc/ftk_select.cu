@@ -347,12 +347,16 @@ __device__ __forceinline__ void pad_row(int32_t *oi, float *ov, int from, int k)
     }
 }
 
-__global__ void __launch_bounds__(kSelThreads) refine_kernel(const RefineArgs p)
+// Shared memory is kept small (keys only; the candidates' key indices are
+// re-read from global memory, eight loads in flight per thread, where the
+// bitmap passes need them) so that several rows' CTAs share an SM: the
+// kernel is latency-bound per row.
+__global__ void __launch_bounds__(kSelThreads, 6) refine_kernel(const RefineArgs p)
 {
     extern __shared__ __align__(16) uint32_t rsm[];
     __shared__ SelShared ss;
     __shared__ uint32_t bitmap[kBitmapWords];
-    __shared__ uint32_t wpre[kBitmapWords];
+    __shared__ uint16_t wpre[kBitmapWords];  // selected keys before each word (<= capacity)
     __shared__ int nan_seen;
     const int64_t t = blockIdx.x;
     const int k = p.topk;
@@ -378,22 +382,19 @@ __global__ void __launch_bounds__(kSelThreads) refine_kernel(const RefineArgs p)
     }
     const int n = c;
     uint32_t *keys = rsm;
-    int32_t *idx = reinterpret_cast<int32_t *>(rsm + p.cap);
     if (threadIdx.x == 0) nan_seen = 0;
     __syncthreads();
     const float *cv = p.cand_val + t * p.cap;
     const int32_t *ci = p.cand_idx + t * p.cap;
     bool nan = false;
     uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;  // bounds of the keys, for the radix select
-    // Eight (value, index) loads in flight per thread, then the stores.
+    // Eight value loads in flight per thread, then the stores.
     for (int i0 = 0; i0 < n; i0 += 8 * kSelThreads) {
         uint32_t v[8];
-        int32_t x[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int i = i0 + j * kSelThreads + threadIdx.x;
             v[j] = i < n ? __float_as_uint(__ldg(cv + i)) : 0u;
-            x[j] = i < n ? __ldg(ci + i) : 0;
         }
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -402,7 +403,6 @@ __global__ void __launch_bounds__(kSelThreads) refine_kernel(const RefineArgs p)
                 nan |= f32_bits_isnan(v[j]);
                 const uint32_t u = f32_key(v[j]);
                 keys[i] = u;
-                idx[i] = x[j];
                 kmin = min(kmin, u);
                 kmax = max(kmax, u);
             }
@@ -448,13 +448,13 @@ __global__ void __launch_bounds__(kSelThreads) refine_kernel(const RefineArgs p)
             uint32_t g2;
             const uint32_t inv = block_kth_largest(
                 n, need,
-                [&](int i) { return keys[i] == ustar ? ~static_cast<uint32_t>(idx[i]) : 0u; }, ss, &g2);
+                [&](int i) { return keys[i] == ustar ? ~static_cast<uint32_t>(__ldg(ci + i)) : 0u; }, ss, &g2);
             idxcut = ~inv;
         }
     }
-    auto selected = [&](int i) {
+    auto selected = [&](int i, int32_t s) {
         const uint32_t u = keys[i];
-        return u > ustar || (u == ustar && static_cast<uint32_t>(idx[i]) <= idxcut);
+        return u > ustar || (u == ustar && static_cast<uint32_t>(s) <= idxcut);
     };
 
     // Ordered output: rank of a selected key = number of selected keys with
@@ -465,11 +465,21 @@ __global__ void __launch_bounds__(kSelThreads) refine_kernel(const RefineArgs p)
         const int words = static_cast<int>((seg1 - seg0 + 31) >> 5);
         for (int w = threadIdx.x; w < words; w += blockDim.x) bitmap[w] = 0;
         __syncthreads();
-        for (int i = threadIdx.x; i < n; i += blockDim.x) {
-            const int64_t s = idx[i];
-            if (s >= seg0 && s < seg1 && selected(i)) {
-                const uint32_t off = static_cast<uint32_t>(s - seg0);
-                atomicOr(&bitmap[off >> 5], 1u << (off & 31u));
+        for (int i0 = 0; i0 < n; i0 += 8 * kSelThreads) {
+            int32_t x[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int i = i0 + j * kSelThreads + threadIdx.x;
+                x[j] = i < n ? __ldg(ci + i) : -1;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int i = i0 + j * kSelThreads + threadIdx.x;
+                const int64_t s = x[j];
+                if (i < n && s >= seg0 && s < seg1 && selected(i, x[j])) {
+                    const uint32_t off = static_cast<uint32_t>(s - seg0);
+                    atomicOr(&bitmap[off >> 5], 1u << (off & 31u));
+                }
             }
         }
         __syncthreads();
@@ -483,23 +493,33 @@ __global__ void __launch_bounds__(kSelThreads) refine_kernel(const RefineArgs p)
 #pragma unroll
         for (int i = 0; i < per; ++i) {
             if (w0 + i < words) {
-                wpre[w0 + i] = run;
+                wpre[w0 + i] = static_cast<uint16_t>(run);
                 run += __popc(bitmap[w0 + i]);
             }
         }
         __syncthreads();
-        for (int i = threadIdx.x; i < n; i += blockDim.x) {
-            const int64_t s = idx[i];
-            if (s >= seg0 && s < seg1 && selected(i)) {
-                const uint32_t off = static_cast<uint32_t>(s - seg0);
-                const uint32_t w = off >> 5;
-                const uint32_t rank =
-                    out_base + wpre[w] + __popc(bitmap[w] & ((1u << (off & 31u)) - 1u));
-                if (rank < static_cast<uint32_t>(k)) {
-                    oi[rank] = static_cast<int32_t>(s);
-                    if (ov) ov[rank] = __uint_as_float(f32_from_key(keys[i]));
-                } else {
-                    atomicOr(&p.info->info.status, FTK_STATUS_INTERNAL);
+        for (int i0 = 0; i0 < n; i0 += 8 * kSelThreads) {
+            int32_t x[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int i = i0 + j * kSelThreads + threadIdx.x;
+                x[j] = i < n ? __ldg(ci + i) : -1;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int i = i0 + j * kSelThreads + threadIdx.x;
+                const int64_t s = x[j];
+                if (i < n && s >= seg0 && s < seg1 && selected(i, x[j])) {
+                    const uint32_t off = static_cast<uint32_t>(s - seg0);
+                    const uint32_t w = off >> 5;
+                    const uint32_t rank =
+                        out_base + wpre[w] + __popc(bitmap[w] & ((1u << (off & 31u)) - 1u));
+                    if (rank < static_cast<uint32_t>(k)) {
+                        oi[rank] = static_cast<int32_t>(s);
+                        if (ov) ov[rank] = __uint_as_float(f32_from_key(keys[i]));
+                    } else {
+                        atomicOr(&p.info->info.status, FTK_STATUS_INTERNAL);
+                    }
                 }
             }
         }
@@ -959,7 +979,7 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
     ra.bad_count = w.bad_count;
     ra.info = w.info;
     {
-        const size_t smem = static_cast<size_t>(c.cap) * 8;
+        const size_t smem = static_cast<size_t>(c.cap) * 4;
         cudaError_t e = cudaFuncSetAttribute(refine_kernel,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              static_cast<int>(smem));
