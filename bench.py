@@ -55,6 +55,8 @@ def parse_args():
     ap.add_argument("--no-rows", action="store_true", help="skip the row top-k section")
     ap.add_argument("--only-rows", action="store_true", help="run only the row top-k section")
     ap.add_argument("--no-decode", action="store_true", help="skip the 64-query (decode-shaped) section")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the decode-shaped, packed-workload and FP8 GEMM reference sections")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--rows", type=int, default=0,
                     help="use only the first ROWS queries of the batch (profiling captures)")
@@ -497,7 +499,7 @@ def run_ours(args):
     # (in-window or not), i.e. minus the pruned ones.
     rt = 16 if c.q.dtype == torch.float8_e4m3fn else 8
     exec_pairs = (int(info["blocks_total"]) - int(info["blocks_pruned"])) * rt * 128
-    fp8_direct = fp8_gemm_peak(dev) if world == 1 else None
+    fp8_direct = fp8_gemm_peak(dev) if world == 1 and not args.no_extras else None
     out = {
         "metric": METRIC,
         "value": value,
@@ -530,7 +532,7 @@ def run_ours(args):
         "gpu_launches": int(info["kernel_launches"]) * K,
         "clocks": clocks,
     }
-    if world == 1 and not args.no_decode:
+    if world == 1 and not (args.no_decode or args.no_extras):
         out["decode_64q"] = bench_decode(c, dev)
         out["fp8_packed"] = bench_config("fp8_packed", dev)
     if world == 1 and not args.no_rows:
