@@ -95,12 +95,27 @@ def profiled_traffic():
     return float(m.group(1))
 
 
-def scan_kernel_hash() -> str:
+def strip_comments(src: str) -> str:
+    """C++ source without comments and with whitespace collapsed."""
+    import re
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    return " ".join(src.split())
+
+
+def scan_kernel_hash(read=None) -> str:
+    """Hash of the scan kernel's sources, comments and layout ignored (a
+    comment edit does not invalidate the profiled counters)."""
     import hashlib
     h = hashlib.sha1()
     for f in ("ftk_score.cuh", "ftk_device.cuh"):
-        with open(os.path.join(ROOT, "sparse_attention_indexer_ftk_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        path = os.path.join("sparse_attention_indexer_ftk_b200", "csrc", f)
+        if read is None:
+            with open(os.path.join(ROOT, path)) as fh:
+                text = fh.read()
+        else:
+            text = read(path)
+        h.update(strip_comments(text).encode())
     return h.hexdigest()[:12]
 
 

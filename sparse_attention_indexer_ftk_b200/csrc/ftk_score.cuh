@@ -11,8 +11,8 @@
 // a TMA ring; each key tile feeds QG MMAs, one per query tile, which halves
 // the key traffic from L2 per FLOP.  The fp32 accumulator (128 lanes x 256
 // columns) alternates between two tensor-memory buffers (2 x 256 of the 512
-// columns), so the MMA of the next (key tile, query tile) overlaps the
-// epilogue of the current one.  TMEM lane = key, so each epilogue thread
+// columns); with QG = 2 one key tile fills both, and an accumulator goes
+// back to the MMA warp as soon as every epilogue warp has loaded it.  TMEM lane = key, so each epilogue thread
 // owns one key and reduces the 32 heads of a query in registers: ReLU, the
 // head weights and sigma are applied and the T x S x 32 intermediate never
 // leaves the SM.
@@ -26,11 +26,14 @@
 //               warps per scheduler so that their dependency chains
 //               interleave.
 //
-// Head reduction: for each (query, key), four partial sums over the heads
-// h = 0, 1, 2, 3 (mod 4), each a chain of correctly rounded fmas in head
-// order, combined as (p0 + p1) + (p2 + p3), times sigma, plus +0.0 (which
-// turns -0.0 into +0.0).  ReLU propagates NaN, so a NaN dot product makes the
-// score NaN, which the candidate test keeps and the refine step reports.
+// Head reduction: for each (query, key), two partial sums over the even and
+// the odd heads (the two lanes of one packed fma chain, correctly rounded,
+// in head order), added, times sigma, plus +0.0 (which turns -0.0 into
+// +0.0).  ReLU propagates NaN, so a NaN dot product makes the score NaN,
+// which the candidate test keeps and the refine step reports.
+//
+// Pruning (PR = true): key tiles that the score bound marks for the item's
+// row tile are skipped by all three roles (see ftk_prune.cuh).
 //
 // Modes (one kernel body, so every mode produces bit-identical scores):
 //   SAMPLE   keys are a strided sample k[j*stride] (a strided TMA view of kv);
