@@ -108,6 +108,7 @@ struct ScoreArgs {
     // kernel start from the rows in the list (make_sched).  SAMPLE and
     // COLLECT run planned, DUMP static.
     int32_t planned;
+    int32_t *work_next;       // planned: shared item counter (dynamic schedule), or NULL
     int32_t chunk_keys;       // planned: keys (SAMPLE: samples) per work item, a multiple of 128
     const int32_t *tile_lo, *tile_hi, *tile_lg, *item_start;
     int32_t ntiles;
@@ -351,9 +352,11 @@ struct ScoreMisc {
     uint64_t kv_full[4], kv_empty[4];
     uint64_t q_full, q_empty;
     uint64_t acc_full[2], acc_empty[2];
+    uint64_t item_full[2], item_empty[2];  // the work-item queue (producer -> all roles)
     uint64_t final_bar;
     uint32_t tmem_base;
     int32_t abort;
+    int32_t item_q[2];                     // item index, -1: no more items
 };
 
 static_assert(sizeof(ScoreMisc) <= ScoreSmemLayout<FTK_F8E4M3>::kMiscBytes, "misc area");
@@ -404,6 +407,10 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             mbar_init(&ms.acc_full[i], 1);
             mbar_init(&ms.acc_empty[i], kEpiWarps);
         }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&ms.item_full[i], 1);
+            mbar_init(&ms.item_empty[i], 1 + kEpiWarps);
+        }
         mbar_init(&ms.final_bar, 1);
         ms.abort = 0;
         fence_barrier_init();
@@ -425,7 +432,30 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             int q_armed = 0;
             uint32_t q_armed_ph = 0;
             Item m;
-            for (int it = blockIdx.x; !*abort && next_item<MODE, RT>(a, sc, it, nlist, m); it += gridDim.x) {
+            // Work items: taken from the shared counter (dynamic: a CTA that
+            // finishes early takes more) or in the static round-robin order,
+            // and handed to the MMA and epilogue roles through the queue.
+            const bool dynamic = a.planned && a.work_next != nullptr;
+            const int32_t total = a.planned ? a.item_start[a.ntiles] : 0;
+            int islot = 0, it_s = blockIdx.x;
+            uint32_t iph = 0;
+            for (;;) {
+                int it = -1;
+                if (!*abort) {
+                    if (dynamic) {
+                        it = atomicAdd(a.work_next, 1);
+                        if (it >= total) it = -1;
+                    } else if (next_item<MODE, RT>(a, sc, it_s, nlist, m)) {
+                        it = it_s;
+                        it_s += gridDim.x;
+                    }
+                }
+                if (!mbar_wait(&ms.item_empty[islot], iph ^ 1u, abort, a.status)) break;
+                ms.item_q[islot] = it;
+                mbar_arrive(&ms.item_full[islot]);
+                if (++islot == 2) { islot = 0; iph ^= 1u; }
+                if (it < 0) break;
+                if (dynamic) get_item<MODE, RT>(a, sc, it, nlist, m);
                 // The query group: the 32 head rows of each of RT queries.
                 if (!mbar_wait(&ms.q_empty, qph ^ 1u, abort, a.status)) break;
                 mbar_arrive_expect_tx(&ms.q_full, Lay::kQBytes);
@@ -470,7 +500,15 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             uint32_t kph = 0, qph = 0, aph = 0;
             bool issued = false, ok = true;
             Item m;
-            for (int it = blockIdx.x; ok && !*abort && next_item<MODE, RT>(a, sc, it, nlist, m); it += gridDim.x) {
+            int islot = 0;
+            uint32_t iph = 0;
+            while (ok && !*abort) {
+                if (!mbar_wait(&ms.item_full[islot], iph, abort, a.status)) break;
+                const int it = *reinterpret_cast<volatile int32_t *>(&ms.item_q[islot]);
+                mbar_arrive(&ms.item_empty[islot]);
+                if (++islot == 2) { islot = 0; iph ^= 1u; }
+                if (it < 0) break;
+                get_item<MODE, RT>(a, sc, it, nlist, m);
                 if (!mbar_wait(&ms.q_full, qph, abort, a.status)) break;
                 qph ^= 1u;
                 tc_fence_after();
@@ -536,7 +574,17 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         uint32_t aph = 0;
         bool bad_scale = false;
         Item m;
-        for (int it = blockIdx.x; !*abort && next_item<MODE, RT>(a, sc, it, nlist, m); it += gridDim.x) {
+        int islot = 0;
+        uint32_t iph = 0;
+        while (!*abort) {
+            const bool got_item = mbar_wait(&ms.item_full[islot], iph, abort, a.status);
+            if (!__all_sync(0xFFFFFFFFu, got_item)) break;
+            const int it = *reinterpret_cast<volatile int32_t *>(&ms.item_q[islot]);
+            __syncwarp();  // every lane has the index before the slot is released
+            if (lane == 0) mbar_arrive(&ms.item_empty[islot]);
+            if (++islot == 2) { islot = 0; iph ^= 1u; }
+            if (it < 0) break;
+            get_item<MODE, RT>(a, sc, it, nlist, m);
             // Per-item parameters of this warp's queries (warp-uniform).  Slot
             // qq = vt * NQ + qi is query qg * NQ + qi of query tile vt.
             int32_t qt[WQ], qpos[WQ], wlo[WQ], wlen[WQ];

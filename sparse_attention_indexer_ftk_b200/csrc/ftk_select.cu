@@ -45,6 +45,7 @@ constexpr int kMaxRowTile = 16;      // largest row_tile_of(dtype)
 struct DevInfo {
     ftk_info info;
     uint32_t est_total, est_pruned;  // sampled (tile, block) pairs of the prune estimate
+    int32_t work_next;               // the scan's shared work-item counter
 };
 
 // ---------------------------------------------------------------------------
@@ -114,6 +115,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanArgs p)
         p.info->info.kernel_launches = p.launches;
         p.info->est_total = 0;
         p.info->est_pruned = 0;
+        p.info->work_next = 0;
     }
     __syncthreads();
     unsigned long long nblocks = 0;  // (row tile, key block) pairs of the scan
@@ -936,8 +938,9 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
     }
     stage_mark(7, s);
 
-    // scan
+    // scan (dynamic schedule over the planned items)
     sa.chunk_keys = pa.chunk_keys;
+    sa.work_next = &w.info->work_next;
     sa.tile_lo = w.c_lo;
     sa.tile_hi = w.c_hi;
     sa.tile_lg = nullptr;
