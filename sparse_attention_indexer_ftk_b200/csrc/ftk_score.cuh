@@ -53,7 +53,7 @@ enum ScoreMode { MODE_SAMPLE = 0, MODE_COLLECT = 1, MODE_DUMP = 2 };
 
 constexpr int kQTile = 8;            // queries per MMA tile -> N = 256
 constexpr int kKeyTile = 128;        // keys per tile -> M = 128
-constexpr int kChunkTiles = 128;     // key tiles per work item (16384 keys)
+constexpr int kChunkTiles = 64;      // key tiles per work item (8192 keys)
 constexpr int kChunkKeys = kChunkTiles * kKeyTile;
 constexpr int kEpiWarps = 16;        // warps 2..17
 constexpr int kEpiThreads = kEpiWarps * 32;
