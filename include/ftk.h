@@ -200,6 +200,58 @@ ftk_status ftk_topk_rows_sorted(ftk_dtype dtype, const void *x, int64_t rows,
                                 uint32_t *status, void *stream);
 
 /*
+ * Options of ftk_topk_rows_ex (DeepSelect README, "Usage" and
+ * "Variable-length rows": sorted, sorted_index, indices_type, the output
+ * buffers' row stride and the out-of-bound fill values).  Fill a struct
+ * with ftk_rows_options_init, then change what differs.
+ *   sorted       0: each row's output in ascending column order (what
+ *                DeepSelect calls sorted_index=True, which also serves
+ *                sorted_index=False); 1: by value descending, ties by
+ *                column ascending, padding last
+ *   index_bits   32: out_idx is int32_t; 64: int64_t (indices_type)
+ *   out_stride   elements between consecutive output rows of out_idx and
+ *                out_val; 0 means topk; otherwise topk .. 2^31 - 1
+ *   idx_fill     index of the padding slots of rows shorter than topk
+ *                (idx_oob_fill_value); within int32 when index_bits = 32
+ *   val_fill     value of those slots (value_oob_fill_value), stored in
+ *                x's dtype (rounded to nearest even for bf16)
+ * Defaults: sorted 0, index_bits 32, out_stride 0, idx_fill -1,
+ * val_fill -inf.
+ */
+typedef struct {
+    int32_t sorted;
+    int32_t index_bits;
+    int64_t out_stride;
+    int64_t idx_fill;
+    float val_fill;
+} ftk_rows_options;
+
+/* Writes the defaults above into *options (no-op on NULL). */
+void ftk_rows_options_init(ftk_rows_options *options);
+
+/*
+ * ftk_topk_rows_ex -- the row top-k with every option: ftk_topk_rows,
+ * ftk_topk_rows_end and ftk_topk_rows_sorted are this call with default
+ * options (and sorted = 1 for the last).
+ *   row_end   device [rows] int32 per-row exclusive end, clamped to
+ *             [0, cols], or NULL (every row has cols columns)
+ *   options   as above, or NULL for the defaults
+ *   out_idx   device [rows, out_stride] int32 or int64 (index_bits),
+ *             aligned to its element size; slots [0, topk) of each row are
+ *             written
+ *   out_val   device [rows, out_stride] of x's dtype, aligned to its
+ *             element size, or NULL; with sorted = 1 and no value output
+ *             the sort reads each selected value from x
+ * Errors: FTK_ERR_INVALID_ARG for an option outside the ranges above,
+ * FTK_ERR_ALIGNMENT for misaligned outputs; the rest as for ftk_topk_rows.
+ */
+ftk_status ftk_topk_rows_ex(ftk_dtype dtype, const void *x, int64_t rows,
+                            int64_t cols, int64_t row_stride,
+                            const int32_t *row_end, int topk,
+                            const ftk_rows_options *options, void *out_idx,
+                            void *out_val, uint32_t *status, void *stream);
+
+/*
  * ftk_score_dense -- the fused scores themselves, for checking: for each
  * listed row r (query t = rows ? rows[r] : r) writes
  *     out[r * ld + (s - ks[t])] = I[t, s]   for s in [ks[t], ke[t])

@@ -56,7 +56,7 @@ ftk_status launch_box(int dtype, const BoxArgs &a, cudaStream_t stream);
 ftk_status launch_bound(int dtype, int mode, const BoundArgs &a, int grid, cudaStream_t stream);
 // Launches the row top-k kernel for the given dtype (FTK_BF16 / FTK_F32)
 // with one cluster of `cluster` CTAs per grid row.
-ftk_status launch_rows_topk(int dtype, const RowsArgs &a, int cluster, cudaStream_t stream);
+ftk_status launch_rows_topk(int dtype, const RowsArgs &a, int cluster, cudaStream_t stream, bool idx64 = false);
 // Cluster size and per-CTA chunk for rows of `cols` columns.
 void rows_plan(int64_t rows, int64_t cols, int k, int *cluster, int *chunk);
 

@@ -1,7 +1,10 @@
 // ftk_rows.cu -- host side of the row top-k (ftk_topk_rows) and the launch
 // helper the dense-recovery step reuses.
+#include <math.h>
+#include <stdint.h>
 #include <stdio.h>
 #include <stdlib.h>
+#include <string.h>
 
 #include "ftk_host.h"
 #include "ftk_rows.cuh"
@@ -46,7 +49,7 @@ void rows_plan(int64_t rows, int64_t cols, int k, int *cluster, int *chunk)
 }
 
 template <int DT>
-static ftk_status launch_rows_dt(const RowsArgs &a, int cluster, cudaStream_t stream)
+static ftk_status launch_rows_dt(const RowsArgs &a, int cluster, bool idx64, cudaStream_t stream)
 {
     // One cluster per row if they all fit at once (two CTAs per SM) and the
     // row count is known here; else as many clusters as fit, striding.
@@ -58,7 +61,8 @@ static ftk_status launch_rows_dt(const RowsArgs &a, int cluster, cudaStream_t st
     const bool loop = a.nrows_dev != nullptr || a.rows > fit;
     const int64_t nclusters = loop ? (a.rows < fit ? a.rows : fit) : a.rows;
     const size_t smem = sizeof(RowsSmem);
-    auto kern = loop ? rows_topk_kernel<DT, true> : rows_topk_kernel<DT, false>;
+    auto kern = idx64 ? (loop ? rows_topk_kernel<DT, true, int64_t> : rows_topk_kernel<DT, false, int64_t>)
+                      : (loop ? rows_topk_kernel<DT, true, int32_t> : rows_topk_kernel<DT, false, int32_t>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return cuda_status(e);
@@ -77,11 +81,12 @@ static ftk_status launch_rows_dt(const RowsArgs &a, int cluster, cudaStream_t st
     return cuda_status(cudaLaunchKernelEx(&cfg, kern, a));
 }
 
-ftk_status launch_rows_topk(int dtype, const RowsArgs &a, int cluster, cudaStream_t stream)
+ftk_status launch_rows_topk(int dtype, const RowsArgs &a, int cluster, cudaStream_t stream, bool idx64)
 {
     if (a.chunk <= 0 || a.chunk % 8) return FTK_ERR_UNSUPPORTED;
-    if (dtype == FTK_BF16) return launch_rows_dt<FTK_BF16>(a, cluster, stream);
-    if (dtype == FTK_F32) return launch_rows_dt<FTK_F32>(a, cluster, stream);
+    if (a.ldo < a.k) return FTK_ERR_INVALID_ARG;
+    if (dtype == FTK_BF16) return launch_rows_dt<FTK_BF16>(a, cluster, idx64, stream);
+    if (dtype == FTK_F32) return launch_rows_dt<FTK_F32>(a, cluster, idx64, stream);
     return FTK_ERR_UNSUPPORTED;
 }
 
@@ -96,22 +101,36 @@ constexpr int kSortThreads = 512;
 // shared memory, padded to kp = the power of two >= k with keys that sort
 // last.  The unsorted output is in ascending column order, so ordering
 // equal values by position orders them by column; the values and columns
-// are then moved by position, bit for bit (-0.0 stays -0.0).  Padding
-// entries (-inf, -1) of short rows stay at the end.
-template <int DT>
-__global__ void __launch_bounds__(kSortThreads) sort_rows_kernel(void *vals, int32_t *idx, int k, int kp)
+// are then moved by position, bit for bit (-0.0 stays -0.0).  The padding
+// slots of a row shorter than k (positions >= its length) keep their place
+// at the end whatever their fill value.  Without a value output the key
+// is read from x at the selected column.
+template <int DT, typename IT>
+__global__ void __launch_bounds__(kSortThreads) sort_rows_kernel(const void *x, int64_t ld,
+                                                                 const int32_t *row_end, int64_t cols,
+                                                                 void *vals, IT *idx, int64_t ldo, int k,
+                                                                 int kp)
 {
     using Tr = RowsTraits<DT>;
     using elem = typename Tr::elem;
     extern __shared__ unsigned long long skey[];
     const int64_t r = blockIdx.x;
-    elem *v = static_cast<elem *>(vals) + r * k;
-    int32_t *ix = idx + r * k;
+    int64_t len = cols;
+    if (row_end) {
+        const int64_t e = row_end[r];
+        len = e < 0 ? 0 : (e < len ? e : len);
+    }
+    const int nreal = len < k ? static_cast<int>(len) : k;
+    elem *v = vals ? static_cast<elem *>(vals) + r * ldo : nullptr;
+    const elem *xr = static_cast<const elem *>(x) + r * ld;
+    IT *ix = idx + r * ldo;
     for (int i = threadIdx.x; i < kp; i += blockDim.x) {
         unsigned long long c = ~0ull;
-        if (i < k) {
-            const uint32_t key = Tr::key(static_cast<uint32_t>(v[i]));
-            c = (static_cast<unsigned long long>(~key) << 32) | static_cast<uint32_t>(i);
+        if (i < nreal) {
+            const uint32_t bits = static_cast<uint32_t>(v ? v[i] : xr[ix[i]]);
+            c = (static_cast<unsigned long long>(~Tr::key(bits)) << 32) | static_cast<uint32_t>(i);
+        } else if (i < k) {
+            c = (0xFFFFFFFFull << 32) | static_cast<uint32_t>(i);
         }
         skey[i] = c;
     }
@@ -133,13 +152,13 @@ __global__ void __launch_bounds__(kSortThreads) sort_rows_kernel(void *vals, int
     }
     constexpr int kPer = FTK_MAX_TOPK / kSortThreads;  // outputs per thread (k <= FTK_MAX_TOPK)
     elem mv[kPer];
-    int32_t mi[kPer];
+    IT mi[kPer];
 #pragma unroll
     for (int j = 0; j < kPer; ++j) {
         const int i = threadIdx.x + j * kSortThreads;
         if (i < k) {
             const int pos = static_cast<int>(static_cast<uint32_t>(skey[i]));
-            mv[j] = v[pos];
+            if (v) mv[j] = v[pos];
             mi[j] = ix[pos];
         }
     }
@@ -148,28 +167,51 @@ __global__ void __launch_bounds__(kSortThreads) sort_rows_kernel(void *vals, int
     for (int j = 0; j < kPer; ++j) {
         const int i = threadIdx.x + j * kSortThreads;
         if (i < k) {
-            v[i] = mv[j];
+            if (v) v[i] = mv[j];
             ix[i] = mi[j];
         }
     }
 }
 
-static ftk_status launch_sort_rows(int dtype, void *vals, int32_t *idx, int64_t rows, int k,
-                                   cudaStream_t stream)
+template <int DT>
+static void launch_sort_dt(const RowsArgs &a, bool idx64, unsigned rows, int kp, size_t smem,
+                           cudaStream_t stream)
+{
+    if (idx64)
+        sort_rows_kernel<DT, int64_t><<<rows, kSortThreads, smem, stream>>>(
+            a.x, a.ld, a.row_end, a.cols, a.out_val, static_cast<int64_t *>(a.out_idx), a.ldo, a.k, kp);
+    else
+        sort_rows_kernel<DT, int32_t><<<rows, kSortThreads, smem, stream>>>(
+            a.x, a.ld, a.row_end, a.cols, a.out_val, static_cast<int32_t *>(a.out_idx), a.ldo, a.k, kp);
+}
+
+// Sorts the output of a finished row top-k call described by `a`.
+static ftk_status launch_sort_rows(int dtype, const RowsArgs &a, bool idx64, cudaStream_t stream)
 {
     int kp = 1;
-    while (kp < k) kp <<= 1;
+    while (kp < a.k) kp <<= 1;
     const size_t smem = static_cast<size_t>(kp) * sizeof(unsigned long long);
+    const unsigned rows = static_cast<unsigned>(a.rows);
     if (dtype == FTK_BF16)
-        sort_rows_kernel<FTK_BF16><<<static_cast<unsigned>(rows), kSortThreads, smem, stream>>>(vals, idx, k, kp);
+        launch_sort_dt<FTK_BF16>(a, idx64, rows, kp, smem, stream);
     else
-        sort_rows_kernel<FTK_F32><<<static_cast<unsigned>(rows), kSortThreads, smem, stream>>>(vals, idx, k, kp);
+        launch_sort_dt<FTK_F32>(a, idx64, rows, kp, smem, stream);
     return cuda_status(cudaGetLastError());
+}
+
+// float -> bf16 bits, round to nearest even (a NaN stays a quiet NaN).
+static uint32_t bf16_bits(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7FFFFFFFu) > 0x7F800000u) return ((u >> 16) | 0x40u) & 0xFFFFu;
+    return (u + 0x7FFFu + ((u >> 16) & 1u)) >> 16;
 }
 
 static ftk_status topk_rows_impl(ftk_dtype dtype, const void *x, int64_t rows, int64_t cols,
                                  int64_t row_stride, const int32_t *row_end, int topk,
-                                 int32_t *out_idx, void *out_val, uint32_t *status, void *stream)
+                                 const ftk_rows_options &o, void *out_idx, void *out_val,
+                                 uint32_t *status, void *stream)
 {
     if (dtype != FTK_BF16 && dtype != FTK_F32) return FTK_ERR_UNSUPPORTED;
     if (!x || !out_idx) return FTK_ERR_INVALID_ARG;
@@ -177,8 +219,16 @@ static ftk_status topk_rows_impl(ftk_dtype dtype, const void *x, int64_t rows, i
         return FTK_ERR_INVALID_ARG;
     if (topk < 1 || topk > FTK_MAX_TOPK) return FTK_ERR_TOPK_RANGE;
     if (cols > kRowsMaxCols) return FTK_ERR_UNSUPPORTED;
+    if ((o.sorted != 0 && o.sorted != 1) || (o.index_bits != 32 && o.index_bits != 64))
+        return FTK_ERR_INVALID_ARG;
+    const int64_t ldo = o.out_stride ? o.out_stride : topk;
+    if (ldo < topk || ldo > INT32_MAX) return FTK_ERR_INVALID_ARG;  // offsets stay within int64
+    if (o.index_bits == 32 && (o.idx_fill < INT32_MIN || o.idx_fill > INT32_MAX)) return FTK_ERR_INVALID_ARG;
     const int esz = dtype == FTK_BF16 ? 2 : 4;
     if (!aligned16(x) || (row_stride * esz) % 16) return FTK_ERR_ALIGNMENT;
+    if (reinterpret_cast<uintptr_t>(out_idx) % (o.index_bits / 8) ||
+        reinterpret_cast<uintptr_t>(out_val) % esz)
+        return FTK_ERR_ALIGNMENT;
     ftk_status st = check_device();
     if (st != FTK_OK) return st;
     RowsArgs a = {};
@@ -189,23 +239,46 @@ static ftk_status topk_rows_impl(ftk_dtype dtype, const void *x, int64_t rows, i
     a.row_end = row_end;
     a.out_idx = out_idx;
     a.out_val = out_val;
+    a.ldo = ldo;
+    a.idx_fill = o.idx_fill;
+    if (dtype == FTK_BF16) {
+        a.val_fill = bf16_bits(o.val_fill);
+    } else {
+        memcpy(&a.val_fill, &o.val_fill, sizeof a.val_fill);
+    }
     a.k = topk;
     a.status = status;
     int cluster = 1, chunk = 8;
     rows_plan(rows, cols, topk, &cluster, &chunk);
     a.chunk = chunk;
-    return launch_rows_topk(dtype, a, cluster, as_stream(stream));
+    const bool idx64 = o.index_bits == 64;
+    st = launch_rows_topk(dtype, a, cluster, as_stream(stream), idx64);
+    if (st != FTK_OK || !o.sorted) return st;
+    return launch_sort_rows(dtype, a, idx64, as_stream(stream));
 }
 
 }  // namespace ftk
 
 using namespace ftk;
 
+extern "C" void ftk_rows_options_init(ftk_rows_options *o)
+{
+    if (!o) return;
+    memset(o, 0, sizeof *o);
+    o->sorted = 0;
+    o->index_bits = 32;
+    o->out_stride = 0;
+    o->idx_fill = -1;
+    o->val_fill = -INFINITY;
+}
+
 extern "C" ftk_status ftk_topk_rows(ftk_dtype dtype, const void *x, int64_t rows, int64_t cols,
                                     int64_t row_stride, int topk, int32_t *out_idx,
                                     void *out_val, uint32_t *status, void *stream)
 {
-    return topk_rows_impl(dtype, x, rows, cols, row_stride, nullptr, topk, out_idx, out_val, status,
+    ftk_rows_options o;
+    ftk_rows_options_init(&o);
+    return topk_rows_impl(dtype, x, rows, cols, row_stride, nullptr, topk, o, out_idx, out_val, status,
                           stream);
 }
 
@@ -215,7 +288,9 @@ extern "C" ftk_status ftk_topk_rows_end(ftk_dtype dtype, const void *x, int64_t 
                                         void *stream)
 {
     if (!row_end) return FTK_ERR_INVALID_ARG;
-    return topk_rows_impl(dtype, x, rows, cols, row_stride, row_end, topk, out_idx, out_val, status,
+    ftk_rows_options o;
+    ftk_rows_options_init(&o);
+    return topk_rows_impl(dtype, x, rows, cols, row_stride, row_end, topk, o, out_idx, out_val, status,
                           stream);
 }
 
@@ -225,8 +300,21 @@ extern "C" ftk_status ftk_topk_rows_sorted(ftk_dtype dtype, const void *x, int64
                                            void *stream)
 {
     if (!out_val) return FTK_ERR_INVALID_ARG;
-    ftk_status st = topk_rows_impl(dtype, x, rows, cols, row_stride, row_end, topk, out_idx, out_val,
-                                   status, stream);
-    if (st != FTK_OK) return st;
-    return launch_sort_rows(dtype, out_val, out_idx, rows, topk, as_stream(stream));
+    ftk_rows_options o;
+    ftk_rows_options_init(&o);
+    o.sorted = 1;
+    return topk_rows_impl(dtype, x, rows, cols, row_stride, row_end, topk, o, out_idx, out_val, status,
+                          stream);
+}
+
+extern "C" ftk_status ftk_topk_rows_ex(ftk_dtype dtype, const void *x, int64_t rows, int64_t cols,
+                                       int64_t row_stride, const int32_t *row_end, int topk,
+                                       const ftk_rows_options *options, void *out_idx, void *out_val,
+                                       uint32_t *status, void *stream)
+{
+    ftk_rows_options o;
+    ftk_rows_options_init(&o);
+    if (options) o = *options;
+    return topk_rows_impl(dtype, x, rows, cols, row_stride, row_end, topk, o, out_idx, out_val, status,
+                          stream);
 }

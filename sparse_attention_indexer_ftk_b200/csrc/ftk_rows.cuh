@@ -47,16 +47,22 @@ struct RowsArgs {
     int64_t rows;               // rows covered by the grid
     const int32_t *nrows_dev;   // optional device count: rows >= *nrows_dev - nrows_off are skipped
     int32_t nrows_off;
+    uint32_t val_fill;          // value bits of the padding slots (x's dtype)
     const int32_t *row_map;     // optional: output row of grid row r (also indexes win_*)
     const int32_t *win_ks;      // optional windows: row length ke - ks,
     const int32_t *win_ke;      //   reported index = ks + column
     const int32_t *row_end;     // optional: row r holds columns [0, row_end[r]) (clamped to [0, cols])
-    int32_t *out_idx;           // [*, k]
-    void *out_val;              // [*, k] of the input dtype (or NULL)
+    void *out_idx;              // [*, ldo] int32 or int64 (the kernel's index type)
+    void *out_val;              // [*, ldo] of the input dtype (or NULL)
     int k;
     int chunk;                  // columns per CTA, multiple of 8
     uint32_t *status;
+    int64_t ldo;                // output row stride in elements (>= k)
+    int64_t idx_fill;           // index of the padding slots of rows shorter than k
 };
+// Kept at 128 bytes: a larger kernel parameter block made the striding
+// (LOOP) kernels spill registers.
+static_assert(sizeof(RowsArgs) <= 128, "RowsArgs grew past 128 bytes");
 
 struct RowsSmem {
     uint32_t cand_bits[kRowsWarps * kRowsCapWarp];  // raw value bits
@@ -77,6 +83,7 @@ struct RowsSmem {
 
 template <int DT>
 struct RowsTraits;
+
 
 template <>
 struct RowsTraits<FTK_BF16> {
@@ -235,7 +242,7 @@ __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.w
 // Top-k of grid row r by the whole cluster.  Returns with every cp.async
 // of this CTA complete and, for rows that used distributed shared memory,
 // with every CTA of the cluster done reading this CTA's shared memory.
-template <int DT>
+template <int DT, typename IT>
 __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, cg::cluster_group &cluster,
                                               unsigned cs, unsigned rank, int64_t r)
 {
@@ -257,8 +264,10 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
     }
     const int k = a.k;
     const elem *row = reinterpret_cast<const elem *>(a.x) + r * a.ld;
-    int32_t *oidx = a.out_idx + orow * k;
-    elem *oval = a.out_val ? reinterpret_cast<elem *>(a.out_val) + orow * k : nullptr;
+    // Every output index is below 2^31 (cols <= 2^30; windows are int32), so
+    // it is formed in 32 bits and only widened by the store when IT is int64.
+    IT *oidx = static_cast<IT *>(a.out_idx) + orow * a.ldo;
+    elem *oval = a.out_val ? static_cast<elem *>(a.out_val) + orow * a.ldo : nullptr;
     const int64_t c0 = static_cast<int64_t>(rank) * a.chunk;
     const int64_t c1 = min(len, c0 + static_cast<int64_t>(a.chunk));
     const int n = c1 > c0 ? static_cast<int>(c1 - c0) : 0;  // my columns
@@ -268,13 +277,13 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
         for (int i = tid; i < n; i += blockDim.x) {
             const uint32_t bits = row[c0 + i];
             if (Tr::isnan_bits(bits)) set_status(a.status, FTK_STATUS_NAN);
-            oidx[c0 + i] = static_cast<int32_t>(base_index + c0 + i);
+            oidx[c0 + i] = static_cast<IT>(static_cast<int32_t>(base_index + c0 + i));
             if (oval) oval[c0 + i] = static_cast<elem>(bits);
         }
         if (rank == 0) {
             for (int64_t j = len + tid; j < k; j += blockDim.x) {
-                oidx[j] = -1;
-                if (oval) oval[j] = DT == FTK_BF16 ? static_cast<elem>(0xFF80u) : static_cast<elem>(0xFF800000u);
+                oidx[j] = static_cast<IT>(a.idx_fill);
+                if (oval) oval[j] = static_cast<elem>(a.val_fill);
             }
         }
         return;
@@ -693,7 +702,7 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
         if (sel) {
             const uint32_t p = pos + __popc(sel_bal & lt_mask);
             if (p < static_cast<uint32_t>(k)) {
-                oidx[p] = static_cast<int32_t>(base_index + c0 + col);
+                oidx[p] = static_cast<IT>(static_cast<int32_t>(base_index + c0 + col));
                 if (oval) oval[p] = static_cast<elem>(bits);
             } else {
                 set_status(a.status, FTK_STATUS_INTERNAL);
@@ -709,8 +718,9 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
 
 // One cluster per row.  LOOP: clusters stride over the rows (the count may
 // be on the device), so a grid sized for the SMs serves any row count;
-// otherwise the grid holds one cluster per row.
-template <int DT, bool LOOP>
+// otherwise the grid holds one cluster per row.  IT: the output index type
+// (int32_t or int64_t).
+template <int DT, bool LOOP, typename IT>
 __global__ void __launch_bounds__(kRowsThreads, 2) rows_topk_kernel(const RowsArgs a)
 {
     extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -726,10 +736,10 @@ __global__ void __launch_bounds__(kRowsThreads, 2) rows_topk_kernel(const RowsAr
     // Row selection is uniform over the cluster: its CTAs walk the same rows.
     if constexpr (!LOOP) {
         const int64_t r = blockIdx.x / cs;
-        if (r < nrows) rows_topk_row<DT>(a, sm, cluster, cs, rank, r);
+        if (r < nrows) rows_topk_row<DT, IT>(a, sm, cluster, cs, rank, r);
     } else {
         for (int64_t r = blockIdx.x / cs; r < nrows; r += gridDim.x / cs) {
-            rows_topk_row<DT>(a, sm, cluster, cs, rank, r);
+            rows_topk_row<DT, IT>(a, sm, cluster, cs, rank, r);
             cp_async_wait<0>();
             __syncthreads();  // shared memory is free for the next row
         }

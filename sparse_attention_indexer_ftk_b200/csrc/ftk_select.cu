@@ -1026,6 +1026,9 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
         ra2.win_ke = ke;
         ra2.out_idx = out_idx;
         ra2.out_val = out_val;
+        ra2.ldo = topk;
+        ra2.idx_fill = -1;
+        ra2.val_fill = 0xFF800000u;  // -inf
         ra2.k = topk;
         ra2.chunk = rchunk;
         ra2.status = status;

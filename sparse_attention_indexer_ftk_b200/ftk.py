@@ -13,9 +13,10 @@ API (names after the pages' own):
       FlashTopK README, "Usage": Selector (owns the workspace)
   windows_from_cu_seqlens(cu_seqlens_q, cu_seqlens_k)
       FlashTopK README, "Usage"
-  topk_rows(x, topk, return_value=True)
-      DeepSelect README, "Usage": deep_select.topk (unsorted values, int32
-      indices; ours come in ascending index order)
+  topk_rows(x, topk, return_value=True, end=None, sorted=False,
+            indices_type=torch.int32, idx_fill=-1, val_fill=-inf)
+      DeepSelect README, "Usage" and "Variable-length rows":
+      deep_select.topk (unsorted output in ascending index order)
   score_dense(q, kv, weights, ks, ke, kv_scales=None, rows=None)
       the fused scores themselves, for checking
 """
@@ -40,6 +41,7 @@ EXPORTS = (
     "ftk_score_dense", "ftk_score_dense_workspace_size", "ftk_windows_from_cu_seqlens",
     "ftk_set_stage_events", "ftk_status_string", "ftk_version", "ftk_select_noalloc",
     "ftk_block_bound", "ftk_block_bound_workspace_size", "ftk_topk_rows_end", "ftk_topk_rows_sorted",
+    "ftk_rows_options_init", "ftk_topk_rows_ex",
 )
 
 
@@ -51,6 +53,15 @@ class FtkConfig(ctypes.Structure):
     _fields_ = [("sample_keys", ctypes.c_int32), ("oversample", ctypes.c_float),
                 ("capacity", ctypes.c_int32), ("prune", ctypes.c_int32),
                 ("recovery_rows", ctypes.c_int32), ("reserved", ctypes.c_int32 * 3)]
+
+
+class FtkRowsOptions(ctypes.Structure):
+    """ftk_rows_options (DeepSelect README, "Usage": sorted, indices_type,
+    the out-of-bound fill values; out_stride: the output buffers' row
+    stride)."""
+    _fields_ = [("sorted", ctypes.c_int32), ("index_bits", ctypes.c_int32),
+                ("out_stride", ctypes.c_int64), ("idx_fill", ctypes.c_int64),
+                ("val_fill", ctypes.c_float)]
 
 
 class FtkInfo(ctypes.Structure):
@@ -95,6 +106,10 @@ def load_library(path: str = LIB_PATH):
     L.ftk_topk_rows_sorted.argtypes = [I32, P, I64, I64, I64, P, I32, P, P, P, P]
     L.ftk_topk_rows_end.restype = I32
     L.ftk_topk_rows_end.argtypes = [I32, P, I64, I64, I64, P, I32, P, P, P, P]
+    L.ftk_rows_options_init.restype = None
+    L.ftk_rows_options_init.argtypes = [P]
+    L.ftk_topk_rows_ex.restype = I32
+    L.ftk_topk_rows_ex.argtypes = [I32, P, I64, I64, I64, P, I32, P, P, P, P, P]
     L.ftk_block_bound.restype = I32
     L.ftk_block_bound.argtypes = [I32, P, P, P, P, I64, I64, P, I64, P, SZ, P]
     L.ftk_block_bound_workspace_size.restype = SZ
@@ -277,41 +292,58 @@ def windows_from_cu_seqlens(cu_seqlens_q: torch.Tensor, cu_seqlens_k: torch.Tens
     return ks, ke
 
 
+def _rows_out(given, rows: int, topk: int, dtype, device, stride: int | None, what: str):
+    """A [rows, >= topk] output with a contiguous last dimension (the given
+    one, checked) and its row stride; new ones get `stride` (or topk)."""
+    if given is None:
+        width = stride or topk
+        full = torch.empty((rows, width), dtype=dtype, device=device)
+        return full[:, :topk], width
+    if (given.dim() != 2 or given.shape[0] != rows or given.shape[1] < topk or given.dtype != dtype
+            or (given.stride(1) != 1 and given.shape[1] > 1) or not given.is_cuda):
+        raise FtkError(f"{what} must be a CUDA [{rows}, >= {topk}] {dtype} tensor with a contiguous last dimension")
+    return given, given.stride(0)
+
+
 def topk_rows(x: torch.Tensor, topk: int, return_value: bool = True, status: torch.Tensor | None = None,
               out_idx: torch.Tensor | None = None, out_val: torch.Tensor | None = None,
-              end: torch.Tensor | None = None, sorted: bool = False):
+              end: torch.Tensor | None = None, sorted: bool = False,
+              indices_type: torch.dtype = torch.int32, idx_fill: int = -1, val_fill: float = float("-inf")):
     """Row top-k of a [rows, cols] bf16/fp32 CUDA tensor (ties to smaller columns).
 
     Returns (values, indices) like deep_select.topk, or indices alone when
-    return_value=False.  Indices are int32 in ascending column order, or,
-    with sorted=True, by value descending (ties by column ascending).
-    end: optional int32 [rows] per-row exclusive end (ftk_topk_rows_end).
+    return_value=False.  Indices (int32 or int64: indices_type) come in
+    ascending column order, or, with sorted=True, by value descending (ties
+    by column ascending).  end: optional int32 [rows] per-row exclusive end.
+    Rows shorter than topk are padded with idx_fill / val_fill (val_fill is
+    stored in x's dtype).  out_idx / out_val: caller-owned outputs, [rows,
+    >= topk] with a contiguous last dimension and one common row stride;
+    only their first topk columns are written.  Calls ftk_topk_rows_ex.
     """
     _need_cuda(x, status, end)
     if x.dim() != 2 or x.stride(1) != 1:
         raise FtkError("x must be 2-D with a contiguous last dimension")
+    if indices_type not in (torch.int32, torch.int64):
+        raise FtkError("indices_type must be torch.int32 or torch.int64")
     rows, cols = x.shape
-    if out_idx is None:
-        out_idx = torch.empty((rows, topk), dtype=torch.int32, device=x.device)
-    if return_value and out_val is None:
-        out_val = torch.empty((rows, topk), dtype=x.dtype, device=x.device)
+    out_idx, stride = _rows_out(out_idx, rows, topk, indices_type, x.device, None, "out_idx")
+    if return_value or out_val is not None:
+        out_val, vstride = _rows_out(out_val, rows, topk, x.dtype, x.device, stride, "out_val")
+        if vstride != stride:
+            raise FtkError("out_idx and out_val must have the same row stride")
     if end is not None and (end.shape != (rows,) or end.dtype != torch.int32 or not end.is_contiguous()):
         raise FtkError("end must be a contiguous int32 [rows] tensor")
-    if sorted:
-        if out_val is None:
-            out_val = torch.empty((rows, topk), dtype=x.dtype, device=x.device)
-        st = lib().ftk_topk_rows_sorted(_dtype_code(x), _ptr(x), rows, cols, x.stride(0), _ptr(end), topk,
-                                        _ptr(out_idx), _ptr(out_val), _ptr(status), _stream(x.device))
-        _check(st, "ftk_topk_rows_sorted")
-    elif end is None:
-        st = lib().ftk_topk_rows(_dtype_code(x), _ptr(x), rows, cols, x.stride(0), topk, _ptr(out_idx),
-                                 _ptr(out_val) if return_value else None, _ptr(status), _stream(x.device))
-        _check(st, "ftk_topk_rows")
-    else:
-        st = lib().ftk_topk_rows_end(_dtype_code(x), _ptr(x), rows, cols, x.stride(0), _ptr(end), topk,
-                                     _ptr(out_idx), _ptr(out_val) if return_value else None, _ptr(status),
-                                     _stream(x.device))
-        _check(st, "ftk_topk_rows_end")
+    opt = FtkRowsOptions()
+    lib().ftk_rows_options_init(ctypes.byref(opt))
+    opt.sorted = 1 if sorted else 0
+    opt.index_bits = 64 if indices_type == torch.int64 else 32
+    opt.out_stride = stride
+    opt.idx_fill = int(idx_fill)
+    opt.val_fill = float(val_fill)
+    st = lib().ftk_topk_rows_ex(_dtype_code(x), _ptr(x), rows, cols, x.stride(0), _ptr(end), topk,
+                                ctypes.byref(opt), _ptr(out_idx), _ptr(out_val), _ptr(status),
+                                _stream(x.device))
+    _check(st, "ftk_topk_rows_ex")
     return (out_val, out_idx) if return_value else out_idx
 
 

@@ -81,6 +81,38 @@ def test_topk_rows_sorted_host_validation(lib):
     assert lib.ftk_topk_rows_sorted(2, P(A), 4, 100, 104, None, 0, P(A), P(A), None, None) == -3
 
 
+def test_rows_options_init_defaults(lib):
+    o = ftk.FtkRowsOptions(sorted=5, index_bits=7, out_stride=9, idx_fill=11, val_fill=13.0)
+    lib.ftk_rows_options_init(ctypes.byref(o))
+    assert (o.sorted, o.index_bits, o.out_stride, o.idx_fill) == (0, 32, 0, -1)
+    assert o.val_fill == float("-inf")
+    lib.ftk_rows_options_init(None)  # no-op
+    assert ctypes.sizeof(ftk.FtkRowsOptions) == 32  # int32, int32, int64, int64, float + padding
+
+
+def test_topk_rows_ex_host_validation(lib):
+    P = ctypes.c_void_p
+
+    def call(idx=A, val=None, topk=8, **opt):
+        o = ftk.FtkRowsOptions()
+        lib.ftk_rows_options_init(ctypes.byref(o))
+        for k, v in opt.items():
+            setattr(o, k, v)
+        return lib.ftk_topk_rows_ex(2, P(A), 4, 100, 104, None, topk, ctypes.byref(o), P(idx),
+                                    None if val is None else P(val), None, None)
+    assert call(sorted=2) == -1
+    assert call(index_bits=16) == -1 and call(index_bits=0) == -1
+    assert call(out_stride=7) == -1 and call(out_stride=-8) == -1 and call(out_stride=1 << 31) == -1
+    assert call(idx_fill=1 << 31) == -1 and call(idx_fill=-(1 << 31) - 1) == -1
+    assert call(topk=0) == -3 and call(topk=4097) == -3
+    assert call(idx=0) == -1
+    assert call(idx=A + 4, index_bits=64) == -4   # int64 output on a 4-byte boundary
+    assert call(idx=A + 2) == -4                   # int32 output on a 2-byte boundary
+    assert call(val=A + 1) == -4                   # bf16 values on an odd address
+    # options=NULL means the defaults; the bad x pointer is still caught first
+    assert lib.ftk_topk_rows_ex(2, None, 4, 100, 104, None, 8, None, P(A), None, None, None) == -1
+
+
 def test_block_bound_host_validation(lib):
     P = ctypes.c_void_p
     need = lib.ftk_block_bound_workspace_size(1000)

@@ -173,3 +173,99 @@ def test_sorted_output(dtype):
             assert torch.equal(val[r, :n].view(bits), ref.view(bits)), f"row {r}: value bits"
         assert np.all(idx[r, n:] == -1)
         assert torch.all(torch.isneginf(val[r, n:].float()))
+
+
+def _options_case(dtype, seed):
+    """Rows with short, empty and full lengths, heavy ties and signed zeros."""
+    rows, cols, k = 20, 7000, 500
+    g = torch.Generator().manual_seed(seed)
+    x_cpu = torch.randn((rows, cols), generator=g).to(dtype)
+    x_cpu[2] = torch.randint(0, 4, (cols,), generator=g).to(dtype) - 1.5
+    x_cpu[3] = 0.0
+    x_cpu[3, ::5] = -0.0
+    ends = torch.full((rows,), cols, dtype=torch.int32)
+    ends[4], ends[5], ends[6], ends[7] = 0, 1, k - 1, 37
+    return x_cpu, ends, k
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("sorted_", [False, True])
+def test_int64_indices_fill_values_and_output_stride(dtype, sorted_):
+    """indices_type=int64, idx_oob_fill_value / value_oob_fill_value and a
+    caller-owned output with a row stride (DeepSelect README, "Usage" and
+    "Variable-length rows").  The fill value 0.5 lies inside the rows'
+    values, so a sort that let padding move would misplace it.  Each row
+    equals the oracle (order included when sorted); padding holds the fills;
+    columns past topk keep their contents."""
+    x_cpu, ends, k = _options_case(dtype, 123)
+    rows, cols = x_cpu.shape
+    x = aligned_rows(x_cpu)
+    width = k + 13
+    idx_buf = torch.full((rows, width), 4242, dtype=torch.int64, device="cuda")
+    val_buf = torch.full((rows, width), 7.0, dtype=dtype, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    val, idx = ftk.topk_rows(x, k, status=status, end=ends.cuda(), sorted=sorted_, indices_type=torch.int64,
+                             idx_fill=-(1 << 40), val_fill=0.5, out_idx=idx_buf, out_val=val_buf)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert idx.dtype == torch.int64 and idx.data_ptr() == idx_buf.data_ptr()
+    bits = torch.int16 if dtype == torch.bfloat16 else torch.int32
+    idx_all, val_all = idx_buf.cpu(), val_buf.cpu()
+    assert torch.all(idx_all[:, k:] == 4242) and torch.all(val_all[:, k:] == 7.0)
+    for r in range(rows):
+        e = int(ends[r])
+        n = min(k, e)
+        got = idx_all[r, :k].numpy()
+        if n:
+            oidx, _, _ = orc.topk_rows(x_cpu[r:r + 1, :e].contiguous(), k)
+            want = oidx[0, :n] if sorted_ else np.sort(oidx[0, :n])
+            assert np.array_equal(got[:n], want.astype(np.int64)), f"row {r}"
+            ref = x_cpu[r, torch.from_numpy(got[:n])]
+            assert torch.equal(val_all[r, :n].view(bits), ref.view(bits)), f"row {r}: value bits"
+        assert np.all(got[n:] == -(1 << 40))
+        assert torch.all(val_all[r, n:k] == 0.5)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_sorted_without_values_reads_x(dtype):
+    """sorted=True with return_value=False: the sort takes each selected
+    value from x; the order equals the sorted call with values."""
+    x_cpu, ends, k = _options_case(dtype, 321)
+    x = aligned_rows(x_cpu)
+    _, want = ftk.topk_rows(x, k, end=ends.cuda(), sorted=True)
+    got = ftk.topk_rows(x, k, end=ends.cuda(), sorted=True, return_value=False)
+    assert torch.equal(got, want)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_fixed_entry_points_equal_the_options_call(dtype):
+    """ftk_topk_rows, ftk_topk_rows_end and ftk_topk_rows_sorted give the
+    same bits as ftk_topk_rows_ex with the matching options."""
+    import ctypes
+    x_cpu, ends, k = _options_case(dtype, 555)
+    rows, cols = x_cpu.shape
+    x = aligned_rows(x_cpu)
+    end_d = ends.cuda()
+    L = ftk.lib()
+    code = ftk.BF16 if dtype == torch.bfloat16 else ftk.F32
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    P = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())  # noqa: E731
+
+    def fresh():
+        return (torch.full((rows, k), 99, dtype=torch.int32, device="cuda"),
+                torch.full((rows, k), 3.0, dtype=dtype, device="cuda"))
+
+    i0, v0 = fresh()
+    assert L.ftk_topk_rows(code, P(x), rows, cols, x.stride(0), k, P(i0), P(v0), None, stream) == 0
+    v, i = ftk.topk_rows(x, k)
+    assert torch.equal(i0, i) and torch.equal(v0.view(torch.uint8), v.contiguous().view(torch.uint8))
+    i1, v1 = fresh()
+    assert L.ftk_topk_rows_end(code, P(x), rows, cols, x.stride(0), P(end_d), k, P(i1), P(v1), None,
+                               stream) == 0
+    v, i = ftk.topk_rows(x, k, end=end_d)
+    assert torch.equal(i1, i) and torch.equal(v1.view(torch.uint8), v.contiguous().view(torch.uint8))
+    i2, v2 = fresh()
+    assert L.ftk_topk_rows_sorted(code, P(x), rows, cols, x.stride(0), P(end_d), k, P(i2), P(v2), None,
+                                  stream) == 0
+    v, i = ftk.topk_rows(x, k, end=end_d, sorted=True)
+    assert torch.equal(i2, i) and torch.equal(v2.view(torch.uint8), v.contiguous().view(torch.uint8))
