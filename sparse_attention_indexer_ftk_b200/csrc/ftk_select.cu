@@ -584,7 +584,11 @@ struct SelectCfg {
     int cap;
     PruneMode prune;
     int rec_rows;
+    int64_t scratch_floats;  // recovery scratch reserved, >= rec_rows * scratch row stride
 };
+
+// Row stride of the recovery scratch (floats): S rounded up to 8.
+static int64_t scratch_ld_of(int64_t S) { return (S + 7) / 8 * 8; }
 
 static SelectCfg resolve_cfg(int64_t T, int64_t S, int topk, const ftk_config *c)
 {
@@ -600,18 +604,22 @@ static SelectCfg resolve_cfg(int64_t T, int64_t S, int topk, const ftk_config *c
     if (r.m < min_m) r.m = static_cast<int>(min_m);
     if (r.m < 32) r.m = 32;
     if (r.m > 32768) r.m = 32768;
-    int64_t rr = c && c->recovery_rows > 0 ? c->recovery_rows : 0;
-    if (rr == 0) {
-        // At most 2^27 floats (512 MB) of recovery scratch, at least 64 rows;
-        // non-increasing in S so that a larger plan serves smaller calls.
-        const int64_t ld = (S + 7) / 8 * 8;
-        rr = ((int64_t(1) << 27) / ld) & ~static_cast<int64_t>(kMaxRowTile - 1);
-        if (rr < 64) rr = 64;
-    }
-    rr = (rr + kMaxRowTile - 1) / kMaxRowTile * kMaxRowTile;
+    // Recovery scratch: rec_rows rows of ld floats.  The reservation is a
+    // non-decreasing function of T and S (so a workspace planned for (T, S)
+    // serves every call with smaller T and S), and rec_rows is what fits.
+    const int64_t ld = scratch_ld_of(S);
     const int64_t tcap = (T + kMaxRowTile - 1) / kMaxRowTile * kMaxRowTile;
-    if (rr > tcap) rr = tcap;
-    r.rec_rows = static_cast<int>(rr);
+    int64_t budget;
+    if (c && c->recovery_rows > 0) {
+        budget = (static_cast<int64_t>(c->recovery_rows) + kMaxRowTile - 1) / kMaxRowTile * kMaxRowTile * ld;
+    } else {
+        // 2^27 floats (512 MB), or 64 rows when rows are longer than 2^21 keys
+        budget = int64_t(1) << 27;
+        if (budget < 64 * ld) budget = 64 * ld;
+    }
+    if (budget > tcap * ld) budget = tcap * ld;
+    r.scratch_floats = budget;
+    r.rec_rows = static_cast<int>(budget / ld / kMaxRowTile * kMaxRowTile);
     return r;
 }
 
@@ -653,8 +661,8 @@ static bool carve_select(Carver &cv, int64_t T, int64_t S, const SelectCfg &c, S
     w.cand_idx = cv.take<int32_t>(T * static_cast<int64_t>(c.cap));
     w.bad_rows = cv.take<int32_t>(T);
     w.bad_count = cv.take<int32_t>(1);
-    w.scratch_ld = (S + 7) / 8 * 8;
-    w.scratch = cv.take<float>(static_cast<int64_t>(c.rec_rows) * w.scratch_ld);
+    w.scratch_ld = scratch_ld_of(S);
+    w.scratch = cv.take<float>(c.scratch_floats);
     w.nblocks = static_cast<int32_t>((S + kBlockKeys - 1) / kBlockKeys);
     w.nwords = (w.nblocks + kBoundWordBlocks - 1) / kBoundWordBlocks;
     if (c.prune != PRUNE_OFF) {

@@ -63,6 +63,23 @@ def test_workspace_size(lib):
     assert lib.ftk_select_workspace_size(4096, 131072, 2048, ctypes.byref(cfg)) >= n1
 
 
+def test_workspace_planned_for_larger_sizes_serves_smaller_calls(lib):
+    """The size is non-decreasing in T and S (the header's promise behind
+    Selector.plan(max_rows, max_kv)): a workspace planned for (T, S) is
+    large enough for every call with smaller T and S.  The recovery scratch
+    once broke this: rows x row length rounded to multiples of 16 rows
+    grew for some smaller S."""
+    cfgs = [None, ftk.FtkConfig(recovery_rows=8), ftk.FtkConfig(recovery_rows=100, capacity=64),
+            ftk.FtkConfig(prune=-1), ftk.FtkConfig(sample_keys=64)]
+    for cfg in cfgs:
+        ref = None if cfg is None else ctypes.byref(cfg)
+        for T, S in [(17, 129), (4096, 1000000), (8192, 262144), (64, 3000000)]:
+            big = lib.ftk_select_workspace_size(T, S, 2048, ref)
+            for S2 in sorted({1, S // 2 + 1} | set(range(S // 2 + 1, S + 1, max(1, S // 61)))):
+                for T2 in (1, T // 2 + 1, T):
+                    assert lib.ftk_select_workspace_size(T2, S2, 2048, ref) <= big, (cfg, T, S, T2, S2)
+
+
 A = 0x10000  # a 16-byte aligned stand-in pointer (never dereferenced on the host)
 
 
