@@ -176,9 +176,35 @@ def _check_select_inputs(q, kv, weights, ks, ke, kv_scales):
     for name, w in (("ks", ks), ("ke", ke)):
         if w.shape != (T,) or w.dtype != torch.int32 or not w.is_contiguous():
             raise FtkError(f"{name} must be a contiguous int32 [T] tensor")
+    for t in (kv, weights, ks, ke, kv_scales):
+        if t is not None and t.device != q.device:
+            raise FtkError("all inputs must be on q's device")
     if kv_scales is not None and (kv_scales.shape != (kv.shape[0],) or kv_scales.dtype != torch.float32
                                   or not kv_scales.is_contiguous()):
         raise FtkError("kv_scales must be a contiguous float32 [S] tensor")
+
+
+def _check_buffer(t: torch.Tensor | None, shape: tuple, dtype: torch.dtype, device: torch.device, what: str):
+    """A caller-provided buffer the kernels write: exactly `shape`, `dtype`,
+    contiguous and on the inputs' device (None passes)."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype or not t.is_contiguous() or t.device != device:
+        raise FtkError(f"{what} must be a contiguous {dtype} tensor of shape {list(shape)} on {device}")
+
+
+def _check_workspace(ws: torch.Tensor | None, device: torch.device):
+    if ws is not None and (ws.dtype != torch.uint8 or ws.dim() != 1 or not ws.is_contiguous()
+                           or ws.device != device):
+        raise FtkError(f"workspace must be a contiguous 1-D uint8 tensor on {device}")
+
+
+def _check_status(status: torch.Tensor | None, device: torch.device):
+    """The status word the kernels OR bits into: a 32-bit integer tensor of
+    at least one element on the inputs' device (None passes)."""
+    if status is not None and (status.dtype not in (torch.int32, torch.uint32) or status.numel() < 1
+                               or not status.is_contiguous() or status.device != device):
+        raise FtkError(f"status must be a contiguous int32 tensor of at least one element on {device}")
 
 
 def select_workspace_size(T: int, S: int, topk: int, config: dict | None = None) -> int:
@@ -197,6 +223,10 @@ def select(q, kv, weights, ks, ke, kv_scales=None, topk: int = 2048, return_scor
     _check_select_inputs(q, kv, weights, ks, ke, kv_scales)
     T, S = q.shape[0], kv.shape[0]
     dev = q.device
+    _check_workspace(workspace, dev)
+    _check_buffer(out_idx, (T, topk), torch.int32, dev, "out_idx")
+    if return_scores:
+        _check_buffer(out_val, (T, topk), torch.float32, dev, "out_val")
     if workspace is None:
         workspace = torch.empty(select_workspace_size(T, S, topk, config), dtype=torch.uint8, device=dev)
     if out_idx is None:
@@ -270,6 +300,8 @@ class Selector:
             self.plan(q.shape[0], kv.shape[0], q.device)
         if q.shape[0] > self.max_rows or kv.shape[0] > self.max_kv:
             raise FtkError("inputs exceed the planned sizes")
+        if q.dtype != self.dtype:
+            raise FtkError(f"this Selector was made for {self.dtype} inputs, not {q.dtype}")
         return select(q, kv, weights, ks, ke, kv_scales, self.topk, return_scores,
                       workspace=self.workspace, config=self.config, out_idx=out_idx, out_val=out_val)
 
@@ -300,8 +332,9 @@ def _rows_out(given, rows: int, topk: int, dtype, device, stride: int | None, wh
         full = torch.empty((rows, width), dtype=dtype, device=device)
         return full[:, :topk], width
     if (given.dim() != 2 or given.shape[0] != rows or given.shape[1] < topk or given.dtype != dtype
-            or (given.stride(1) != 1 and given.shape[1] > 1) or not given.is_cuda):
-        raise FtkError(f"{what} must be a CUDA [{rows}, >= {topk}] {dtype} tensor with a contiguous last dimension")
+            or (given.stride(1) != 1 and given.shape[1] > 1) or given.device != device):
+        raise FtkError(f"{what} must be a [{rows}, >= {topk}] {dtype} tensor on {device} with a contiguous "
+                       "last dimension")
     return given, given.stride(0)
 
 
@@ -331,8 +364,10 @@ def topk_rows(x: torch.Tensor, topk: int, return_value: bool = True, status: tor
         out_val, vstride = _rows_out(out_val, rows, topk, x.dtype, x.device, stride, "out_val")
         if vstride != stride:
             raise FtkError("out_idx and out_val must have the same row stride")
-    if end is not None and (end.shape != (rows,) or end.dtype != torch.int32 or not end.is_contiguous()):
-        raise FtkError("end must be a contiguous int32 [rows] tensor")
+    if end is not None and (end.shape != (rows,) or end.dtype != torch.int32 or not end.is_contiguous()
+                            or end.device != x.device):
+        raise FtkError("end must be a contiguous int32 [rows] tensor on x's device")
+    _check_status(status, x.device)
     opt = FtkRowsOptions()
     lib().ftk_rows_options_init(ctypes.byref(opt))
     opt.sorted = 1 if sorted else 0

@@ -44,3 +44,88 @@ def test_block_structured_keys():
     assert torch.equal(c.kv_scales[hot], base.kv_scales[hot])
     assert torch.allclose(c.kv_scales[~hot], base.kv_scales[~hot] * 2.0 ** -7)
     assert bool(torch.all(c.weights[:, 1:8] >= 0)) and bool(torch.all(c.weights[:, ::8] <= 0))
+
+
+def test_binding_rejects_buffers_the_kernels_would_overrun():
+    """Caller-provided outputs, workspaces and status words are checked in
+    the binding before any pointer reaches the library (CPU tensors stand in
+    for device ones: the checks compare shapes, dtypes, layout, devices)."""
+    import pytest
+    from sparse_attention_indexer_ftk_b200 import ftk
+    cpu = torch.device("cpu")
+    ok = torch.empty((5, 7), dtype=torch.int32)
+    ftk._check_buffer(ok, (5, 7), torch.int32, cpu, "out_idx")
+    ftk._check_buffer(None, (5, 7), torch.int32, cpu, "out_idx")
+    for bad in (torch.empty((5, 6), dtype=torch.int32), torch.empty((4, 7), dtype=torch.int32),
+                torch.empty((5, 7), dtype=torch.int64), torch.empty((7, 5), dtype=torch.int32).t(),
+                torch.empty(35, dtype=torch.int32)):
+        with pytest.raises(ftk.FtkError):
+            ftk._check_buffer(bad, (5, 7), torch.int32, cpu, "out_idx")
+    ftk._check_workspace(torch.empty(100, dtype=torch.uint8), cpu)
+    for bad in (torch.empty(100, dtype=torch.float32), torch.empty((10, 10), dtype=torch.uint8),
+                torch.empty(200, dtype=torch.uint8)[::2]):
+        with pytest.raises(ftk.FtkError):
+            ftk._check_workspace(bad, cpu)
+    ftk._check_status(torch.zeros(1, dtype=torch.int32), cpu)
+    ftk._check_status(None, cpu)
+    for bad in (torch.zeros(0, dtype=torch.int32), torch.zeros(1, dtype=torch.int16),
+                torch.zeros(1, dtype=torch.float32)):
+        with pytest.raises(ftk.FtkError):
+            ftk._check_status(bad, cpu)
+    with pytest.raises(ftk.FtkError):
+        ftk._check_status(torch.zeros(1, dtype=torch.int32), torch.device("cuda", 0))
+
+
+class _FakeLib:
+    """Stands in for libftk: records calls, returns FTK_OK."""
+
+    def __init__(self):
+        self.calls = []
+
+    def __getattr__(self, name):
+        def fn(*args):
+            self.calls.append(name)
+            return 1024 if name.endswith("workspace_size") else 0
+        return fn
+
+
+def test_binding_accepts_the_calls_bench_and_tests_make(monkeypatch):
+    """select(), Selector.run() and topk_rows() with conforming buffers (the
+    patterns bench.py and the GPU tests use) pass the binding's checks and
+    reach the library; CPU tensors and a fake library stand in for the GPU."""
+    import pytest
+    from sparse_attention_indexer_ftk_b200 import ftk
+    fake = _FakeLib()
+    monkeypatch.setattr(ftk, "lib", lambda: fake)
+    monkeypatch.setattr(ftk, "_need_cuda", lambda *ts: None)
+    monkeypatch.setattr(ftk, "_stream", lambda dev: None)
+    c = wl.small_case(seed=3, dtype="fp8", T=9, S=300, topk=16, windows="causal")
+    T, k = c.T, c.topk
+    ws = torch.empty(ftk.select_workspace_size(T, c.S, k), dtype=torch.uint8)
+    oi = torch.empty((T, k), dtype=torch.int32)
+    ov = torch.empty((T, k), dtype=torch.float32)
+    ftk.select(c.q, c.kv, c.weights, c.ks, c.ke, c.kv_scales, k, return_scores=True, workspace=ws,
+               out_idx=oi, out_val=ov)
+    ftk.select(c.q, c.kv, c.weights, c.ks, c.ke, c.kv_scales, k, return_scores=True, workspace=ws,
+               config={"prune": 1})
+    ftk.select(c.q, c.kv, c.weights, c.ks, c.ke, None, k)
+    sel = ftk.Selector(topk=k, dtype=torch.float8_e4m3fn).plan(32, 8000, device="cpu")
+    sel.run(c.q, c.kv, c.weights, c.ks, c.ke, c.kv_scales)
+    assert fake.calls.count("ftk_select") == 4
+    with pytest.raises(ftk.FtkError):
+        ftk.select(c.q, c.kv, c.weights, c.ks, c.ke, c.kv_scales, k, out_idx=oi[:, :-1])
+    with pytest.raises(ftk.FtkError):
+        ftk.Selector(topk=k, dtype=torch.bfloat16).plan(32, 8000, device="cpu").run(
+            c.q, c.kv, c.weights, c.ks, c.ke, c.kv_scales)
+    x = torch.randn(6, 1000).to(torch.bfloat16)
+    st = torch.zeros(1, dtype=torch.int32)
+    end = torch.full((6,), 500, dtype=torch.int32)
+    xi = torch.empty((6, 64), dtype=torch.int32)
+    xv = torch.empty((6, 64), dtype=torch.bfloat16)
+    ftk.topk_rows(x, 64, out_idx=xi, out_val=xv)
+    ftk.topk_rows(x, 64, status=st, end=end, sorted=True)
+    ftk.topk_rows(x, 64, return_value=False)
+    val, idx = ftk.topk_rows(x, 64, end=end, indices_type=torch.int64, idx_fill=-5, val_fill=0.0,
+                             out_idx=torch.empty((6, 70), dtype=torch.int64))
+    assert val.shape == (6, 64) and val.stride(0) == 70 and idx.dtype == torch.int64
+    assert fake.calls.count("ftk_topk_rows_ex") == 4
