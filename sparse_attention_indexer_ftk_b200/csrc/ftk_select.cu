@@ -819,7 +819,7 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
     pa.ntiles = ntiles;
     pa.rt = rt;
     pa.sample_keys = c.m;
-    // Scan work items: up to 128 key tiles each, fewer when the call is
+    // Scan work items: up to kChunkTiles key tiles each, fewer when the call is
     // small (few query rows, decode-like) so that the items still cover
     // every SM about twice.
     {
