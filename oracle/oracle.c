@@ -13,9 +13,13 @@
  *
  * Sources (web pages; cited by page title and section):
  *   [FTK-QS]  FlashTopK README, "Quick start": the score
- *             I[t,s] = sigma_s * sum_{h=1..32} w[t,h] * ReLU(q[t,h] . k[s]),
- *             head dimension 128, window [ks[t], ke[t]), sigma = kv_scales,
- *             1 for BF16 keys; output int32 indices [T, topk].
+ *             I[t,s] = sigma_s * sum_{h=1..H} w[t,h] * ReLU(q[t,h] . k[s]),
+ *             H = 32 heads of dimension 128, window [ks[t], ke[t]),
+ *             sigma = kv_scales, 1 for BF16 keys; output int32 indices
+ *             [T, topk].
+ *   [FTK-RM]  FlashTopK README, "Roadmap": indexers with other head counts,
+ *             such as 64 heads.  The head count H is an argument here
+ *             (the sum runs over every head of q[t]).
  *   [FTK-HL]  FlashTopK README, "Highlights": exact top-k; ties at the k-th
  *             score keep the smallest key indices.
  *   [FTK-SUP] FlashTopK README, "Support": 32 heads x 128, FP8 or BF16,
@@ -45,7 +49,7 @@
 #endif
 
 enum { ORC_E4M3 = 1, ORC_BF16 = 2, ORC_F32 = 3 };
-enum { ORC_HEADS = 32, ORC_DIM = 128 };
+enum { ORC_DIM = 128 };  /* head dimension; the head count H is an argument */
 
 /* ---------------------------------------------------------------------- */
 /* Value decoding                                                           */
@@ -108,12 +112,12 @@ void orc_decode(int dtype, const void *src, int64_t n, double *dst)
 
 /* Score of one (t, s) pair and its rounding-error scale
  *   E = sigma_s * sum_h |w[t,h]| * sum_d |q[t,h,d] * k[s,d]|.
- * qd: the 32x128 decoded heads of q[t]; wt: the 32 weights of row t. */
-static void score_pair(const double *qd, const double *wt, const double *kd,
+ * qd: the heads x 128 decoded heads of q[t]; wt: the heads weights of row t. */
+static void score_pair(int heads, const double *qd, const double *wt, const double *kd,
                        double sigma, double *I_out, double *E_out)
 {
     double acc = 0.0, err = 0.0;
-    for (int h = 0; h < ORC_HEADS; ++h) {
+    for (int h = 0; h < heads; ++h) {
         double dot = 0.0, absdot = 0.0;
         for (int d = 0; d < ORC_DIM; ++d) {
             double p = qd[h * ORC_DIM + d] * kd[d];
@@ -135,16 +139,17 @@ static int window_ok(int32_t ks, int32_t ke, int64_t S)
 
 /*
  * Scores of the windows of the listed rows.
- *   q        [T, 32, 128] of dtype, row-major
+ *   heads    H >= 1, the head count of the indexer
+ *   q        [T, H, 128] of dtype, row-major
  *   kv       [S, 128] of dtype
  *   kv_scales [S] float32, or NULL for all-ones
- *   weights  [T, 32] float32
+ *   weights  [T, H] float32
  *   rows     the nrows query indices to score
  *   out_I, out_E  [nrows, ld]: entry (r, s - ks[t]) for s in [ks[t], ke[t])
  * Returns the number of listed rows with an invalid window (those rows are
  * left untouched).
  */
-int64_t orc_index_scores(int dtype, const void *q, const void *kv,
+int64_t orc_index_scores(int dtype, int heads, const void *q, const void *kv,
                          const float *kv_scales, const float *weights,
                          int64_t T, int64_t S, const int32_t *ks,
                          const int32_t *ke, const int64_t *rows,
@@ -159,21 +164,25 @@ int64_t orc_index_scores(int dtype, const void *q, const void *kv,
             bad += 1;
             continue;
         }
-        double qd[ORC_HEADS * ORC_DIM], wt[ORC_HEADS], kd[ORC_DIM];
-        for (int i = 0; i < ORC_HEADS * ORC_DIM; ++i)
-            qd[i] = element(dtype, q, t * ORC_HEADS * ORC_DIM + i);
-        for (int h = 0; h < ORC_HEADS; ++h)
-            wt[h] = (double)weights[t * ORC_HEADS + h];
+        double *qd = (double *)malloc(sizeof(double) * heads * ORC_DIM);
+        double *wt = (double *)malloc(sizeof(double) * heads);
+        double kd[ORC_DIM];
+        for (int64_t i = 0; i < (int64_t)heads * ORC_DIM; ++i)
+            qd[i] = element(dtype, q, t * heads * ORC_DIM + i);
+        for (int h = 0; h < heads; ++h)
+            wt[h] = (double)weights[t * heads + h];
         for (int64_t s = ks[t]; s < ke[t]; ++s) {
             for (int d = 0; d < ORC_DIM; ++d)
                 kd[d] = element(dtype, kv, s * ORC_DIM + d);
             double sigma = kv_scales ? (double)kv_scales[s] : 1.0;
             double I, E;
-            score_pair(qd, wt, kd, sigma, &I, &E);
+            score_pair(heads, qd, wt, kd, sigma, &I, &E);
             out_I[r * ld + (s - ks[t])] = I;
             if (out_E)
                 out_E[r * ld + (s - ks[t])] = E;
         }
+        free(qd);
+        free(wt);
     }
     return bad;
 }
@@ -197,7 +206,7 @@ int64_t orc_index_scores(int dtype, const void *q, const void *kv,
  *   out_scale [nrows, nblocks] or NULL: sum_h |w| sum_d |q| max(|hi|, |lo|),
  *             the size of the terms UB is summed from
  */
-void orc_block_bound(int dtype, const void *q, const void *kv, const float *kv_scales,
+void orc_block_bound(int dtype, int heads, const void *q, const void *kv, const float *kv_scales,
                      const float *weights, int64_t T, int64_t S, int64_t block,
                      const int64_t *rows, int64_t nrows, double *out_ub, double *out_scale)
 {
@@ -221,15 +230,16 @@ void orc_block_bound(int dtype, const void *q, const void *kv, const float *kv_s
 #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t r = 0; r < nrows; ++r) {
         int64_t t = rows[r];
-        double qd[ORC_HEADS * ORC_DIM], wt[ORC_HEADS];
-        for (int i = 0; i < ORC_HEADS * ORC_DIM; ++i)
-            qd[i] = element(dtype, q, t * ORC_HEADS * ORC_DIM + i);
-        for (int h = 0; h < ORC_HEADS; ++h)
-            wt[h] = weights[(int64_t)t * ORC_HEADS + h];
+        double *qd = (double *)malloc(sizeof(double) * heads * ORC_DIM);
+        double *wt = (double *)malloc(sizeof(double) * heads);
+        for (int64_t i = 0; i < (int64_t)heads * ORC_DIM; ++i)
+            qd[i] = element(dtype, q, t * heads * ORC_DIM + i);
+        for (int h = 0; h < heads; ++h)
+            wt[h] = weights[(int64_t)t * heads + h];
         for (int64_t b = 0; b < nb; ++b) {
             const double *bh = hi + b * ORC_DIM, *bl = lo + b * ORC_DIM;
             double ub = 0.0, scale = 0.0;
-            for (int h = 0; h < ORC_HEADS; ++h) {
+            for (int h = 0; h < heads; ++h) {
                 double U = 0.0, L = 0.0, mag = 0.0;
                 for (int d = 0; d < ORC_DIM; ++d) {
                     double x = qd[h * ORC_DIM + d] * bh[d];
@@ -248,6 +258,8 @@ void orc_block_bound(int dtype, const void *q, const void *kv, const float *kv_s
             if (out_scale)
                 out_scale[r * nb + b] = scale;
         }
+        free(qd);
+        free(wt);
     }
     free(hi);
     free(lo);
@@ -346,7 +358,7 @@ int64_t orc_select_f32_rows(const float *scores, int64_t rows, int64_t ld,
  * [nrows]) gets 1 for a NaN score, 2 for an invalid window.
  * Returns the number of flagged rows.
  */
-int64_t orc_fused_select(int dtype, const void *q, const void *kv,
+int64_t orc_fused_select(int dtype, int heads, const void *q, const void *kv,
                          const float *kv_scales, const float *weights,
                          int64_t T, int64_t S, const int32_t *ks,
                          const int32_t *ke, const int64_t *rows, int64_t nrows,
@@ -368,7 +380,7 @@ int64_t orc_fused_select(int dtype, const void *q, const void *kv,
             int64_t L = (int64_t)ke[t] - ks[t];
             double *I = (double *)malloc((size_t)(L > 0 ? L : 1) * sizeof(double));
             int64_t one = t;
-            orc_index_scores(dtype, q, kv, kv_scales, weights, T, S, ks, ke,
+            orc_index_scores(dtype, heads, q, kv, kv_scales, weights, T, S, ks, ke,
                              &one, 1, L > 0 ? L : 1, I, NULL);
             if (orc_select_f64(I, L, ks[t], k, out_idx + r * k,
                                out_val + r * k))

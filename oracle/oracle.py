@@ -7,7 +7,8 @@ imports this module and shares no code with it.
 The oracle computes, in IEEE double, the plain definitions from the pages:
 
 * FlashTopK README, "Quick start": I[t,s] = sigma_s * sum_h w[t,h] *
-  ReLU(q[t,h] . k[s]) over the window [ks[t], ke[t]);
+  ReLU(q[t,h] . k[s]) over the window [ks[t], ke[t]); the head count H is
+  q.shape[1] (32 on the pages; "Roadmap": other head counts, such as 64);
 * FlashTopK README, "Highlights": the exact top-k, ties at the k-th score
   to the smallest key indices;
 * DeepSelect README, "Usage": the row top-k of a bf16 / fp32 matrix.
@@ -55,17 +56,17 @@ def load(path: str):
     L.orc_decode.restype = None
     L.orc_decode.argtypes = [I32, P, I64, P]
     L.orc_index_scores.restype = I64
-    L.orc_index_scores.argtypes = [I32, P, P, P, P, I64, I64, P, P, P, I64, I64, P, P]
+    L.orc_index_scores.argtypes = [I32, I32, P, P, P, P, I64, I64, P, P, P, I64, I64, P, P]
     L.orc_select_f64.restype = I32
     L.orc_select_f64.argtypes = [P, I64, I64, I32, P, P]
     L.orc_select_f32_rows.restype = I64
     L.orc_select_f32_rows.argtypes = [P, I64, I64, P, P, I64, P, I32, P, P]
     L.orc_fused_select.restype = I64
-    L.orc_fused_select.argtypes = [I32, P, P, P, P, I64, I64, P, P, P, I64, I32, P, P, P]
+    L.orc_fused_select.argtypes = [I32, I32, P, P, P, P, I64, I64, P, P, P, I64, I32, P, P, P]
     L.orc_topk_rows.restype = I64
     L.orc_topk_rows.argtypes = [I32, P, I64, I64, I64, I32, P, P, P]
     L.orc_num_threads.restype = I32
-    L.orc_block_bound.argtypes = [I32, P, P, P, P, I64, I64, I64, P, I64, P, P]
+    L.orc_block_bound.argtypes = [I32, I32, P, P, P, P, I64, I64, I64, P, I64, P, P]
     L.orc_block_bound.restype = None
     L.orc_num_threads.argtypes = []
     return L
@@ -149,6 +150,15 @@ def decode(x) -> np.ndarray:
     return out.reshape(tuple(x.shape))
 
 
+def _heads(q, weights) -> int:
+    """H of a [T, H, 128] q, checked against the [T, H] weights."""
+    if q.dim() != 3 or q.shape[2] != 128 or q.shape[1] < 1:
+        raise ValueError("q must be [T, H, 128]")
+    if tuple(weights.shape) != (q.shape[0], q.shape[1]):
+        raise ValueError("weights must be [T, H] for q of shape [T, H, 128]")
+    return int(q.shape[1])
+
+
 def _rows_arg(rows, T):
     if rows is None:
         rows = np.arange(T, dtype=np.int64)
@@ -171,7 +181,7 @@ def index_scores(q, kv, kv_scales, weights, ks, ke, rows=None, ld=None):
         ld = int(max(1, max((int(ke_[t]) - int(ks_[t]) for t in rows), default=1)))
     I = np.full((rows.size, ld), np.nan)
     E = np.full((rows.size, ld), np.nan)
-    lib().orc_index_scores(dtype_code(q), _ptr(qr), _ptr(kr), _ptr(sc), _ptr(w), T, S,
+    lib().orc_index_scores(dtype_code(q), _heads(q, weights), _ptr(qr), _ptr(kr), _ptr(sc), _ptr(w), T, S,
                            _ptr(ks_), _ptr(ke_), _ptr(rows), rows.size, ld, _ptr(I), _ptr(E))
     return I, E
 
@@ -190,7 +200,7 @@ def block_bound(q, kv, kv_scales, weights, block: int = 128, rows=None):
     nb = (S + block - 1) // block
     ub = np.empty((rows.size, nb))
     scale = np.empty((rows.size, nb))
-    lib().orc_block_bound(dtype_code(q), _ptr(qr), _ptr(kr), _ptr(sc), _ptr(w), T, S, block,
+    lib().orc_block_bound(dtype_code(q), _heads(q, weights), _ptr(qr), _ptr(kr), _ptr(sc), _ptr(w), T, S, block,
                           _ptr(rows), rows.size, _ptr(ub), _ptr(scale))
     return ub, scale
 
@@ -232,7 +242,7 @@ def fused_select(q, kv, kv_scales, weights, ks, ke, k: int, rows=None):
     idx = np.empty((rows.size, k), dtype=np.int64)
     val = np.empty((rows.size, k), dtype=np.float64)
     flags = np.zeros(rows.size, dtype=np.int32)
-    lib().orc_fused_select(dtype_code(q), _ptr(qr), _ptr(kr), _ptr(sc), _ptr(w), T, S,
+    lib().orc_fused_select(dtype_code(q), _heads(q, weights), _ptr(qr), _ptr(kr), _ptr(sc), _ptr(w), T, S,
                            _ptr(ks_), _ptr(ke_), _ptr(rows), rows.size, k,
                            _ptr(idx), _ptr(val), _ptr(flags))
     return idx, val, flags

@@ -263,18 +263,19 @@ def fp8_packed(gamma: float = 6.0) -> SelectInputs:
 
 def small_case(seed: int, dtype: str, T: int, S: int, topk: int,
                windows: str = "causal", scales: bool = True,
-               kv_levels: int = 0) -> SelectInputs:
+               kv_levels: int = 0, heads: int = 32) -> SelectInputs:
     """A generic small case.
 
     windows: "causal" | "random" | "short" | "empty_mix" | "packed".
     kv_levels > 0 rounds key entries onto that many levels (forces ties).
+    heads: the indexer's head count H (q [T, H, 128], weights [T, H]).
     """
     g = torch.Generator(device="cpu")
     g.manual_seed(SEED_BASE + 1000 + seed)
-    q = _normal(g, (T, 32, 128))
+    q = _normal(g, (T, heads, 128))
     kv = _normal(g, (S, 128))
     sc = _scales(g, S) if scales else None
-    w = _weights(g, T)
+    w = _weights(g, T, heads)
     if kv_levels:
         kv = (kv.clamp(-2, 2) * (kv_levels / 4)).round() / (kv_levels / 4)
     if windows == "causal":

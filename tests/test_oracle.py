@@ -80,9 +80,9 @@ def _decoded(t):
     return t.to(torch.float32).double().numpy()
 
 
-def _case(seed, dtype, T, S, nonneg=False):
+def _case(seed, dtype, T, S, nonneg=False, heads=32):
     g = torch.Generator().manual_seed(seed)
-    q = torch.randn((T, 32, 128), generator=g)
+    q = torch.randn((T, heads, 128), generator=g)
     kv = torch.randn((S, 128), generator=g)
     if nonneg:
         q, kv = q.abs(), kv.abs()
@@ -141,6 +141,51 @@ def check_score_linear_in_weights(dtype):
         Ih, _ = orc.index_scores(q, kv, sc, eh, ks, ke)
         acc += w[:, h].double().numpy()[:, None] * Ih
     np.testing.assert_allclose(I, acc, rtol=1e-12, atol=1e-12)
+
+
+def check_score_single_head(dtype):
+    """H = 1 (FlashTopK README, "Roadmap": other head counts): the score is
+    the closed form w * sigma * ReLU(q . k) and E = |w| * sigma * (|q| . |k|),
+    one numpy matmul each; weights of both signs (one row per call)."""
+    S = 60
+    q, kv, sc = _case(15, dtype, 1, S, heads=1)
+    ks, ke = _full_windows(1, S)
+    qd, kd, s = _decoded(q)[:, 0, :], _decoded(kv), sc.double().numpy()
+    for c in (0.625, -1.375):
+        w = torch.full((1, 1), c)
+        I, E = orc.index_scores(q, kv, sc, w, ks, ke)
+        np.testing.assert_allclose(I[0], c * s * np.maximum(qd @ kd.T, 0.0)[0], rtol=1e-12, atol=1e-300)
+        np.testing.assert_allclose(E[0], abs(c) * s * (np.abs(qd) @ np.abs(kd).T)[0], rtol=1e-12, atol=0)
+
+
+def check_score_heads_split(dtype):
+    """A 64-head score is the sum of the scores of its two 32-head halves
+    (and so is E): the head sum covers every head of q[t], with the row
+    stride of H heads."""
+    T, S = 4, 45
+    q, kv, sc = _case(16, dtype, T, S, heads=64)
+    w = torch.randn((T, 64), generator=torch.Generator().manual_seed(8)) / 8
+    ks, ke = _full_windows(T, S)
+    I, E = orc.index_scores(q, kv, sc, w, ks, ke)
+    Ia, Ea = orc.index_scores(q[:, :32].contiguous(), kv, sc, w[:, :32].contiguous(), ks, ke)
+    Ib, Eb = orc.index_scores(q[:, 32:].contiguous(), kv, sc, w[:, 32:].contiguous(), ks, ke)
+    np.testing.assert_allclose(I, Ia + Ib, rtol=0, atol=1e-12 * E.max())
+    np.testing.assert_allclose(E, Ea + Eb, rtol=1e-12, atol=0)
+    assert np.abs(Ib).max() > 0 and np.abs(Ia).max() > 0
+
+
+def check_score_head_permutation():
+    """Permuting the heads of q and w together leaves the score unchanged
+    (H = 48, not a power of two)."""
+    T, S = 3, 37
+    q, kv, sc = _case(17, "bf16", T, S, heads=48)
+    w = torch.randn((T, 48), generator=torch.Generator().manual_seed(9))
+    perm = torch.randperm(48, generator=torch.Generator().manual_seed(10))
+    ks, ke = _full_windows(T, S)
+    I, E = orc.index_scores(q, kv, sc, w, ks, ke)
+    Ip, Ep = orc.index_scores(q[:, perm].contiguous(), kv, sc, w[:, perm].contiguous(), ks, ke)
+    np.testing.assert_allclose(Ip, I, rtol=0, atol=1e-12 * E.max())
+    np.testing.assert_allclose(Ep, E, rtol=1e-12, atol=0)
 
 
 def check_score_homogeneity():
@@ -203,6 +248,27 @@ def test_score_one_hot_heads(dtype):
 @pytest.mark.parametrize("dtype", ["fp8", "bf16"])
 def test_score_linear_in_weights(dtype):
     check_score_linear_in_weights(dtype)
+
+
+@pytest.mark.parametrize("dtype", ["fp8", "bf16"])
+def test_score_single_head(dtype):
+    check_score_single_head(dtype)
+
+
+@pytest.mark.parametrize("dtype", ["fp8", "bf16"])
+def test_score_heads_split(dtype):
+    check_score_heads_split(dtype)
+
+
+def test_score_head_permutation():
+    check_score_head_permutation()
+
+
+def test_heads_shape_checked():
+    q, kv, sc = _case(18, "bf16", 2, 10, heads=64)
+    ks, ke = _full_windows(2, 10)
+    with pytest.raises(ValueError):
+        orc.index_scores(q, kv, sc, torch.ones((2, 32)), ks, ke)
 
 
 def test_score_homogeneity():
@@ -444,16 +510,16 @@ def test_fused_window_locality():
 # block score bound
 # ---------------------------------------------------------------------------
 
-def _bound_case(dtype, seed=21, T=3, S=300):
-    q, kv, sc = _case(seed, dtype, T, S)
-    w = torch.randn((T, 32), generator=torch.Generator().manual_seed(seed + 1)) / math.sqrt(32)
+def _bound_case(dtype, seed=21, T=3, S=300, heads=32):
+    q, kv, sc = _case(seed, dtype, T, S, heads=heads)
+    w = torch.randn((T, heads), generator=torch.Generator().manual_seed(seed + 1)) / math.sqrt(heads)
     return q, kv, sc, w
 
 
-def check_bound_dominates_scores(dtype):
+def check_bound_dominates_scores(dtype, heads=32):
     """UB(t, b) >= I(t, s) for every key s of block b (blocks of 128 and a
     ragged last block of 44 keys), with weights of both signs."""
-    q, kv, sc, w = _bound_case(dtype)
+    q, kv, sc, w = _bound_case(dtype, heads=heads)
     T, S = q.shape[0], kv.shape[0]
     ks, ke = _full_windows(T, S)
     I, _ = orc.index_scores(q, kv, sc, w, ks, ke)
@@ -496,6 +562,10 @@ def check_bound_hand_example():
     ks, ke = _full_windows(1, 2)
     I, _ = orc.index_scores(qb, kb, None, w, ks, ke)
     assert I[0].tolist() == [-4.0, -2.0]
+
+
+def test_bound_dominates_scores_64_heads():
+    check_bound_dominates_scores("fp8", heads=64)
 
 
 @pytest.mark.parametrize("dtype", ["fp8", "bf16"])

@@ -17,9 +17,9 @@ MUTATIONS = [
     ("weight_sign", "acc += wt[h] * relu;", "acc -= wt[h] * relu;"),
     ("sigma_dropped", "*I_out = sigma * acc;", "*I_out = acc;"),
     ("q_transposed", "double p = qd[h * ORC_DIM + d] * kd[d];",
-     "double p = qd[d * ORC_HEADS + h] * kd[d];"),
-    ("weight_index", "wt[h] = (double)weights[t * ORC_HEADS + h];",
-     "wt[h] = (double)weights[t * ORC_HEADS + (h ^ 1)];"),
+     "double p = qd[d * heads + h] * kd[d];"),
+    ("weight_index", "wt[h] = (double)weights[t * heads + h];",
+     "wt[h] = (double)weights[t * heads + (h + 1) % heads];"),
     ("first_key_dropped", "for (int64_t s = ks[t]; s < ke[t]; ++s) {",
      "for (int64_t s = ks[t] + 1; s < ke[t]; ++s) {"),
     ("error_scale_signed", "err += fabs(wt[h]) * absdot;", "err += wt[h] * absdot;"),
@@ -40,6 +40,15 @@ MUTATIONS = [
      "double v = element(dtype, kv, s * ORC_DIM + d);"),
     ("bound_last_key_dropped", "for (int64_t s = b * block; s < S && s < (b + 1) * block; ++s) {",
      "for (int64_t s = b * block; s < S && s < (b + 1) * block - 1; ++s) {"),
+    ("last_head_dropped", "for (int h = 0; h < heads; ++h) {\n        double dot = 0.0, absdot = 0.0;",
+     "for (int h = 0; h < heads - 1; ++h) {\n        double dot = 0.0, absdot = 0.0;"),
+    ("q_row_stride_of_32_heads",
+     "qd[i] = element(dtype, q, t * heads * ORC_DIM + i);\n        for (int h = 0; h < heads; ++h)\n"
+     "            wt[h] = (double)weights",
+     "qd[i] = element(dtype, q, t * 32 * ORC_DIM + i);\n        for (int h = 0; h < heads; ++h)\n"
+     "            wt[h] = (double)weights"),
+    ("weight_row_stride_of_32_heads", "wt[h] = (double)weights[t * heads + h];",
+     "wt[h] = (double)weights[t * 32 + h];"),
     ("bound_scale_smaller_side",
      "(fabs(bh[d]) > fabs(bl[d]) ? fabs(bh[d]) : fabs(bl[d]))",
      "(fabs(bh[d]) < fabs(bl[d]) ? fabs(bh[d]) : fabs(bl[d]))"),
@@ -53,6 +62,9 @@ CHECKS = [
     lambda: pins.check_score_one_hot_heads("fp8"),
     lambda: pins.check_score_one_hot_heads("bf16"),
     lambda: pins.check_score_linear_in_weights("fp8"),
+    lambda: pins.check_score_single_head("fp8"),
+    lambda: pins.check_score_heads_split("bf16"),
+    pins.check_score_head_permutation,
     pins.check_score_homogeneity,
     pins.check_hand_example,
     pins.check_select_brute_force,
