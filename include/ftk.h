@@ -108,9 +108,10 @@ typedef struct {
  *   kv         device [S, 128] of dtype, contiguous, 16-byte aligned
  *   kv_scales  device [S] float32 sigma_s, or NULL for all ones (BF16 keys);
  *              values must be > 0 (checked, FTK_STATUS_BAD_SCALE)
- *   weights    device [T, 32] float32
+ *   weights    device [T, 32] float32, 16-byte aligned
  *   ks, ke     device [T] int32 windows, 0 <= ks <= ke <= S
- *   T, S       1 <= T, S and T, S < 2^31
+ *   T, S       1 <= T < 2^26 (the T * 32 head rows stay below 2^31) and
+ *              1 <= S < 2^31 - 8192
  *   topk       1 .. FTK_MAX_TOPK
  *   out_idx    device [T, topk] int32: selected key indices in ascending
  *              order; rows whose window holds L < topk keys get the L keys
@@ -258,7 +259,8 @@ ftk_status ftk_topk_rows_ex(ftk_dtype dtype, const void *x, int64_t rows,
  * with exactly the arithmetic ftk_select uses (same kernel, same bits).
  * Entries past a row's window are left untouched.
  *   rows   device [nrows] int32 query indices, or NULL for 0 .. nrows-1
- *   out    device float32 [nrows, ld], ld >= max window length, ld % 4 == 0
+ *   out    device float32 [nrows, ld], ld >= S (so that every valid window
+ *          fits its row), ld % 4 == 0
  *   workspace  as for ftk_select, sized by ftk_score_dense_workspace_size
  * Other arguments as for ftk_select.
  */

@@ -1061,7 +1061,9 @@ extern "C" ftk_status ftk_score_dense(ftk_dtype dtype, const void *q, const void
 {
     ftk_status st = check_select_args(dtype, q, kv, weights, ks, ke, T, S, 1, rows ? rows : ks);
     if (st != FTK_OK) return st;
-    if (!out || nrows < 1 || nrows > T * 64 || ld < 1 || (ld & 3)) return FTK_ERR_INVALID_ARG;
+    // ld >= S: every valid window (ke <= S) fits its row, whatever the
+    // windows hold on the device
+    if (!out || nrows < 1 || nrows > T * 64 || ld < S || (ld & 3)) return FTK_ERR_INVALID_ARG;
     if (!rows && nrows > T) return FTK_ERR_INVALID_ARG;
     if (!workspace || workspace_bytes < 256 || (reinterpret_cast<uintptr_t>(workspace) & 255u))
         return FTK_ERR_WORKSPACE;

@@ -191,6 +191,9 @@ def test_score_dense_host_validation(lib):
     r = lib.ftk_score_dense(1, P(A), P(A), None, P(A), P(A), P(A), 16, 1000, None, 17, P(A), 1000,
                             P(A), 256, None)
     assert r == -1  # more rows than T without a row list
+    r = lib.ftk_score_dense(1, P(A), P(A), None, P(A), P(A), P(A), 16, 1000, None, 16, P(A), 996,
+                            P(A), 256, None)
+    assert r == -1  # ld < S: a window could run past its row
 
 
 def test_windows_host_validation(lib):

@@ -51,10 +51,8 @@ def check_case(c: wl.SelectInputs, rows=None, fp64_rows=None, config=None, expec
         else:
             assert np.all(idx[t] == -1)
     # bit-exact against the oracle's selection of the GPU's own scores
-    Lmax = int(max(1, max(ke[t] - ks[t] for t in rows)))
-    ld = (Lmax + 3) // 4 * 4
     dump = ftk.score_dense(g.q, g.kv, g.weights, g.ks, g.ke, g.kv_scales,
-                           rows=torch.tensor(rows, dtype=torch.int32), ld=ld)
+                           rows=torch.tensor(rows, dtype=torch.int32))
     dump = to_np(dump)
     oidx, oval, nflag = orc.select_f32_rows(dump, c.ks, c.ke, c.S, c.topk, row_ids=rows)
     for r, t in enumerate(rows):
