@@ -352,8 +352,9 @@ ftk_status ftk_select_noalloc(ftk_dtype dtype, const void *q, const void *kv,
  * the score-bound kernels, before the scan; right after 3 when pruning is
  * off).  n must be 0 (or events NULL) to stop, else >= 7 with non-NULL
  * events (the first min(n, 8) are used; FTK_ERR_INVALID_ARG otherwise).
- * If recording fails the hook switches itself off.  The library does not
- * own the events. */
+ * If recording fails the hook switches itself off.  The handles are copied
+ * (the array itself need not outlive this call); the events must stay valid
+ * while the hook is set.  The library does not own the events. */
 ftk_status ftk_set_stage_events(void *const *events, int n);
 
 /* Human-readable name of an ftk_status value (static string). */

@@ -727,14 +727,16 @@ static ftk_status check_select_args(int dtype, const void *q, const void *kv, co
     return FTK_OK;
 }
 
-thread_local void *const *g_stage_events = nullptr;
+// The caller's event handles, copied (the caller's array need not outlive
+// ftk_set_stage_events); g_stage_count == 0 means the hook is off.
+thread_local void *g_stage_events[8];
 thread_local int g_stage_count = 0;
 
 static void stage_mark(int i, cudaStream_t s)
 {
-    if (g_stage_events && i < g_stage_count && cudaEventRecord(static_cast<cudaEvent_t>(g_stage_events[i]), s) != cudaSuccess) {
+    if (i < g_stage_count && cudaEventRecord(static_cast<cudaEvent_t>(g_stage_events[i]), s) != cudaSuccess) {
         (void)cudaGetLastError();  // a bad event must not poison the launch checks
-        g_stage_events = nullptr;
+        g_stage_count = 0;
     }
 }
 
@@ -745,7 +747,6 @@ using namespace ftk;
 extern "C" ftk_status ftk_set_stage_events(void *const *events, int n)
 {
     if (events == nullptr || n == 0) {
-        g_stage_events = nullptr;
         g_stage_count = 0;
         return FTK_OK;
     }
@@ -753,7 +754,7 @@ extern "C" ftk_status ftk_set_stage_events(void *const *events, int n)
     const int used = n < 8 ? n : 8;
     for (int i = 0; i < used; ++i)
         if (events[i] == nullptr) return FTK_ERR_INVALID_ARG;
-    g_stage_events = events;
+    for (int i = 0; i < used; ++i) g_stage_events[i] = events[i];
     g_stage_count = used;
     return FTK_OK;
 }

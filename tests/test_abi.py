@@ -196,6 +196,23 @@ def test_score_dense_host_validation(lib):
     assert r == -1  # ld < S: a window could run past its row
 
 
+def test_stage_events_host_validation(lib):
+    """The hook takes 7 or 8 non-NULL handles (copied), and n = 0 or NULL
+    switches it off; nothing is recorded until an ftk_select call."""
+    P = ctypes.c_void_p
+    fake = (P * 8)(*[P(A + 64 * i) for i in range(8)])  # never recorded: no select runs here
+    try:
+        assert lib.ftk_set_stage_events(fake, 6) == -1
+        holes = (P * 8)(*[P(A + 64 * i) for i in range(8)])
+        holes[3] = None
+        assert lib.ftk_set_stage_events(holes, 8) == -1
+        assert lib.ftk_set_stage_events(fake, 7) == 0
+        assert lib.ftk_set_stage_events(fake, 12) == 0
+    finally:
+        assert lib.ftk_set_stage_events(None, 0) == 0
+    assert lib.ftk_set_stage_events(fake, 0) == 0
+
+
 def test_windows_host_validation(lib):
     P = ctypes.c_void_p
     assert lib.ftk_windows_from_cu_seqlens(None, P(A), 2, 10, P(A), P(A), None) == -1
