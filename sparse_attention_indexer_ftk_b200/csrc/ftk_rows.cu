@@ -2,6 +2,8 @@
 // helper the dense-recovery step reuses.
 #include <math.h>
 #include <stdint.h>
+
+#include <atomic>
 #include <stdio.h>
 #include <stdlib.h>
 #include <string.h>
@@ -15,14 +17,15 @@ ftk_status check_device()
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return cuda_status(cudaErrorInvalidDevice);
-    static int cached[64];  // 0 unknown, 1 ok, 2 wrong arch
-    if (dev >= 0 && dev < 64 && cached[dev]) return cached[dev] == 1 ? FTK_OK : FTK_ERR_DEVICE;
+    static std::atomic<int> cached[64];  // 0 unknown, 1 ok, 2 wrong arch (threads may race here)
+    const int c = dev >= 0 && dev < 64 ? cached[dev].load(std::memory_order_relaxed) : 0;
+    if (c) return c == 1 ? FTK_OK : FTK_ERR_DEVICE;
     int major = 0, minor = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
         return cuda_status(cudaErrorInvalidDevice);
     const bool ok = major == 10 && minor == 0;
-    if (dev >= 0 && dev < 64) cached[dev] = ok ? 1 : 2;
+    if (dev >= 0 && dev < 64) cached[dev].store(ok ? 1 : 2, std::memory_order_relaxed);
     return ok ? FTK_OK : FTK_ERR_DEVICE;
 }
 

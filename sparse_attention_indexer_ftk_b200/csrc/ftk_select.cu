@@ -29,6 +29,8 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "ftk_host.h"
 #include "ftk_prune.cuh"
 #include "ftk_rows.cuh"
@@ -537,14 +539,18 @@ __global__ void __launch_bounds__(kSelThreads, 6) refine_kernel(const RefineArgs
 
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
 {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    // Looked up once; a failed lookup is retried on the next call.
+    static std::atomic<PFN_cuTensorMapEncodeTiled_v12000> cached{nullptr};
+    PFN_cuTensorMapEncodeTiled_v12000 fn = cached.load(std::memory_order_acquire);
     if (!fn) {
         void *p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
                 cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
+            q == cudaDriverEntryPointSuccess) {
             fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+            cached.store(fn, std::memory_order_release);
+        }
     }
     return fn;
 }
