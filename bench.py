@@ -58,6 +58,8 @@ def parse_args():
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the decode-shaped, packed-workload and FP8 GEMM reference sections")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--oracle-configs", action="store_true",
+                    help="time only the CPU oracle on every workload configuration (no GPU)")
     ap.add_argument("--rows", type=int, default=0,
                     help="use only the first ROWS queries of the batch (profiling captures)")
     return ap.parse_args()
@@ -207,6 +209,46 @@ def cpu_baseline(c, seconds: float):
     return {"value": rows_total / t_total, "unit": "queries/s", "cores": threads, "kind": "oracle",
             "sample": f"{rows_total} seeded query rows of the {c.T}-row batch (first and last "
                       f"included), fp64 score + full sort per row, {t_total:.1f} s on {threads} threads"}
+
+
+# Oracle timing per workload configuration: the small BF16 and row top-k
+# workloads on all rows, the FP8 workloads on 64 seeded rows (first and
+# last included).
+ORACLE_CONFIGS = [("bf16_small", None), ("rows_bf16", None), ("rows_f32", None),
+                  ("fp8_prefill", 64), ("fp8_packed", 64), ("fp8_large", 64)]
+
+
+def oracle_configs():
+    """--oracle-configs: one JSON line per configuration with the oracle's
+    rows/s on the host cores (no GPU involved)."""
+    from oracle import oracle as orc
+    from sparse_attention_indexer_ftk_b200 import workloads as wl
+
+    threads = orc.num_threads()
+    for name, nrows in ORACLE_CONFIGS:
+        c = wl.get(name)
+        if isinstance(c, wl.RowsInputs):
+            t0 = time.perf_counter()
+            orc.topk_rows(c.x, c.topk)
+            dt = time.perf_counter() - t0
+            rows = c.x.shape[0]
+            extra = {"cols": c.x.shape[1], "input_mb": c.x.numel() * c.x.element_size() / 1e6}
+        else:
+            sel = wl.sample_rows(c.T, nrows or c.T, seed=0)
+            t0 = time.perf_counter()
+            orc.fused_select(c.q, c.kv, c.kv_scales, c.weights, c.ks, c.ke, c.topk, rows=sel)
+            dt = time.perf_counter() - t0
+            rows = len(sel)
+            L = (c.ke - c.ks).double()
+            pairs = float(L[torch_index(sel)].sum())
+            extra = {"T": c.T, "S": c.S, "dense_eq_gflops": pairs * 2 * 32 * 128 / dt / 1e9}
+        print(json.dumps({"workload": name, "kind": "oracle", "rows": rows, "seconds": round(dt, 3),
+                          "rows_per_s": rows / dt, "threads": threads, "topk": c.topk, **extra}), flush=True)
+
+
+def torch_index(rows):
+    import torch
+    return torch.tensor(rows, dtype=torch.long)
 
 
 def run_reference(args):
@@ -562,6 +604,9 @@ def run_ours(args):
 
 def main():
     args = parse_args()
+    if args.oracle_configs:
+        oracle_configs()
+        return
     if args.only_rows:
         import torch
         dev = torch.device("cuda")
