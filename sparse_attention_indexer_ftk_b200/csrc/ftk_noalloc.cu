@@ -10,6 +10,8 @@
 // g_noalloc_scratch, a file-scope __device__ array of
 // FTK_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds until
 // the process exits.
+#include <atomic>
+
 #include "ftk_host.h"
 
 namespace ftk {
@@ -21,17 +23,17 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[FTK_NOALLOC_SCRATCH_B
 // cudaGetSymbolAddress, once per device, with that device current.
 static void *scratch_on_device(int dev)
 {
-    static void *addr[64];
+    static std::atomic<void *> addr[64];  // host threads may race here
     if (dev < 0 || dev >= 64) return nullptr;
-    if (!addr[dev]) {
-        void *p = nullptr;
+    void *p = addr[dev].load(std::memory_order_acquire);
+    if (!p) {
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
             (void)cudaGetLastError();
             return nullptr;
         }
-        addr[dev] = p;
+        addr[dev].store(p, std::memory_order_release);
     }
-    return addr[dev];
+    return p;
 }
 
 }  // namespace ftk
