@@ -599,6 +599,8 @@ def run_ours(args):
         out["cpu_baseline"] = cpu_baseline(c, args.cpu_seconds)
     print(json.dumps(out), flush=True)
     if world > 1:
+        dist.destroy_process_group()  # rank 0 too (its collectives all ended above)
+    if world > 1:
         dist.destroy_process_group()
 
 
