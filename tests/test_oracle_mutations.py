@@ -2,7 +2,6 @@
 and check that the pins in tests/test_oracle.py catch every one of them."""
 from __future__ import annotations
 
-import os
 import subprocess
 
 import pytest
