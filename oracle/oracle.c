@@ -202,7 +202,8 @@ int64_t orc_index_scores(int dtype, int heads, const void *q, const void *kv,
  *   UB  = sum_h (w[t,h] >= 0 ? w[t,h] * ReLU(U_h) : w[t,h] * ReLU(L_h))
  * For sigma_s > 0, sigma_s * sum_h w_h ReLU(x_h) = sum_h w_h ReLU(sigma_s x_h),
  * so UB >= I[t,s] for every key of the block.
- *   out_ub    [nrows, nblocks]: UB of (rows[r], b)
+ *   out_ub    [nrows, nblocks]: UB of (rows[r], b); NaN for a listed row
+ *             outside [0, T)
  *   out_scale [nrows, nblocks] or NULL: sum_h |w| sum_d |q| max(|hi|, |lo|),
  *             the size of the terms UB is summed from
  */
@@ -230,6 +231,14 @@ void orc_block_bound(int dtype, int heads, const void *q, const void *kv, const 
 #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t r = 0; r < nrows; ++r) {
         int64_t t = rows[r];
+        if (t < 0 || t >= T) {
+            for (int64_t b = 0; b < nb; ++b) {
+                out_ub[r * nb + b] = NAN;
+                if (out_scale)
+                    out_scale[r * nb + b] = NAN;
+            }
+            continue;
+        }
         double *qd = (double *)malloc(sizeof(double) * heads * ORC_DIM);
         double *wt = (double *)malloc(sizeof(double) * heads);
         for (int64_t i = 0; i < (int64_t)heads * ORC_DIM; ++i)

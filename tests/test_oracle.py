@@ -564,6 +564,12 @@ def check_bound_hand_example():
     assert I[0].tolist() == [-4.0, -2.0]
 
 
+def test_bound_rows_outside_the_batch_are_nan():
+    q, kv, sc, w = _bound_case("bf16", T=2, S=200)
+    ub, scale = orc.block_bound(q, kv, sc, w, rows=[1, 2, -1])
+    assert np.all(np.isfinite(ub[0])) and np.all(np.isnan(ub[1:])) and np.all(np.isnan(scale[1:]))
+
+
 def test_bound_dominates_scores_64_heads():
     check_bound_dominates_scores("fp8", heads=64)
 
