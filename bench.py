@@ -449,6 +449,69 @@ def bench_config(name: str, dev, reps: int = 10):
             "rows_recovered": info["rows_overflow"] + info["rows_underflow"]}
 
 
+def e2e_pipelined(ftk, host: dict, ws, T: int, k: int, E: int, dev, ref_idx, ref_val):
+    """End to end through the public API with the copies overlapped: while
+    step j computes, the inputs of step j+1 go up on one stream and the
+    results of step j-1 come back on another (device inputs and outputs
+    double-buffered, ordered by events).  Every step still copies its own
+    inputs from pinned host memory and its own results back.  Returns
+    (ms per step, ok): ok says the last step's results, as copied back,
+    equal ref_idx / ref_val bit for bit (the same inputs, computed without
+    overlap)."""
+    import torch
+    comp = torch.cuda.current_stream(dev)
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    names = list(host)
+    din = [{n: torch.empty(host[n].shape, dtype=host[n].dtype, device=dev) for n in names} for _ in range(2)]
+    oidx = [torch.empty((T, k), dtype=torch.int32, device=dev) for _ in range(2)]
+    oval = [torch.empty((T, k), dtype=torch.float32, device=dev) for _ in range(2)]
+    hidx = [torch.empty((T, k), dtype=torch.int32).pin_memory() for _ in range(2)]
+    hval = [torch.empty((T, k), dtype=torch.float32).pin_memory() for _ in range(2)]
+    ev_up = [torch.cuda.Event() for _ in range(2)]    # inputs of buffer b are on the device
+    ev_comp = [torch.cuda.Event() for _ in range(2)]  # step on buffer b done (inputs free, results ready)
+    ev_down = [torch.cuda.Event() for _ in range(2)]  # results of buffer b are on the host
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def issue_up(j):
+        b = j % 2
+        with torch.cuda.stream(up):
+            if j >= 2:
+                up.wait_event(ev_comp[b])  # step j-2 has finished reading din[b]
+            for n in names:
+                din[b][n].copy_(host[n], non_blocking=True)
+            ev_up[b].record(up)
+
+    torch.cuda.synchronize(dev)
+    e0.record(comp)
+    up.wait_event(e0)
+    down.wait_event(e0)
+    issue_up(0)
+    for j in range(E):
+        b = j % 2
+        if j + 1 < E:
+            issue_up(j + 1)
+        comp.wait_event(ev_up[b])
+        if j >= 2:
+            comp.wait_event(ev_down[b])  # the results of step j-2 have left oidx[b] / oval[b]
+        d = din[b]
+        ftk.select(d["q"], d["kv"], d["weights"], d["ks"], d["ke"], d["kv_scales"], k, return_scores=True,
+                   workspace=ws, out_idx=oidx[b], out_val=oval[b])
+        ev_comp[b].record(comp)
+        with torch.cuda.stream(down):
+            down.wait_event(ev_comp[b])
+            hidx[b].copy_(oidx[b], non_blocking=True)
+            hval[b].copy_(oval[b], non_blocking=True)
+            ev_down[b].record(down)
+    for j in range(max(0, E - 2), E):
+        comp.wait_event(ev_down[j % 2])
+    e1.record(comp)
+    torch.cuda.synchronize(dev)
+    last = (E - 1) % 2
+    ok = bool(torch.equal(hidx[last], ref_idx.cpu())
+              and torch.equal(hval[last].view(torch.int32), ref_val.cpu().view(torch.int32)))
+    return e0.elapsed_time(e1) / E, ok
+
+
 def run_ours(args):
     import torch
 
@@ -537,8 +600,29 @@ def run_ours(args):
         h_val.copy_(out_val, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / E
-    e2e_ms = shard.max_over_ranks(e2e_ms, dev)
+    serial_ms = e0.elapsed_time(e1) / E
+    serial_ms = shard.max_over_ranks(serial_ms, dev)
+    # The same with the copies overlapped across steps (a serving loop).
+    # Self-checked: the copied-back results must equal the timed run's bits,
+    # and no end-to-end step can beat the device-only step; otherwise (or on
+    # any error) the serial figure stands.  Every rank takes the same
+    # collective steps either way.
+    ref_idx, ref_val = out_idx.clone(), out_val.clone()
+    pipe_note = ""
+    try:
+        pipe_ms, pipe_ok = e2e_pipelined(ftk, host, ws, T, k, E, dev, ref_idx, ref_val)
+        if not pipe_ok:
+            pipe_note = "results differ from the plain run"
+        elif pipe_ms < 0.98 * mean_ms:
+            pipe_note = f"faster than the device-only step ({pipe_ms:.3f} < {mean_ms:.3f} ms)"
+    except Exception as ex:  # noqa: BLE001 -- any failure falls back to the serial figure
+        pipe_ms, pipe_note = float("inf"), f"{type(ex).__name__}: {ex}"
+    pipe_ms = shard.max_over_ranks(pipe_ms if not pipe_note else float("inf"), dev)
+    if pipe_ms != float("inf"):
+        e2e_ms, e2e_mode = pipe_ms, ("pipelined: inputs of step j+1 and results of step j-1 copied "
+                                      "while step j computes; last step's results checked bit-exact")
+    else:
+        e2e_ms, e2e_mode = serial_ms, "serial" + (f" (pipelined run rejected: {pipe_note})" if pipe_note else "")
 
     if rank != 0:
         if world > 1:
@@ -585,7 +669,9 @@ def run_ours(args):
                      "frac_of_fp8_gemm_measured": (achieved / fp8_direct["tflops"])
                      if fp8_direct and "tflops" in fp8_direct else None},
         "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": "queries/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "mode": e2e_mode, "steps": E,
+                "serial": {"value": world * T / (serial_ms * 1e-3), "ms_per_step": serial_ms}},
         "gpu_launches": int(info["kernel_launches"]) * K,
         "clocks": clocks,
     }
