@@ -28,6 +28,18 @@ def declared_functions():
     return sorted(set(re.findall(r"\b(ftk_[a-z0-9_]+)\s*\(", text)))
 
 
+def test_header_is_plain_c_and_links(lib, tmp_path):
+    """A C11 program includes include/ftk.h, links libftk.so and calls the
+    host-side entry points (no GPU): the boundary needs no C++ or torch."""
+    exe = tmp_path / "c_abi_check"
+    libdir = os.path.dirname(ftk.LIB_PATH)
+    subprocess.check_call(["gcc", "-std=c11", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                           os.path.join(ROOT, "tests", "c_abi_check.c"), "-o", str(exe), "-L", libdir, "-lftk",
+                           "-Wl,-rpath," + libdir, "-lm"])
+    out = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert out.returncode == 0 and out.stdout.strip() == "OK", out.stdout + out.stderr
+
+
 def test_header_matches_binding_list():
     assert declared_functions() == sorted(ftk.EXPORTS)
 
