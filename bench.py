@@ -176,8 +176,14 @@ class ClockSampler:
         sm = [int(r[1]) for r in rows]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        power = []
+        for r in rows:
+            try:
+                power.append(float(r[3]))
+            except ValueError:  # "[N/A]" or empty
+                pass
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": int(rows[0][2]), "reasons": reasons,
-                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows if r[3] not in ("", "[N/A]"))}
+                "samples": len(rows), "power_w_max": max(power) if power else None}
 
 
 def gpu_index(local_rank: int) -> int:

@@ -129,3 +129,26 @@ def test_binding_accepts_the_calls_bench_and_tests_make(monkeypatch):
                              out_idx=torch.empty((6, 70), dtype=torch.int64))
     assert val.shape == (6, 64) and val.stride(0) == 70 and idx.dtype == torch.int64
     assert fake.calls.count("ftk_topk_rows_ex") == 4
+
+
+def test_clock_summary(tmp_path):
+    """The clock record beside every bench number: median SM clock under
+    load, the max clock, and the throttle reasons seen in any sample."""
+    s = bench.ClockSampler(0)
+    s.path = str(tmp_path / "clocks.csv")
+    with open(s.path, "w") as f:
+        f.write("0, 1965, 1965, 800.5, 0x0, Not Active, Not Active, Not Active, Not Active\n")
+        f.write("0, 1800, 1965, 1001.2, 0x4, Not Active, Not Active, Not Active, Active\n")
+        f.write("garbage line\n")
+        f.write("0, 1900, 1965, [N/A], 0x0, Not Active, Not Active, Not Active, Not Active\n")
+    out = s.summary()
+    assert out["sm_mhz"] == 1900 and out["sm_max_mhz"] == 1965 and out["samples"] == 3
+    assert out["reasons"] == ["sw_power_cap"] and out["power_w_max"] == 1001.2
+    assert not os.path.exists(s.path)
+    s.path = str(tmp_path / "none.csv")
+    with open(s.path, "w") as f:
+        f.write("0, 1965, 1965, [N/A], 0x0, Not Active, Active, Not Active, Not Active\n")
+    out = s.summary()
+    assert out["power_w_max"] is None and out["reasons"] == ["hw_thermal_slowdown"]
+    s.path = str(tmp_path / "missing.csv")
+    assert s.summary()["reasons"] == ["unsampled"]
