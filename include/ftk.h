@@ -165,6 +165,9 @@ ftk_status ftk_read_info(const void *workspace, ftk_info *out, void *stream);
  *               (OR-ed in; DeepSelect README, "NaN handling" aborts instead),
  *               or NULL
  *   stream      cudaStream_t
+ * Diagnostics: the environment variable FTK_ROWS_CLUSTER = 1, 2, 4 or 8
+ * forces the number of CTAs (one thread-block cluster) per row instead of
+ * the planned one; the result is the same, only the speed changes.
  */
 ftk_status ftk_topk_rows(ftk_dtype dtype, const void *x, int64_t rows,
                          int64_t cols, int64_t row_stride, int topk,
