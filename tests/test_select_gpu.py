@@ -28,7 +28,7 @@ def gpu_inputs(c: wl.SelectInputs):
 
 
 def run_select(g: wl.SelectInputs, config=None):
-    ws = torch.empty(ftk.select_workspace_size(g.T, g.S, g.topk, config), dtype=torch.uint8,
+    ws = torch.empty(ftk.select_workspace_size(g.T, g.S, g.topk, config, g.q.shape[1]), dtype=torch.uint8,
                      device="cuda")
     idx, val = ftk.select(g.q, g.kv, g.weights, g.ks, g.ke, g.kv_scales, g.topk,
                           return_scores=True, workspace=ws, config=config)
