@@ -83,3 +83,16 @@ def test_selector_64_heads_and_determinism():
     assert np.array_equal(a, ref)
     with pytest.raises(ftk.FtkError):  # a 32-head Selector refuses 64-head inputs
         ftk.Selector(topk=512).plan(64, 20000).run(g.q, g.kv, g.weights, g.ks, g.ke, g.kv_scales)
+
+
+def test_full_size_64_heads():
+    """fp8_prefill_64h (4096 queries x 128K FP8 keys, 64 heads, topk 2048):
+    every row against the invariants, 64 seeded rows bit-exact against the
+    oracle's selection of the GPU's dumped scores, 8 of them against the
+    fp64 oracle."""
+    c = wl.get("fp8_prefill_64h")
+    rows = wl.sample_rows(c.T, 64, seed=2)
+    fp64_rows = rows[:: len(rows) // 8][:8] + [rows[-1]]
+    _, _, info, worst, overlaps = check_case(c, rows=rows, fp64_rows=fp64_rows)
+    assert worst < 1e-4 and min(overlaps) >= 0.99
+    assert info["prune_enabled"] == 0
