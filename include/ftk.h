@@ -80,8 +80,7 @@ typedef struct {
     int32_t recovery_rows; /* rows rescored densely per recovery pass (0: auto) */
     int32_t heads;         /* indexer heads H: 32 (or 0, the default) or 64 (FlashTopK
                             * README, "Roadmap": other head counts such as 64); q is then
-                            * [T, H, 128] and weights [T, H].  With 64 heads the call
-                            * scans without key pruning. */
+                            * [T, H, 128] and weights [T, H]. */
     int32_t reserved[2];   /* must be 0 */
 } ftk_config;
 
@@ -315,6 +314,15 @@ ftk_status ftk_block_bound(ftk_dtype dtype, const void *q, const void *kv,
                            void *stream);
 
 size_t ftk_block_bound_workspace_size(int64_t S);
+
+/* ftk_block_bound for an indexer of `heads` heads (32 or 64): q
+ * [T, heads, 128], weights [T, heads], the sums over h run over every head;
+ * otherwise as ftk_block_bound (which is this call with heads = 32). */
+ftk_status ftk_block_bound_heads(ftk_dtype dtype, int heads, const void *q,
+                                 const void *kv, const float *kv_scales,
+                                 const float *weights, int64_t T, int64_t S,
+                                 float *out, int64_t ld, void *workspace,
+                                 size_t workspace_bytes, void *stream);
 
 /*
  * ftk_windows_from_cu_seqlens -- causal windows of packed sequences

@@ -607,7 +607,6 @@ static SelectCfg resolve_cfg(int64_t T, int64_t S, int topk, const ftk_config *c
     if (r.cap > 2 * FTK_MAX_TOPK) r.cap = 2 * FTK_MAX_TOPK;
     const int pr = c ? c->prune : 0;
     r.prune = pr == 0 ? PRUNE_AUTO : pr > 0 ? PRUNE_ON : PRUNE_OFF;
-    if (r.heads != 32) r.prune = PRUNE_OFF;  // the bound kernels hold one head per lane
     // Strides are powers of two up to 2^(kNumStrideMaps - 1).
     const int64_t min_m = (S + (int64_t(1) << (kNumStrideMaps - 1)) - 1) >> (kNumStrideMaps - 1);
     if (r.m < min_m) r.m = static_cast<int>(min_m);
@@ -961,12 +960,12 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
         ba.prune_enabled = &w.info->info.prune_enabled;
         ba.blocks_pruned = reinterpret_cast<unsigned long long *>(&w.info->info.blocks_pruned);
         if (c.prune == PRUNE_AUTO) {
-            st = launch_bound(dtype, BOUND_EST, ba, ba.est_tiles * (kEstBlocks / kEstChunk), s);
+            st = launch_bound(dtype, BOUND_EST, ba, ba.est_tiles * (kEstBlocks / kEstChunk), s, heads);
             if (st != FTK_OK) return st;
         }
         const int64_t items = static_cast<int64_t>(ntiles) * w.nwords;
         const int64_t cap = static_cast<int64_t>(sms) * 2;
-        st = launch_bound(dtype, BOUND_FULL, ba, static_cast<int>(items < cap ? items : cap), s);
+        st = launch_bound(dtype, BOUND_FULL, ba, static_cast<int>(items < cap ? items : cap), s, heads);
         if (st != FTK_OK) return st;
     }
     stage_mark(7, s);

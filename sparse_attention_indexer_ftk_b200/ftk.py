@@ -42,7 +42,7 @@ EXPORTS = (
     "ftk_score_dense", "ftk_score_dense_workspace_size", "ftk_windows_from_cu_seqlens",
     "ftk_set_stage_events", "ftk_status_string", "ftk_version", "ftk_select_noalloc",
     "ftk_block_bound", "ftk_block_bound_workspace_size", "ftk_topk_rows_end", "ftk_topk_rows_sorted",
-    "ftk_rows_options_init", "ftk_topk_rows_ex", "ftk_score_dense_heads",
+    "ftk_rows_options_init", "ftk_topk_rows_ex", "ftk_score_dense_heads", "ftk_block_bound_heads",
 )
 
 
@@ -116,6 +116,8 @@ def load_library(path: str = LIB_PATH):
     L.ftk_topk_rows_ex.argtypes = [I32, P, I64, I64, I64, P, I32, P, P, P, P, P]
     L.ftk_block_bound.restype = I32
     L.ftk_block_bound.argtypes = [I32, P, P, P, P, I64, I64, P, I64, P, SZ, P]
+    L.ftk_block_bound_heads.restype = I32
+    L.ftk_block_bound_heads.argtypes = [I32, I32, P, P, P, P, I64, I64, P, I64, P, SZ, P]
     L.ftk_block_bound_workspace_size.restype = SZ
     L.ftk_block_bound_workspace_size.argtypes = [I64]
     L.ftk_status_string.restype = ctypes.c_char_p
@@ -427,7 +429,7 @@ def block_bound(q, kv, weights, kv_scales=None) -> torch.Tensor:
     nb = (S + 127) // 128
     out = torch.empty((T, nb), dtype=torch.float32, device=dev)
     ws = torch.empty(int(lib().ftk_block_bound_workspace_size(S)), dtype=torch.uint8, device=dev)
-    st = lib().ftk_block_bound(_dtype_code(q), _ptr(q), _ptr(kv), _ptr(kv_scales), _ptr(weights), T, S,
-                               _ptr(out), nb, _ptr(ws), ws.numel(), _stream(dev))
-    _check(st, "ftk_block_bound")
+    st = lib().ftk_block_bound_heads(_dtype_code(q), q.shape[1], _ptr(q), _ptr(kv), _ptr(kv_scales),
+                                     _ptr(weights), T, S, _ptr(out), nb, _ptr(ws), ws.numel(), _stream(dev))
+    _check(st, "ftk_block_bound_heads")
     return out

@@ -340,16 +340,17 @@ def sample_rows(T: int, n: int, seed: int = 0) -> list[int]:
 
 
 def block_structured(seed: int, dtype: str, T: int, S: int, topk: int, hot_every: int = 8,
-                     cold: float = 2.0 ** -7) -> SelectInputs:
+                     cold: float = 2.0 ** -7, heads: int = 32) -> SelectInputs:
     """Keys in 128-key blocks where only every hot_every-th block keeps its
     kv_scales and the others have theirs multiplied by `cold`, with causal
     windows and mostly positive weights (|N(0,1)|/sqrt(32), negated on the
     heads h % 8 == 0): the top-k lies in the hot blocks and the cold blocks'
     scores stay far below the threshold, the case score-bound pruning is for."""
-    c = small_case(seed, dtype, T, S, topk, windows="causal")
+    c = small_case(seed, dtype, T, S, topk, windows="causal", heads=heads)
     sc = c.kv_scales.clone()
     blk = torch.arange(S) // 128
     sc[blk % hot_every != 0] *= cold
     w = c.weights.abs()
     w[:, ::8] = -w[:, ::8]
-    return SelectInputs(f"blocks{seed}_{dtype}", c.q, c.kv, sc, w.contiguous(), c.ks, c.ke, topk)
+    name = f"blocks{seed}_{dtype}" + ("" if heads == 32 else f"_{heads}h")
+    return SelectInputs(name, c.q, c.kv, sc, w.contiguous(), c.ks, c.ke, topk)

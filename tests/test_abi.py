@@ -221,6 +221,8 @@ def test_head_count_validation(lib):
                               1 << 30, ctypes.byref(cfg), None) == -1
         assert lib.ftk_score_dense_heads(1, h, P(A), P(A), None, P(A), P(A), P(A), 16, 1000, None, 16,
                                          P(A), 1000, P(A), 256, None) == -1
+        assert lib.ftk_block_bound_heads(1, h, P(A), P(A), None, P(A), 4, 1000, P(A), 8, P(A), 1 << 20,
+                                         None) == -1
     # 64 heads: twice the row tiles (4 or 8 queries per tile instead of 8 or 16)
     n32 = lib.ftk_select_workspace_size(4096, 131072, 2048, None)
     n64 = lib.ftk_select_workspace_size(4096, 131072, 2048, ctypes.byref(ftk.FtkConfig(heads=64)))

@@ -34,7 +34,6 @@ def test_small_cases_64_heads(spec):
     c = wl.small_case(heads=64, **spec)
     assert c.q.shape[1] == 64 and c.weights.shape[1] == 64
     _, _, info, worst, overlaps = check_case(c)
-    assert info["prune_enabled"] == 0
     assert worst < 1e-4
 
 
@@ -51,7 +50,6 @@ def test_config_does_not_change_the_result_64_heads(config):
         assert info["rows_overflow"] > 0
     if "oversample" in config:
         assert info["rows_underflow"] > 0
-    assert info["prune_enabled"] == 0  # no key pruning with 64 heads
     check_case(c, config=config)
 
 
@@ -95,4 +93,29 @@ def test_full_size_64_heads():
     fp64_rows = rows[:: len(rows) // 8][:8] + [rows[-1]]
     _, _, info, worst, overlaps = check_case(c, rows=rows, fp64_rows=fp64_rows)
     assert worst < 1e-4 and min(overlaps) >= 0.99
-    assert info["prune_enabled"] == 0
+
+
+@pytest.mark.parametrize("dtype", ["fp8", "bf16"])
+def test_block_bound_64_heads_matches_oracle(dtype):
+    """The 64-head score bound (both halves of every row) against the
+    oracle's fp64 box bound over all 64 heads."""
+    c = wl.small_case(seed=41, dtype=dtype, T=21, S=1000, topk=8, windows="causal", heads=64)
+    g = c.to("cuda")
+    ub = to_np(ftk.block_bound(g.q, g.kv, g.weights, g.kv_scales)).astype(np.float64)
+    oub, scale = orc.block_bound(c.q, c.kv, c.kv_scales, c.weights, block=128)
+    assert ub.shape == oub.shape == (21, 8)
+    assert (np.abs(ub - oub) / scale).max() <= 1e-5
+
+
+@pytest.mark.parametrize("dtype,T,S,topk", [("fp8", 70, 9000, 128), ("bf16", 29, 5000, 64)])
+def test_pruning_64_heads_fires_and_changes_nothing(dtype, T, S, topk):
+    c = wl.block_structured(seed=42, dtype=dtype, T=T, S=S, topk=topk, heads=64)
+    idx, val, info, worst, overlaps = check_case(c)
+    assert info["prune_enabled"] == 1, info
+    assert info["blocks_pruned"] >= info["blocks_total"] // 2, info
+    g = c.to("cuda")
+    off = run_select(g, {"prune": -1})
+    on = run_select(g, {"prune": 1})
+    assert off[2]["prune_enabled"] == 0 and on[2]["blocks_pruned"] == info["blocks_pruned"]
+    for r in (off, on):
+        assert np.array_equal(idx, r[0]) and np.array_equal(val.view(np.int32), r[1].view(np.int32))
