@@ -221,7 +221,7 @@ def cpu_baseline(c, seconds: float):
 # workloads on all rows, the FP8 workloads on 64 seeded rows (first and
 # last included).
 ORACLE_CONFIGS = [("bf16_small", None), ("rows_bf16", None), ("rows_f32", None),
-                  ("fp8_prefill", 64), ("fp8_packed", 64), ("fp8_large", 64)]
+                  ("fp8_prefill", 64), ("fp8_packed", 64), ("fp8_large", 64), ("fp8_prefill_64h", 64)]
 
 
 def oracle_configs():
@@ -247,7 +247,8 @@ def oracle_configs():
             rows = len(sel)
             L = (c.ke - c.ks).double()
             pairs = float(L[torch_index(sel)].sum())
-            extra = {"T": c.T, "S": c.S, "dense_eq_gflops": pairs * 2 * 32 * 128 / dt / 1e9}
+            heads = c.q.shape[1]
+            extra = {"T": c.T, "S": c.S, "heads": heads, "dense_eq_gflops": pairs * 2 * heads * 128 / dt / 1e9}
         print(json.dumps({"workload": name, "kind": "oracle", "rows": rows, "seconds": round(dt, 3),
                           "rows_per_s": rows / dt, "threads": threads, "topk": c.topk, **extra}), flush=True)
 
