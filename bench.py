@@ -221,7 +221,7 @@ def cpu_baseline(c, seconds: float):
 # workloads on all rows, the FP8 workloads on 64 seeded rows (first and
 # last included).
 ORACLE_CONFIGS = [("bf16_small", None), ("rows_bf16", None), ("rows_f32", None),
-                  ("fp8_prefill", 64), ("fp8_packed", 64), ("fp8_large", 64)]
+                  ("fp8_prefill", 64), ("fp8_packed", 64), ("fp8_large", 64), ("fp8_prefill_64h", 64)]
 
 
 def oracle_configs():
@@ -247,7 +247,8 @@ def oracle_configs():
             rows = len(sel)
             L = (c.ke - c.ks).double()
             pairs = float(L[torch_index(sel)].sum())
-            extra = {"T": c.T, "S": c.S, "dense_eq_gflops": pairs * 2 * 32 * 128 / dt / 1e9}
+            heads = c.q.shape[1]
+            extra = {"T": c.T, "S": c.S, "heads": heads, "dense_eq_gflops": pairs * 2 * heads * 128 / dt / 1e9}
         print(json.dumps({"workload": name, "kind": "oracle", "rows": rows, "seconds": round(dt, 3),
                           "rows_per_s": rows / dt, "threads": threads, "topk": c.topk, **extra}), flush=True)
 
@@ -430,7 +431,8 @@ def bench_config(name: str, dev, reps: int = 10):
     from sparse_attention_indexer_ftk_b200 import workloads as wl
 
     d = wl.get(name).to(dev)
-    ws = torch.empty(ftk.select_workspace_size(d.T, d.S, d.topk), dtype=torch.uint8, device=dev)
+    heads = d.q.shape[1]
+    ws = torch.empty(ftk.select_workspace_size(d.T, d.S, d.topk, None, heads), dtype=torch.uint8, device=dev)
     oi = torch.empty((d.T, d.topk), dtype=torch.int32, device=dev)
     ov = torch.empty((d.T, d.topk), dtype=torch.float32, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -447,9 +449,9 @@ def bench_config(name: str, dev, reps: int = 10):
     torch.cuda.synchronize()
     ms = sum(a.elapsed_time(b) for a, b in ev) / reps
     info = ftk.read_info(ws)
-    return {"workload": name, "T": d.T, "S": d.S, "topk": d.topk, "ms_per_call": ms,
+    return {"workload": name, "T": d.T, "S": d.S, "topk": d.topk, "heads": heads, "ms_per_call": ms,
             "queries_per_s": d.T / (ms * 1e-3),
-            "dense_eq_tflops": 2.0 * 32 * 128 * d.pairs() / (ms * 1e-3) / 1e12,
+            "dense_eq_tflops": 2.0 * heads * 128 * d.pairs() / (ms * 1e-3) / 1e12,
             "prune_enabled": info["prune_enabled"], "blocks_total": info["blocks_total"],
             "blocks_pruned": info["blocks_pruned"],
             "rows_recovered": info["rows_overflow"] + info["rows_underflow"]}
@@ -684,6 +686,7 @@ def run_ours(args):
     if world == 1 and not (args.no_decode or args.no_extras):
         out["decode_64q"] = bench_decode(c, dev)
         out["fp8_packed"] = bench_config("fp8_packed", dev)
+        out["fp8_prefill_64h"] = bench_config("fp8_prefill_64h", dev)
     if world == 1 and not args.no_rows:
         out["row_topk"] = [bench_rows("rows_bf16", dev), bench_rows("rows_f32", dev),
                            bench_rows("rows_bf16_1024", dev, reps=16)]

@@ -78,7 +78,10 @@ typedef struct {
                           * default (estimate the skippable share of key blocks on
                           * a sample and prune if it is >= 25%), 1 always, -1 off */
     int32_t recovery_rows; /* rows rescored densely per recovery pass (0: auto) */
-    int32_t reserved[3];   /* must be 0 */
+    int32_t heads;         /* indexer heads H: 32 (or 0, the default) or 64 (FlashTopK
+                            * README, "Roadmap": other head counts such as 64); q is then
+                            * [T, H, 128] and weights [T, H]. */
+    int32_t reserved[2];   /* must be 0 */
 } ftk_config;
 
 /* Per-call information (FlashTopK README, "Usage": last_info), filled on
@@ -276,6 +279,17 @@ ftk_status ftk_score_dense(ftk_dtype dtype, const void *q, const void *kv,
 
 size_t ftk_score_dense_workspace_size(int64_t nrows);
 
+/* ftk_score_dense for an indexer of `heads` heads (32 or 64): q
+ * [T, heads, 128], weights [T, heads]; otherwise as ftk_score_dense (which
+ * is this call with heads = 32). */
+ftk_status ftk_score_dense_heads(ftk_dtype dtype, int heads, const void *q,
+                                 const void *kv, const float *kv_scales,
+                                 const float *weights, const int32_t *ks,
+                                 const int32_t *ke, int64_t T, int64_t S,
+                                 const int32_t *rows, int64_t nrows, float *out,
+                                 int64_t ld, void *workspace,
+                                 size_t workspace_bytes, void *stream);
+
 /*
  * ftk_block_bound -- the score bound that ftk_select's key pruning uses
  * (FlashTopK README, "Highlights": keys are skipped by a score bound; the
@@ -300,6 +314,15 @@ ftk_status ftk_block_bound(ftk_dtype dtype, const void *q, const void *kv,
                            void *stream);
 
 size_t ftk_block_bound_workspace_size(int64_t S);
+
+/* ftk_block_bound for an indexer of `heads` heads (32 or 64): q
+ * [T, heads, 128], weights [T, heads], the sums over h run over every head;
+ * otherwise as ftk_block_bound (which is this call with heads = 32). */
+ftk_status ftk_block_bound_heads(ftk_dtype dtype, int heads, const void *q,
+                                 const void *kv, const float *kv_scales,
+                                 const float *weights, int64_t T, int64_t S,
+                                 float *out, int64_t ld, void *workspace,
+                                 size_t workspace_bytes, void *stream);
 
 /*
  * ftk_windows_from_cu_seqlens -- causal windows of packed sequences

@@ -53,7 +53,7 @@ struct BoundArgs;
 // Score-bound pruning kernels (ftk_prune.cu): the box of every key block,
 // and the bound in mode BOUND_EST / BOUND_FULL / BOUND_OUT.
 ftk_status launch_box(int dtype, const BoxArgs &a, cudaStream_t stream);
-ftk_status launch_bound(int dtype, int mode, const BoundArgs &a, int grid, cudaStream_t stream);
+ftk_status launch_bound(int dtype, int mode, const BoundArgs &a, int grid, cudaStream_t stream, int heads = 32);
 // Launches the row top-k kernel for the given dtype (FTK_BF16 / FTK_F32)
 // with one cluster of `cluster` CTAs per grid row.
 ftk_status launch_rows_topk(int dtype, const RowsArgs &a, int cluster, cudaStream_t stream, bool idx64 = false);

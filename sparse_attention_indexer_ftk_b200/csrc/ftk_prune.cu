@@ -174,13 +174,16 @@ struct BoundSmem {
     float mb[kBoundWordBlocks];
     int32_t blk[kBoundWordBlocks];
     uint32_t pass[kBoundWarps];
+    float ub[kBoundWarps][kBoundWordBlocks];  // 64 heads: a row's bound, summed over its two halves
     int32_t nblk;
 };
 
 // Work items.  EST: (sampled tile, chunk of kEstChunk sampled blocks).
 // FULL: (row tile, bitmap word) over every word meeting the tile's scan
 // range.  OUT: (row tile, word) over all blocks.
-template <int DT, int MODE>
+// H: the indexer's heads.  32: lane = head.  64: lane = heads lane and
+// lane + 32, taken in two passes (q of one head is 128 floats in registers).
+template <int DT, int MODE, int H>
 __global__ void __launch_bounds__(kBoundWarps * 32, 1) bound_kernel(const BoundArgs a)
 {
     __shared__ BoundSmem sm;
@@ -256,54 +259,127 @@ __global__ void __launch_bounds__(kBoundWarps * 32, 1) bound_kernel(const BoundA
                 tau = a.tau[t];
             }
             if (!row_ok) continue;  // masked row: no constraint
-            float qf[kDim];
-            load_q<DT>(a.q, t * kHeads + lane, qf);
-            const float w = a.weights[t * kHeads + lane];
-            float l1 = 0.f;
-#pragma unroll
-            for (int i = 0; i < kDim; ++i) l1 += fabsf(qf[i]);
-            const float A = warp_sum(fabsf(w) * l1);            // sum_h |w_h| |q_h|_1
-            const float P = warp_sum(w >= 0.f ? w * l1 : 0.f);  // sum_{w_h >= 0} w_h |q_h|_1
             uint32_t row_pass = 0;
-            for (int j = 0; j < nblk; ++j) {
-                const int32_t B = sm.blk[j];
-                const float M = sm.mb[j];
-                if (MODE != BOUND_OUT) {
-                    const int32_t k0 = B * kBlockKeys;
-                    if (!(wks < k0 + kBlockKeys && wke > k0)) {  // window misses the block
-                        row_pass |= 1u << j;
-                        continue;
-                    }
-                    if (!(M < INFINITY)) continue;  // never skipped
-                    if (P * M + kPruneEps * A * M < tau) {
-                        row_pass |= 1u << j;  // |U_h| <= |q_h|_1 M_B: the coarse bound decides
-                        continue;
-                    }
-                }
-                const float4 *c4 = reinterpret_cast<const float4 *>(sm.box[j]);
-                const float4 *r4 = c4 + kDim / 4;
-                float a0 = 0.f, a1 = 0.f, e0 = 0.f, e1 = 0.f;
+            if constexpr (H == 32) {
+                float qf[kDim];
+                load_q<DT>(a.q, t * kHeads + lane, qf);
+                const float w = a.weights[t * kHeads + lane];
+                float l1 = 0.f;
 #pragma unroll
-                for (int i = 0; i < kDim / 4; ++i) {
-                    const float4 c = c4[i], r = r4[i];
-                    const float *x = qf + 4 * i;
-                    a0 = fmaf(x[0], c.x, a0);
-                    e0 = fmaf(fabsf(x[0]), r.x, e0);
-                    a1 = fmaf(x[1], c.y, a1);
-                    e1 = fmaf(fabsf(x[1]), r.y, e1);
-                    a0 = fmaf(x[2], c.z, a0);
-                    e0 = fmaf(fabsf(x[2]), r.z, e0);
-                    a1 = fmaf(x[3], c.w, a1);
-                    e1 = fmaf(fabsf(x[3]), r.w, e1);
+                for (int i = 0; i < kDim; ++i) l1 += fabsf(qf[i]);
+                const float A = warp_sum(fabsf(w) * l1);            // sum_h |w_h| |q_h|_1
+                const float P = warp_sum(w >= 0.f ? w * l1 : 0.f);  // sum_{w_h >= 0} w_h |q_h|_1
+                for (int j = 0; j < nblk; ++j) {
+                    const int32_t B = sm.blk[j];
+                    const float M = sm.mb[j];
+                    if (MODE != BOUND_OUT) {
+                        const int32_t k0 = B * kBlockKeys;
+                        if (!(wks < k0 + kBlockKeys && wke > k0)) {  // window misses the block
+                            row_pass |= 1u << j;
+                            continue;
+                        }
+                        if (!(M < INFINITY)) continue;  // never skipped
+                        if (P * M + kPruneEps * A * M < tau) {
+                            row_pass |= 1u << j;  // |U_h| <= |q_h|_1 M_B: the coarse bound decides
+                            continue;
+                        }
+                    }
+                    const float4 *c4 = reinterpret_cast<const float4 *>(sm.box[j]);
+                    const float4 *r4 = c4 + kDim / 4;
+                    float a0 = 0.f, a1 = 0.f, e0 = 0.f, e1 = 0.f;
+#pragma unroll
+                    for (int i = 0; i < kDim / 4; ++i) {
+                        const float4 c = c4[i], r = r4[i];
+                        const float *x = qf + 4 * i;
+                        a0 = fmaf(x[0], c.x, a0);
+                        e0 = fmaf(fabsf(x[0]), r.x, e0);
+                        a1 = fmaf(x[1], c.y, a1);
+                        e1 = fmaf(fabsf(x[1]), r.y, e1);
+                        a0 = fmaf(x[2], c.z, a0);
+                        e0 = fmaf(fabsf(x[2]), r.z, e0);
+                        a1 = fmaf(x[3], c.w, a1);
+                        e1 = fmaf(fabsf(x[3]), r.w, e1);
+                    }
+                    const float mid = a0 + a1, rad = e0 + e1;
+                    const float term = w >= 0.f ? w * fmaxf(mid + rad, 0.f) : w * fmaxf(mid - rad, 0.f);
+                    const float ub = warp_sum(term);
+                    if (MODE == BOUND_OUT) {
+                        if (lane == 0) a.out[t * a.ld + B] = M < INFINITY ? ub : INFINITY;
+                    } else if (ub + kPruneEps * A * M < tau) {
+                        row_pass |= 1u << j;
+                    }
                 }
-                const float mid = a0 + a1, rad = e0 + e1;
-                const float term = w >= 0.f ? w * fmaxf(mid + rad, 0.f) : w * fmaxf(mid - rad, 0.f);
-                const float ub = warp_sum(term);
-                if (MODE == BOUND_OUT) {
-                    if (lane == 0) a.out[t * a.ld + B] = M < INFINITY ? ub : INFINITY;
-                } else if (ub + kPruneEps * A * M < tau) {
-                    row_pass |= 1u << j;
+            } else {
+                constexpr int NH = H / kHeads;  // head halves per lane
+                float A = 0.f, P = 0.f;          // sum_h |w_h| |q_h|_1 and sum_{w_h >= 0} w_h |q_h|_1
+#pragma unroll 1
+                for (int hh = 0; hh < NH; ++hh) {
+                    float qf[kDim];
+                    load_q<DT>(a.q, (t * NH + hh) * kHeads + lane, qf);
+                    const float w = a.weights[t * H + hh * kHeads + lane];
+                    float l1 = 0.f;
+#pragma unroll
+                    for (int i = 0; i < kDim; ++i) l1 += fabsf(qf[i]);
+                    A += warp_sum(fabsf(w) * l1);
+                    P += warp_sum(w >= 0.f ? w * l1 : 0.f);
                 }
+                uint32_t fine = 0;  // blocks the coarse bound does not decide
+                for (int j = 0; j < nblk; ++j) {
+                    if (MODE != BOUND_OUT) {
+                        const float M = sm.mb[j];
+                        const int32_t k0 = sm.blk[j] * kBlockKeys;
+                        if (!(wks < k0 + kBlockKeys && wke > k0)) {  // window misses the block
+                            row_pass |= 1u << j;
+                            continue;
+                        }
+                        if (!(M < INFINITY)) continue;  // never skipped
+                        if (P * M + kPruneEps * A * M < tau) {
+                            row_pass |= 1u << j;
+                            continue;
+                        }
+                    }
+                    fine |= 1u << j;
+                }
+#pragma unroll 1
+                for (int hh = 0; hh < NH; ++hh) {
+                    float qf[kDim];
+                    load_q<DT>(a.q, (t * NH + hh) * kHeads + lane, qf);
+                    const float w = a.weights[t * H + hh * kHeads + lane];
+                    for (int j = 0; j < nblk; ++j) {
+                        if (!((fine >> j) & 1u)) continue;
+                        const float4 *c4 = reinterpret_cast<const float4 *>(sm.box[j]);
+                        const float4 *r4 = c4 + kDim / 4;
+                        float a0 = 0.f, a1 = 0.f, e0 = 0.f, e1 = 0.f;
+#pragma unroll
+                        for (int i = 0; i < kDim / 4; ++i) {
+                            const float4 c = c4[i], r = r4[i];
+                            const float *x = qf + 4 * i;
+                            a0 = fmaf(x[0], c.x, a0);
+                            e0 = fmaf(fabsf(x[0]), r.x, e0);
+                            a1 = fmaf(x[1], c.y, a1);
+                            e1 = fmaf(fabsf(x[1]), r.y, e1);
+                            a0 = fmaf(x[2], c.z, a0);
+                            e0 = fmaf(fabsf(x[2]), r.z, e0);
+                            a1 = fmaf(x[3], c.w, a1);
+                            e1 = fmaf(fabsf(x[3]), r.w, e1);
+                        }
+                        const float mid = a0 + a1, rad = e0 + e1;
+                        const float term = w >= 0.f ? w * fmaxf(mid + rad, 0.f) : w * fmaxf(mid - rad, 0.f);
+                        const float part = warp_sum(term);
+                        if (lane == 0) sm.ub[warp][j] = hh == 0 ? part : sm.ub[warp][j] + part;
+                    }
+                }
+                __syncwarp();
+                for (int j = 0; j < nblk; ++j) {
+                    if (!((fine >> j) & 1u)) continue;
+                    const float ub = sm.ub[warp][j], M = sm.mb[j];
+                    if (MODE == BOUND_OUT) {
+                        if (lane == 0) a.out[t * a.ld + sm.blk[j]] = M < INFINITY ? ub : INFINITY;
+                    } else if (ub + kPruneEps * A * M < tau) {
+                        row_pass |= 1u << j;
+                    }
+                }
+                __syncwarp();  // sm.ub is read before the next row writes it
             }
             pass &= row_pass;
         }
@@ -343,20 +419,23 @@ ftk_status launch_box(int dtype, const BoxArgs &a, cudaStream_t s)
     return dtype == FTK_F8E4M3 ? launch_box_dt<FTK_F8E4M3>(a, s) : launch_box_dt<FTK_BF16>(a, s);
 }
 
-template <int DT>
+template <int DT, int H>
 static ftk_status launch_bound_dt(int mode, const BoundArgs &a, int grid, cudaStream_t s)
 {
     const int threads = kBoundWarps * 32;
-    if (mode == BOUND_EST) bound_kernel<DT, BOUND_EST><<<grid, threads, 0, s>>>(a);
-    else if (mode == BOUND_FULL) bound_kernel<DT, BOUND_FULL><<<grid, threads, 0, s>>>(a);
-    else bound_kernel<DT, BOUND_OUT><<<grid, threads, 0, s>>>(a);
+    if (mode == BOUND_EST) bound_kernel<DT, BOUND_EST, H><<<grid, threads, 0, s>>>(a);
+    else if (mode == BOUND_FULL) bound_kernel<DT, BOUND_FULL, H><<<grid, threads, 0, s>>>(a);
+    else bound_kernel<DT, BOUND_OUT, H><<<grid, threads, 0, s>>>(a);
     return cuda_status(cudaGetLastError());
 }
 
-ftk_status launch_bound(int dtype, int mode, const BoundArgs &a, int grid, cudaStream_t s)
+ftk_status launch_bound(int dtype, int mode, const BoundArgs &a, int grid, cudaStream_t s, int heads)
 {
-    return dtype == FTK_F8E4M3 ? launch_bound_dt<FTK_F8E4M3>(mode, a, grid, s)
-                               : launch_bound_dt<FTK_BF16>(mode, a, grid, s);
+    if (heads == 64)
+        return dtype == FTK_F8E4M3 ? launch_bound_dt<FTK_F8E4M3, 64>(mode, a, grid, s)
+                                   : launch_bound_dt<FTK_BF16, 64>(mode, a, grid, s);
+    return dtype == FTK_F8E4M3 ? launch_bound_dt<FTK_F8E4M3, 32>(mode, a, grid, s)
+                               : launch_bound_dt<FTK_BF16, 32>(mode, a, grid, s);
 }
 
 static int sm_count()
@@ -379,14 +458,15 @@ extern "C" size_t ftk_block_bound_workspace_size(int64_t S)
            align_up(static_cast<size_t>(nb) * sizeof(float), 256);
 }
 
-extern "C" ftk_status ftk_block_bound(ftk_dtype dtype, const void *q, const void *kv,
-                                      const float *kv_scales, const float *weights, int64_t T,
-                                      int64_t S, float *out, int64_t ld, void *workspace,
-                                      size_t workspace_bytes, void *stream)
+extern "C" ftk_status ftk_block_bound_heads(ftk_dtype dtype, int heads, const void *q, const void *kv,
+                                            const float *kv_scales, const float *weights, int64_t T,
+                                            int64_t S, float *out, int64_t ld, void *workspace,
+                                            size_t workspace_bytes, void *stream)
 {
     if (dtype != FTK_F8E4M3 && dtype != FTK_BF16) return FTK_ERR_UNSUPPORTED;
+    if (heads != 32 && heads != 64) return FTK_ERR_INVALID_ARG;
     if (!q || !kv || !weights || !out) return FTK_ERR_INVALID_ARG;
-    if (T < 1 || S < 1 || T >= (int64_t(1) << 31) / kHeads || S >= (int64_t(1) << 31) - kBlockKeys)
+    if (T < 1 || S < 1 || T >= (int64_t(1) << 31) / heads || S >= (int64_t(1) << 31) - kBlockKeys)
         return FTK_ERR_INVALID_ARG;
     const int64_t nb = (S + kBlockKeys - 1) / kBlockKeys;
     if (ld < nb) return FTK_ERR_INVALID_ARG;
@@ -421,5 +501,14 @@ extern "C" ftk_status ftk_block_bound(ftk_dtype dtype, const void *q, const void
     a.ld = ld;
     const int64_t items = static_cast<int64_t>(a.ntiles) * a.nwords;
     const int64_t cap = static_cast<int64_t>(sm_count()) * 4;
-    return launch_bound(dtype, BOUND_OUT, a, static_cast<int>(items < cap ? items : cap), s);
+    return launch_bound(dtype, BOUND_OUT, a, static_cast<int>(items < cap ? items : cap), s, heads);
+}
+
+extern "C" ftk_status ftk_block_bound(ftk_dtype dtype, const void *q, const void *kv,
+                                      const float *kv_scales, const float *weights, int64_t T,
+                                      int64_t S, float *out, int64_t ld, void *workspace,
+                                      size_t workspace_bytes, void *stream)
+{
+    return ftk_block_bound_heads(dtype, 32, q, kv, kv_scales, weights, T, S, out, ld, workspace,
+                                 workspace_bytes, stream);
 }

@@ -32,6 +32,15 @@
 // +0.0).  ReLU propagates NaN, so a NaN dot product makes the score NaN,
 // which the candidate test keeps and the refine step reports.
 //
+// 64 heads (H64 = true; FlashTopK README, "Roadmap": other head counts
+// such as 64): q [T, 64, 128] is the same bytes as [2T, 32, 128], so query
+// t occupies MMA rows 2t and 2t + 1 (heads 0..31 and 32..63) and the
+// tiles, TMA loads and TMEM layout stay as they are (4 queries per MMA
+// tile).  The epilogue warp that holds those two rows finishes one score
+//     I = sigma * ((even_a + odd_a) + (even_b + odd_b)) + 0.0
+// from the two halves' partial sums and makes one threshold decision per
+// query.
+//
 // Pruning (PR = true): key tiles that the score bound marks for the item's
 // row tile are skipped by all three roles (see ftk_prune.cuh).
 //
@@ -84,16 +93,18 @@ struct ScoreCfg<FTK_BF16> {
     static constexpr uint32_t kIdesc = instr_desc(1, 1, 128, 256);  // bf16 x bf16 -> f32
 };
 
-// Rows of the row list per work item (the planning granularity).
-__host__ __device__ constexpr int row_tile_of(int dtype)
+// Rows of the row list per work item (the planning granularity): the
+// queries of the item's MMA tiles (a 64-head query takes two MMA rows).
+__host__ __device__ constexpr int row_tile_of(int dtype, int heads = 32)
 {
-    return dtype == FTK_F8E4M3 ? ScoreCfg<FTK_F8E4M3>::kQG * kQTile : ScoreCfg<FTK_BF16>::kQG * kQTile;
+    return (dtype == FTK_F8E4M3 ? ScoreCfg<FTK_F8E4M3>::kQG : ScoreCfg<FTK_BF16>::kQG) * kQTile /
+           (heads == 64 ? 2 : 1);
 }
 
 struct ScoreArgs {
     int64_t T, S;
     const float *kv_scales;   // [S] or NULL (all ones)
-    const float *weights;     // [T, 32]
+    const float *weights;     // [T, heads]
     const int32_t *ks, *ke;   // [T]
     // Row list: position p of the list is query rows[p] (identity if NULL).
     // The list holds min(nrows, *count_dev - count_off) rows when count_dev
@@ -330,6 +341,17 @@ __device__ __forceinline__ float head_finish(uint64_t p, float sigma)
     return __fmaf_rn(sigma, __fadd_rn(even, odd), 0.0f);
 }
 
+// The score of a 64-head query held as two 32-head halves (p: heads 0..31,
+// q: heads 32..63, each an even/odd pair of partial sums):
+//   I = sigma * ((p.even + p.odd) + (q.even + q.odd)) + 0.0.
+__device__ __forceinline__ float head_finish_pair(uint64_t p, uint64_t q, float sigma)
+{
+    float pe, po, qe, qo;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(pe), "=f"(po) : "l"(p));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(qe), "=f"(qo) : "l"(q));
+    return __fmaf_rn(sigma, __fadd_rn(__fadd_rn(pe, po), __fadd_rn(qe, qo)), 0.0f);
+}
+
 template <int DT>
 struct ScoreSmemLayout {
     using C = ScoreCfg<DT>;
@@ -368,7 +390,7 @@ static_assert(ScoreCfg<FTK_F8E4M3>::kKStages <= 4 && ScoreCfg<FTK_BF16>::kKStage
 // COLLECT variants are launched and the one that does not match the
 // device-side decision (*prune_on) returns at once, so an unpruned scan runs
 // exactly the plain tile loop.
-template <int DT, int MODE, bool PR>
+template <int DT, int MODE, bool PR, bool H64>
 __global__ void __launch_bounds__(kScoreThreads, 1)
     score_kernel(const __grid_constant__ ScoreArgs a, const __grid_constant__ CUtensorMap tm_q,
                  const __grid_constant__ KvMaps kvm)
@@ -377,7 +399,11 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     using C = ScoreCfg<DT>;
     using Lay = ScoreSmemLayout<DT>;
     constexpr int QG = C::kQG;
-    constexpr int RT = QG * kQTile;  // rows per work item
+    // H64: a 64-head query is two consecutive 32-head rows of the MMA tile
+    // (the same bytes: q [T, 64, 128] == [2T, 32, 128]).
+    constexpr int VPQ = H64 ? 2 : 1;     // MMA rows (32 heads each) per query
+    constexpr int QPT = kQTile / VPQ;    // queries per MMA tile
+    constexpr int RT = QG * QPT;         // queries per work item
     extern __shared__ uint8_t smem_dyn[];
     // 1024-byte alignment: the 128-byte swizzle pattern repeats every 8 rows.
     // (Offsetting the __shared__ array itself keeps every derived pointer
@@ -462,13 +488,14 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                 q_armed = 1;
                 q_armed_ph = qph;
                 for (int vt = 0; vt < QG; ++vt) {
-                    for (int j = 0; j < kQTile; ++j) {
-                        int32_t t = list_query(a, static_cast<int64_t>(m.tile) * RT + vt * kQTile + j, nlist);
+                    for (int j = 0; j < kQTile; ++j) {  // MMA row j: half j % VPQ of query j / VPQ
+                        int32_t t = list_query(a, static_cast<int64_t>(m.tile) * RT + vt * QPT + j / VPQ,
+                                               nlist);
                         if (t < 0) t = 0;  // placeholder rows are masked in the epilogue
                         for (int at = 0; at < C::kAtoms; ++at)
                             tma_load_2d(sq + vt * Lay::kQTileBytes + at * (Lay::kQTileBytes / C::kAtoms) +
                                             j * kHeads * 128,
-                                        &tm_q, &ms.q_full, at * 64, t * kHeads);
+                                        &tm_q, &ms.q_full, at * 64, (t * VPQ + j % VPQ) * kHeads);
                     }
                 }
                 qph ^= 1u;
@@ -559,15 +586,16 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         // Each epilogue warp works on its own: its queries' parameters and
         // weights, and its own candidate staging, so the tile loop has no
         // cross-warp synchronisation besides releasing the accumulator.
-        constexpr int NQ = kEpiQueries;          // queries per warp per query tile
-        constexpr int WQ = QG * NQ;              // queries per warp
+        constexpr int NQ = kEpiQueries;          // MMA rows per warp per query tile (2)
+        constexpr int NR = NQ / VPQ;             // queries per warp per query tile
+        constexpr int WQ = QG * NR;              // queries per warp
         const int ew = warp - 2;                 // 0..15
         const int quad = warp & 3;               // TMEM lane quarter
         const int qg = ew >> 2;                  // query pair within each query tile
         const int key_lane = quad * 32 + lane;   // row of the 128-key tile
         const uint32_t tlane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
         const uint32_t lt_mask = (1u << lane) - 1u;
-        float *my_w = sw + ew * WQ * kHeads;
+        float *my_w = sw + ew * QG * NQ * kHeads;  // by MMA row: (vt * NQ + r) * 32 + head
         float *my_sv = stage_val + ew * WQ * C::kWarpStage;
         int32_t *my_si = stage_idx + ew * WQ * C::kWarpStage;
         int ab = 0;
@@ -586,12 +614,13 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             if (it < 0) break;
             get_item<MODE, RT>(a, sc, it, nlist, m);
             // Per-item parameters of this warp's queries (warp-uniform).  Slot
-            // qq = vt * NQ + qi is query qg * NQ + qi of query tile vt.
+            // qq = vt * NR + qi is query qg * NR + qi of query tile vt, whose
+            // MMA rows are qg * NQ + qi * VPQ + (0 .. VPQ - 1).
             int32_t qt[WQ], qpos[WQ], wlo[WQ], wlen[WQ];
             float qtau[WQ];
             {
                 const int sl = lane % WQ;
-                const int64_t p = static_cast<int64_t>(m.tile) * RT + (sl / NQ) * kQTile + qg * NQ + (sl % NQ);
+                const int64_t p = static_cast<int64_t>(m.tile) * RT + (sl / NR) * QPT + qg * NR + (sl % NR);
                 int32_t t_l = -1, ks_l = 0, ke_l = 0;
                 float tau_l = 0.f;
                 if (lane < WQ) {
@@ -608,10 +637,14 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                     wlo[qq] = __shfl_sync(0xFFFFFFFFu, ks_l, qq);
                     wlen[qq] = __shfl_sync(0xFFFFFFFFu, ke_l, qq) - wlo[qq];
                     qtau[qq] = __shfl_sync(0xFFFFFFFFu, tau_l, qq);
-                    qpos[qq] = m.tile * RT + (qq / NQ) * kQTile + qg * NQ + (qq % NQ);
-                    my_w[qq * kHeads + lane] =
-                        qt[qq] >= 0 ? stored_weight(a.weights[static_cast<int64_t>(qt[qq]) * kHeads + lane], lane)
-                                    : 0.f;
+                    qpos[qq] = m.tile * RT + (qq / NR) * QPT + qg * NR + (qq % NR);
+#pragma unroll
+                    for (int v = 0; v < VPQ; ++v)
+                        my_w[((qq / NR) * NQ + (qq % NR) * VPQ + v) * kHeads + lane] =
+                            qt[qq] >= 0 ? stored_weight(a.weights[(static_cast<int64_t>(qt[qq]) * VPQ + v) * kHeads +
+                                                                  lane],
+                                                        lane)
+                                        : 0.f;
                 }
                 __syncwarp();
             }
@@ -679,17 +712,21 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                         ab = 0;
                         aph ^= 1u;
                     }
-                    float I[NQ];
-                    I[0] = head_finish(p, sigma);
-                    I[1] = head_finish(q, sigma);
+                    float I[NR];
+                    if constexpr (H64) {
+                        I[0] = head_finish_pair(p, q, sigma);
+                    } else {
+                        I[0] = head_finish(p, sigma);
+                        I[1] = head_finish(q, sigma);
+                    }
                     if (MODE == MODE_COLLECT) {
                         // Candidates are rare: one vote for both queries, the
                         // staging only when some lane has one.
-                        bool take[NQ];
+                        bool take[NR];
                         bool anyt = false;
 #pragma unroll
-                        for (int qi = 0; qi < NQ; ++qi) {
-                            const int qq = vt * NQ + qi;
+                        for (int qi = 0; qi < NR; ++qi) {
+                            const int qq = vt * NR + qi;
                             // s in [wlo, wlo + wlen) as one unsigned compare
                             const bool valid = static_cast<uint32_t>(s - wlo[qq]) < static_cast<uint32_t>(wlen[qq]);
                             take[qi] = valid && !(I[qi] < qtau[qq]);  // NaN is kept, to be seen
@@ -697,8 +734,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                         }
                         if (__any_sync(0xFFFFFFFFu, anyt)) {
 #pragma unroll
-                            for (int qi = 0; qi < NQ; ++qi) {
-                                const int qq = vt * NQ + qi;
+                            for (int qi = 0; qi < NR; ++qi) {
+                                const int qq = vt * NR + qi;
                                 const uint32_t bal = __ballot_sync(0xFFFFFFFFu, take[qi]);
                                 const int pos = cnt[qq] + __popc(bal & lt_mask);
                                 if (take[qi]) {
@@ -711,8 +748,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                         }
                     }
 #pragma unroll
-                    for (int qi = 0; qi < (MODE == MODE_COLLECT ? 0 : NQ); ++qi) {
-                        const int qq = vt * NQ + qi;
+                    for (int qi = 0; qi < (MODE == MODE_COLLECT ? 0 : NR); ++qi) {
+                        const int qq = vt * NR + qi;
                         const bool valid = static_cast<uint32_t>(s - wlo[qq]) < static_cast<uint32_t>(wlen[qq]);
                         if (MODE == MODE_SAMPLE) {
                             if (qt[qq] >= 0 && kidx < m.kend)

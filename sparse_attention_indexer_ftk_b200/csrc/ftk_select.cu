@@ -585,6 +585,7 @@ static int num_sms()
 enum PruneMode { PRUNE_AUTO = 0, PRUNE_ON = 1, PRUNE_OFF = 2 };
 
 struct SelectCfg {
+    int heads;      // 32 or 64
     int m;          // sample keys
     float beta;
     int cap;
@@ -599,6 +600,7 @@ static int64_t scratch_ld_of(int64_t S) { return (S + 7) / 8 * 8; }
 static SelectCfg resolve_cfg(int64_t T, int64_t S, int topk, const ftk_config *c)
 {
     SelectCfg r;
+    r.heads = c && c->heads == 64 ? 64 : 32;
     r.m = c && c->sample_keys > 0 ? c->sample_keys : 4096;
     r.beta = c && c->oversample > 0.f ? c->oversample : 1.5f;
     r.cap = c && c->capacity > 0 ? c->capacity : 2 * topk;
@@ -650,7 +652,12 @@ struct SelectWs {
 
 static bool carve_select(Carver &cv, int64_t T, int64_t S, const SelectCfg &c, SelectWs &w)
 {
-    const int64_t ntiles = (T + kQTile - 1) / kQTile;
+    // Row tiles of the smallest row tile of either dtype (the size query
+    // does not know the dtype).
+    const int64_t min_rt = row_tile_of(FTK_BF16, c.heads) < row_tile_of(FTK_F8E4M3, c.heads)
+                               ? row_tile_of(FTK_BF16, c.heads)
+                               : row_tile_of(FTK_F8E4M3, c.heads);
+    const int64_t ntiles = (T + min_rt - 1) / min_rt;
     w.info = cv.take<DevInfo>(1);
     w.s_lo = cv.take<int32_t>(ntiles);
     w.s_hi = cv.take<int32_t>(ntiles);
@@ -683,12 +690,12 @@ static bool carve_select(Carver &cv, int64_t T, int64_t S, const SelectCfg &c, S
     return cv.ok;
 }
 
-template <int DT, int MODE, bool PR>
+template <int DT, int MODE, bool PR, bool H64>
 static ftk_status launch_score(const ScoreArgs &a, const CUtensorMap &tq, const KvMaps &kvm,
                                int grid, cudaStream_t st)
 {
     const int smem = ScoreSmemLayout<DT>::kBytes;
-    auto kern = score_kernel<DT, MODE, PR>;
+    auto kern = score_kernel<DT, MODE, PR, H64>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_status(e);
     kern<<<grid, kScoreThreads, smem, st>>>(a, tq, kvm);
@@ -696,18 +703,24 @@ static ftk_status launch_score(const ScoreArgs &a, const CUtensorMap &tq, const 
 }
 
 template <int MODE, bool PR = false>
-static ftk_status launch_score_dt(int dtype, const ScoreArgs &a, const CUtensorMap &tq,
+static ftk_status launch_score_dt(int dtype, int heads, const ScoreArgs &a, const CUtensorMap &tq,
                                   const KvMaps &kvm, int grid, cudaStream_t st)
 {
-    if (dtype == FTK_F8E4M3) return launch_score<FTK_F8E4M3, MODE, PR>(a, tq, kvm, grid, st);
-    return launch_score<FTK_BF16, MODE, PR>(a, tq, kvm, grid, st);
+    if (heads == 64) {
+        if (dtype == FTK_F8E4M3) return launch_score<FTK_F8E4M3, MODE, PR, true>(a, tq, kvm, grid, st);
+        return launch_score<FTK_BF16, MODE, PR, true>(a, tq, kvm, grid, st);
+    }
+    if (dtype == FTK_F8E4M3) return launch_score<FTK_F8E4M3, MODE, PR, false>(a, tq, kvm, grid, st);
+    return launch_score<FTK_BF16, MODE, PR, false>(a, tq, kvm, grid, st);
 }
 
-static bool build_maps(int dtype, const void *q, const void *kv, int64_t T, int64_t S, int max_lg,
+// q as rows of 128 elements (T * heads of them, boxes of 32 = one MMA row
+// each), and kv at every sample stride.
+static bool build_maps(int dtype, int heads, const void *q, const void *kv, int64_t T, int64_t S, int max_lg,
                        CUtensorMap *tq, KvMaps *kvm)
 {
     const uint64_t esz = dtype == FTK_F8E4M3 ? 1 : 2;
-    if (!make_map(tq, dtype, q, static_cast<uint64_t>(T) * kHeads, kDim * esz, kHeads)) return false;
+    if (!make_map(tq, dtype, q, static_cast<uint64_t>(T) * heads, kDim * esz, kHeads)) return false;
     for (int i = 0; i < kNumStrideMaps; ++i) {
         if (i > max_lg) {
             kvm->m[i] = kvm->m[0];
@@ -720,13 +733,14 @@ static bool build_maps(int dtype, const void *q, const void *kv, int64_t T, int6
     return true;
 }
 
-static ftk_status check_select_args(int dtype, const void *q, const void *kv, const float *w,
+static ftk_status check_select_args(int dtype, int heads, const void *q, const void *kv, const float *w,
                                     const int32_t *ks, const int32_t *ke, int64_t T, int64_t S,
                                     int topk, const int32_t *out_idx)
 {
     if (dtype != FTK_F8E4M3 && dtype != FTK_BF16) return FTK_ERR_UNSUPPORTED;
+    if (heads != 32 && heads != 64) return FTK_ERR_INVALID_ARG;
     if (!q || !kv || !w || !ks || !ke || !out_idx) return FTK_ERR_INVALID_ARG;
-    if (T < 1 || S < 1 || T >= (int64_t(1) << 31) / kHeads || S >= (int64_t(1) << 31) - kChunkKeys)
+    if (T < 1 || S < 1 || T >= (int64_t(1) << 31) / heads || S >= (int64_t(1) << 31) - kChunkKeys)
         return FTK_ERR_INVALID_ARG;
     if (topk < 1 || topk > FTK_MAX_TOPK) return FTK_ERR_TOPK_RANGE;
     if (!aligned16(q) || !aligned16(kv) || !aligned16(w)) return FTK_ERR_ALIGNMENT;
@@ -768,6 +782,7 @@ extern "C" ftk_status ftk_set_stage_events(void *const *events, int n)
 extern "C" size_t ftk_select_workspace_size(int64_t T, int64_t S, int topk, const ftk_config *config)
 {
     if (T < 1 || S < 1 || topk < 1 || topk > FTK_MAX_TOPK) return 0;
+    if (config && config->heads != 0 && config->heads != 32 && config->heads != 64) return 0;
     const SelectCfg c = resolve_cfg(T, S, topk, config);
     Carver cv{nullptr, 0};
     SelectWs w;
@@ -790,10 +805,12 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
                                  int32_t *out_idx, float *out_val, void *workspace,
                                  size_t workspace_bytes, const ftk_config *config, void *stream)
 {
-    ftk_status st = check_select_args(dtype, q, kv, weights, ks, ke, T, S, topk, out_idx);
-    if (st != FTK_OK) return st;
-    if (config && (config->reserved[0] || config->reserved[1] || config->reserved[2]))
+    if (config && (config->reserved[0] || config->reserved[1] ||
+                   (config->heads != 0 && config->heads != 32 && config->heads != 64)))
         return FTK_ERR_INVALID_ARG;
+    const int heads = config && config->heads == 64 ? 64 : 32;
+    ftk_status st = check_select_args(dtype, heads, q, kv, weights, ks, ke, T, S, topk, out_idx);
+    if (st != FTK_OK) return st;
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return FTK_ERR_WORKSPACE;
     const SelectCfg c = resolve_cfg(T, S, topk, config);
     if (c.cap < topk) return FTK_ERR_INVALID_ARG;
@@ -810,9 +827,9 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
     if (max_lg >= kNumStrideMaps) return FTK_ERR_UNSUPPORTED;
     CUtensorMap tq;
     KvMaps kvm;
-    if (!build_maps(dtype, q, kv, T, S, max_lg, &tq, &kvm)) return FTK_ERR_CUDA;
+    if (!build_maps(dtype, heads, q, kv, T, S, max_lg, &tq, &kvm)) return FTK_ERR_CUDA;
 
-    const int rt = row_tile_of(dtype);
+    const int rt = row_tile_of(dtype, heads);
     const int32_t ntiles = static_cast<int32_t>((T + rt - 1) / rt);
     const int sms = num_sms();
     uint32_t *status = &w.info->info.status;
@@ -880,7 +897,7 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
     sa.item_start = w.s_start;
     sa.out = w.samp;
     sa.ld = w.sld;
-    st = launch_score_dt<MODE_SAMPLE>(dtype, sa, tq, kvm, sms, s);  // CTAs without an item exit
+    st = launch_score_dt<MODE_SAMPLE>(dtype, heads, sa, tq, kvm, sms, s);  // CTAs without an item exit
     if (st != FTK_OK) return st;
     stage_mark(2, s);
 
@@ -943,12 +960,12 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
         ba.prune_enabled = &w.info->info.prune_enabled;
         ba.blocks_pruned = reinterpret_cast<unsigned long long *>(&w.info->info.blocks_pruned);
         if (c.prune == PRUNE_AUTO) {
-            st = launch_bound(dtype, BOUND_EST, ba, ba.est_tiles * (kEstBlocks / kEstChunk), s);
+            st = launch_bound(dtype, BOUND_EST, ba, ba.est_tiles * (kEstBlocks / kEstChunk), s, heads);
             if (st != FTK_OK) return st;
         }
         const int64_t items = static_cast<int64_t>(ntiles) * w.nwords;
         const int64_t cap = static_cast<int64_t>(sms) * 2;
-        st = launch_bound(dtype, BOUND_FULL, ba, static_cast<int>(items < cap ? items : cap), s);
+        st = launch_bound(dtype, BOUND_FULL, ba, static_cast<int>(items < cap ? items : cap), s, heads);
         if (st != FTK_OK) return st;
     }
     stage_mark(7, s);
@@ -972,11 +989,11 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
     // auto: both variants, the device-side decision picks one (the other
     // returns at once); always: the pruned one; off: the plain one
     if (c.prune != PRUNE_ON) {
-        st = launch_score_dt<MODE_COLLECT, false>(dtype, sa, tq, kvm, sms, s);
+        st = launch_score_dt<MODE_COLLECT, false>(dtype, heads, sa, tq, kvm, sms, s);
         if (st != FTK_OK) return st;
     }
     if (c.prune != PRUNE_OFF) {
-        st = launch_score_dt<MODE_COLLECT, true>(dtype, sa, tq, kvm, sms, s);
+        st = launch_score_dt<MODE_COLLECT, true>(dtype, heads, sa, tq, kvm, sms, s);
         if (st != FTK_OK) return st;
     }
     stage_mark(4, s);
@@ -1027,7 +1044,7 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
         da.out = w.scratch;
         da.ld = w.scratch_ld;
         da.status = status;
-        st = launch_score_dt<MODE_DUMP>(dtype, da, tq, kvm, sms, s);
+        st = launch_score_dt<MODE_DUMP>(dtype, heads, da, tq, kvm, sms, s);
         if (st != FTK_OK) return st;
         RowsArgs ra2 = {};
         ra2.x = w.scratch;
@@ -1060,13 +1077,13 @@ extern "C" size_t ftk_score_dense_workspace_size(int64_t nrows)
     return 256;
 }
 
-extern "C" ftk_status ftk_score_dense(ftk_dtype dtype, const void *q, const void *kv,
-                                      const float *kv_scales, const float *weights,
-                                      const int32_t *ks, const int32_t *ke, int64_t T, int64_t S,
-                                      const int32_t *rows, int64_t nrows, float *out, int64_t ld,
-                                      void *workspace, size_t workspace_bytes, void *stream)
+extern "C" ftk_status ftk_score_dense_heads(ftk_dtype dtype, int heads, const void *q, const void *kv,
+                                            const float *kv_scales, const float *weights,
+                                            const int32_t *ks, const int32_t *ke, int64_t T, int64_t S,
+                                            const int32_t *rows, int64_t nrows, float *out, int64_t ld,
+                                            void *workspace, size_t workspace_bytes, void *stream)
 {
-    ftk_status st = check_select_args(dtype, q, kv, weights, ks, ke, T, S, 1, rows ? rows : ks);
+    ftk_status st = check_select_args(dtype, heads, q, kv, weights, ks, ke, T, S, 1, rows ? rows : ks);
     if (st != FTK_OK) return st;
     // ld >= S: every valid window (ke <= S) fits its row, whatever the
     // windows hold on the device
@@ -1078,7 +1095,7 @@ extern "C" ftk_status ftk_score_dense(ftk_dtype dtype, const void *q, const void
     if (st != FTK_OK) return st;
     CUtensorMap tq;
     KvMaps kvm;
-    if (!build_maps(dtype, q, kv, T, S, 0, &tq, &kvm)) return FTK_ERR_CUDA;
+    if (!build_maps(dtype, heads, q, kv, T, S, 0, &tq, &kvm)) return FTK_ERR_CUDA;
     ScoreArgs da = {};
     da.T = T;
     da.S = S;
@@ -1094,5 +1111,15 @@ extern "C" ftk_status ftk_score_dense(ftk_dtype dtype, const void *q, const void
     cudaStream_t s = as_stream(stream);
     cudaError_t e = cudaMemsetAsync(workspace, 0, 4, s);
     if (e != cudaSuccess) return cuda_status(e);
-    return launch_score_dt<MODE_DUMP>(dtype, da, tq, kvm, num_sms(), s);
+    return launch_score_dt<MODE_DUMP>(dtype, heads, da, tq, kvm, num_sms(), s);
+}
+
+extern "C" ftk_status ftk_score_dense(ftk_dtype dtype, const void *q, const void *kv,
+                                      const float *kv_scales, const float *weights,
+                                      const int32_t *ks, const int32_t *ke, int64_t T, int64_t S,
+                                      const int32_t *rows, int64_t nrows, float *out, int64_t ld,
+                                      void *workspace, size_t workspace_bytes, void *stream)
+{
+    return ftk_score_dense_heads(dtype, 32, q, kv, kv_scales, weights, ks, ke, T, S, rows, nrows, out, ld,
+                                 workspace, workspace_bytes, stream);
 }

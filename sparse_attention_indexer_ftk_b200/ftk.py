@@ -34,6 +34,7 @@ LIB_PATH = os.path.join(HERE, "libftk.so")
 F8E4M3, BF16, F32 = 1, 2, 3
 STATUS_BAD_WINDOW, STATUS_NAN, STATUS_TIMEOUT, STATUS_BAD_SCALE, STATUS_INTERNAL = 1, 2, 4, 8, 16
 HEADS, DIM, MAX_TOPK = 32, 128, 4096
+HEAD_COUNTS = (32, 64)  # indexer head counts the kernels take
 
 # Every symbol include/ftk.h declares.
 EXPORTS = (
@@ -41,7 +42,7 @@ EXPORTS = (
     "ftk_score_dense", "ftk_score_dense_workspace_size", "ftk_windows_from_cu_seqlens",
     "ftk_set_stage_events", "ftk_status_string", "ftk_version", "ftk_select_noalloc",
     "ftk_block_bound", "ftk_block_bound_workspace_size", "ftk_topk_rows_end", "ftk_topk_rows_sorted",
-    "ftk_rows_options_init", "ftk_topk_rows_ex",
+    "ftk_rows_options_init", "ftk_topk_rows_ex", "ftk_score_dense_heads", "ftk_block_bound_heads",
 )
 
 
@@ -52,7 +53,8 @@ class FtkError(RuntimeError):
 class FtkConfig(ctypes.Structure):
     _fields_ = [("sample_keys", ctypes.c_int32), ("oversample", ctypes.c_float),
                 ("capacity", ctypes.c_int32), ("prune", ctypes.c_int32),
-                ("recovery_rows", ctypes.c_int32), ("reserved", ctypes.c_int32 * 3)]
+                ("recovery_rows", ctypes.c_int32), ("heads", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 2)]
 
 
 class FtkRowsOptions(ctypes.Structure):
@@ -94,6 +96,8 @@ def load_library(path: str = LIB_PATH):
     L.ftk_topk_rows.argtypes = [I32, P, I64, I64, I64, I32, P, P, P, P]
     L.ftk_score_dense.restype = I32
     L.ftk_score_dense.argtypes = [I32, P, P, P, P, P, P, I64, I64, P, I64, P, I64, P, SZ, P]
+    L.ftk_score_dense_heads.restype = I32
+    L.ftk_score_dense_heads.argtypes = [I32, I32, P, P, P, P, P, P, I64, I64, P, I64, P, I64, P, SZ, P]
     L.ftk_score_dense_workspace_size.restype = SZ
     L.ftk_score_dense_workspace_size.argtypes = [I64]
     L.ftk_windows_from_cu_seqlens.restype = I32
@@ -112,6 +116,8 @@ def load_library(path: str = LIB_PATH):
     L.ftk_topk_rows_ex.argtypes = [I32, P, I64, I64, I64, P, I32, P, P, P, P, P]
     L.ftk_block_bound.restype = I32
     L.ftk_block_bound.argtypes = [I32, P, P, P, P, I64, I64, P, I64, P, SZ, P]
+    L.ftk_block_bound_heads.restype = I32
+    L.ftk_block_bound_heads.argtypes = [I32, I32, P, P, P, P, I64, I64, P, I64, P, SZ, P]
     L.ftk_block_bound_workspace_size.restype = SZ
     L.ftk_block_bound_workspace_size.argtypes = [I64]
     L.ftk_status_string.restype = ctypes.c_char_p
@@ -155,24 +161,29 @@ def _need_cuda(*ts):
             raise FtkError("inputs must be CUDA tensors")
 
 
-def _config(cfg: dict | None):
-    if not cfg:
+def _config(cfg: dict | None, heads: int = HEADS):
+    """ftk_config from a dict of knobs plus the indexer's head count (None:
+    the library defaults)."""
+    if not cfg and heads == HEADS:
         return None
     c = FtkConfig()
-    for k, v in cfg.items():
+    for k, v in (cfg or {}).items():
         setattr(c, k, v)
+    if cfg and cfg.get("heads", heads) != heads:
+        raise FtkError(f"config heads={cfg['heads']} but q has {heads} heads")
+    c.heads = heads
     return c
 
 
 def _check_select_inputs(q, kv, weights, ks, ke, kv_scales):
     _need_cuda(q, kv, weights, ks, ke, kv_scales)
-    if q.dim() != 3 or q.shape[1:] != (HEADS, DIM) or not q.is_contiguous():
-        raise FtkError("q must be a contiguous [T, 32, 128] tensor")
+    if q.dim() != 3 or q.shape[1] not in HEAD_COUNTS or q.shape[2] != DIM or not q.is_contiguous():
+        raise FtkError("q must be a contiguous [T, H, 128] tensor, H = 32 or 64")
     if kv.dim() != 2 or kv.shape[1] != DIM or not kv.is_contiguous() or kv.dtype != q.dtype:
         raise FtkError("kv must be a contiguous [S, 128] tensor of q's dtype")
     T = q.shape[0]
-    if weights.shape != (T, HEADS) or weights.dtype != torch.float32 or not weights.is_contiguous():
-        raise FtkError("weights must be a contiguous float32 [T, 32] tensor")
+    if weights.shape != (T, q.shape[1]) or weights.dtype != torch.float32 or not weights.is_contiguous():
+        raise FtkError("weights must be a contiguous float32 [T, H] tensor (H: q's heads)")
     for name, w in (("ks", ks), ("ke", ke)):
         if w.shape != (T,) or w.dtype != torch.int32 or not w.is_contiguous():
             raise FtkError(f"{name} must be a contiguous int32 [T] tensor")
@@ -207,8 +218,8 @@ def _check_status(status: torch.Tensor | None, device: torch.device):
         raise FtkError(f"status must be a contiguous int32 tensor of at least one element on {device}")
 
 
-def select_workspace_size(T: int, S: int, topk: int, config: dict | None = None) -> int:
-    c = _config(config)
+def select_workspace_size(T: int, S: int, topk: int, config: dict | None = None, heads: int = HEADS) -> int:
+    c = _config(config, heads)
     return int(lib().ftk_select_workspace_size(T, S, topk, ctypes.byref(c) if c else None))
 
 
@@ -228,12 +239,13 @@ def select(q, kv, weights, ks, ke, kv_scales=None, topk: int = 2048, return_scor
     if return_scores:
         _check_buffer(out_val, (T, topk), torch.float32, dev, "out_val")
     if workspace is None:
-        workspace = torch.empty(select_workspace_size(T, S, topk, config), dtype=torch.uint8, device=dev)
+        workspace = torch.empty(select_workspace_size(T, S, topk, config, q.shape[1]), dtype=torch.uint8,
+                                device=dev)
     if out_idx is None:
         out_idx = torch.empty((T, topk), dtype=torch.int32, device=dev)
     if return_scores and out_val is None:
         out_val = torch.empty((T, topk), dtype=torch.float32, device=dev)
-    c = _config(config)
+    c = _config(config, q.shape[1])
     st = lib().ftk_select(_dtype_code(q), _ptr(q), _ptr(kv), _ptr(kv_scales), _ptr(weights), _ptr(ks),
                           _ptr(ke), T, S, topk, _ptr(out_idx), _ptr(out_val) if return_scores else None,
                           _ptr(workspace), workspace.numel(), ctypes.byref(c) if c else None,
@@ -285,13 +297,14 @@ class Selector:
     topk: int = 2048
     dtype: torch.dtype = torch.float8_e4m3fn
     config: dict | None = None
+    heads: int = HEADS
     workspace: torch.Tensor | None = None
     max_rows: int = 0
     max_kv: int = 0
 
     def plan(self, max_rows: int, max_kv: int, device="cuda") -> "Selector":
         self.max_rows, self.max_kv = max_rows, max_kv
-        nbytes = select_workspace_size(max_rows, max_kv, self.topk, self.config)
+        nbytes = select_workspace_size(max_rows, max_kv, self.topk, self.config, self.heads)
         self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
         return self
 
@@ -300,8 +313,9 @@ class Selector:
             self.plan(q.shape[0], kv.shape[0], q.device)
         if q.shape[0] > self.max_rows or kv.shape[0] > self.max_kv:
             raise FtkError("inputs exceed the planned sizes")
-        if q.dtype != self.dtype:
-            raise FtkError(f"this Selector was made for {self.dtype} inputs, not {q.dtype}")
+        if q.dtype != self.dtype or q.shape[1] != self.heads:
+            raise FtkError(f"this Selector was made for {self.dtype} inputs of {self.heads} heads, "
+                           f"not {q.dtype} of {q.shape[1]}")
         return select(q, kv, weights, ks, ke, kv_scales, self.topk, return_scores,
                       workspace=self.workspace, config=self.config, out_idx=out_idx, out_val=out_val)
 
@@ -398,10 +412,10 @@ def score_dense(q, kv, weights, ks, ke, kv_scales=None, rows: torch.Tensor | Non
         ld = (S + 3) // 4 * 4
     out = torch.full((nrows, ld), float("nan"), dtype=torch.float32, device=dev)
     ws = torch.empty(int(lib().ftk_score_dense_workspace_size(nrows)), dtype=torch.uint8, device=dev)
-    st = lib().ftk_score_dense(_dtype_code(q), _ptr(q), _ptr(kv), _ptr(kv_scales), _ptr(weights), _ptr(ks),
-                               _ptr(ke), T, S, _ptr(rows), nrows, _ptr(out), ld, _ptr(ws), ws.numel(),
-                               _stream(dev))
-    _check(st, "ftk_score_dense")
+    st = lib().ftk_score_dense_heads(_dtype_code(q), q.shape[1], _ptr(q), _ptr(kv), _ptr(kv_scales),
+                                     _ptr(weights), _ptr(ks), _ptr(ke), T, S, _ptr(rows), nrows, _ptr(out), ld,
+                                     _ptr(ws), ws.numel(), _stream(dev))
+    _check(st, "ftk_score_dense_heads")
     return out
 
 
@@ -415,7 +429,7 @@ def block_bound(q, kv, weights, kv_scales=None) -> torch.Tensor:
     nb = (S + 127) // 128
     out = torch.empty((T, nb), dtype=torch.float32, device=dev)
     ws = torch.empty(int(lib().ftk_block_bound_workspace_size(S)), dtype=torch.uint8, device=dev)
-    st = lib().ftk_block_bound(_dtype_code(q), _ptr(q), _ptr(kv), _ptr(kv_scales), _ptr(weights), T, S,
-                               _ptr(out), nb, _ptr(ws), ws.numel(), _stream(dev))
-    _check(st, "ftk_block_bound")
+    st = lib().ftk_block_bound_heads(_dtype_code(q), q.shape[1], _ptr(q), _ptr(kv), _ptr(kv_scales),
+                                     _ptr(weights), T, S, _ptr(out), nb, _ptr(ws), ws.numel(), _stream(dev))
+    _check(st, "ftk_block_bound_heads")
     return out

@@ -208,12 +208,12 @@ def _fp8(x: torch.Tensor) -> torch.Tensor:
     return x.to(torch.float8_e4m3fn)
 
 
-def fp8_causal(n: int, name: str, T: int, S: int, topk: int) -> SelectInputs:
+def fp8_causal(n: int, name: str, T: int, S: int, topk: int, heads: int = 32) -> SelectInputs:
     g = _gen(n)
-    q = _fp8(_normal(g, (T, 32, 128)))
+    q = _fp8(_normal(g, (T, heads, 128)))
     kv = _fp8(_normal(g, (S, 128)))
     sc = _scales(g, S)
-    w = _weights(g, T)
+    w = _weights(g, T, heads)
     ks, ke = causal_windows(T, S)
     return SelectInputs(name, q, kv, sc, w, ks, ke, topk)
 
@@ -224,6 +224,13 @@ def fp8_prefill() -> SelectInputs:
 
 def fp8_large() -> SelectInputs:
     return fp8_causal(5, "fp8_large", 8192, 262144, 4096)
+
+
+def fp8_prefill_64h() -> SelectInputs:
+    """The fp8_prefill shape for a 64-head indexer (FlashTopK README,
+    "Roadmap": other head counts such as 64): q [4096, 64, 128], weights
+    N(0,1)/sqrt(64)."""
+    return fp8_causal(6, "fp8_prefill_64h", 4096, 131072, 2048, heads=64)
 
 
 def fp8_packed(gamma: float = 6.0) -> SelectInputs:
@@ -317,6 +324,7 @@ def get(name: str):
         "bf16_small": bf16_small, "bf16_ties": bf16_ties, "bf16_all_equal": bf16_all_equal,
         "rows_bf16": rows_bf16, "rows_f32": rows_f32, "rows_bf16_1024": rows_bf16_1024,
         "fp8_prefill": fp8_prefill, "fp8_packed": fp8_packed, "fp8_large": fp8_large,
+        "fp8_prefill_64h": fp8_prefill_64h,
     }
     return table[name]()
 
@@ -332,16 +340,17 @@ def sample_rows(T: int, n: int, seed: int = 0) -> list[int]:
 
 
 def block_structured(seed: int, dtype: str, T: int, S: int, topk: int, hot_every: int = 8,
-                     cold: float = 2.0 ** -7) -> SelectInputs:
+                     cold: float = 2.0 ** -7, heads: int = 32) -> SelectInputs:
     """Keys in 128-key blocks where only every hot_every-th block keeps its
     kv_scales and the others have theirs multiplied by `cold`, with causal
     windows and mostly positive weights (|N(0,1)|/sqrt(32), negated on the
     heads h % 8 == 0): the top-k lies in the hot blocks and the cold blocks'
     scores stay far below the threshold, the case score-bound pruning is for."""
-    c = small_case(seed, dtype, T, S, topk, windows="causal")
+    c = small_case(seed, dtype, T, S, topk, windows="causal", heads=heads)
     sc = c.kv_scales.clone()
     blk = torch.arange(S) // 128
     sc[blk % hot_every != 0] *= cold
     w = c.weights.abs()
     w[:, ::8] = -w[:, ::8]
-    return SelectInputs(f"blocks{seed}_{dtype}", c.q, c.kv, sc, w.contiguous(), c.ks, c.ke, topk)
+    name = f"blocks{seed}_{dtype}" + ("" if heads == 32 else f"_{heads}h")
+    return SelectInputs(name, c.q, c.kv, sc, w.contiguous(), c.ks, c.ke, topk)

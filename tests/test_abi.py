@@ -208,6 +208,27 @@ def test_score_dense_host_validation(lib):
     assert r == -1  # ld < S: a window could run past its row
 
 
+def test_head_count_validation(lib):
+    """ftk_config.heads: 0 or 32 (default) or 64; anything else is refused
+    by ftk_select, by the workspace query (0) and by ftk_score_dense_heads."""
+    P = ctypes.c_void_p
+    for h in (0, 32, 64):
+        assert lib.ftk_select_workspace_size(100, 1000, 16, ctypes.byref(ftk.FtkConfig(heads=h))) > 0
+    for h in (-1, 1, 16, 48, 128):
+        cfg = ftk.FtkConfig(heads=h)
+        assert lib.ftk_select_workspace_size(100, 1000, 16, ctypes.byref(cfg)) == 0
+        assert lib.ftk_select(1, P(A), P(A), None, P(A), P(A), P(A), 100, 1000, 16, P(A), None, P(A),
+                              1 << 30, ctypes.byref(cfg), None) == -1
+        assert lib.ftk_score_dense_heads(1, h, P(A), P(A), None, P(A), P(A), P(A), 16, 1000, None, 16,
+                                         P(A), 1000, P(A), 256, None) == -1
+        assert lib.ftk_block_bound_heads(1, h, P(A), P(A), None, P(A), 4, 1000, P(A), 8, P(A), 1 << 20,
+                                         None) == -1
+    # 64 heads: twice the row tiles (4 or 8 queries per tile instead of 8 or 16)
+    n32 = lib.ftk_select_workspace_size(4096, 131072, 2048, None)
+    n64 = lib.ftk_select_workspace_size(4096, 131072, 2048, ctypes.byref(ftk.FtkConfig(heads=64)))
+    assert n64 > 0 and n32 > 0
+
+
 def test_stage_events_host_validation(lib):
     """The hook takes 7 or 8 non-NULL handles (copied), and n = 0 or NULL
     switches it off; nothing is recorded until an ftk_select call."""

@@ -28,7 +28,7 @@ def gpu_inputs(c: wl.SelectInputs):
 
 
 def run_select(g: wl.SelectInputs, config=None):
-    ws = torch.empty(ftk.select_workspace_size(g.T, g.S, g.topk, config), dtype=torch.uint8,
+    ws = torch.empty(ftk.select_workspace_size(g.T, g.S, g.topk, config, g.q.shape[1]), dtype=torch.uint8,
                      device="cuda")
     idx, val = ftk.select(g.q, g.kv, g.weights, g.ks, g.ke, g.kv_scales, g.topk,
                           return_scores=True, workspace=ws, config=config)
@@ -85,6 +85,10 @@ SMALL = [
     # sample and scan work items, candidates merged across items)
     dict(seed=11, dtype="fp8", T=3, S=100000, topk=2048, windows="causal"),
     dict(seed=12, dtype="bf16", T=5, S=40000, topk=512, windows="random"),
+    # edge sizes: one query, one key; topk above every window; one query over a long window
+    dict(seed=21, dtype="fp8", T=1, S=1, topk=1, windows="causal"),
+    dict(seed=22, dtype="bf16", T=2, S=300, topk=4096, windows="random"),
+    dict(seed=23, dtype="fp8", T=1, S=70000, topk=4096, windows="causal"),
 ]
 
 
