@@ -695,8 +695,6 @@ def run_ours(args):
     print(json.dumps(out), flush=True)
     if world > 1:
         dist.destroy_process_group()  # rank 0 too (its collectives all ended above)
-    if world > 1:
-        dist.destroy_process_group()
 
 
 def main():
