@@ -355,12 +355,16 @@ ftk_status ftk_windows_from_cu_seqlens(const int32_t *cu_q,
  * the recovery batch is the largest that fits the array.
  * Returns FTK_ERR_WORKSPACE when the problem needs more scratch than
  * FTK_NOALLOC_SCRATCH_BYTES (smaller T, S or topk fit).
- * The first call on each device looks up the array's device address
- * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * The array's device address is looked up (cudaGetSymbolAddress) on the
+ * first call in each CUDA context of a device and again whenever the
+ * context changes (say after cudaDeviceReset); make the first call on a
+ * device before any stream capture.  Argument errors are those of
+ * ftk_select and are reported first.
  * All calls share the one array and leave their state in it (each call
  * clears what it needs): calls that overlap on the same GPU, for example
- * on two streams, race on it, so serialise them.  There is no
- * ftk_read_info for this entry point.
+ * on two streams, race on it, so serialise them.  The per-call information
+ * (status bits such as FTK_STATUS_BAD_WINDOW or FTK_STATUS_NAN included)
+ * is read with ftk_noalloc_read_info.
  */
 #define FTK_NOALLOC_SCRATCH_BYTES (64u << 20)
 ftk_status ftk_select_noalloc(ftk_dtype dtype, const void *q, const void *kv,
@@ -369,6 +373,13 @@ ftk_status ftk_select_noalloc(ftk_dtype dtype, const void *q, const void *kv,
                               int64_t S, int topk, int32_t *out_idx,
                               float *out_val, const ftk_config *config,
                               void *stream);
+
+/* The ftk_info of the last ftk_select_noalloc call on the current device,
+ * copied from the start of the fixed array after the stream completes
+ * (synchronises the stream, like ftk_read_info); it allocates nothing.
+ * Valid only when no other ftk_select_noalloc call on this device ran in
+ * between. */
+ftk_status ftk_noalloc_read_info(ftk_info *out, void *stream);
 
 /* Diagnostic timing hook.  While set, every ftk_select call made from the
  * calling host thread records events[i] (cudaEvent_t values created by the

@@ -47,6 +47,13 @@ struct Carver {
     }
 };
 
+// The host-visible argument checks of ftk_select (dtype, head count and
+// reserved config fields, pointers, sizes, topk range, alignment), in the
+// order ftk_select reports them; FTK_OK if the call may proceed.
+ftk_status check_select_call(int dtype, const void *q, const void *kv, const float *w, const int32_t *ks,
+                             const int32_t *ke, int64_t T, int64_t S, int topk, const int32_t *out_idx,
+                             const ftk_config *config);
+
 struct RowsArgs;
 struct BoxArgs;
 struct BoundArgs;

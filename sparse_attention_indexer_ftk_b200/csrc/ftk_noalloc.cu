@@ -10,7 +10,10 @@
 // g_noalloc_scratch, a file-scope __device__ array of
 // FTK_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds until
 // the process exits.
+#include <cudaTypedefs.h>
+
 #include <atomic>
+#include <mutex>
 
 #include "ftk_host.h"
 
@@ -18,21 +21,56 @@ namespace ftk {
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[FTK_NOALLOC_SCRATCH_BYTES];
 
-// Device address of g_noalloc_scratch per device.  In host code the array's
-// name is only a host-side stand-in, so the address comes from
-// cudaGetSymbolAddress, once per device, with that device current.
+// cuCtxGetCurrent, through the runtime's driver entry point (the library
+// does not link the driver library itself).
+static PFN_cuCtxGetCurrent_v4000 ctx_get_current_fn()
+{
+    static std::atomic<PFN_cuCtxGetCurrent_v4000> cached{nullptr};
+    PFN_cuCtxGetCurrent_v4000 fn = cached.load(std::memory_order_acquire);
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess) {
+            fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+            cached.store(fn, std::memory_order_release);
+        }
+    }
+    return fn;
+}
+
+// Device address of g_noalloc_scratch in the current context.  In host code
+// the array's name is only a host-side stand-in, so the address comes from
+// cudaGetSymbolAddress, with the device current.  It is cached per device
+// together with the context it was taken in: a context that was destroyed
+// and created again (cudaDeviceReset, a released and re-retained primary
+// context) reloads the module at another address, and the next call looks
+// the address up again instead of using a stale one.
 static void *scratch_on_device(int dev)
 {
-    static std::atomic<void *> addr[64];  // host threads may race here
+    struct Entry {
+        CUcontext ctx;
+        void *addr;
+    };
+    static Entry cache[64] = {};
+    static std::mutex mu;  // host threads may race here
     if (dev < 0 || dev >= 64) return nullptr;
-    void *p = addr[dev].load(std::memory_order_acquire);
-    if (!p) {
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
-            (void)cudaGetLastError();
-            return nullptr;
-        }
-        addr[dev].store(p, std::memory_order_release);
+    PFN_cuCtxGetCurrent_v4000 get = ctx_get_current_fn();
+    if (!get) return nullptr;
+    CUcontext ctx = nullptr;
+    if (get(&ctx) != CUDA_SUCCESS) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (ctx && cache[dev].ctx == ctx && cache[dev].addr) return cache[dev].addr;
+    // (Also makes the device's primary context current on this thread if no
+    // context was.)
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return nullptr;
     }
+    if (get(&ctx) != CUDA_SUCCESS || !ctx) return nullptr;
+    cache[dev].ctx = ctx;
+    cache[dev].addr = p;
     return p;
 }
 
@@ -46,11 +84,9 @@ extern "C" ftk_status ftk_select_noalloc(ftk_dtype dtype, const void *q, const v
                                          int64_t S, int topk, int32_t *out_idx, float *out_val,
                                          const ftk_config *config, void *stream)
 {
-    if (T < 1 || S < 1 || topk < 1 || topk > FTK_MAX_TOPK) {
-        // Same argument errors as ftk_select (it reports them first).
-        return ftk_select(dtype, q, kv, kv_scales, weights, ks, ke, T, S, topk, out_idx, out_val,
-                          nullptr, 0, config, stream);
-    }
+    // ftk_select's argument errors come first, as ftk_select reports them.
+    ftk_status st = check_select_call(dtype, q, kv, weights, ks, ke, T, S, topk, out_idx, config);
+    if (st != FTK_OK) return st;
     // With the default recovery batch the scratch would be sized for up to
     // 512 MB of recovery rows; within the fixed array, use the largest batch
     // that fits (at least one 16-row tile), unless the caller chose one.
@@ -75,4 +111,16 @@ extern "C" ftk_status ftk_select_noalloc(ftk_dtype dtype, const void *q, const v
     if (!scratch) return FTK_ERR_CUDA;
     return ftk_select(dtype, q, kv, kv_scales, weights, ks, ke, T, S, topk, out_idx, out_val,
                       scratch, FTK_NOALLOC_SCRATCH_BYTES, &cfg, stream);
+}
+
+// The ftk_info of the last ftk_select_noalloc call on the current device:
+// ftk_select keeps it at the start of its scratch.
+extern "C" ftk_status ftk_noalloc_read_info(ftk_info *out, void *stream)
+{
+    if (!out) return FTK_ERR_INVALID_ARG;
+    cudaStream_t st = as_stream(stream);
+    cudaError_t e = cudaMemcpyFromSymbolAsync(out, g_noalloc_scratch, sizeof(ftk_info), 0,
+                                              cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    return cuda_status(e);
 }

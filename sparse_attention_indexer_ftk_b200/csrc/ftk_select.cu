@@ -747,6 +747,17 @@ static ftk_status check_select_args(int dtype, int heads, const void *q, const v
     return FTK_OK;
 }
 
+ftk_status check_select_call(int dtype, const void *q, const void *kv, const float *w, const int32_t *ks,
+                             const int32_t *ke, int64_t T, int64_t S, int topk, const int32_t *out_idx,
+                             const ftk_config *config)
+{
+    if (config && (config->reserved[0] || config->reserved[1] ||
+                   (config->heads != 0 && config->heads != 32 && config->heads != 64)))
+        return FTK_ERR_INVALID_ARG;
+    const int heads = config && config->heads == 64 ? 64 : 32;
+    return check_select_args(dtype, heads, q, kv, w, ks, ke, T, S, topk, out_idx);
+}
+
 // The caller's event handles, copied (the caller's array need not outlive
 // ftk_set_stage_events); g_stage_count == 0 means the hook is off.
 thread_local void *g_stage_events[8];
@@ -805,12 +816,9 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
                                  int32_t *out_idx, float *out_val, void *workspace,
                                  size_t workspace_bytes, const ftk_config *config, void *stream)
 {
-    if (config && (config->reserved[0] || config->reserved[1] ||
-                   (config->heads != 0 && config->heads != 32 && config->heads != 64)))
-        return FTK_ERR_INVALID_ARG;
-    const int heads = config && config->heads == 64 ? 64 : 32;
-    ftk_status st = check_select_args(dtype, heads, q, kv, weights, ks, ke, T, S, topk, out_idx);
+    ftk_status st = check_select_call(dtype, q, kv, weights, ks, ke, T, S, topk, out_idx, config);
     if (st != FTK_OK) return st;
+    const int heads = config && config->heads == 64 ? 64 : 32;
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return FTK_ERR_WORKSPACE;
     const SelectCfg c = resolve_cfg(T, S, topk, config);
     if (c.cap < topk) return FTK_ERR_INVALID_ARG;

@@ -43,6 +43,7 @@ EXPORTS = (
     "ftk_set_stage_events", "ftk_status_string", "ftk_version", "ftk_select_noalloc",
     "ftk_block_bound", "ftk_block_bound_workspace_size", "ftk_topk_rows_end", "ftk_topk_rows_sorted",
     "ftk_rows_options_init", "ftk_topk_rows_ex", "ftk_score_dense_heads", "ftk_block_bound_heads",
+    "ftk_noalloc_read_info",
 )
 
 
@@ -104,6 +105,8 @@ def load_library(path: str = LIB_PATH):
     L.ftk_windows_from_cu_seqlens.argtypes = [P, P, I64, I64, P, P, P]
     L.ftk_select_noalloc.restype = I32
     L.ftk_select_noalloc.argtypes = [I32, P, P, P, P, P, P, I64, I64, I32, P, P, P, P]
+    L.ftk_noalloc_read_info.restype = I32
+    L.ftk_noalloc_read_info.argtypes = [P, P]
     L.ftk_set_stage_events.restype = I32
     L.ftk_set_stage_events.argtypes = [P, I32]
     L.ftk_topk_rows_sorted.restype = I32
