@@ -21,7 +21,10 @@ trivial read-reduce over the same bytes, and the CPU oracle's rate.
 
 Multi-GPU (launched with torch.distributed.run): every rank runs its own
 independent batch of the same shape (weak scaling; no data-path collective);
-the step time is the max over ranks.
+the step time is the max over ranks.  Beside it, one batch split into
+contiguous row blocks across the ranks (strong scaling), its blocks gathered
+on rank 0 after the timed region and checked bit for bit against the
+single-GPU result.
 
 Prints one JSON line (rank 0).
 """
@@ -384,16 +387,23 @@ def bench_decode(c, dev, rows: int = 64, reps: int = 50):
     for _ in range(3):
         step()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    stage_evs = [ftk.stage_events() for _ in range(reps)]
     for i in range(reps):
         flush.zero_()
-        ev[i][0].record()
-        step()
-        ev[i][1].record()
+        with stage_evs[i]:
+            ev[i][0].record()
+            step()
+            ev[i][1].record()
     torch.cuda.synchronize()
     ms = sum(a.elapsed_time(b) for a, b in ev) / reps
+    stages = [s.times_ms() for s in stage_evs]
+    info = ftk.read_info(ws)
     pairs = d.pairs()
     return {"workload": d.name, "T": d.T, "S": d.S, "topk": d.topk, "ms_per_call": ms,
-            "queries_per_s": d.T / (ms * 1e-3), "dense_eq_tflops": 2.0 * 32 * 128 * pairs / (ms * 1e-3) / 1e12}
+            "queries_per_s": d.T / (ms * 1e-3), "dense_eq_tflops": 2.0 * 32 * 128 * pairs / (ms * 1e-3) / 1e12,
+            "stage_ms": {name: sum(s[name] for s in stages) / reps for name in stages[0]},
+            "kernel_launches": int(info["kernel_launches"]), "prune_enabled": info["prune_enabled"],
+            "rows_recovered": info["rows_overflow"] + info["rows_underflow"]}
 
 
 def fp8_gemm_peak(dev, n: int = 8192, reps: int = 10):
@@ -520,16 +530,62 @@ def e2e_pipelined(ftk, host: dict, ws, T: int, k: int, E: int, dev, ref_idx, ref
     return e0.elapsed_time(e1) / E, ok
 
 
-def run_ours(args):
+def bench_sharded(c, g, dev, pg, world: int, rank: int, ref_idx, ref_val, reps: int = 20):
+    """One batch split across the ranks: rank r runs ftk_select on its
+    contiguous block of query rows (shard.row_shard; kv replicated), the
+    step time is the max over ranks, and the blocks gathered on rank 0
+    (NCCL, outside the timed region) must equal the single-GPU result of the
+    whole batch bit for bit.  Every rank takes the same collective steps."""
     import torch
+    from sparse_attention_indexer_ftk_b200 import ftk, shard
+    from sparse_attention_indexer_ftk_b200 import workloads as wl
+
+    lo, hi = shard.row_shard(c.T, world, rank)
+    d = wl.SelectInputs(c.name + f"[{lo}:{hi}]", g.q[lo:hi].contiguous(), g.kv, g.kv_scales,
+                        g.weights[lo:hi].contiguous(), g.ks[lo:hi].contiguous(), g.ke[lo:hi].contiguous(),
+                        c.topk)
+    ws = torch.empty(ftk.select_workspace_size(d.T, d.S, d.topk), dtype=torch.uint8, device=dev)
+    oi = torch.empty((d.T, d.topk), dtype=torch.int32, device=dev)
+    ov = torch.empty((d.T, d.topk), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    step = lambda: ftk.select(d.q, d.kv, d.weights, d.ks, d.ke, d.kv_scales, d.topk, return_scores=True,
+                              workspace=ws, out_idx=oi, out_val=ov)
+    for _ in range(3):
+        step()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    pg.barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(reps):
+        flush.zero_()
+        ev[i][0].record()
+        step()
+        ev[i][1].record()
+    torch.cuda.synchronize(dev)
+    pg.barrier()
+    ms = shard.max_over_ranks(sum(a.elapsed_time(b) for a, b in ev) / reps, dev)
+    got_idx = shard.gather_rows(oi, c.T, dev)
+    got_val = shard.gather_rows(ov, c.T, dev)
+    out = {"T": c.T, "rows_per_rank": hi - lo, "ms_per_step": ms, "value": c.T / (ms * 1e-3),
+           "unit": "queries/s", "scaling": "strong",
+           "gather": "out_idx / out_val gathered on rank 0 (NCCL) after the timed region"}
+    if rank == 0:
+        out["matches_single_gpu"] = bool(torch.equal(got_idx, ref_idx)
+                                         and torch.equal(got_val.view(torch.int32), ref_val.view(torch.int32)))
+    return out
+
+
+def run_ours(args):
+    from sparse_attention_indexer_ftk_b200 import shard
 
     world, rank, local = dist_env()
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+    # Set up once, destroyed exactly once on the way out (errors included).
+    with shard.ProcessGroup(world, local, "nccl") as pg:
+        _run_ours(args, pg, world, rank, local)
+
+
+def _run_ours(args, pg, world, rank, local):
+    import torch
+
     dev = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(dev)
 
@@ -559,10 +615,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     info = ftk.read_info(ws)
 
-    def barrier():
-        if world > 1:
-            import torch.distributed as dist
-            dist.barrier()
+    barrier = pg.barrier
 
     K = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
@@ -632,9 +685,12 @@ def run_ours(args):
     else:
         e2e_ms, e2e_mode = serial_ms, "serial" + (f" (pipelined run rejected: {pipe_note})" if pipe_note else "")
 
+    # One batch split over the ranks (strong scaling), checked against the
+    # single-GPU result of the whole batch; every rank takes part.
+    sharded = None
+    if world > 1:
+        sharded = bench_sharded(c, g, dev, pg, world, rank, ref_idx, ref_val)
     if rank != 0:
-        if world > 1:
-            dist.destroy_process_group()
         return
 
     peaks, peak_src = measured_peaks()
@@ -692,9 +748,9 @@ def run_ours(args):
                            bench_rows("rows_bf16_1024", dev, reps=16)]
     if world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(c, args.cpu_seconds)
+    if sharded is not None:
+        out["sharded_one_batch"] = sharded
     print(json.dumps(out), flush=True)
-    if world > 1:
-        dist.destroy_process_group()  # rank 0 too (its collectives all ended above)
 
 
 def main():

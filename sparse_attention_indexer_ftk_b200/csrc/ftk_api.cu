@@ -1,9 +1,65 @@
 // ftk_api.cu -- small C-ABI entry points: status strings, version, packed
 // causal windows.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <mutex>
+
 #include "ftk_device.cuh"
 #include "ftk_host.h"
 
 namespace ftk {
+
+void *current_context()
+{
+    // cuCtxGetCurrent through the runtime's driver entry point (the library
+    // does not link the driver library itself).
+    static std::atomic<PFN_cuCtxGetCurrent_v4000> cached{nullptr};
+    PFN_cuCtxGetCurrent_v4000 fn = cached.load(std::memory_order_acquire);
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+        cached.store(fn, std::memory_order_release);
+    }
+    CUcontext ctx = nullptr;
+    return fn(&ctx) == CUDA_SUCCESS ? static_cast<void *>(ctx) : nullptr;
+}
+
+ftk_status ensure_smem_limit(const void *func, int bytes)
+{
+    struct Entry {
+        const void *func;
+        void *ctx;
+        int bytes;
+    };
+    static Entry table[256];
+    static int used = 0;
+    static std::mutex mu;
+    void *ctx = current_context();
+    if (ctx) {
+        std::lock_guard<std::mutex> lock(mu);
+        for (int i = 0; i < used; ++i)
+            if (table[i].func == func && table[i].ctx == ctx && table[i].bytes >= bytes) return FTK_OK;
+    }
+    const cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return cuda_status(e);
+    ctx = current_context();  // (the call above may have made the context current)
+    if (ctx) {
+        std::lock_guard<std::mutex> lock(mu);
+        for (int i = 0; i < used; ++i) {
+            if (table[i].func == func && table[i].ctx == ctx) {
+                if (table[i].bytes < bytes) table[i].bytes = bytes;
+                return FTK_OK;
+            }
+        }
+        if (used < 256) table[used++] = Entry{func, ctx, bytes};
+    }
+    return FTK_OK;
+}
 
 // One thread per query row: finds its sequence by binary search over cu_q
 // and writes the causal window of a query that is among its sequence's last

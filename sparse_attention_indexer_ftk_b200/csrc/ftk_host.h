@@ -47,6 +47,15 @@ struct Carver {
     }
 };
 
+// The calling thread's current CUDA context (a driver handle), or NULL.
+void *current_context();
+
+// Raises the dynamic shared-memory limit of kernel `func` to at least
+// `bytes`, once per (kernel, context): later calls find it in a small table
+// instead of calling cudaFuncSetAttribute again.  A context that is
+// destroyed and created again is a new context, so the limit is set anew.
+ftk_status ensure_smem_limit(const void *func, int bytes);
+
 // The host-visible argument checks of ftk_select (dtype, head count and
 // reserved config fields, pointers, sizes, topk range, alignment), in the
 // order ftk_select reports them; FTK_OK if the call may proceed.

@@ -10,8 +10,6 @@
 // g_noalloc_scratch, a file-scope __device__ array of
 // FTK_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds until
 // the process exits.
-#include <cudaTypedefs.h>
-
 #include <atomic>
 #include <mutex>
 
@@ -20,24 +18,6 @@
 namespace ftk {
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[FTK_NOALLOC_SCRATCH_BYTES];
-
-// cuCtxGetCurrent, through the runtime's driver entry point (the library
-// does not link the driver library itself).
-static PFN_cuCtxGetCurrent_v4000 ctx_get_current_fn()
-{
-    static std::atomic<PFN_cuCtxGetCurrent_v4000> cached{nullptr};
-    PFN_cuCtxGetCurrent_v4000 fn = cached.load(std::memory_order_acquire);
-    if (!fn) {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess) {
-            fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
-            cached.store(fn, std::memory_order_release);
-        }
-    }
-    return fn;
-}
 
 // Device address of g_noalloc_scratch in the current context.  In host code
 // the array's name is only a host-side stand-in, so the address comes from
@@ -49,16 +29,13 @@ static PFN_cuCtxGetCurrent_v4000 ctx_get_current_fn()
 static void *scratch_on_device(int dev)
 {
     struct Entry {
-        CUcontext ctx;
+        void *ctx;
         void *addr;
     };
     static Entry cache[64] = {};
     static std::mutex mu;  // host threads may race here
     if (dev < 0 || dev >= 64) return nullptr;
-    PFN_cuCtxGetCurrent_v4000 get = ctx_get_current_fn();
-    if (!get) return nullptr;
-    CUcontext ctx = nullptr;
-    if (get(&ctx) != CUDA_SUCCESS) return nullptr;
+    void *ctx = current_context();
     std::lock_guard<std::mutex> lock(mu);
     if (ctx && cache[dev].ctx == ctx && cache[dev].addr) return cache[dev].addr;
     // (Also makes the device's primary context current on this thread if no
@@ -68,7 +45,8 @@ static void *scratch_on_device(int dev)
         (void)cudaGetLastError();
         return nullptr;
     }
-    if (get(&ctx) != CUDA_SUCCESS || !ctx) return nullptr;
+    ctx = current_context();
+    if (!ctx) return nullptr;
     cache[dev].ctx = ctx;
     cache[dev].addr = p;
     return p;

@@ -66,9 +66,8 @@ static ftk_status launch_rows_dt(const RowsArgs &a, int cluster, bool idx64, cud
     const size_t smem = sizeof(RowsSmem);
     auto kern = idx64 ? (loop ? rows_topk_kernel<DT, true, int64_t> : rows_topk_kernel<DT, false, int64_t>)
                       : (loop ? rows_topk_kernel<DT, true, int32_t> : rows_topk_kernel<DT, false, int32_t>);
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return cuda_status(e);
+    const ftk_status e = ensure_smem_limit(reinterpret_cast<const void *>(kern), static_cast<int>(smem));
+    if (e != FTK_OK) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(nclusters * cluster), 1, 1);
     cfg.blockDim = dim3(kRowsThreads, 1, 1);

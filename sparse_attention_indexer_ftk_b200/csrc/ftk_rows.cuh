@@ -2,26 +2,33 @@
 // "Supported Cases" and "Usage"; also the selection step of dense recovery).
 //
 // One thread-block cluster per row; CTA c of the cluster owns a contiguous
-// chunk of the row, and each of its warps a contiguous segment of the chunk.
-// The row is streamed from HBM once:
-//   1. a spread sample of the chunk (1024 values) gives a threshold F with no
-//      atomics: the minimum over groups of the group maxima, the group size
-//      chosen so that about >= 2 * topk * chunk / row elements lie above F;
-//   2. the stream (cp.async into a 4-stage shared-memory ring) checks each
-//      16-byte vector with a packed max against F and, only for the rare
-//      vectors that reach it, writes the elements >= F, in column order,
-//      into the warp's candidate list in shared memory;
-//   3. the cluster finds the exact k-th largest candidate key u*: every CTA
-//      gathers all candidate keys of the cluster through distributed shared
-//      memory and radix-selects them locally (or, with very many
-//      candidates, sums per-CTA histograms across the cluster).  If every
-//      CTA kept all its elements >= u* (u* >= each F) and no candidate list
-//      overflowed, u* is the row's k-th largest value; otherwise an exact
-//      multi-pass radix select re-reads the row (L2);
-//   4. ties at u* go to the smallest columns (CTA order, then segment order)
-//      and an ordered compaction writes the selected columns in ascending
-//      order.
-// No sort, no global scratch.
+// chunk of the row and each of its 8 warps a contiguous segment of the
+// chunk.  The row is read from HBM once, in the common case:
+//   1. stream: every warp streams its segment through its own ring of
+//      shared-memory stages filled by bulk copies (cp.async.bulk, no
+//      multicast; lane 0 issues them, an mbarrier per stage), so about 8 KB
+//      per warp are in flight without any thread issuing loads;
+//   2. threshold F, while the first stages are in flight: a spread sample of
+//      the chunk (one 16-byte vector per thread) and F = the smallest sampled
+//      key of the 11-bit bin that holds the r-th largest sample, r chosen so
+//      that the whole row very likely keeps >= topk elements >= F;
+//   3. filter: each vector is tested against F with one packed compare; the
+//      rare elements >= F go, in column order, to the warp's candidate list
+//      in shared memory.  Elements equal to F that find the list full are
+//      only counted (heavy ties);
+//   4. exact k-th key u*: every CTA gathers all candidate keys of the
+//      cluster through distributed shared memory and radix-selects them
+//      locally (11-bit digits), counting the uncounted ties at F as well;
+//      u* is the row's k-th largest key if every CTA kept every element
+//      >= u* (u* >= every F, no list overflowed);
+//   5. output: the counts of each list (> u*, == u*) give every warp its
+//      output slots; ties at u* go to the smallest columns (CTA order, then
+//      warp order, then list order), written in ascending column order.
+// Rows where step 4's conditions fail (adversarial or structured rows, very
+// many candidates) take an exact fallback: multi-pass radix select over the
+// chunk (8-bit digits, histograms summed over the cluster), a counting pass
+// and an ordered writing pass, each streaming the chunk through the same
+// rings.  No sort, no global scratch.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -32,12 +39,16 @@ namespace ftk {
 
 namespace cg = cooperative_groups;
 
-constexpr int kRowsThreads = 512;
+constexpr int kRowsThreads = 256;
 constexpr int kRowsWarps = kRowsThreads / 32;
 constexpr int kRowsMaxCluster = 8;
-constexpr int kRowsCapWarp = 512;    // candidates per warp
-constexpr int kRowsStages = 4;       // cp.async ring stages (one 16-byte vector per thread each)
-constexpr int kRowsGather = kRowsStages * kRowsThreads * 4;  // keys gathered into the (free) ring
+constexpr int kRowsLists = kRowsMaxCluster * kRowsWarps;  // candidate lists of a cluster
+constexpr int kRowsCapWarp = 512;      // candidates per warp list
+constexpr int kRowsStages = 4;         // ring stages per warp
+constexpr int kRowsStageVecs = 128;    // 16-byte vectors per stage (2 KB)
+constexpr int kRowsGather = kRowsWarps * kRowsStages * kRowsStageVecs * 4;  // keys that fit the rings
+constexpr int kRowsBins = 2048;        // 11-bit digits
+constexpr int kRowsKeepAll = 4096;     // chunks of at most this many elements keep all of them
 constexpr int64_t kRowsMaxCols = int64_t(1) << 30;
 
 struct RowsArgs {
@@ -65,25 +76,27 @@ struct RowsArgs {
 static_assert(sizeof(RowsArgs) <= 128, "RowsArgs grew past 128 bytes");
 
 struct RowsSmem {
-    uint32_t cand_bits[kRowsWarps * kRowsCapWarp];  // raw value bits
-    int32_t cand_col[kRowsWarps * kRowsCapWarp];    // column within the chunk
-    uint4 ring[kRowsStages][kRowsThreads];           // stream staging; later the gathered keys
-    uint32_t wmin[kRowsWarps];
-    uint32_t hist[256];
-    uint32_t tot[256];
-    uint32_t warp_cnt[kRowsWarps];
-    uint32_t warp_gt[kRowsWarps];
-    uint32_t warp_eq[kRowsWarps];
-    uint32_t sel_bin, sel_above;
-    uint32_t r_gt[kRowsMaxCluster], r_eq[kRowsMaxCluster];  // per-CTA counts, this CTA's view
-    // published to the cluster
-    uint32_t cta_cnt, cta_fkey, cta_over, cta_gt, cta_eq;
+    uint4 ring[kRowsWarps][kRowsStages][kRowsStageVecs];  // stream stages; later the gathered keys
+    uint32_t cand_bits[kRowsWarps][kRowsCapWarp];         // raw value bits
+    int32_t cand_col[kRowsWarps][kRowsCapWarp];           // column within the chunk
+    uint32_t hist[kRowsBins];
+    uint64_t full[kRowsWarps][kRowsStages];               // one mbarrier per ring stage
+    // this CTA's lists, read by the other CTAs of the cluster
+    uint32_t w_cnt[kRowsWarps];    // stored entries
+    uint32_t w_lost[kRowsWarps];   // entries equal to F past the end of a full list
+    uint32_t cta_fkey, cta_over, cta_gt, cta_eq;
+    // every list of the cluster in column order (index rank * kRowsWarps + warp)
+    uint32_t l_off[kRowsLists + 1], l_cnt[kRowsLists], l_lost[kRowsLists], l_fkey[kRowsLists];
+    uint32_t l_gt[kRowsLists], l_eq[kRowsLists], l_take[kRowsLists], l_selb[kRowsLists];
+    uint32_t wsum[kRowsWarps];
+    uint32_t red[2 * kRowsWarps];
+    uint32_t sel_bin, sel_above, fmin, short_eq;
+    uint32_t g_total, g_lost, g_fmax, g_over;
     uint32_t nan_seen, overflow;
 };
 
 template <int DT>
 struct RowsTraits;
-
 
 template <>
 struct RowsTraits<FTK_BF16> {
@@ -180,71 +193,359 @@ __device__ __forceinline__ void hist_add(uint32_t *hist, uint32_t bin, bool acti
     }
 }
 
-__device__ __forceinline__ void cp_async16(void *dst, const void *src, bool pred)
+__device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v)
 {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
-                 "r"(pred ? 16 : 0)
-                 : "memory");
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t t = __shfl_up_sync(0xFFFFFFFFu, v, o);
+        if (lane >= o) v += t;
+    }
+    return v;
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-// Finds the bin b holding the k-th largest element of tot[0..256):
-// sum(tot[b+1..]) < k <= sum(tot[b..]); writes sm.sel_bin / sm.sel_above.
-// Block-wide.
-__device__ __forceinline__ void find_kth_bin256(RowsSmem &sm, uint32_t k)
+// Finds the bin b of h[0 .. NB) holding the r-th largest counted element:
+// sum(h[b+1 ..]) < r <= sum(h[b ..]).  Sets sm.sel_bin (0xFFFFFFFF if the
+// counts sum to less than r) and sm.sel_above = sum(h[b+1 ..]).  Block-wide
+// (two barriers); h must not change during the call.
+template <int NB>
+__device__ __forceinline__ bool find_bin_top(RowsSmem &sm, const uint32_t *h, uint32_t r)
 {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (warp == 0) {
-        uint32_t c[8], sum = 0;
+    constexpr int B = NB / kRowsThreads;
+    static_assert(B >= 1 && B * kRowsThreads == NB, "bins per thread");
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint32_t c[B], sum = 0;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            c[i] = sm.tot[255 - 8 * lane - i];
-            sum += c[i];
-        }
-        uint32_t inc = sum;
+    for (int i = 0; i < B; ++i) {
+        c[i] = h[NB - 1 - B * tid - i];
+        sum += c[i];
+    }
+    uint32_t inc = warp_incl_scan(sum);
+    if (lane == 31) sm.wsum[warp] = inc;
+    if (tid == 0) sm.sel_bin = 0xFFFFFFFFu;
+    __syncthreads();
+    uint32_t wb = 0;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t u = __shfl_up_sync(0xFFFFFFFFu, inc, o);
-            if (lane >= o) inc += u;
-        }
-        uint32_t above = inc - sum;
-        if (above < k && inc >= k) {
+    for (int w = 0; w < kRowsWarps; ++w) wb += w < warp ? sm.wsum[w] : 0u;
+    inc += wb;
+    uint32_t ab = inc - sum;
+    if (ab < r && inc >= r) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                if (above + c[i] >= k) {
-                    sm.sel_bin = 255 - 8 * lane - i;
-                    sm.sel_above = above;
-                    break;
-                }
-                above += c[i];
+        for (int i = 0; i < B; ++i) {
+            if (ab + c[i] >= r) {
+                sm.sel_bin = static_cast<uint32_t>(NB - 1 - B * tid - i);
+                sm.sel_above = ab;
+                break;
             }
+            ab += c[i];
         }
     }
     __syncthreads();
+    return sm.sel_bin != 0xFFFFFFFFu;
 }
 
-// Sums hist over the cluster into tot (every CTA computes the same totals).
-__device__ __forceinline__ void cluster_sum256(cg::cluster_group &cluster, RowsSmem &sm)
+// Block-wide sum of one value per thread (two barriers).
+__device__ __forceinline__ uint32_t block_sum(RowsSmem &sm, uint32_t v)
 {
-    const unsigned cs = cluster.num_blocks();
-    for (int b = threadIdx.x; b < 256; b += blockDim.x) {
-        uint32_t s = 0;
-        for (unsigned r = 0; r < cs; ++r) s += cluster.map_shared_rank(sm.hist, r)[b];
-        sm.tot[b] = s;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    v = __reduce_add_sync(0xFFFFFFFFu, v);
+    if (lane == 0) sm.red[warp] = v;
+    __syncthreads();
+    uint32_t s = 0;
+#pragma unroll
+    for (int w = 0; w < kRowsWarps; ++w) s += sm.red[w];
+    __syncthreads();
+    return s;
+}
+
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// Bounded wait for a ring stage (bulk copies from valid memory always
+// land; a wait that outlasts kWaitNs reports FTK_STATUS_TIMEOUT and gives up).
+__device__ __forceinline__ bool stage_wait(uint64_t *bar, uint32_t parity, uint32_t *status)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = global_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 63u) == 0 && global_ns() - t0 > kWaitNs) {
+            set_status(status, FTK_STATUS_TIMEOUT);
+            return false;
+        }
     }
 }
 
 __device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 
-// Top-k of grid row r by the whole cluster.  Returns with every cp.async
-// of this CTA complete and, for rows that used distributed shared memory,
-// with every CTA of the cluster done reading this CTA's shared memory.
+// One warp's stream of the vectors [wv0, wv1) of src through its ring.
+// prologue(): lane 0 issues the first stages.  run(visit): waits for each
+// stage in order, calls visit(x, valid, v) on every lane for each of its
+// vectors (v: index into src; warp-collective), and refills the stage.
+// ph holds the parity each stage's barrier waits for next (warp-uniform);
+// every issued copy is waited for exactly once.
+struct WarpStream {
+    RowsSmem &sm;
+    const uint4 *src;
+    int wv0, nv, nst, warp, lane;
+    uint32_t &ph;
+    uint32_t *status;
+
+    __device__ __forceinline__ void issue(int j) const
+    {
+        const int s = j % kRowsStages;
+        const int cnt = min(kRowsStageVecs, nv - j * kRowsStageVecs);
+        const uint32_t bytes = static_cast<uint32_t>(cnt) * 16u;
+        mbar_arrive_expect_tx(&sm.full[warp][s], bytes);
+        bulk_load(&sm.ring[warp][s][0], src + wv0 + j * kRowsStageVecs, bytes, &sm.full[warp][s]);
+    }
+
+    __device__ __forceinline__ void prologue() const
+    {
+        if (lane == 0) {
+            fence_proxy_async();  // earlier generic accesses of the ring precede the copies
+            for (int j = 0; j < min(kRowsStages, nst); ++j) issue(j);
+        }
+    }
+
+    template <typename Visit>
+    __device__ __forceinline__ bool run(Visit &&visit) const
+    {
+        bool ok = true;
+        int issued = min(kRowsStages, nst);
+        for (int j = 0; j < issued; ++j) {
+            const int s = j % kRowsStages;
+            const bool got = stage_wait(&sm.full[warp][s], (ph >> s) & 1u, status);
+            ph ^= 1u << s;
+            ok = __all_sync(0xFFFFFFFFu, ok && got);
+            if (ok) {
+                const uint4 *buf = sm.ring[warp][s];
+                const int cnt = min(kRowsStageVecs, nv - j * kRowsStageVecs);
+                const int vb = wv0 + j * kRowsStageVecs;
+#pragma unroll
+                for (int it = 0; it < kRowsStageVecs / 32; ++it) {
+                    const int i = it * 32 + lane;
+                    const bool valid = i < cnt;
+                    const uint4 x = valid ? buf[i] : make_uint4(0u, 0u, 0u, 0u);
+                    visit(x, valid, vb + i);
+                }
+            }
+            __syncwarp();
+            if (ok && j + kRowsStages < nst) {
+                if (lane == 0) {
+                    fence_proxy_async();
+                    issue(j + kRowsStages);
+                }
+                ++issued;
+            }
+        }
+        return ok;
+    }
+};
+
+// Per-lane masks of the elements of x that are > u (gt) and == u (eq).
+template <int DT>
+__device__ __forceinline__ void cmp_masks(const uint4 &x, uint32_t u, uint32_t &gt, uint32_t &eq)
+{
+    using Tr = RowsTraits<DT>;
+    gt = 0;
+    eq = 0;
+#pragma unroll
+    for (int j = 0; j < Tr::kVec; ++j) {
+        const uint32_t k = Tr::key(Tr::element(x, j));
+        gt |= (k > u ? 1u : 0u) << j;
+        eq |= (k == u ? 1u : 0u) << j;
+    }
+}
+
+// Exact fallback for the cluster's row: u* by radix select over the chunks
+// (8-bit digits, histograms summed over the cluster), then a counting pass
+// and an ordered writing pass, all streamed through the rings.  Every CTA of
+// the cluster calls it (it holds cluster barriers).  Ends with
+// cluster_arrive() (no more reads of other CTAs' shared memory).
+template <int DT, typename IT>
+__device__ __noinline__ void rows_fallback(const RowsArgs &a, RowsSmem &sm, cg::cluster_group &cluster,
+                                           unsigned cs, unsigned rank, const typename RowsTraits<DT>::elem *row,
+                                           int64_t c0, int n, int64_t base_index, IT *oidx,
+                                           typename RowsTraits<DT>::elem *oval, uint32_t &ph)
+{
+    using Tr = RowsTraits<DT>;
+    using elem = typename Tr::elem;
+    constexpr int VEC = Tr::kVec;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int k = a.k;
+    const int nvec = n / VEC;
+    const int per = (nvec + kRowsWarps - 1) / kRowsWarps;
+    const int wv0 = min(nvec, warp * per), wv1 = min(nvec, wv0 + per);
+    const uint4 *src = reinterpret_cast<const uint4 *>(row + c0);
+    const WarpStream ws{sm, src, wv0, wv1 - wv0, (wv1 - wv0 + kRowsStageVecs - 1) / kRowsStageVecs,
+                        warp, lane, ph, a.status};
+    const bool tail_warp = warp == kRowsWarps - 1;
+    uint32_t *tot = sm.hist + 256;
+
+    // ---- u*: radix select over the row, 8-bit digits ----
+    const int passes = DT == FTK_BF16 ? 2 : 4;
+    uint32_t prefix = 0, mask = 0, krem = static_cast<uint32_t>(k), above = 0;
+    for (int p = 0; p < passes; ++p) {
+        const int shift = 24 - 8 * p;
+        if (tid < 256) sm.hist[tid] = 0;
+        __syncthreads();
+        ws.prologue();
+        ws.run([&](const uint4 &x, bool valid, int) {
+#pragma unroll
+            for (int j = 0; j < VEC; ++j) {
+                const uint32_t u = Tr::key(Tr::element(x, j));
+                hist_add(sm.hist, (u >> shift) & 255u, valid && (u & mask) == prefix);
+            }
+        });
+        if (tail_warp) {
+            for (int e0 = nvec * VEC; e0 < n; e0 += 32) {
+                const int e = e0 + lane;
+                const uint32_t u = e < n ? Tr::key(row[c0 + e]) : 0u;
+                hist_add(sm.hist, (u >> shift) & 255u, e < n && (u & mask) == prefix);
+            }
+        }
+        cluster.sync();
+        if (tid < 256) {
+            uint32_t s = 0;
+            for (unsigned rr = 0; rr < cs; ++rr) s += cluster.map_shared_rank(sm.hist, rr)[tid];
+            tot[tid] = s;
+        }
+        __syncthreads();
+        find_bin_top<256>(sm, tot, krem);
+        const uint32_t b = sm.sel_bin == 0xFFFFFFFFu ? 0u : sm.sel_bin;  // (always found: k < len)
+        if (sm.sel_bin == 0xFFFFFFFFu && tid == 0) set_status(a.status, FTK_STATUS_INTERNAL);
+        prefix |= b << shift;
+        mask |= 255u << shift;
+        krem -= sm.sel_bin == 0xFFFFFFFFu ? 0u : sm.sel_above;
+        above += sm.sel_bin == 0xFFFFFFFFu ? 0u : sm.sel_above;
+        cluster.sync();  // every CTA is done reading my histogram
+    }
+    const uint32_t ustar = prefix;
+    const uint32_t need = static_cast<uint32_t>(k) - above;  // ties at u* to take, >= 1
+
+    // ---- counts of > u* and == u* per warp segment ----
+    uint32_t g = 0, q = 0;
+    ws.prologue();
+    ws.run([&](const uint4 &x, bool valid, int) {
+        uint32_t gt, eq;
+        cmp_masks<DT>(x, ustar, gt, eq);
+        if (valid) {
+            g += __popc(gt);
+            q += __popc(eq);
+        }
+    });
+    if (tail_warp) {
+        for (int e = nvec * VEC + lane; e < n; e += 32) {
+            const uint32_t u = Tr::key(row[c0 + e]);
+            g += u > ustar ? 1u : 0u;
+            q += u == ustar ? 1u : 0u;
+        }
+    }
+    g = __reduce_add_sync(0xFFFFFFFFu, g);
+    q = __reduce_add_sync(0xFFFFFFFFu, q);
+    if (lane == 0) {
+        sm.l_gt[warp] = g;
+        sm.l_eq[warp] = q;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        uint32_t tg = 0, tq = 0;
+        for (int w = 0; w < kRowsWarps; ++w) {
+            const uint32_t a0 = sm.l_gt[w], b0 = sm.l_eq[w];
+            sm.l_gt[w] = tg;  // exclusive prefixes within the CTA
+            sm.l_eq[w] = tq;
+            tg += a0;
+            tq += b0;
+        }
+        sm.cta_gt = tg;
+        sm.cta_eq = tq;
+    }
+    cluster.sync();
+    uint32_t eq_before = 0, sel_before = 0;
+    for (unsigned rr = 0; rr < rank; ++rr) {
+        const RowsSmem *o = cluster.map_shared_rank(&sm, rr);
+        const uint32_t og = o->cta_gt, oq = o->cta_eq;
+        const uint32_t take = eq_before >= need ? 0u : min(oq, need - eq_before);
+        sel_before += og + take;
+        eq_before += oq;
+    }
+    __syncthreads();
+    cluster_arrive();  // no more reads of other CTAs' shared memory
+
+    // ---- ordered writing pass ----
+    const uint32_t my_take = eq_before >= need ? 0u : min(sm.cta_eq, need - eq_before);
+    const uint32_t w_gt = sm.l_gt[warp], w_eq = sm.l_eq[warp];
+    uint32_t pos = sel_before + w_gt + min(w_eq, my_take);  // next output slot of this warp
+    uint32_t eq_rank = w_eq;                                // CTA-local tie rank
+    auto emit = [&](uint32_t gt, uint32_t eq, const uint4 &x, int col0) {
+        // this lane's elements in column order, ranks from warp prefix sums
+        const uint32_t ce = __popc(eq);
+        const uint32_t eb = warp_incl_scan(ce) - ce;
+        uint32_t sel = gt;
+        uint32_t er = eq_rank + eb;
+        uint32_t m = eq;
+        while (m) {
+            const int j = __ffs(m) - 1;
+            m &= m - 1u;
+            if (er < my_take) sel |= 1u << j;
+            ++er;
+        }
+        const uint32_t cnt = __popc(sel);
+        const uint32_t incl = warp_incl_scan(cnt);
+        uint32_t p = pos + incl - cnt;
+        while (sel) {
+            const int j = __ffs(sel) - 1;
+            sel &= sel - 1u;
+            if (p < static_cast<uint32_t>(k)) {
+                oidx[p] = static_cast<IT>(static_cast<int32_t>(base_index + c0 + col0 + j));
+                if (oval) oval[p] = static_cast<elem>(Tr::element(x, j));
+            } else {
+                set_status(a.status, FTK_STATUS_INTERNAL);
+            }
+            ++p;
+        }
+        pos += __shfl_sync(0xFFFFFFFFu, incl, 31);
+        eq_rank += __shfl_sync(0xFFFFFFFFu, eb + ce, 31);
+    };
+    ws.prologue();
+    ws.run([&](const uint4 &x, bool valid, int v) {
+        uint32_t gt = 0, eq = 0;
+        if (valid) cmp_masks<DT>(x, ustar, gt, eq);
+        if (__ballot_sync(0xFFFFFFFFu, (gt | eq) != 0u)) emit(gt, eq, x, v * VEC);
+    });
+    if (tail_warp) {
+        for (int e0 = nvec * VEC; e0 < n; e0 += 32) {
+            const int e = e0 + lane;
+            uint32_t gt = 0, eq = 0, bits = 0;
+            if (e < n) {
+                bits = row[c0 + e];
+                const uint32_t u = Tr::key(bits);
+                gt = u > ustar ? 1u : 0u;
+                eq = u == ustar ? 1u : 0u;
+            }
+            // one element per lane: element 0 of a vector whose .x holds it
+            const uint4 x = make_uint4(bits, 0u, 0u, 0u);
+            if (__ballot_sync(0xFFFFFFFFu, (gt | eq) != 0u)) emit(gt, eq, x, e - 0);
+        }
+    }
+}
+
+// Top-k of grid row r by the whole cluster.  Returns with every bulk copy
+// of this CTA landed and every CTA of the cluster done with this CTA's
+// shared memory.
 template <int DT, typename IT>
 __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, cg::cluster_group &cluster,
-                                              unsigned cs, unsigned rank, int64_t r)
+                                              unsigned cs, unsigned rank, int64_t r, uint32_t &ph)
 {
     using Tr = RowsTraits<DT>;
     using elem = typename Tr::elem;
@@ -289,95 +590,85 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
         return;
     }
 
+    const int nvec = n / VEC;
+    const int per = (nvec + kRowsWarps - 1) / kRowsWarps;
+    const int wv0 = min(nvec, warp * per), wv1 = min(nvec, wv0 + per);
+    const uint4 *src = reinterpret_cast<const uint4 *>(row + c0);
+    const WarpStream ws{sm, src, wv0, wv1 - wv0, (wv1 - wv0 + kRowsStageVecs - 1) / kRowsStageVecs,
+                        warp, lane, ph, a.status};
     if (tid == 0) {
         sm.nan_seen = 0;
         sm.overflow = 0;
+        sm.fmin = 0xFFFFFFFFu;
     }
+    ws.prologue();  // the first stages are in flight while F is found
 
-    // ---- 1. threshold F from a spread sample (no atomics) ----
-    const int nvec = n / VEC;
-    const int per = (nvec + kRowsWarps - 1) / kRowsWarps;
-    const int v0 = min(nvec, warp * per), v1 = min(nvec, v0 + per);
-    const uint4 *src = reinterpret_cast<const uint4 *>(row + c0);
-    constexpr int kSampleThreads = 128;                 // warps 0..3, 8 samples per lane
-    constexpr int kSampleVecs = 8 / VEC;                // vectors per sampling lane
-    const bool sampled = nvec >= kSampleThreads * kSampleVecs;
-    uint32_t lmax = 0;
-    if (sampled && tid < kSampleThreads) {
+    // ---- threshold F from a spread sample of the chunk ----
+    uint32_t fkey = 0u;  // 0: keep every element
+    if (nvec >= kRowsThreads && n > kRowsKeepAll) {
+        const uint4 sx = __ldg(src + static_cast<int64_t>(tid) * nvec / kRowsThreads);
+        // Samples above the row's k-th largest value: about
+        // lam = k * m / len; F is the r-th largest sample with r a few
+        // standard deviations above lam.
+        const float m = static_cast<float>(kRowsThreads * VEC);
+        const float lam = static_cast<float>(k) * m / static_cast<float>(len);
+        const float rf = ceilf(lam + 4.f * sqrtf(lam) + 4.f);
+        if (rf < m) {
+            for (int b = tid; b < kRowsBins; b += kRowsThreads) sm.hist[b] = 0;
+            __syncthreads();
+            uint32_t keys[VEC];
 #pragma unroll
-        for (int q = 0; q < kSampleVecs; ++q) {
-            const int64_t sv = static_cast<int64_t>(tid * kSampleVecs + q) * nvec / (kSampleThreads * kSampleVecs);
-            const uint4 x = __ldg(src + sv);
+            for (int j = 0; j < VEC; ++j) {
+                keys[j] = Tr::key(Tr::element(sx, j));
+                hist_add(sm.hist, keys[j] >> 21, true);
+            }
+            __syncthreads();
+            find_bin_top<kRowsBins>(sm, sm.hist, static_cast<uint32_t>(rf));
+            const uint32_t b = sm.sel_bin;  // found: the counts sum to m > r
+            uint32_t mn = 0xFFFFFFFFu;
 #pragma unroll
-            for (int j = 0; j < VEC; ++j) lmax = max(lmax, Tr::key(Tr::element(x, j)));
+            for (int j = 0; j < VEC; ++j)
+                if ((keys[j] >> 21) == b) mn = min(mn, keys[j]);
+            mn = __reduce_min_sync(0xFFFFFFFFu, mn);
+            if (lane == 0) atomicMin(&sm.fmin, mn);
+            __syncthreads();
+            fkey = sm.fmin == 0xFFFFFFFFu ? 0u : sm.fmin;
         }
     }
-    // Stream prologue: the first ring stages are in flight while F is found.
-    const int nb = (v1 - v0 + 31) / 32;  // 32-vector batches of my warp
-#pragma unroll
-    for (int b = 0; b < kRowsStages; ++b) {
-        const int v = v0 + b * 32 + lane;
-        cp_async16(&sm.ring[b][tid], v < v1 ? src + v : src, b < nb && v < v1);
-        cp_async_commit();
-    }
-    // F = min over groups of the group maxima.  With G samples per group and
-    // M groups, about ln(M / ln 2) / G of the values lie above it; take the
-    // largest group that still leaves >= 2 * k / len of them.
-    const double want = 2.0 * static_cast<double>(k) / static_cast<double>(len);
-    int g = -1;  // log2 of lanes per group (0..7); -1: keep everything
-    for (int gg = 7; gg >= 0; --gg) {
-        const double G = 8.0 * (1 << gg), M = 1024.0 / G;
-        if (log(M / 0.6931471805599453) / G >= want) {
-            g = gg;
-            break;
-        }
-    }
-    if (warp < 4) {
-        uint32_t m = lmax;
-        const int gl = g < 0 ? 0 : (g > 5 ? 5 : g);  // lanes per group inside a warp: 2^gl
-        for (int o = 1; o < (1 << gl); o <<= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-        // min over the groups inside this warp (g < 5), or the warp max (g >= 5)
-        uint32_t w = m;
-        for (int o = (1 << gl); o < 32; o <<= 1) w = min(w, __shfl_xor_sync(0xFFFFFFFFu, w, o));
-        if (lane == 0) sm.wmin[warp] = w;
-    }
-    __syncthreads();
-    uint32_t fkey;
-    if (n == 0) {
-        fkey = 0xFFFFFFFFu;  // no elements, no candidates
-    } else if (!sampled || g < 0) {
-        fkey = 0u;           // keep everything
-    } else if (g <= 5) {
-        fkey = min(min(sm.wmin[0], sm.wmin[1]), min(sm.wmin[2], sm.wmin[3]));
-    } else if (g == 6) {
-        fkey = min(max(sm.wmin[0], sm.wmin[1]), max(sm.wmin[2], sm.wmin[3]));
-    } else {
-        fkey = max(max(sm.wmin[0], sm.wmin[1]), max(sm.wmin[2], sm.wmin[3]));
-    }
-    if (DT == FTK_BF16 && fkey != 0xFFFFFFFFu) fkey &= 0xFFFF0000u;
-    if (tid == 0) sm.cta_fkey = fkey;
     // A strictly positive F allows the packed raw-bits test.
-    const bool fpos = fkey > 0x80000000u && fkey != 0xFFFFFFFFu;
-    const uint32_t fbits = f32_from_key(fkey);  // F as f32 bits
+    const bool fpos = fkey > 0x80000000u;
+    const uint32_t fbits = f32_from_key(fkey);  // F as f32 bits (bf16: its top half)
     const uint32_t fraw = DT == FTK_BF16 ? ((fbits >> 16) | (fbits & 0xFFFF0000u)) : fbits;
 
-    // ---- 2. stream the chunk; keep the elements >= F in column order ----
+    // ---- stream the chunk; keep the elements >= F in column order ----
     {
-        uint32_t *cb = sm.cand_bits + warp * kRowsCapWarp;
-        int32_t *cc = sm.cand_col + warp * kRowsCapWarp;
-        uint32_t wcnt = 0, mag = 0;
-        for (int b = 0; b < nb; ++b) {
-            cp_async_wait<kRowsStages - 1>();  // batch b has landed (my own slot)
-            const int slot = b % kRowsStages;
-            const uint4 x = sm.ring[slot][tid];
-            {
-                const int vn = v0 + (b + kRowsStages) * 32 + lane;
-                cp_async16(&sm.ring[slot][tid], vn < v1 ? src + vn : src, vn < v1);
-                cp_async_commit();
+        uint32_t *cb = sm.cand_bits[warp];
+        int32_t *cc = sm.cand_col[warp];
+        uint32_t wcnt = 0, lost = 0, mag = 0;
+        bool over = false;
+        auto append = [&](uint32_t msk, const uint4 &x, int col0) {
+            const uint32_t c = __popc(msk);
+            const uint32_t incl = warp_incl_scan(c);
+            uint32_t pos = wcnt + incl - c;
+            while (msk) {  // the set bits, in column order
+                const int j = __ffs(msk) - 1;
+                msk &= msk - 1u;
+                const uint32_t bits = Tr::element(x, j);
+                if (pos < static_cast<uint32_t>(kRowsCapWarp)) {
+                    cb[pos] = bits;
+                    cc[pos] = col0 + j;
+                } else if (Tr::key(bits) == fkey) {
+                    ++lost;  // a tie at F past the list's end: counted only
+                } else {
+                    over = true;
+                }
+                ++pos;
             }
-            const int v = v0 + b * 32 + lane;
+            wcnt += __shfl_sync(0xFFFFFFFFu, incl, 31);
+        };
+        ws.run([&](const uint4 &x, bool valid, int v) {
             bool hit = false;
-            if (v < v1) {
+            if (valid) {
                 mag = Tr::mag_max(mag, x);
                 if (fpos) {
                     hit = Tr::any_ge_pos(x, fraw);
@@ -387,38 +678,19 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
                 }
             }
             if (__ballot_sync(0xFFFFFFFFu, hit)) {
-                uint32_t m = 0;
+                uint32_t msk = 0;
                 if (hit) {
                     if (fpos) {
-                        m = Tr::ge_mask_pos(x, fraw);
+                        msk = Tr::ge_mask_pos(x, fraw);
                     } else {
 #pragma unroll
                         for (int j = 0; j < VEC; ++j)
-                            if (Tr::key(Tr::element(x, j)) >= fkey) m |= 1u << j;
+                            if (Tr::key(Tr::element(x, j)) >= fkey) msk |= 1u << j;
                     }
                 }
-                const uint32_t c = __popc(m);
-                uint32_t incl = c;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const uint32_t t = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-                    if (lane >= o) incl += t;
-                }
-                uint32_t pos = wcnt + incl - c;
-                const int col0 = v * VEC;
-                while (m) {  // the set bits, in column order
-                    const int j = __ffs(m) - 1;
-                    m &= m - 1u;
-                    if (pos < static_cast<uint32_t>(kRowsCapWarp)) {
-                        cb[pos] = Tr::element(x, j);
-                        cc[pos] = col0 + j;
-                    }
-                    ++pos;
-                }
-                wcnt += __shfl_sync(0xFFFFFFFFu, incl, 31);
+                append(msk, x, v * VEC);
             }
-        }
-        cp_async_wait<0>();
+        });
         // ragged tail (n not a multiple of VEC): the last warp, in order
         bool tail_nan = false;
         if (warp == kRowsWarps - 1) {
@@ -431,287 +703,249 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
                     tail_nan |= Tr::isnan_bits(bits);
                     hit = Tr::key(bits) >= fkey;
                 }
-                const uint32_t bal = __ballot_sync(0xFFFFFFFFu, hit);
-                const uint32_t pos = wcnt + __popc(bal & lt_mask);
-                if (hit && pos < static_cast<uint32_t>(kRowsCapWarp)) {
-                    cb[pos] = bits;
-                    cc[pos] = e;
-                }
-                wcnt += __popc(bal);
+                append(hit ? 1u : 0u, make_uint4(bits, 0u, 0u, 0u), e - 0);
             }
         }
         if (Tr::mag_has_nan(mag) || tail_nan) sm.nan_seen = 1;
+        lost = __reduce_add_sync(0xFFFFFFFFu, lost);
+        over = __any_sync(0xFFFFFFFFu, over);
         if (lane == 0) {
-            sm.warp_cnt[warp] = min(wcnt, static_cast<uint32_t>(kRowsCapWarp));
-            if (wcnt > static_cast<uint32_t>(kRowsCapWarp)) sm.overflow = 1;
+            sm.w_cnt[warp] = min(wcnt, static_cast<uint32_t>(kRowsCapWarp));
+            sm.w_lost[warp] = lost;
+            if (over) sm.overflow = 1;
         }
     }
     __syncthreads();
     if (tid == 0) {
-        uint32_t t = 0;
-        for (int ww = 0; ww < kRowsWarps; ++ww) t += sm.warp_cnt[ww];
-        sm.cta_cnt = t;
+        sm.cta_fkey = fkey;
         sm.cta_over = sm.overflow;
-    }
-    if (tid < kRowsMaxCluster) {
-        sm.r_gt[tid] = 0;
-        sm.r_eq[tid] = 0;
     }
     cluster.sync();  // every candidate list of the cluster is final from here on
 
-    // ---- 3. exact threshold key u* ----
-    uint32_t total = 0, fmax = 0, over = 0;
-    for (unsigned rr = 0; rr < cs; ++rr) {
-        const RowsSmem *o = cluster.map_shared_rank(&sm, rr);
-        total += o->cta_cnt;
-        fmax = max(fmax, o->cta_fkey == 0xFFFFFFFFu ? 0u : o->cta_fkey);
-        over |= o->cta_over;
-    }
-    // Uniform across the cluster: every CTA reads the same values.
-    bool exact_ok = !over && total >= static_cast<uint32_t>(k);
-    uint32_t ustar = 0, above = 0;
-    const int passes = DT == FTK_BF16 ? 2 : 4;
-    if (exact_ok && total <= static_cast<uint32_t>(kRowsGather)) {
-        uint32_t *gath = reinterpret_cast<uint32_t *>(sm.ring);  // the ring is free now
-        // Few candidates: every CTA gathers all candidate keys of the cluster
-        // into its own shared memory once and selects locally (identical
-        // result in every CTA, no cluster barrier between passes).
-        uint32_t off = 0;  // start of list (rr, warp) in gath
-        uint32_t kmn = 0xFFFFFFFFu, kmx = 0u;  // bounds of the gathered keys
-        for (unsigned rr = 0; rr < cs; ++rr) {
-            const RowsSmem *o = cluster.map_shared_rank(&sm, rr);
-            uint32_t before = 0;
-            for (int ww = 0; ww < warp; ++ww) before += o->warp_cnt[ww];
-            const uint32_t cnt = o->warp_cnt[warp];
-            const uint32_t *cb = o->cand_bits + warp * kRowsCapWarp;
-            for (uint32_t i = lane; i < cnt; i += 32) {
-                const uint32_t u = Tr::key(cb[i]);
-                gath[off + before + i] = u;
-                kmn = min(kmn, u);
-                kmx = max(kmx, u);
-            }
-            off += o->cta_cnt;
-        }
+    // ---- the cluster's lists, in column order ----
+    const int nl = static_cast<int>(cs) * kRowsWarps;
+    if (warp == 0) {
+        uint32_t cnt[2], lst[2], fk[2], ov = 0, fmax = 0;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            kmn = min(kmn, __shfl_xor_sync(0xFFFFFFFFu, kmn, o));
-            kmx = max(kmx, __shfl_xor_sync(0xFFFFFFFFu, kmx, o));
+        for (int h = 0; h < 2; ++h) {
+            const int L = lane + 32 * h;
+            cnt[h] = lst[h] = fk[h] = 0;
+            if (L < nl) {
+                const RowsSmem *o = cluster.map_shared_rank(&sm, static_cast<unsigned>(L / kRowsWarps));
+                cnt[h] = o->w_cnt[L % kRowsWarps];
+                lst[h] = o->w_lost[L % kRowsWarps];
+                fk[h] = o->cta_fkey;
+                ov |= o->cta_over;
+                fmax = max(fmax, fk[h]);
+            }
         }
+        const uint32_t i0 = warp_incl_scan(cnt[0]);
+        const uint32_t t0 = __shfl_sync(0xFFFFFFFFu, i0, 31);
+        const uint32_t i1 = warp_incl_scan(cnt[1]) + t0;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int L = lane + 32 * h;
+            if (L < nl) {
+                sm.l_off[L] = (h == 0 ? i0 : i1) - cnt[h];
+                sm.l_cnt[L] = cnt[h];
+                sm.l_lost[L] = lst[h];
+                sm.l_fkey[L] = fk[h];
+            }
+        }
+        const uint32_t lost_all = __reduce_add_sync(0xFFFFFFFFu, lst[0] + lst[1]);
+        ov = __reduce_or_sync(0xFFFFFFFFu, ov);
+        fmax = __reduce_max_sync(0xFFFFFFFFu, fmax);
+        if (lane == 31) sm.l_off[nl] = i1;
         if (lane == 0) {
-            sm.tot[warp] = kmn;
-            sm.tot[kRowsWarps + warp] = kmx;
+            sm.g_lost = lost_all;
+            sm.g_over = ov;
+            sm.g_fmax = fmax;
+        }
+    }
+    __syncthreads();
+    const uint32_t total = sm.l_off[nl];
+    bool exact_ok = !sm.g_over && total <= static_cast<uint32_t>(kRowsGather) &&
+                    total + sm.g_lost >= static_cast<uint32_t>(k);
+    uint32_t ustar = 0, above = 0;
+    if (exact_ok) {
+        // Every CTA gathers all candidate keys of the cluster (the rings are
+        // free now) and finds u* locally: the same result in every CTA.
+        uint32_t *gath = reinterpret_cast<uint32_t *>(sm.ring);
+        uint32_t kmn = 0xFFFFFFFFu, kmx = 0u;
+        for (int L = warp; L < nl; L += kRowsWarps) {
+            const RowsSmem *o = cluster.map_shared_rank(&sm, static_cast<unsigned>(L / kRowsWarps));
+            const uint32_t *cb = o->cand_bits[L % kRowsWarps];
+            const uint32_t cnt = sm.l_cnt[L], off = sm.l_off[L];
+            for (uint32_t i0 = 0; i0 < cnt; i0 += 128) {
+                uint32_t v[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const uint32_t i = i0 + u * 32 + lane;
+                    v[u] = i < cnt ? cb[i] : 0u;
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const uint32_t i = i0 + u * 32 + lane;
+                    if (i < cnt) {
+                        const uint32_t key = Tr::key(v[u]);
+                        gath[off + i] = key;
+                        kmn = min(kmn, key);
+                        kmx = max(kmx, key);
+                    }
+                }
+            }
+        }
+        if (tid < nl && sm.l_lost[tid]) {  // uncounted ties at F take part too
+            kmn = min(kmn, sm.l_fkey[tid]);
+            kmx = max(kmx, sm.l_fkey[tid]);
+        }
+        kmn = __reduce_min_sync(0xFFFFFFFFu, kmn);
+        kmx = __reduce_max_sync(0xFFFFFFFFu, kmx);
+        if (lane == 0) {
+            sm.red[warp] = kmn;
+            sm.red[kRowsWarps + warp] = kmx;
         }
         __syncthreads();
-        for (int ww = 0; ww < kRowsWarps; ++ww) {
-            kmn = min(kmn, sm.tot[ww]);
-            kmx = max(kmx, sm.tot[kRowsWarps + ww]);
+#pragma unroll
+        for (int w = 0; w < kRowsWarps; ++w) {
+            kmn = min(kmn, sm.red[w]);
+            kmx = max(kmx, sm.red[kRowsWarps + w]);
         }
         // Bits above the highest one where the keys differ are common to
-        // all of them: the 8-bit radix digits start below those.
-        const int lo_bit = 32 - 8 * passes;  // bf16 keys sit in the upper half
+        // all of them: the 11-bit radix digits start below those.
+        const int lo_bit = DT == FTK_BF16 ? 16 : 0;  // bf16 keys sit in the upper half
         const uint32_t diff = kmn ^ kmx;
         const int top = diff ? 31 - __clz(diff) : -1;
         uint32_t mask = top < 0 ? 0xFFFFFFFFu : (top == 31 ? 0u : ~((2u << top) - 1u));
         uint32_t prefix = kmx & mask, krem = static_cast<uint32_t>(k);
-        for (int hi = top; hi >= lo_bit; hi -= 8) {
-            const int shift = hi - 7 >= lo_bit ? hi - 7 : lo_bit;
+        bool found = true;
+        for (int hi = top; hi >= lo_bit && found; hi -= 11) {
+            const int shift = hi - 10 >= lo_bit ? hi - 10 : lo_bit;
             const uint32_t dmask = (2u << (hi - shift)) - 1u;
-            for (int b = tid; b < 256; b += blockDim.x) sm.hist[b] = 0;
+            for (int b = tid; b < kRowsBins; b += kRowsThreads) sm.hist[b] = 0;
             __syncthreads();
-            for (uint32_t i0 = 0; i0 < total; i0 += blockDim.x) {
+            for (uint32_t i0 = 0; i0 < total; i0 += kRowsThreads) {
                 const uint32_t i = i0 + tid;
                 const uint32_t u = i < total ? gath[i] : 0u;
                 hist_add(sm.hist, (u >> shift) & dmask, i < total && (u & mask) == prefix);
             }
+            if (tid < nl && sm.l_lost[tid] && (sm.l_fkey[tid] & mask) == prefix)
+                atomicAdd(&sm.hist[(sm.l_fkey[tid] >> shift) & dmask], sm.l_lost[tid]);
             __syncthreads();
-            for (int b = tid; b < 256; b += blockDim.x) sm.tot[b] = sm.hist[b];
-            __syncthreads();
-            find_kth_bin256(sm, krem);
-            prefix |= sm.sel_bin << shift;
-            mask |= dmask << shift;
-            krem -= sm.sel_above;
-            above += sm.sel_above;
-            __syncthreads();
+            found = find_bin_top<kRowsBins>(sm, sm.hist, krem);
+            if (found) {
+                prefix |= sm.sel_bin << shift;
+                mask |= dmask << shift;
+                krem -= sm.sel_above;
+                above += sm.sel_above;
+            }
         }
         ustar = prefix;
-        // The candidates are exactly each chunk's elements >= its F, so they
-        // hold every element >= u* iff u* >= every F.
-        exact_ok = ustar >= fmax;
-    } else if (exact_ok) {
-        // Many candidates (heavy ties): per-CTA histograms of my own lists,
-        // summed over the cluster through distributed shared memory.
-        uint32_t prefix = 0, mask = 0, krem = static_cast<uint32_t>(k);
-        for (int p = 0; p < passes; ++p) {
-            const int shift = 24 - 8 * p;
-            for (int b = tid; b < 256; b += blockDim.x) sm.hist[b] = 0;
-            __syncthreads();
-            {
-                const uint32_t cnt = sm.warp_cnt[warp];
-                const uint32_t *cb = sm.cand_bits + warp * kRowsCapWarp;
+        // The candidates are exactly each chunk's elements >= its F (ties at
+        // F counted), so they hold every element >= u* iff u* >= every F.
+        exact_ok = found && ustar >= sm.g_fmax;
+        if (exact_ok) {
+            // Per list: keys > u* and stored keys == u*; then, in column
+            // order, each list's share of the ties and its first output slot.
+            for (int L = warp; L < nl; L += kRowsWarps) {
+                const uint32_t cnt = sm.l_cnt[L], off = sm.l_off[L];
+                uint32_t g = 0, q = 0;
                 for (uint32_t i0 = 0; i0 < cnt; i0 += 32) {
                     const uint32_t i = i0 + lane;
-                    const uint32_t u = i < cnt ? Tr::key(cb[i]) : 0u;
-                    hist_add(sm.hist, (u >> shift) & 255u, i < cnt && (u & mask) == prefix);
+                    const uint32_t u = i < cnt ? gath[off + i] : 0u;
+                    g += __popc(__ballot_sync(0xFFFFFFFFu, i < cnt && u > ustar));
+                    q += __popc(__ballot_sync(0xFFFFFFFFu, i < cnt && u == ustar));
+                }
+                if (lane == 0) {
+                    sm.l_gt[L] = g;
+                    sm.l_eq[L] = q;
                 }
             }
-            cluster.sync();
-            cluster_sum256(cluster, sm);
             __syncthreads();
-            find_kth_bin256(sm, krem);
-            prefix |= sm.sel_bin << shift;
-            mask |= 255u << shift;
-            krem -= sm.sel_above;
-            above += sm.sel_above;
-            cluster.sync();  // every CTA is done reading my hist
+            if (warp == 0) {
+                const uint32_t need = static_cast<uint32_t>(k) - above;  // ties at u* to take, >= 1
+                uint32_t eqt[2], sel[2], take[2];
+                bool shrt = false;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int L = lane + 32 * h;
+                    eqt[h] = 0;
+                    if (L < nl) eqt[h] = sm.l_eq[L] + (sm.l_fkey[L] == ustar ? sm.l_lost[L] : 0u);
+                }
+                const uint32_t e0 = warp_incl_scan(eqt[0]);
+                const uint32_t et = __shfl_sync(0xFFFFFFFFu, e0, 31);
+                const uint32_t e1 = warp_incl_scan(eqt[1]) + et;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int L = lane + 32 * h;
+                    const uint32_t eb = (h == 0 ? e0 : e1) - eqt[h];  // ties before list L
+                    take[h] = eb >= need ? 0u : min(eqt[h], need - eb);
+                    sel[h] = 0;
+                    if (L < nl) {
+                        shrt |= take[h] > sm.l_eq[L];  // needs ties it did not store
+                        sel[h] = sm.l_gt[L] + take[h];
+                    }
+                }
+                const uint32_t s0 = warp_incl_scan(sel[0]);
+                const uint32_t st = __shfl_sync(0xFFFFFFFFu, s0, 31);
+                const uint32_t s1 = warp_incl_scan(sel[1]) + st;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int L = lane + 32 * h;
+                    if (L < nl) {
+                        sm.l_take[L] = take[h];
+                        sm.l_selb[L] = (h == 0 ? s0 : s1) - sel[h];
+                    }
+                }
+                shrt = __any_sync(0xFFFFFFFFu, shrt);
+                if (lane == 0) sm.short_eq = shrt ? 1u : 0u;
+            }
+            __syncthreads();
+            exact_ok = sm.short_eq == 0;
         }
-        ustar = prefix;
-        exact_ok = ustar >= fmax;
     }
+    // exact_ok is uniform over the cluster: every CTA decided it from the
+    // same published lists.
     if (!exact_ok) {
-        // Exact multi-pass radix select over the whole row (re-read from L2).
-        uint32_t prefix = 0, mask = 0, krem = static_cast<uint32_t>(k);
-        above = 0;
-        for (int p = 0; p < passes; ++p) {
-            const int shift = 24 - 8 * p;
-            for (int b = tid; b < 256; b += blockDim.x) sm.hist[b] = 0;
-            __syncthreads();
-            for (int e0 = 0; e0 < n; e0 += blockDim.x) {
-                const int e = e0 + tid;
-                const uint32_t u = e < n ? Tr::key(row[c0 + e]) : 0u;
-                hist_add(sm.hist, (u >> shift) & 255u, e < n && (u & mask) == prefix);
-            }
-            cluster.sync();
-            cluster_sum256(cluster, sm);
-            __syncthreads();
-            find_kth_bin256(sm, krem);
-            prefix |= sm.sel_bin << shift;
-            mask |= 255u << shift;
-            krem -= sm.sel_above;
-            above += sm.sel_above;
-            cluster.sync();
-        }
-        ustar = prefix;
-    }
-    const uint32_t need = static_cast<uint32_t>(k) - above;  // ties at u* to take, >= 1
-
-    // ---- 4. ordered selection ----
-    // Segment order is column order: the fast path walks each warp's
-    // candidate list, the fallback each warp's contiguous slice of the chunk.
-    const int seg = ((n + kRowsWarps - 1) / kRowsWarps + 31) & ~31;
-    const int s0 = min(n, warp * seg), s1 = min(n, s0 + seg);
-    const uint32_t wlen = exact_ok ? sm.warp_cnt[warp] : static_cast<uint32_t>(s1 - s0);
-    auto item = [&](uint32_t i, uint32_t &bits, int &col) {
-        if (exact_ok) {
-            bits = sm.cand_bits[warp * kRowsCapWarp + i];
-            col = sm.cand_col[warp * kRowsCapWarp + i];
-        } else {
-            col = s0 + static_cast<int>(i);
-            bits = row[c0 + col];
-        }
-    };
-    uint32_t my_gt = 0, my_eq = 0;
-    for (uint32_t i0 = 0; i0 < wlen; i0 += 32) {
-        const uint32_t i = i0 + lane;
-        bool gt = false, eq = false;
-        if (i < wlen) {
-            uint32_t bits;
-            int col;
-            item(i, bits, col);
-            const uint32_t u = Tr::key(bits);
-            gt = u > ustar;
-            eq = u == ustar;
-        }
-        my_gt += __popc(__ballot_sync(0xFFFFFFFFu, gt));
-        my_eq += __popc(__ballot_sync(0xFFFFFFFFu, eq));
-    }
-    if (lane == 0) {
-        sm.warp_gt[warp] = my_gt;
-        sm.warp_eq[warp] = my_eq;
-    }
-    if (exact_ok) {
-        // Counts of the CTAs before me, from their lists in place.
-        for (unsigned rr = 0; rr < rank; ++rr) {
-            const RowsSmem *o = cluster.map_shared_rank(&sm, rr);
-            const uint32_t cnt = o->warp_cnt[warp];
-            const uint32_t *cb = o->cand_bits + warp * kRowsCapWarp;
-            uint32_t g = 0, q = 0;
-            for (uint32_t i0 = 0; i0 < cnt; i0 += 32) {
-                const uint32_t i = i0 + lane;
-                const uint32_t u = i < cnt ? Tr::key(cb[i]) : 0u;
-                g += __popc(__ballot_sync(0xFFFFFFFFu, i < cnt && u > ustar));
-                q += __popc(__ballot_sync(0xFFFFFFFFu, i < cnt && u == ustar));
-            }
-            if (lane == 0 && (g | q)) {
-                atomicAdd(&sm.r_gt[rr], g);
-                atomicAdd(&sm.r_eq[rr], q);
-            }
-        }
-    }
-    __syncthreads();
-    if (tid == 0) {
-        uint32_t g = 0, q = 0;
-        for (int ww = 0; ww < kRowsWarps; ++ww) {
-            const uint32_t tg = sm.warp_gt[ww], tq = sm.warp_eq[ww];
-            sm.warp_gt[ww] = g;  // exclusive prefixes
-            sm.warp_eq[ww] = q;
-            g += tg;
-            q += tq;
-        }
-        sm.cta_gt = g;
-        sm.cta_eq = q;
-    }
-    if (exact_ok) {
+        __syncthreads();
+        rows_fallback<DT, IT>(a, sm, cluster, cs, rank, row, c0, n, base_index, oidx, oval, ph);
+    } else {
         __syncthreads();
         cluster_arrive();  // no more reads of other CTAs' shared memory
-    } else {
-        cluster.sync();
-        for (unsigned rr = tid; rr < rank; rr += blockDim.x) {
-            const RowsSmem *o = cluster.map_shared_rank(&sm, rr);
-            sm.r_gt[rr] = o->cta_gt;
-            sm.r_eq[rr] = o->cta_eq;
-        }
-        __syncthreads();
-        cluster_arrive();
-    }
-    uint32_t eq_before = 0, sel_before = 0;
-    for (unsigned rr = 0; rr < rank; ++rr) {
-        const uint32_t g = sm.r_gt[rr], q = sm.r_eq[rr];
-        const uint32_t take = eq_before >= need ? 0u : min(q, need - eq_before);
-        sel_before += g + take;
-        eq_before += q;
-    }
-    const uint32_t my_take = eq_before >= need ? 0u : min(sm.cta_eq, need - eq_before);
-    const uint32_t w_gt = sm.warp_gt[warp], w_eq = sm.warp_eq[warp];
-    uint32_t pos = sel_before + w_gt + min(w_eq, my_take);  // next output slot of this warp
-    uint32_t eq_rank = w_eq;                                // CTA-local tie rank
-    for (uint32_t i0 = 0; i0 < wlen; i0 += 32) {
-        const uint32_t i = i0 + lane;
-        uint32_t bits = 0;
-        int col = 0;
-        bool gt = false, eq = false;
-        if (i < wlen) {
-            item(i, bits, col);
-            const uint32_t u = Tr::key(bits);
-            gt = u > ustar;
-            eq = u == ustar;
-        }
-        const uint32_t eq_bal = __ballot_sync(0xFFFFFFFFu, eq);
-        const uint32_t rank_eq = eq_rank + __popc(eq_bal & lt_mask);
-        const bool sel = gt || (eq && rank_eq < my_take);
-        const uint32_t sel_bal = __ballot_sync(0xFFFFFFFFu, sel);
-        if (sel) {
-            const uint32_t p = pos + __popc(sel_bal & lt_mask);
-            if (p < static_cast<uint32_t>(k)) {
-                oidx[p] = static_cast<IT>(static_cast<int32_t>(base_index + c0 + col));
-                if (oval) oval[p] = static_cast<elem>(bits);
-            } else {
-                set_status(a.status, FTK_STATUS_INTERNAL);
+        // ---- ordered output of my lists ----
+        const int L = static_cast<int>(rank) * kRowsWarps + warp;
+        const uint32_t cnt = sm.w_cnt[warp], take = sm.l_take[L];
+        uint32_t pos = sm.l_selb[L], eq_rank = 0;
+        for (uint32_t i0 = 0; i0 < cnt; i0 += 32) {
+            const uint32_t i = i0 + lane;
+            uint32_t bits = 0;
+            int col = 0;
+            bool gt = false, eq = false;
+            if (i < cnt) {
+                bits = sm.cand_bits[warp][i];
+                col = sm.cand_col[warp][i];
+                const uint32_t u = Tr::key(bits);
+                gt = u > ustar;
+                eq = u == ustar;
             }
+            const uint32_t eq_bal = __ballot_sync(0xFFFFFFFFu, eq);
+            const bool sel = gt || (eq && eq_rank + __popc(eq_bal & lt_mask) < take);
+            const uint32_t sel_bal = __ballot_sync(0xFFFFFFFFu, sel);
+            if (sel) {
+                const uint32_t p = pos + __popc(sel_bal & lt_mask);
+                if (p < static_cast<uint32_t>(k)) {
+                    oidx[p] = static_cast<IT>(static_cast<int32_t>(base_index + c0 + col));
+                    if (oval) oval[p] = static_cast<elem>(bits);
+                } else {
+                    set_status(a.status, FTK_STATUS_INTERNAL);
+                }
+            }
+            pos += __popc(sel_bal);
+            eq_rank += __popc(eq_bal);
         }
-        pos += __popc(sel_bal);
-        eq_rank += __popc(eq_bal);
     }
     if (tid == 0 && sm.nan_seen) set_status(a.status, FTK_STATUS_NAN);
+    fence_proxy_async();  // generic writes of the rings precede later bulk copies into them
     __syncwarp();
     cluster_wait();  // keep my shared memory alive until every CTA is done with it
 }
@@ -733,14 +967,20 @@ __global__ void __launch_bounds__(kRowsThreads, 2) rows_topk_kernel(const RowsAr
         const int64_t c = static_cast<int64_t>(*a.nrows_dev) - a.nrows_off;
         nrows = c < nrows ? c : nrows;
     }
+    if (static_cast<int64_t>(blockIdx.x / cs) >= nrows) return;  // whole clusters exit together
+    if (threadIdx.x == 0) {
+        for (int w = 0; w < kRowsWarps; ++w)
+            for (int s = 0; s < kRowsStages; ++s) mbar_init(&sm.full[w][s], 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    uint32_t ph = 0;  // parity each stage barrier of my warp waits for next
     // Row selection is uniform over the cluster: its CTAs walk the same rows.
     if constexpr (!LOOP) {
-        const int64_t r = blockIdx.x / cs;
-        if (r < nrows) rows_topk_row<DT, IT>(a, sm, cluster, cs, rank, r);
+        rows_topk_row<DT, IT>(a, sm, cluster, cs, rank, blockIdx.x / cs, ph);
     } else {
         for (int64_t r = blockIdx.x / cs; r < nrows; r += gridDim.x / cs) {
-            rows_topk_row<DT, IT>(a, sm, cluster, cs, rank, r);
-            cp_async_wait<0>();
+            rows_topk_row<DT, IT>(a, sm, cluster, cs, rank, r, ph);
             __syncthreads();  // shared memory is free for the next row
         }
     }

@@ -419,6 +419,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t nlist = list_rows(a);
+    if (nlist <= 0) return;  // e.g. a recovery pass with no rows left: no TMEM, no barriers
     const Sched sc = make_sched<MODE, RT>(a, nlist);
     constexpr bool pruned = MODE == MODE_COLLECT && PR;
 

@@ -696,8 +696,8 @@ static ftk_status launch_score(const ScoreArgs &a, const CUtensorMap &tq, const 
 {
     const int smem = ScoreSmemLayout<DT>::kBytes;
     auto kern = score_kernel<DT, MODE, PR, H64>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return cuda_status(e);
+    const ftk_status e = ensure_smem_limit(reinterpret_cast<const void *>(kern), smem);
+    if (e != FTK_OK) return e;
     kern<<<grid, kScoreThreads, smem, st>>>(a, tq, kvm);
     return cuda_status(cudaGetLastError());
 }
@@ -926,10 +926,8 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
     ta.oversample = c.beta;
     {
         const size_t smem = static_cast<size_t>(w.sld) * 4;
-        cudaError_t e = cudaFuncSetAttribute(threshold_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem));
-        if (e != cudaSuccess) return cuda_status(e);
+        st = ensure_smem_limit(reinterpret_cast<const void *>(threshold_kernel), static_cast<int>(smem));
+        if (st != FTK_OK) return st;
         threshold_kernel<<<static_cast<unsigned>(T), kSelThreads, smem, s>>>(ta);
         if ((st = cuda_status(cudaGetLastError())) != FTK_OK) return st;
     }
@@ -1023,10 +1021,8 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
     ra.info = w.info;
     {
         const size_t smem = static_cast<size_t>(c.cap) * 4;
-        cudaError_t e = cudaFuncSetAttribute(refine_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem));
-        if (e != cudaSuccess) return cuda_status(e);
+        st = ensure_smem_limit(reinterpret_cast<const void *>(refine_kernel), static_cast<int>(smem));
+        if (st != FTK_OK) return st;
         refine_kernel<<<static_cast<unsigned>(T), kSelThreads, smem, s>>>(ra);
         if ((st = cuda_status(cudaGetLastError())) != FTK_OK) return st;
     }

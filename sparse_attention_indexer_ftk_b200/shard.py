@@ -9,8 +9,42 @@ caller wants every row's result on one rank, a gather after the fact.
 """
 from __future__ import annotations
 
+import datetime
+
 import torch
 import torch.distributed as dist
+
+
+class ProcessGroup:
+    """One process per GPU: the default process group for `world` ranks,
+    set up on entry and destroyed exactly once on exit (also when the body
+    raises).  With world == 1 nothing is set up.  backend "nccl" makes
+    cuda:local_rank current first; "gloo" runs on the CPU.  The timeout is
+    short so that ranks waiting for a rank that died end with an error."""
+
+    def __init__(self, world: int, local_rank: int = 0, backend: str = "nccl", timeout_s: float = 120.0):
+        self.world, self.local, self.backend, self.timeout_s = world, local_rank, backend, timeout_s
+        self.active = False
+
+    def __enter__(self) -> "ProcessGroup":
+        if self.world > 1:
+            kw = {}
+            if self.backend == "nccl":
+                torch.cuda.set_device(self.local)
+                kw["device_id"] = torch.device("cuda", self.local)
+            dist.init_process_group(self.backend, timeout=datetime.timedelta(seconds=self.timeout_s), **kw)
+            self.active = True
+        return self
+
+    def barrier(self) -> None:
+        if self.active:
+            dist.barrier()
+
+    def __exit__(self, *exc) -> bool:
+        if self.active and dist.is_initialized():
+            dist.destroy_process_group()
+        self.active = False
+        return False
 
 
 def row_shard(T: int, world: int, rank: int) -> tuple[int, int]:
