@@ -459,9 +459,22 @@ def bench_config(name: str, dev, reps: int = 10):
     torch.cuda.synchronize()
     ms = sum(a.elapsed_time(b) for a, b in ev) / reps
     info = ftk.read_info(ws)
-    return {"workload": name, "T": d.T, "S": d.S, "topk": d.topk, "heads": heads, "ms_per_call": ms,
-            "queries_per_s": d.T / (ms * 1e-3),
-            "dense_eq_tflops": 2.0 * heads * 128 * d.pairs() / (ms * 1e-3) / 1e12,
+    # Tensor roofline of the whole call: the BF16 dense peak for BF16 operands,
+    # 2 x that (nominal FP8 : BF16 ratio) for FP8.
+    peaks, src = measured_peaks()
+    bf16 = d.q.dtype == torch.bfloat16
+    peak = peaks["bf16_tflops"] * (1.0 if bf16 else 2.0)
+    dense = 2.0 * heads * 128 * d.pairs() / (ms * 1e-3) / 1e12
+    rt = (8 if bf16 else 16) // (2 if heads == 64 else 1)
+    executed = 2.0 * heads * 128 * (int(info["blocks_total"]) - int(info["blocks_pruned"])) * rt * 128 \
+        / (ms * 1e-3) / 1e12
+    return {"workload": name, "T": d.T, "S": d.S, "topk": d.topk, "heads": heads,
+            "dtype": "bf16 x bf16 -> f32" if bf16 else "fp8_e4m3 x fp8_e4m3 -> f32", "ms_per_call": ms,
+            "queries_per_s": d.T / (ms * 1e-3), "dense_eq_tflops": dense, "executed_tflops": executed,
+            "roofline": {"bound": "tensor", "achieved": dense, "peak": peak, "unit": "TFLOP/s",
+                         "frac": dense / peak,
+                         "peak_source": f"{'1' if bf16 else '2'} x bf16_tflops ({src}, burst)",
+                         "scope": "whole call (every stage), dense-equivalent work"},
             "prune_enabled": info["prune_enabled"], "blocks_total": info["blocks_total"],
             "blocks_pruned": info["blocks_pruned"],
             "rows_recovered": info["rows_overflow"] + info["rows_underflow"]}
@@ -741,7 +754,9 @@ def _run_ours(args, pg, world, rank, local):
     }
     if world == 1 and not (args.no_decode or args.no_extras):
         out["decode_64q"] = bench_decode(c, dev)
+        out["bf16_small"] = bench_config("bf16_small", dev, reps=50)
         out["fp8_packed"] = bench_config("fp8_packed", dev)
+        out["fp8_large"] = bench_config("fp8_large", dev, reps=5)
         out["fp8_prefill_64h"] = bench_config("fp8_prefill_64h", dev)
     if world == 1 and not args.no_rows:
         out["row_topk"] = [bench_rows("rows_bf16", dev), bench_rows("rows_f32", dev),

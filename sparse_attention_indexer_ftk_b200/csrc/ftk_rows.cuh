@@ -16,11 +16,13 @@
 //      rare elements >= F go, in column order, to the warp's candidate list
 //      in shared memory.  Elements equal to F that find the list full are
 //      only counted (heavy ties);
-//   4. exact k-th key u*: every CTA gathers all candidate keys of the
-//      cluster through distributed shared memory and radix-selects them
-//      locally (11-bit digits), counting the uncounted ties at F as well;
-//      u* is the row's k-th largest key if every CTA kept every element
-//      >= u* (u* >= every F, no list overflowed);
+//   4. exact k-th key u*: with Fu the cluster's largest F, every list holds
+//      all of its chunk's elements > Fu and its elements == Fu are stored
+//      or counted.  If at least topk elements are >= Fu, the k-th largest is
+//      >= Fu: when fewer than topk are > Fu it is Fu itself (heavy ties need
+//      no selection), otherwise every CTA gathers all candidate keys of the
+//      cluster through distributed shared memory and radix-selects those
+//      > Fu locally (11-bit digits);
 //   5. output: the counts of each list (> u*, == u*) give every warp its
 //      output slots; ties at u* go to the smallest columns (CTA order, then
 //      warp order, then list order), written in ascending column order.
@@ -80,18 +82,26 @@ struct RowsSmem {
     uint32_t cand_bits[kRowsWarps][kRowsCapWarp];         // raw value bits
     int32_t cand_col[kRowsWarps][kRowsCapWarp];           // column within the chunk
     uint32_t hist[kRowsBins];
+    uint4 samp[kRowsThreads];                             // the spread sample (one vector per thread)
     uint64_t full[kRowsWarps][kRowsStages];               // one mbarrier per ring stage
     // this CTA's lists, read by the other CTAs of the cluster
     uint32_t w_cnt[kRowsWarps];    // stored entries
     uint32_t w_lost[kRowsWarps];   // entries equal to F past the end of a full list
+    uint32_t w_gtf[kRowsWarps];    // stored entries > Fu (the cluster's largest F)
+    uint32_t w_eqs[kRowsWarps];    // stored entries == Fu
+    uint32_t w_eqf[kRowsWarps];    // entries == Fu, stored or counted
+    uint32_t w_kmax[kRowsWarps];   // largest stored key
     uint32_t cta_fkey, cta_over, cta_gt, cta_eq;
     // every list of the cluster in column order (index rank * kRowsWarps + warp)
-    uint32_t l_off[kRowsLists + 1], l_cnt[kRowsLists], l_lost[kRowsLists], l_fkey[kRowsLists];
-    uint32_t l_gt[kRowsLists], l_eq[kRowsLists], l_take[kRowsLists], l_selb[kRowsLists];
+    uint32_t l_off[kRowsLists + 1], l_cnt[kRowsLists], l_fkey[kRowsLists];
+    uint32_t l_gt[kRowsLists];     // entries > u*
+    uint32_t l_eq[kRowsLists];     // stored entries == u*
+    uint32_t l_eqt[kRowsLists];    // entries == u*, stored or counted
+    uint32_t l_take[kRowsLists], l_selb[kRowsLists];
     uint32_t wsum[kRowsWarps];
     uint32_t red[2 * kRowsWarps];
     uint32_t sel_bin, sel_above, fmin, short_eq;
-    uint32_t g_total, g_lost, g_fmax, g_over;
+    uint32_t g_gt, g_eqt, g_fmax, g_over, g_kmax;
     uint32_t nan_seen, overflow;
 };
 
@@ -111,14 +121,30 @@ struct RowsTraits<FTK_BF16> {
         const uint32_t w = q == 0 ? v.x : q == 1 ? v.y : q == 2 ? v.z : v.w;
         return (j & 1) ? (w >> 16) : (w & 0xFFFFu);
     }
-    // True if some element of the vector may be >= F, for a strictly
-    // positive F whose raw bits are in both halves of f2 (positive bf16
-    // values order like signed 16-bit integers, negative ones are negative).
-    __device__ static bool any_ge_pos(const uint4 &v, uint32_t f2)
+    // Packed signed / unsigned 16-bit maxima.
+    __device__ static uint32_t smax(uint32_t a, uint32_t b)
     {
-        const uint32_t m = __vmaxs2(__vmaxs2(v.x, v.y), __vmaxs2(v.z, v.w));
-        return __vcmpges2(m, f2) != 0u;
+        uint32_t d;
+        asm("max.s16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+        return d;
     }
+    __device__ static uint32_t umax(uint32_t a, uint32_t b)
+    {
+        uint32_t d;
+        asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+        return d;
+    }
+    // The vector's elements as signed / unsigned 16-bit integers, reduced
+    // to their maxima (two halves).
+    __device__ static uint32_t vsmax(const uint4 &v) { return smax(smax(v.x, v.y), smax(v.z, v.w)); }
+    __device__ static uint32_t vumax(const uint4 &v) { return umax(umax(v.x, v.y), umax(v.z, v.w)); }
+    static constexpr uint32_t kSmaxInit = 0x80008000u;
+    // For a strictly positive F: true if some element of the vector whose
+    // signed maxima are m is >= F.  Positive bf16 values order like signed
+    // 16-bit integers, negative ones are negative.  fm1 holds F's raw bits
+    // minus one in both halves.
+    __device__ static bool ge_from_smax(uint32_t m, uint32_t fm1) { return smax(m, fm1) != fm1; }
+    __device__ static uint32_t fm1_of(uint32_t fraw16) { return (fraw16 - 1u) * 0x10001u; }
     // Bit j set for each element j >= F (strictly positive F, raw bits in
     // both halves of f2).
     __device__ static uint32_t ge_mask_pos(const uint4 &v, uint32_t f2)
@@ -132,15 +158,13 @@ struct RowsTraits<FTK_BF16> {
         }
         return m;
     }
-    // Running max of the magnitudes (NaN detection).
-    __device__ static uint32_t mag_max(uint32_t acc, const uint4 &v)
+    // NaN seen, from the running maxima of the raw elements as signed
+    // (a positive NaN is above 0x7F80) and unsigned (a negative NaN is
+    // above 0xFF80) 16-bit integers.
+    __device__ static bool nan_from(uint32_t s, uint32_t u)
     {
-        const uint32_t m = 0x7FFF7FFFu;
-        return __vmaxu2(__vmaxu2(acc, __vmaxu2(v.x & m, v.y & m)), __vmaxu2(v.z & m, v.w & m));
-    }
-    __device__ static bool mag_has_nan(uint32_t acc)
-    {
-        return (acc & 0xFFFFu) > 0x7F80u || (acc >> 16) > 0x7F80u;
+        return static_cast<int16_t>(s & 0xFFFFu) > 0x7F80 || static_cast<int16_t>(s >> 16) > 0x7F80 ||
+               (u & 0xFFFFu) > 0xFF80u || (u >> 16) > 0xFF80u;
     }
 };
 
@@ -154,25 +178,30 @@ struct RowsTraits<FTK_F32> {
     {
         return j == 0 ? v.x : j == 1 ? v.y : j == 2 ? v.z : v.w;
     }
-    // Positive floats order like signed 32-bit integers.
-    __device__ static bool any_ge_pos(const uint4 &v, uint32_t f)
+    __device__ static uint32_t smax(uint32_t a, uint32_t b)
     {
-        const int32_t m = max(max(static_cast<int32_t>(v.x), static_cast<int32_t>(v.y)),
-                              max(static_cast<int32_t>(v.z), static_cast<int32_t>(v.w)));
-        return m >= static_cast<int32_t>(f);
+        return static_cast<uint32_t>(max(static_cast<int32_t>(a), static_cast<int32_t>(b)));
     }
+    __device__ static uint32_t umax(uint32_t a, uint32_t b) { return max(a, b); }
+    __device__ static uint32_t vsmax(const uint4 &v) { return smax(smax(v.x, v.y), smax(v.z, v.w)); }
+    __device__ static uint32_t vumax(const uint4 &v) { return umax(umax(v.x, v.y), umax(v.z, v.w)); }
+    static constexpr uint32_t kSmaxInit = 0x80000000u;
+    // Positive floats order like signed 32-bit integers.
+    __device__ static bool ge_from_smax(uint32_t m, uint32_t fm1)
+    {
+        return static_cast<int32_t>(m) > static_cast<int32_t>(fm1);
+    }
+    __device__ static uint32_t fm1_of(uint32_t fraw) { return fraw - 1u; }
     __device__ static uint32_t ge_mask_pos(const uint4 &v, uint32_t f)
     {
         const int32_t fi = static_cast<int32_t>(f);
         return (static_cast<int32_t>(v.x) >= fi ? 1u : 0u) | (static_cast<int32_t>(v.y) >= fi ? 2u : 0u) |
                (static_cast<int32_t>(v.z) >= fi ? 4u : 0u) | (static_cast<int32_t>(v.w) >= fi ? 8u : 0u);
     }
-    __device__ static uint32_t mag_max(uint32_t acc, const uint4 &v)
+    __device__ static bool nan_from(uint32_t s, uint32_t u)
     {
-        const uint32_t m = 0x7FFFFFFFu;
-        return max(max(acc, max(v.x & m, v.y & m)), max(v.z & m, v.w & m));
+        return static_cast<int32_t>(s) > 0x7F800000 || u > 0xFF800000u;
     }
-    __device__ static bool mag_has_nan(uint32_t acc) { return acc > 0x7F800000u; }
 };
 
 // Adds 1 to hist[bin] for every active lane.  When all active lanes of the
@@ -317,6 +346,17 @@ struct WarpStream {
         }
     }
 
+    // Waits for the stages prologue() issued, without using them.
+    __device__ __forceinline__ void drain() const
+    {
+        for (int j = 0; j < min(kRowsStages, nst); ++j) {
+            const int s = j % kRowsStages;
+            (void)stage_wait(&sm.full[warp][s], (ph >> s) & 1u, status);
+            ph ^= 1u << s;
+        }
+        __syncwarp();
+    }
+
     template <typename Visit>
     __device__ __forceinline__ bool run(Visit &&visit) const
     {
@@ -341,10 +381,9 @@ struct WarpStream {
             }
             __syncwarp();
             if (ok && j + kRowsStages < nst) {
-                if (lane == 0) {
-                    fence_proxy_async();
-                    issue(j + kRowsStages);
-                }
+                // The warp's reads of the stage are complete (their values
+                // are in registers): the copy may overwrite it.
+                if (lane == 0) issue(j + kRowsStages);
                 ++issued;
             }
         }
@@ -540,40 +579,90 @@ __device__ __noinline__ void rows_fallback(const RowsArgs &a, RowsSmem &sm, cg::
     }
 }
 
+// Where row r's data and this CTA's chunk of it are, and its warp
+// segment (vectors [wv0, wv1) of the chunk).
+template <int DT>
+struct RowGeom {
+    int64_t orow, len, base_index, c0;
+    int n, nvec, wv0, wv1;
+    const typename RowsTraits<DT>::elem *row;
+
+    __device__ __forceinline__ RowGeom(const RowsArgs &a, int64_t r, unsigned rank, int warp)
+    {
+        constexpr int VEC = RowsTraits<DT>::kVec;
+        orow = a.row_map ? a.row_map[r] : r;
+        len = a.cols;
+        base_index = 0;
+        if (a.win_ks) {
+            base_index = a.win_ks[orow];
+            len = static_cast<int64_t>(a.win_ke[orow]) - base_index;
+            if (len < 0) len = 0;
+        }
+        if (a.row_end) {
+            const int64_t e = a.row_end[orow];
+            len = e < 0 ? 0 : (e < len ? e : len);
+        }
+        row = reinterpret_cast<const typename RowsTraits<DT>::elem *>(a.x) + r * a.ld;
+        c0 = static_cast<int64_t>(rank) * a.chunk;
+        const int64_t c1 = min(len, c0 + static_cast<int64_t>(a.chunk));
+        n = c1 > c0 ? static_cast<int>(c1 - c0) : 0;
+        nvec = n / VEC;
+        const int per = (nvec + kRowsWarps - 1) / kRowsWarps;
+        wv0 = min(nvec, warp * per);
+        wv1 = min(nvec, wv0 + per);
+    }
+    __device__ __forceinline__ const uint4 *src() const { return reinterpret_cast<const uint4 *>(row + c0); }
+    // The spread sample of the chunk is taken (else every element is kept).
+    __device__ __forceinline__ bool sampled() const { return nvec >= kRowsThreads && n > kRowsKeepAll; }
+    // Issues this CTA's first ring stages and its sample load (cp.async into
+    // sm.samp) for the row.
+    __device__ __forceinline__ void prefetch(RowsSmem &sm, int warp, int lane, uint32_t &ph, uint32_t *status) const
+    {
+        const WarpStream ws{sm, src(), wv0, wv1 - wv0, (wv1 - wv0 + kRowsStageVecs - 1) / kRowsStageVecs,
+                            warp, lane, ph, status};
+        ws.prologue();
+        if (sampled()) {
+            const int t = threadIdx.x;
+            const uint4 *p = src() + static_cast<int64_t>(t) * nvec / kRowsThreads;
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(&sm.samp[t])), "l"(p) : "memory");
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    }
+};
+
 // Top-k of grid row r by the whole cluster.  Returns with every bulk copy
 // of this CTA landed and every CTA of the cluster done with this CTA's
 // shared memory.
+// Top-k of grid row r by the whole cluster.  Returns with every bulk copy
+// of this CTA landed (but those of the next row, see below) and every CTA
+// of the cluster done with this CTA's shared memory.
+// pre: on entry, whether row r's first stages and sample were issued
+// already (RowGeom::prefetch); on return, whether those of row rnext were.
+// With one CTA per row (cs == 1) the rings are idle once the row has
+// streamed, so the next row's first stages load while this row's
+// candidates are selected and written (rnext < 0: no next row).
 template <int DT, typename IT>
 __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, cg::cluster_group &cluster,
-                                              unsigned cs, unsigned rank, int64_t r, uint32_t &ph)
+                                              unsigned cs, unsigned rank, int64_t r, uint32_t &ph, bool &pre,
+                                              int64_t rnext)
 {
     using Tr = RowsTraits<DT>;
     using elem = typename Tr::elem;
     constexpr int VEC = Tr::kVec;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint32_t lt_mask = (1u << lane) - 1u;
-    const int64_t orow = a.row_map ? a.row_map[r] : r;
-    int64_t len = a.cols, base_index = 0;
-    if (a.win_ks) {
-        base_index = a.win_ks[orow];
-        len = static_cast<int64_t>(a.win_ke[orow]) - base_index;
-        if (len < 0) len = 0;
-    }
-    if (a.row_end) {
-        const int64_t e = a.row_end[orow];
-        len = e < 0 ? 0 : (e < len ? e : len);
-    }
+    const RowGeom<DT> gm(a, r, rank, warp);
+    const int64_t orow = gm.orow, len = gm.len, base_index = gm.base_index, c0 = gm.c0;
+    const int n = gm.n;  // my columns
     const int k = a.k;
-    const elem *row = reinterpret_cast<const elem *>(a.x) + r * a.ld;
+    const elem *row = gm.row;
     // Every output index is below 2^31 (cols <= 2^30; windows are int32), so
     // it is formed in 32 bits and only widened by the store when IT is int64.
     IT *oidx = static_cast<IT *>(a.out_idx) + orow * a.ldo;
     elem *oval = a.out_val ? static_cast<elem *>(a.out_val) + orow * a.ldo : nullptr;
-    const int64_t c0 = static_cast<int64_t>(rank) * a.chunk;
-    const int64_t c1 = min(len, c0 + static_cast<int64_t>(a.chunk));
-    const int n = c1 > c0 ? static_cast<int>(c1 - c0) : 0;  // my columns
 
     // Short row: everything is selected, in column order, then padding.
+    // (Rows like this are never prefetched.)
     if (len <= k) {
         for (int i = tid; i < n; i += blockDim.x) {
             const uint32_t bits = row[c0 + i];
@@ -587,13 +676,13 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
                 if (oval) oval[j] = static_cast<elem>(a.val_fill);
             }
         }
+        pre = false;
         return;
     }
 
-    const int nvec = n / VEC;
-    const int per = (nvec + kRowsWarps - 1) / kRowsWarps;
-    const int wv0 = min(nvec, warp * per), wv1 = min(nvec, wv0 + per);
-    const uint4 *src = reinterpret_cast<const uint4 *>(row + c0);
+    const int nvec = gm.nvec;
+    const int wv0 = gm.wv0, wv1 = gm.wv1;
+    const uint4 *src = gm.src();
     const WarpStream ws{sm, src, wv0, wv1 - wv0, (wv1 - wv0 + kRowsStageVecs - 1) / kRowsStageVecs,
                         warp, lane, ph, a.status};
     if (tid == 0) {
@@ -601,12 +690,14 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
         sm.overflow = 0;
         sm.fmin = 0xFFFFFFFFu;
     }
-    ws.prologue();  // the first stages are in flight while F is found
+    if (!pre) gm.prefetch(sm, warp, lane, ph, a.status);  // the first stages load while F is found
+    pre = false;
 
     // ---- threshold F from a spread sample of the chunk ----
     uint32_t fkey = 0u;  // 0: keep every element
-    if (nvec >= kRowsThreads && n > kRowsKeepAll) {
-        const uint4 sx = __ldg(src + static_cast<int64_t>(tid) * nvec / kRowsThreads);
+    asm volatile("cp.async.wait_all;" ::: "memory");  // my sample vector has landed
+    if (gm.sampled()) {
+        const uint4 sx = sm.samp[tid];
         // Samples above the row's k-th largest value: about
         // lam = k * m / len; F is the r-th largest sample with r a few
         // standard deviations above lam.
@@ -644,8 +735,9 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
     {
         uint32_t *cb = sm.cand_bits[warp];
         int32_t *cc = sm.cand_col[warp];
-        uint32_t wcnt = 0, lost = 0, mag = 0;
+        uint32_t wcnt = 0, lost = 0, smx = Tr::kSmaxInit, umx = 0u;
         bool over = false;
+        const uint32_t fm1 = Tr::fm1_of(DT == FTK_BF16 ? (fraw & 0xFFFFu) : fraw);
         auto append = [&](uint32_t msk, const uint4 &x, int col0) {
             const uint32_t c = __popc(msk);
             const uint32_t incl = warp_incl_scan(c);
@@ -669,9 +761,11 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
         ws.run([&](const uint4 &x, bool valid, int v) {
             bool hit = false;
             if (valid) {
-                mag = Tr::mag_max(mag, x);
+                const uint32_t vs = Tr::vsmax(x);
+                smx = Tr::smax(smx, vs);
+                umx = Tr::umax(umx, Tr::vumax(x));
                 if (fpos) {
-                    hit = Tr::any_ge_pos(x, fraw);
+                    hit = Tr::ge_from_smax(vs, fm1);
                 } else {
 #pragma unroll
                     for (int j = 0; j < VEC; ++j) hit |= Tr::key(Tr::element(x, j)) >= fkey;
@@ -706,7 +800,7 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
                 append(hit ? 1u : 0u, make_uint4(bits, 0u, 0u, 0u), e - 0);
             }
         }
-        if (Tr::mag_has_nan(mag) || tail_nan) sm.nan_seen = 1;
+        if (Tr::nan_from(smx, umx) || tail_nan) sm.nan_seen = 1;
         lost = __reduce_add_sync(0xFFFFFFFFu, lost);
         over = __any_sync(0xFFFFFFFFu, over);
         if (lane == 0) {
@@ -715,6 +809,15 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
             if (over) sm.overflow = 1;
         }
     }
+    // One CTA per row: the rings are idle from here on, so the next row's
+    // first stages and sample load while this row's candidates are selected.
+    const bool has_next = cs == 1 && rnext >= 0;
+    const RowGeom<DT> gn(a, has_next ? rnext : r, rank, warp);
+    bool pre_next = false;
+    if (has_next && gn.len > k) {
+        gn.prefetch(sm, warp, lane, ph, a.status);
+        pre_next = true;
+    }
     __syncthreads();
     if (tid == 0) {
         sm.cta_fkey = fkey;
@@ -722,21 +825,25 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
     }
     cluster.sync();  // every candidate list of the cluster is final from here on
 
-    // ---- the cluster's lists, in column order ----
+    // ---- the cluster's lists in column order, and the common threshold ----
+    // Fu = the largest F of the cluster.  Every CTA stored all of its
+    // elements > Fu (its own F is <= Fu); its elements == Fu are stored or,
+    // only where its F == Fu, counted as ties past a full list.
     const int nl = static_cast<int>(cs) * kRowsWarps;
     if (warp == 0) {
-        uint32_t cnt[2], lst[2], fk[2], ov = 0, fmax = 0;
+        uint32_t cnt[2], ov = 0, fmax = 0;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const int L = lane + 32 * h;
-            cnt[h] = lst[h] = fk[h] = 0;
+            cnt[h] = 0;
             if (L < nl) {
                 const RowsSmem *o = cluster.map_shared_rank(&sm, static_cast<unsigned>(L / kRowsWarps));
                 cnt[h] = o->w_cnt[L % kRowsWarps];
-                lst[h] = o->w_lost[L % kRowsWarps];
-                fk[h] = o->cta_fkey;
+                const uint32_t fk = o->cta_fkey;
                 ov |= o->cta_over;
-                fmax = max(fmax, fk[h]);
+                fmax = max(fmax, fk);
+                sm.l_cnt[L] = cnt[h];
+                sm.l_fkey[L] = fk;
             }
         }
         const uint32_t i0 = warp_incl_scan(cnt[0]);
@@ -745,168 +852,239 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const int L = lane + 32 * h;
-            if (L < nl) {
-                sm.l_off[L] = (h == 0 ? i0 : i1) - cnt[h];
-                sm.l_cnt[L] = cnt[h];
-                sm.l_lost[L] = lst[h];
-                sm.l_fkey[L] = fk[h];
-            }
+            if (L < nl) sm.l_off[L] = (h == 0 ? i0 : i1) - cnt[h];
         }
-        const uint32_t lost_all = __reduce_add_sync(0xFFFFFFFFu, lst[0] + lst[1]);
         ov = __reduce_or_sync(0xFFFFFFFFu, ov);
         fmax = __reduce_max_sync(0xFFFFFFFFu, fmax);
         if (lane == 31) sm.l_off[nl] = i1;
         if (lane == 0) {
-            sm.g_lost = lost_all;
             sm.g_over = ov;
             sm.g_fmax = fmax;
         }
     }
     __syncthreads();
+    const uint32_t fu = sm.g_fmax;
+    {
+        // My lists against Fu, published to the cluster.
+        const uint32_t cnt = sm.w_cnt[warp];
+        uint32_t g = 0, q = 0, mx = 0;
+        for (uint32_t i0 = 0; i0 < cnt; i0 += 32) {
+            const uint32_t i = i0 + lane;
+            const uint32_t u = i < cnt ? Tr::key(sm.cand_bits[warp][i]) : 0u;
+            g += __popc(__ballot_sync(0xFFFFFFFFu, i < cnt && u > fu));
+            q += __popc(__ballot_sync(0xFFFFFFFFu, i < cnt && u == fu));
+            mx = max(mx, u);
+        }
+        mx = __reduce_max_sync(0xFFFFFFFFu, mx);
+        if (lane == 0) {
+            sm.w_kmax[warp] = mx;
+            sm.w_gtf[warp] = g;
+            sm.w_eqs[warp] = q;
+            sm.w_eqf[warp] = q + (fkey == fu ? sm.w_lost[warp] : 0u);
+        }
+    }
+    cluster.sync();
+    if (warp == 0) {
+        uint32_t gsum = 0, esum = 0, kmax = 0;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int L = lane + 32 * h;
+            if (L < nl) {
+                const RowsSmem *o = cluster.map_shared_rank(&sm, static_cast<unsigned>(L / kRowsWarps));
+                kmax = max(kmax, o->w_kmax[L % kRowsWarps]);
+                const uint32_t g = o->w_gtf[L % kRowsWarps];
+                const uint32_t et = o->w_eqf[L % kRowsWarps];
+                sm.l_gt[L] = g;
+                sm.l_eq[L] = o->w_eqs[L % kRowsWarps];
+                sm.l_eqt[L] = et;
+                gsum += g;
+                esum += et;
+            }
+        }
+        gsum = __reduce_add_sync(0xFFFFFFFFu, gsum);
+        esum = __reduce_add_sync(0xFFFFFFFFu, esum);
+        kmax = __reduce_max_sync(0xFFFFFFFFu, kmax);
+        if (lane == 0) {
+            sm.g_gt = gsum;
+            sm.g_eqt = esum;
+            sm.g_kmax = kmax;
+        }
+    }
+    __syncthreads();
+    // At least topk elements >= Fu makes the k-th largest >= Fu, so the
+    // lists hold it and everything above it.  Fewer than topk elements > Fu
+    // make it equal to Fu: no selection is needed.
     const uint32_t total = sm.l_off[nl];
-    bool exact_ok = !sm.g_over && total <= static_cast<uint32_t>(kRowsGather) &&
-                    total + sm.g_lost >= static_cast<uint32_t>(k);
-    uint32_t ustar = 0, above = 0;
-    if (exact_ok) {
-        // Every CTA gathers all candidate keys of the cluster (the rings are
-        // free now) and finds u* locally: the same result in every CTA.
-        uint32_t *gath = reinterpret_cast<uint32_t *>(sm.ring);
-        uint32_t kmn = 0xFFFFFFFFu, kmx = 0u;
-        for (int L = warp; L < nl; L += kRowsWarps) {
-            const RowsSmem *o = cluster.map_shared_rank(&sm, static_cast<unsigned>(L / kRowsWarps));
-            const uint32_t *cb = o->cand_bits[L % kRowsWarps];
-            const uint32_t cnt = sm.l_cnt[L], off = sm.l_off[L];
-            for (uint32_t i0 = 0; i0 < cnt; i0 += 128) {
-                uint32_t v[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const uint32_t i = i0 + u * 32 + lane;
-                    v[u] = i < cnt ? cb[i] : 0u;
+    bool exact_ok = !sm.g_over && sm.g_gt + sm.g_eqt >= static_cast<uint32_t>(k);
+    uint32_t ustar = fu, above = sm.g_gt;
+    if (exact_ok && sm.g_gt >= static_cast<uint32_t>(k)) {
+        // u* > Fu: every CTA gathers all candidate keys of the cluster (the
+        // rings are free now) and radix-selects those > Fu locally: the same
+        // result in every CTA.
+        exact_ok = total <= static_cast<uint32_t>(kRowsGather);
+        if (exact_ok) {
+            // cs > 1: the keys gathered into the rings; cs == 1: my own lists
+            // in place (the rings hold the next row's first stages).
+            uint32_t *gath = reinterpret_cast<uint32_t *>(sm.ring);
+            auto for_keys = [&](auto &&fn) {  // fn(key, active) on every thread, uniformly
+                if (cs > 1) {
+                    for (uint32_t i0 = 0; i0 < total; i0 += kRowsThreads) {
+                        const uint32_t i = i0 + tid;
+                        fn(i < total ? gath[i] : 0u, i < total);
+                    }
+                } else {
+                    for (int w = 0; w < kRowsWarps; ++w) {
+                        const uint32_t cnt = sm.w_cnt[w];
+                        for (uint32_t i0 = 0; i0 < cnt; i0 += kRowsThreads) {
+                            const uint32_t i = i0 + tid;
+                            fn(i < cnt ? Tr::key(sm.cand_bits[w][i]) : 0u, i < cnt);
+                        }
+                    }
                 }
+            };
+            if (cs > 1) {
+                // Warp w gathers the lists (rr, w), rr < cs: entry f of its
+                // share is entry f - pf[rr] of list rr, pf[rr] <= f < pf[rr + 1];
+                // eight loads in flight per lane.
+                uint32_t pf[kRowsMaxCluster + 1];
+                pf[0] = 0;
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const uint32_t i = i0 + u * 32 + lane;
-                    if (i < cnt) {
-                        const uint32_t key = Tr::key(v[u]);
-                        gath[off + i] = key;
-                        kmn = min(kmn, key);
-                        kmx = max(kmx, key);
+                for (int rr = 0; rr < kRowsMaxCluster; ++rr)
+                    pf[rr + 1] = pf[rr] + (rr < static_cast<int>(cs) ? sm.l_cnt[rr * kRowsWarps + warp] : 0u);
+                const uint32_t mine = pf[kRowsMaxCluster];
+                for (uint32_t f0 = 0; f0 < mine; f0 += 32 * 8) {
+                    uint32_t v[8], dst[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const uint32_t f = f0 + 32 * u + lane;
+                        v[u] = 0u;
+                        dst[u] = 0xFFFFFFFFu;
+                        if (f < mine) {
+                            int rr = 0;
+                            uint32_t base = 0;
+#pragma unroll
+                            for (int q = 1; q < kRowsMaxCluster; ++q)
+                                if (f >= pf[q]) {
+                                    rr = q;
+                                    base = pf[q];
+                                }
+                            const uint32_t *cb =
+                                cluster.map_shared_rank(&sm.cand_bits[warp][0], static_cast<unsigned>(rr));
+                            v[u] = cb[f - base];
+                            dst[u] = sm.l_off[rr * kRowsWarps + warp] + (f - base);
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        if (dst[u] != 0xFFFFFFFFu) gath[dst[u]] = Tr::key(v[u]);
+                }
+                __syncthreads();
+            }
+            const uint32_t kmx = sm.g_kmax;
+            // Keys > Fu lie in [Fu + one step, kmx]: bits above the highest
+            // one where those bounds differ are common to all of them, and
+            // the 11-bit radix digits start below those.
+            const int lo_bit = DT == FTK_BF16 ? 16 : 0;  // bf16 keys sit in the upper half
+            const uint32_t kmn = fu + (DT == FTK_BF16 ? 0x10000u : 1u);
+            const uint32_t diff = kmn ^ kmx;
+            const int top = diff ? 31 - __clz(diff) : -1;
+            uint32_t mask = top < 0 ? 0xFFFFFFFFu : (top == 31 ? 0u : ~((2u << top) - 1u));
+            uint32_t prefix = kmx & mask, krem = static_cast<uint32_t>(k);
+            above = 0;
+            bool found = true;
+            for (int hi = top; hi >= lo_bit && found; hi -= 11) {
+                const int shift = hi - 10 >= lo_bit ? hi - 10 : lo_bit;
+                const uint32_t dmask = (2u << (hi - shift)) - 1u;
+                for (int b = tid; b < kRowsBins; b += kRowsThreads) sm.hist[b] = 0;
+                __syncthreads();
+                for_keys([&](uint32_t u, bool act) {
+                    hist_add(sm.hist, (u >> shift) & dmask, act && u > fu && (u & mask) == prefix);
+                });
+                __syncthreads();
+                found = find_bin_top<kRowsBins>(sm, sm.hist, krem);
+                if (found) {
+                    prefix |= sm.sel_bin << shift;
+                    mask |= dmask << shift;
+                    krem -= sm.sel_above;
+                    above += sm.sel_above;
+                }
+            }
+            ustar = prefix;
+            exact_ok = found;
+            if (exact_ok) {
+                // Per list: keys > u* and keys == u* (all stored: u* > Fu).
+                for (int l = warp; l < nl; l += kRowsWarps) {
+                    const uint32_t cnt = sm.l_cnt[l], off = sm.l_off[l];
+                    uint32_t g = 0, q = 0;
+                    for (uint32_t i0 = 0; i0 < cnt; i0 += 32) {
+                        const uint32_t i = i0 + lane;
+                        const uint32_t u = i >= cnt ? 0u : cs > 1 ? gath[off + i] : Tr::key(sm.cand_bits[l][i]);
+                        g += __popc(__ballot_sync(0xFFFFFFFFu, i < cnt && u > ustar));
+                        q += __popc(__ballot_sync(0xFFFFFFFFu, i < cnt && u == ustar));
+                    }
+                    if (lane == 0) {
+                        sm.l_gt[l] = g;
+                        sm.l_eq[l] = q;
+                        sm.l_eqt[l] = q;
                     }
                 }
             }
-        }
-        if (tid < nl && sm.l_lost[tid]) {  // uncounted ties at F take part too
-            kmn = min(kmn, sm.l_fkey[tid]);
-            kmx = max(kmx, sm.l_fkey[tid]);
-        }
-        kmn = __reduce_min_sync(0xFFFFFFFFu, kmn);
-        kmx = __reduce_max_sync(0xFFFFFFFFu, kmx);
-        if (lane == 0) {
-            sm.red[warp] = kmn;
-            sm.red[kRowsWarps + warp] = kmx;
         }
         __syncthreads();
+    }
+    if (exact_ok) {
+        // In column order, each list's share of the ties at u* and its first
+        // output slot.
+        if (warp == 0) {
+            const uint32_t need = static_cast<uint32_t>(k) - above;  // ties at u* to take, >= 1
+            uint32_t eqt[2], sel[2], take[2];
+            bool shrt = false;
 #pragma unroll
-        for (int w = 0; w < kRowsWarps; ++w) {
-            kmn = min(kmn, sm.red[w]);
-            kmx = max(kmx, sm.red[kRowsWarps + w]);
+            for (int h = 0; h < 2; ++h) {
+                const int L = lane + 32 * h;
+                eqt[h] = L < nl ? sm.l_eqt[L] : 0u;
+            }
+            const uint32_t e0 = warp_incl_scan(eqt[0]);
+            const uint32_t et = __shfl_sync(0xFFFFFFFFu, e0, 31);
+            const uint32_t e1 = warp_incl_scan(eqt[1]) + et;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int L = lane + 32 * h;
+                const uint32_t eb = (h == 0 ? e0 : e1) - eqt[h];  // ties before list L
+                take[h] = eb >= need ? 0u : min(eqt[h], need - eb);
+                sel[h] = 0;
+                if (L < nl) {
+                    shrt |= take[h] > sm.l_eq[L];  // needs ties it did not store
+                    sel[h] = sm.l_gt[L] + take[h];
+                }
+            }
+            const uint32_t s0 = warp_incl_scan(sel[0]);
+            const uint32_t st = __shfl_sync(0xFFFFFFFFu, s0, 31);
+            const uint32_t s1 = warp_incl_scan(sel[1]) + st;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int L = lane + 32 * h;
+                if (L < nl) {
+                    sm.l_take[L] = take[h];
+                    sm.l_selb[L] = (h == 0 ? s0 : s1) - sel[h];
+                }
+            }
+            shrt = __any_sync(0xFFFFFFFFu, shrt);
+            if (lane == 0) sm.short_eq = shrt ? 1u : 0u;
         }
-        // Bits above the highest one where the keys differ are common to
-        // all of them: the 11-bit radix digits start below those.
-        const int lo_bit = DT == FTK_BF16 ? 16 : 0;  // bf16 keys sit in the upper half
-        const uint32_t diff = kmn ^ kmx;
-        const int top = diff ? 31 - __clz(diff) : -1;
-        uint32_t mask = top < 0 ? 0xFFFFFFFFu : (top == 31 ? 0u : ~((2u << top) - 1u));
-        uint32_t prefix = kmx & mask, krem = static_cast<uint32_t>(k);
-        bool found = true;
-        for (int hi = top; hi >= lo_bit && found; hi -= 11) {
-            const int shift = hi - 10 >= lo_bit ? hi - 10 : lo_bit;
-            const uint32_t dmask = (2u << (hi - shift)) - 1u;
-            for (int b = tid; b < kRowsBins; b += kRowsThreads) sm.hist[b] = 0;
-            __syncthreads();
-            for (uint32_t i0 = 0; i0 < total; i0 += kRowsThreads) {
-                const uint32_t i = i0 + tid;
-                const uint32_t u = i < total ? gath[i] : 0u;
-                hist_add(sm.hist, (u >> shift) & dmask, i < total && (u & mask) == prefix);
-            }
-            if (tid < nl && sm.l_lost[tid] && (sm.l_fkey[tid] & mask) == prefix)
-                atomicAdd(&sm.hist[(sm.l_fkey[tid] >> shift) & dmask], sm.l_lost[tid]);
-            __syncthreads();
-            found = find_bin_top<kRowsBins>(sm, sm.hist, krem);
-            if (found) {
-                prefix |= sm.sel_bin << shift;
-                mask |= dmask << shift;
-                krem -= sm.sel_above;
-                above += sm.sel_above;
-            }
-        }
-        ustar = prefix;
-        // The candidates are exactly each chunk's elements >= its F (ties at
-        // F counted), so they hold every element >= u* iff u* >= every F.
-        exact_ok = found && ustar >= sm.g_fmax;
-        if (exact_ok) {
-            // Per list: keys > u* and stored keys == u*; then, in column
-            // order, each list's share of the ties and its first output slot.
-            for (int L = warp; L < nl; L += kRowsWarps) {
-                const uint32_t cnt = sm.l_cnt[L], off = sm.l_off[L];
-                uint32_t g = 0, q = 0;
-                for (uint32_t i0 = 0; i0 < cnt; i0 += 32) {
-                    const uint32_t i = i0 + lane;
-                    const uint32_t u = i < cnt ? gath[off + i] : 0u;
-                    g += __popc(__ballot_sync(0xFFFFFFFFu, i < cnt && u > ustar));
-                    q += __popc(__ballot_sync(0xFFFFFFFFu, i < cnt && u == ustar));
-                }
-                if (lane == 0) {
-                    sm.l_gt[L] = g;
-                    sm.l_eq[L] = q;
-                }
-            }
-            __syncthreads();
-            if (warp == 0) {
-                const uint32_t need = static_cast<uint32_t>(k) - above;  // ties at u* to take, >= 1
-                uint32_t eqt[2], sel[2], take[2];
-                bool shrt = false;
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int L = lane + 32 * h;
-                    eqt[h] = 0;
-                    if (L < nl) eqt[h] = sm.l_eq[L] + (sm.l_fkey[L] == ustar ? sm.l_lost[L] : 0u);
-                }
-                const uint32_t e0 = warp_incl_scan(eqt[0]);
-                const uint32_t et = __shfl_sync(0xFFFFFFFFu, e0, 31);
-                const uint32_t e1 = warp_incl_scan(eqt[1]) + et;
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int L = lane + 32 * h;
-                    const uint32_t eb = (h == 0 ? e0 : e1) - eqt[h];  // ties before list L
-                    take[h] = eb >= need ? 0u : min(eqt[h], need - eb);
-                    sel[h] = 0;
-                    if (L < nl) {
-                        shrt |= take[h] > sm.l_eq[L];  // needs ties it did not store
-                        sel[h] = sm.l_gt[L] + take[h];
-                    }
-                }
-                const uint32_t s0 = warp_incl_scan(sel[0]);
-                const uint32_t st = __shfl_sync(0xFFFFFFFFu, s0, 31);
-                const uint32_t s1 = warp_incl_scan(sel[1]) + st;
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int L = lane + 32 * h;
-                    if (L < nl) {
-                        sm.l_take[L] = take[h];
-                        sm.l_selb[L] = (h == 0 ? s0 : s1) - sel[h];
-                    }
-                }
-                shrt = __any_sync(0xFFFFFFFFu, shrt);
-                if (lane == 0) sm.short_eq = shrt ? 1u : 0u;
-            }
-            __syncthreads();
-            exact_ok = sm.short_eq == 0;
-        }
+        __syncthreads();
+        exact_ok = sm.short_eq == 0;
     }
     // exact_ok is uniform over the cluster: every CTA decided it from the
     // same published lists.
     if (!exact_ok) {
+        if (pre_next) {  // the fallback streams through the rings again
+            const WarpStream wn{sm, gn.src(), gn.wv0, gn.wv1 - gn.wv0,
+                                (gn.wv1 - gn.wv0 + kRowsStageVecs - 1) / kRowsStageVecs, warp, lane, ph, a.status};
+            wn.drain();
+            asm volatile("cp.async.wait_all;" ::: "memory");
+            pre_next = false;
+        }
         __syncthreads();
         rows_fallback<DT, IT>(a, sm, cluster, cs, rank, row, c0, n, base_index, oidx, oval, ph);
     } else {
@@ -948,6 +1126,7 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
     fence_proxy_async();  // generic writes of the rings precede later bulk copies into them
     __syncwarp();
     cluster_wait();  // keep my shared memory alive until every CTA is done with it
+    pre = pre_next;
 }
 
 // One cluster per row.  LOOP: clusters stride over the rows (the count may
@@ -974,13 +1153,15 @@ __global__ void __launch_bounds__(kRowsThreads, 2) rows_topk_kernel(const RowsAr
         fence_barrier_init();
     }
     __syncthreads();
-    uint32_t ph = 0;  // parity each stage barrier of my warp waits for next
+    uint32_t ph = 0;   // parity each stage barrier of my warp waits for next
+    bool pre = false;  // the row's first stages and sample were issued already
     // Row selection is uniform over the cluster: its CTAs walk the same rows.
     if constexpr (!LOOP) {
-        rows_topk_row<DT, IT>(a, sm, cluster, cs, rank, blockIdx.x / cs, ph);
+        rows_topk_row<DT, IT>(a, sm, cluster, cs, rank, blockIdx.x / cs, ph, pre, -1);
     } else {
-        for (int64_t r = blockIdx.x / cs; r < nrows; r += gridDim.x / cs) {
-            rows_topk_row<DT, IT>(a, sm, cluster, cs, rank, r, ph);
+        const int64_t step = gridDim.x / cs;
+        for (int64_t r = blockIdx.x / cs; r < nrows; r += step) {
+            rows_topk_row<DT, IT>(a, sm, cluster, cs, rank, r, ph, pre, r + step < nrows ? r + step : -1);
             __syncthreads();  // shared memory is free for the next row
         }
     }

@@ -304,7 +304,9 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const ThreshArgs
         return;
     }
     const float *row = p.samp + t * p.sld;
-    // Eight loads in flight per thread, then the conversions.
+    // Eight loads in flight per thread, then the conversions; the bounds of
+    // the keys let the radix passes skip their common leading bits.
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
     for (int i0 = 0; i0 < J; i0 += 8 * kSelThreads) {
         uint32_t v[8];
 #pragma unroll
@@ -315,12 +317,29 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const ThreshArgs
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int i = i0 + j * kSelThreads + threadIdx.x;
-            if (i < J) tkeys[i] = f32_key(v[j]);
+            if (i < J) {
+                const uint32_t u = f32_key(v[j]);
+                tkeys[i] = u;
+                kmin = min(kmin, u);
+                kmax = max(kmax, u);
+            }
         }
     }
+    kmin = __reduce_min_sync(0xFFFFFFFFu, kmin);
+    kmax = __reduce_max_sync(0xFFFFFFFFu, kmax);
+    if ((threadIdx.x & 31) == 0) {
+        ss.red[threadIdx.x >> 5] = kmin;
+        ss.red[32 + (threadIdx.x >> 5)] = kmax;
+    }
     __syncthreads();
+    for (int w = 0; w < kSelThreads / 32; ++w) {
+        kmin = min(kmin, ss.red[w]);
+        kmax = max(kmax, ss.red[32 + w]);
+    }
+    __syncthreads();  // ss.red is free again
     uint32_t gt;
-    const uint32_t u = block_kth_largest(J, static_cast<uint32_t>(r), [&](int i) { return tkeys[i]; }, ss, &gt);
+    const uint32_t u = block_kth_largest(J, static_cast<uint32_t>(r), [&](int i) { return tkeys[i]; }, ss, &gt,
+                                         kmin, kmax);
     if (threadIdx.x == 0) p.tau[t] = __uint_as_float(f32_from_key(u));
 }
 
