@@ -145,16 +145,17 @@ struct RowsTraits<FTK_BF16> {
     // minus one in both halves.
     __device__ static bool ge_from_smax(uint32_t m, uint32_t fm1) { return smax(m, fm1) != fm1; }
     __device__ static uint32_t fm1_of(uint32_t fraw16) { return (fraw16 - 1u) * 0x10001u; }
-    // Bit j set for each element j >= F (strictly positive F, raw bits in
-    // both halves of f2).
-    __device__ static uint32_t ge_mask_pos(const uint4 &v, uint32_t f2)
+    // Bit j set for each element j >= F (strictly positive F; fm1 as for
+    // ge_from_smax).
+    __device__ static uint32_t ge_mask_pos(const uint4 &v, uint32_t fm1)
     {
         uint32_t m = 0;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const uint32_t w = i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
-            const uint32_t c = __vcmpges2(w, f2);  // 0xFFFF per matching half
-            m |= ((c & 1u) | ((c >> 15) & 2u)) << (2 * i);
+            const uint32_t d = smax(w, fm1) ^ fm1;  // a half is non-zero iff it is >= F
+            m |= ((d & 0xFFFFu) ? 1u : 0u) << (2 * i);
+            m |= ((d >> 16) ? 2u : 0u) << (2 * i);
         }
         return m;
     }
@@ -192,11 +193,11 @@ struct RowsTraits<FTK_F32> {
         return static_cast<int32_t>(m) > static_cast<int32_t>(fm1);
     }
     __device__ static uint32_t fm1_of(uint32_t fraw) { return fraw - 1u; }
-    __device__ static uint32_t ge_mask_pos(const uint4 &v, uint32_t f)
+    __device__ static uint32_t ge_mask_pos(const uint4 &v, uint32_t fm1)
     {
-        const int32_t fi = static_cast<int32_t>(f);
-        return (static_cast<int32_t>(v.x) >= fi ? 1u : 0u) | (static_cast<int32_t>(v.y) >= fi ? 2u : 0u) |
-               (static_cast<int32_t>(v.z) >= fi ? 4u : 0u) | (static_cast<int32_t>(v.w) >= fi ? 8u : 0u);
+        const int32_t fi = static_cast<int32_t>(fm1);
+        return (static_cast<int32_t>(v.x) > fi ? 1u : 0u) | (static_cast<int32_t>(v.y) > fi ? 2u : 0u) |
+               (static_cast<int32_t>(v.z) > fi ? 4u : 0u) | (static_cast<int32_t>(v.w) > fi ? 8u : 0u);
     }
     __device__ static bool nan_from(uint32_t s, uint32_t u)
     {
@@ -360,6 +361,15 @@ struct WarpStream {
     template <typename Visit>
     __device__ __forceinline__ bool run(Visit &&visit) const
     {
+        return run(visit, [](const uint4 *, int) {});
+    }
+
+    // end(buf, vb) runs on every lane after the stage's vectors were
+    // visited and before the stage is refilled (buf: the stage, vb: the
+    // index of its first vector).
+    template <typename Visit, typename End>
+    __device__ __forceinline__ bool run(Visit &&visit, End &&end) const
+    {
         bool ok = true;
         int issued = min(kRowsStages, nst);
         for (int j = 0; j < issued; ++j) {
@@ -378,6 +388,7 @@ struct WarpStream {
                     const uint4 x = valid ? buf[i] : make_uint4(0u, 0u, 0u, 0u);
                     visit(x, valid, vb + i);
                 }
+                end(buf, vb);
             }
             __syncwarp();
             if (ok && j + kRowsStages < nst) {
@@ -758,33 +769,54 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
             }
             wcnt += __shfl_sync(0xFFFFFFFFu, incl, 31);
         };
-        ws.run([&](const uint4 &x, bool valid, int v) {
-            bool hit = false;
-            if (valid) {
-                const uint32_t vs = Tr::vsmax(x);
-                smx = Tr::smax(smx, vs);
-                umx = Tr::umax(umx, Tr::vumax(x));
-                if (fpos) {
-                    hit = Tr::ge_from_smax(vs, fm1);
-                } else {
-#pragma unroll
-                    for (int j = 0; j < VEC; ++j) hit |= Tr::key(Tr::element(x, j)) >= fkey;
-                }
-            }
-            if (__ballot_sync(0xFFFFFFFFu, hit)) {
-                uint32_t msk = 0;
-                if (hit) {
+        // A vector with an element >= F is rare, but with 32 lanes some lane
+        // has one in most iterations: the stage's hit vectors are noted (their
+        // index in the stage, in column order) and appended once per stage,
+        // before the stage is refilled.  The notes use the histogram's space,
+        // idle while the row streams.
+        uint32_t *note = sm.hist + warp * kRowsStageVecs;
+        uint32_t nhit = 0;  // warp-uniform
+        ws.run(
+            [&](const uint4 &x, bool valid, int v) {
+                bool hit = false;
+                if (valid) {
+                    const uint32_t vs = Tr::vsmax(x);
+                    smx = Tr::smax(smx, vs);
+                    umx = Tr::umax(umx, Tr::vumax(x));
                     if (fpos) {
-                        msk = Tr::ge_mask_pos(x, fraw);
+                        hit = Tr::ge_from_smax(vs, fm1);
                     } else {
 #pragma unroll
-                        for (int j = 0; j < VEC; ++j)
-                            if (Tr::key(Tr::element(x, j)) >= fkey) msk |= 1u << j;
+                        for (int j = 0; j < VEC; ++j) hit |= Tr::key(Tr::element(x, j)) >= fkey;
                     }
                 }
-                append(msk, x, v * VEC);
-            }
-        });
+                const uint32_t bal = __ballot_sync(0xFFFFFFFFu, hit);
+                if (hit) note[nhit + __popc(bal & lt_mask)] = static_cast<uint32_t>(v - wv0) % kRowsStageVecs;
+                nhit += __popc(bal);
+            },
+            [&](const uint4 *buf, int vb) {
+                __syncwarp();  // the notes are visible to every lane
+                for (uint32_t h0 = 0; h0 < nhit; h0 += 32) {
+                    const uint32_t h = h0 + lane;
+                    uint32_t msk = 0;
+                    uint4 x = make_uint4(0u, 0u, 0u, 0u);
+                    int i = 0;
+                    if (h < nhit) {
+                        i = static_cast<int>(note[h]);
+                        x = buf[i];
+                        if (fpos) {
+                            msk = Tr::ge_mask_pos(x, fm1);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < VEC; ++j)
+                                if (Tr::key(Tr::element(x, j)) >= fkey) msk |= 1u << j;
+                        }
+                    }
+                    append(msk, x, (vb + i) * VEC);
+                }
+                nhit = 0;
+                __syncwarp();  // every note is read before the next stage writes them
+            });
         // ragged tail (n not a multiple of VEC): the last warp, in order
         bool tail_nan = false;
         if (warp == kRowsWarps - 1) {
