@@ -75,8 +75,10 @@ typedef struct {
     int32_t capacity;    /* C: candidate slots per row (0: 2*topk) */
     int32_t prune;       /* score-bound key pruning (FlashTopK README, "Highlights":
                           * adaptive key pruning by a score bound): 0 auto, the
-                          * default (estimate the skippable share of key blocks on
-                          * a sample and prune if it is >= 25%), 1 always, -1 off */
+                          * default (for calls of at least 128 query rows,
+                          * estimate the skippable share of key blocks on a
+                          * sample and prune if it is >= 25%; smaller calls scan
+                          * densely), 1 always, -1 off */
     int32_t recovery_rows; /* rows rescored densely per recovery pass (0: auto) */
     int32_t heads;         /* indexer heads H: 32 (or 0, the default) or 64 (FlashTopK
                             * README, "Roadmap": other head counts such as 64); q is then

@@ -16,13 +16,14 @@
 //      rare elements >= F go, in column order, to the warp's candidate list
 //      in shared memory.  Elements equal to F that find the list full are
 //      only counted (heavy ties);
-//   4. exact k-th key u*: with Fu the cluster's largest F, every list holds
-//      all of its chunk's elements > Fu and its elements == Fu are stored
-//      or counted.  If at least topk elements are >= Fu, the k-th largest is
-//      >= Fu: when fewer than topk are > Fu it is Fu itself (heavy ties need
-//      no selection), otherwise every CTA gathers all candidate keys of the
-//      cluster through distributed shared memory and radix-selects those
-//      > Fu locally (11-bit digits);
+//   4. exact k-th key u*: the cluster filters with one F (the largest of
+//      its CTAs' estimates, exchanged while the first stages load), so every
+//      list holds all of its chunk's elements > F and its elements == F are
+//      stored or counted.  If at least topk elements are >= F, the k-th
+//      largest is >= F: when fewer than topk are > F it is F itself (heavy
+//      ties need no selection), otherwise every CTA gathers all candidate
+//      keys of the cluster through distributed shared memory and
+//      radix-selects those > F locally (11-bit digits);
 //   5. output: the counts of each list (> u*, == u*) give every warp its
 //      output slots; ties at u* go to the smallest columns (CTA order, then
 //      warp order, then list order), written in ascending column order.
@@ -86,14 +87,13 @@ struct RowsSmem {
     uint64_t full[kRowsWarps][kRowsStages];               // one mbarrier per ring stage
     // this CTA's lists, read by the other CTAs of the cluster
     uint32_t w_cnt[kRowsWarps];    // stored entries
-    uint32_t w_lost[kRowsWarps];   // entries equal to F past the end of a full list
-    uint32_t w_gtf[kRowsWarps];    // stored entries > Fu (the cluster's largest F)
-    uint32_t w_eqs[kRowsWarps];    // stored entries == Fu
-    uint32_t w_eqf[kRowsWarps];    // entries == Fu, stored or counted
+    uint32_t w_gtf[kRowsWarps];    // stored entries > F
+    uint32_t w_eqs[kRowsWarps];    // stored entries == F
+    uint32_t w_eqf[kRowsWarps];    // entries == F, stored or counted past the end of a full list
     uint32_t w_kmax[kRowsWarps];   // largest stored key
     uint32_t cta_fkey, cta_over, cta_gt, cta_eq;
     // every list of the cluster in column order (index rank * kRowsWarps + warp)
-    uint32_t l_off[kRowsLists + 1], l_cnt[kRowsLists], l_fkey[kRowsLists];
+    uint32_t l_off[kRowsLists + 1], l_cnt[kRowsLists];
     uint32_t l_gt[kRowsLists];     // entries > u*
     uint32_t l_eq[kRowsLists];     // stored entries == u*
     uint32_t l_eqt[kRowsLists];    // entries == u*, stored or counted
@@ -101,7 +101,7 @@ struct RowsSmem {
     uint32_t wsum[kRowsWarps];
     uint32_t red[2 * kRowsWarps];
     uint32_t sel_bin, sel_above, fmin, short_eq;
-    uint32_t g_gt, g_eqt, g_fmax, g_over, g_kmax;
+    uint32_t g_gt, g_eqt, g_over, g_kmax;
     uint32_t nan_seen, overflow;
 };
 
@@ -737,6 +737,19 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
             fkey = sm.fmin == 0xFFFFFFFFu ? 0u : sm.fmin;
         }
     }
+    if (cs > 1) {
+        // One threshold for the whole row: the largest F of the cluster
+        // (exchanged while the first stages are still in flight).  Every
+        // list then holds its chunk's elements >= F, ties at F stored or
+        // counted.
+        if (tid == 0) sm.cta_fkey = fkey;
+        cluster.sync();
+        if (lane < static_cast<int>(cs))
+            fkey = cluster.map_shared_rank(&sm, static_cast<unsigned>(lane))->cta_fkey;
+        else
+            fkey = 0u;
+        fkey = __reduce_max_sync(0xFFFFFFFFu, fkey);
+    }
     // A strictly positive F allows the packed raw-bits test.
     const bool fpos = fkey > 0x80000000u;
     const uint32_t fbits = f32_from_key(fkey);  // F as f32 bits (bf16: its top half)
@@ -747,6 +760,7 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
         uint32_t *cb = sm.cand_bits[warp];
         int32_t *cc = sm.cand_col[warp];
         uint32_t wcnt = 0, lost = 0, smx = Tr::kSmaxInit, umx = 0u;
+        uint32_t ngt = 0, neq = 0, kmx = 0u;  // stored entries > F and == F, largest key
         bool over = false;
         const uint32_t fm1 = Tr::fm1_of(DT == FTK_BF16 ? (fraw & 0xFFFFu) : fraw);
         auto append = [&](uint32_t msk, const uint4 &x, int col0) {
@@ -757,10 +771,14 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
                 const int j = __ffs(msk) - 1;
                 msk &= msk - 1u;
                 const uint32_t bits = Tr::element(x, j);
+                const uint32_t key = Tr::key(bits);
                 if (pos < static_cast<uint32_t>(kRowsCapWarp)) {
                     cb[pos] = bits;
                     cc[pos] = col0 + j;
-                } else if (Tr::key(bits) == fkey) {
+                    ngt += key > fkey ? 1u : 0u;
+                    neq += key == fkey ? 1u : 0u;
+                    kmx = max(kmx, key);
+                } else if (key == fkey) {
                     ++lost;  // a tie at F past the list's end: counted only
                 } else {
                     over = true;
@@ -834,10 +852,16 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
         }
         if (Tr::nan_from(smx, umx) || tail_nan) sm.nan_seen = 1;
         lost = __reduce_add_sync(0xFFFFFFFFu, lost);
+        ngt = __reduce_add_sync(0xFFFFFFFFu, ngt);
+        neq = __reduce_add_sync(0xFFFFFFFFu, neq);
+        kmx = __reduce_max_sync(0xFFFFFFFFu, kmx);
         over = __any_sync(0xFFFFFFFFu, over);
         if (lane == 0) {
             sm.w_cnt[warp] = min(wcnt, static_cast<uint32_t>(kRowsCapWarp));
-            sm.w_lost[warp] = lost;
+            sm.w_gtf[warp] = ngt;
+            sm.w_eqs[warp] = neq;
+            sm.w_eqf[warp] = neq + lost;
+            sm.w_kmax[warp] = kmx;
             if (over) sm.overflow = 1;
         }
     }
@@ -851,31 +875,31 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
         pre_next = true;
     }
     __syncthreads();
-    if (tid == 0) {
-        sm.cta_fkey = fkey;
-        sm.cta_over = sm.overflow;
-    }
+    if (tid == 0) sm.cta_over = sm.overflow;
     cluster.sync();  // every candidate list of the cluster is final from here on
 
-    // ---- the cluster's lists in column order, and the common threshold ----
-    // Fu = the largest F of the cluster.  Every CTA stored all of its
-    // elements > Fu (its own F is <= Fu); its elements == Fu are stored or,
-    // only where its F == Fu, counted as ties past a full list.
+    // ---- the cluster's lists in column order ----
     const int nl = static_cast<int>(cs) * kRowsWarps;
+    const uint32_t fu = fkey;
     if (warp == 0) {
-        uint32_t cnt[2], ov = 0, fmax = 0;
+        uint32_t cnt[2], ov = 0, gsum = 0, esum = 0, kmax = 0;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const int L = lane + 32 * h;
             cnt[h] = 0;
             if (L < nl) {
                 const RowsSmem *o = cluster.map_shared_rank(&sm, static_cast<unsigned>(L / kRowsWarps));
-                cnt[h] = o->w_cnt[L % kRowsWarps];
-                const uint32_t fk = o->cta_fkey;
-                ov |= o->cta_over;
-                fmax = max(fmax, fk);
+                const int w = L % kRowsWarps;
+                cnt[h] = o->w_cnt[w];
+                const uint32_t g = o->w_gtf[w], et = o->w_eqf[w];
                 sm.l_cnt[L] = cnt[h];
-                sm.l_fkey[L] = fk;
+                sm.l_gt[L] = g;
+                sm.l_eq[L] = o->w_eqs[w];
+                sm.l_eqt[L] = et;
+                gsum += g;
+                esum += et;
+                kmax = max(kmax, o->w_kmax[w]);
+                ov |= o->cta_over;
             }
         }
         const uint32_t i0 = warp_incl_scan(cnt[0]);
@@ -887,65 +911,21 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
             if (L < nl) sm.l_off[L] = (h == 0 ? i0 : i1) - cnt[h];
         }
         ov = __reduce_or_sync(0xFFFFFFFFu, ov);
-        fmax = __reduce_max_sync(0xFFFFFFFFu, fmax);
-        if (lane == 31) sm.l_off[nl] = i1;
-        if (lane == 0) {
-            sm.g_over = ov;
-            sm.g_fmax = fmax;
-        }
-    }
-    __syncthreads();
-    const uint32_t fu = sm.g_fmax;
-    {
-        // My lists against Fu, published to the cluster.
-        const uint32_t cnt = sm.w_cnt[warp];
-        uint32_t g = 0, q = 0, mx = 0;
-        for (uint32_t i0 = 0; i0 < cnt; i0 += 32) {
-            const uint32_t i = i0 + lane;
-            const uint32_t u = i < cnt ? Tr::key(sm.cand_bits[warp][i]) : 0u;
-            g += __popc(__ballot_sync(0xFFFFFFFFu, i < cnt && u > fu));
-            q += __popc(__ballot_sync(0xFFFFFFFFu, i < cnt && u == fu));
-            mx = max(mx, u);
-        }
-        mx = __reduce_max_sync(0xFFFFFFFFu, mx);
-        if (lane == 0) {
-            sm.w_kmax[warp] = mx;
-            sm.w_gtf[warp] = g;
-            sm.w_eqs[warp] = q;
-            sm.w_eqf[warp] = q + (fkey == fu ? sm.w_lost[warp] : 0u);
-        }
-    }
-    cluster.sync();
-    if (warp == 0) {
-        uint32_t gsum = 0, esum = 0, kmax = 0;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int L = lane + 32 * h;
-            if (L < nl) {
-                const RowsSmem *o = cluster.map_shared_rank(&sm, static_cast<unsigned>(L / kRowsWarps));
-                kmax = max(kmax, o->w_kmax[L % kRowsWarps]);
-                const uint32_t g = o->w_gtf[L % kRowsWarps];
-                const uint32_t et = o->w_eqf[L % kRowsWarps];
-                sm.l_gt[L] = g;
-                sm.l_eq[L] = o->w_eqs[L % kRowsWarps];
-                sm.l_eqt[L] = et;
-                gsum += g;
-                esum += et;
-            }
-        }
         gsum = __reduce_add_sync(0xFFFFFFFFu, gsum);
         esum = __reduce_add_sync(0xFFFFFFFFu, esum);
         kmax = __reduce_max_sync(0xFFFFFFFFu, kmax);
+        if (lane == 31) sm.l_off[nl] = i1;
         if (lane == 0) {
+            sm.g_over = ov;
             sm.g_gt = gsum;
             sm.g_eqt = esum;
             sm.g_kmax = kmax;
         }
     }
     __syncthreads();
-    // At least topk elements >= Fu makes the k-th largest >= Fu, so the
-    // lists hold it and everything above it.  Fewer than topk elements > Fu
-    // make it equal to Fu: no selection is needed.
+    // At least topk elements >= F makes the k-th largest >= F, so the
+    // lists hold it and everything above it.  Fewer than topk elements > F
+    // make it equal to F: no selection is needed.
     const uint32_t total = sm.l_off[nl];
     bool exact_ok = !sm.g_over && sm.g_gt + sm.g_eqt >= static_cast<uint32_t>(k);
     uint32_t ustar = fu, above = sm.g_gt;

@@ -450,6 +450,18 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
+        if (MODE == MODE_SAMPLE && lane != 0 && a.kv_scales) {
+            // The idle lanes of the producer warp check a share of the
+            // scales, which must be > 0 and finite (FTK_STATUS_BAD_SCALE:
+            // the pruning's score bound assumes sigma > 0).
+            bool bad = false;
+            const int64_t stride = static_cast<int64_t>(gridDim.x) * 31;
+            for (int64_t i = static_cast<int64_t>(blockIdx.x) * 31 + (lane - 1); i < a.S; i += stride) {
+                const float sg = __ldg(a.kv_scales + i);
+                bad |= !(sg > 0.f) || isinf(sg);
+            }
+            if (bad) set_status(a.status, FTK_STATUS_BAD_SCALE);
+        }
         if (lane == 0) {
             tma_prefetch_desc(&tm_q);
             int ks_ = 0;
@@ -677,7 +689,10 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                     }
                 }
                 const bool skip = pruned && tile_pruned(a, m, kt);  // warp-uniform
-                bad_scale |= !skip && scales && kidx < m.kend && (!(sigma > 0.f) || isinf(sigma));
+                // (The sample pass validates every scale; the dense dump
+                // checks the ones it reads.)
+                if (MODE == MODE_DUMP)
+                    bad_scale |= !skip && scales && kidx < m.kend && (!(sigma > 0.f) || isinf(sigma));
                 const int32_t s = MODE == MODE_SAMPLE ? (kidx << m.lg) : kidx;
                 if (!skip) {
 #pragma unroll

@@ -304,9 +304,7 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const ThreshArgs
         return;
     }
     const float *row = p.samp + t * p.sld;
-    // Eight loads in flight per thread, then the conversions; the bounds of
-    // the keys let the radix passes skip their common leading bits.
-    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+    // Eight loads in flight per thread, then the conversions.
     for (int i0 = 0; i0 < J; i0 += 8 * kSelThreads) {
         uint32_t v[8];
 #pragma unroll
@@ -317,29 +315,12 @@ __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const ThreshArgs
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int i = i0 + j * kSelThreads + threadIdx.x;
-            if (i < J) {
-                const uint32_t u = f32_key(v[j]);
-                tkeys[i] = u;
-                kmin = min(kmin, u);
-                kmax = max(kmax, u);
-            }
+            if (i < J) tkeys[i] = f32_key(v[j]);
         }
     }
-    kmin = __reduce_min_sync(0xFFFFFFFFu, kmin);
-    kmax = __reduce_max_sync(0xFFFFFFFFu, kmax);
-    if ((threadIdx.x & 31) == 0) {
-        ss.red[threadIdx.x >> 5] = kmin;
-        ss.red[32 + (threadIdx.x >> 5)] = kmax;
-    }
     __syncthreads();
-    for (int w = 0; w < kSelThreads / 32; ++w) {
-        kmin = min(kmin, ss.red[w]);
-        kmax = max(kmax, ss.red[32 + w]);
-    }
-    __syncthreads();  // ss.red is free again
     uint32_t gt;
-    const uint32_t u = block_kth_largest(J, static_cast<uint32_t>(r), [&](int i) { return tkeys[i]; }, ss, &gt,
-                                         kmin, kmax);
+    const uint32_t u = block_kth_largest(J, static_cast<uint32_t>(r), [&](int i) { return tkeys[i]; }, ss, &gt);
     if (threadIdx.x == 0) p.tau[t] = __uint_as_float(f32_from_key(u));
 }
 
@@ -602,6 +583,7 @@ static int num_sms()
 }
 
 enum PruneMode { PRUNE_AUTO = 0, PRUNE_ON = 1, PRUNE_OFF = 2 };
+constexpr int64_t kAutoPruneRows = 128;
 
 struct SelectCfg {
     int heads;      // 32 or 64
@@ -626,6 +608,11 @@ static SelectCfg resolve_cfg(int64_t T, int64_t S, int topk, const ftk_config *c
     if (r.cap > 2 * FTK_MAX_TOPK) r.cap = 2 * FTK_MAX_TOPK;
     const int pr = c ? c->prune : 0;
     r.prune = pr == 0 ? PRUNE_AUTO : pr > 0 ? PRUNE_ON : PRUNE_OFF;
+    // The automatic decision needs its sampled estimate, and the bound's
+    // fixed cost (the box of every key block) pays only over enough query
+    // rows: calls of fewer than kAutoPruneRows rows scan densely unless
+    // pruning is asked for.
+    if (r.prune == PRUNE_AUTO && T < kAutoPruneRows) r.prune = PRUNE_OFF;
     // Strides are powers of two up to 2^(kNumStrideMaps - 1).
     const int64_t min_m = (S + (int64_t(1) << (kNumStrideMaps - 1)) - 1) >> (kNumStrideMaps - 1);
     if (r.m < min_m) r.m = static_cast<int>(min_m);
@@ -875,7 +862,7 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
     // every SM about twice.
     {
         const int64_t pairs = static_cast<int64_t>(ntiles) * ((S + kKeyTile - 1) / kKeyTile);
-        int64_t ct = pairs / (2 * static_cast<int64_t>(sms));
+        int64_t ct = (pairs + 2 * static_cast<int64_t>(sms) - 1) / (2 * static_cast<int64_t>(sms));
         ct = ct < kMinChunkTiles ? kMinChunkTiles : (ct > kChunkTiles ? kChunkTiles : ct);
         pa.chunk_keys = static_cast<int32_t>(ct * kKeyTile);
         // The sample pass has one item per row tile; with fewer row tiles

@@ -107,7 +107,7 @@ def test_block_bound_64_heads_matches_oracle(dtype):
     assert (np.abs(ub - oub) / scale).max() <= 1e-5
 
 
-@pytest.mark.parametrize("dtype,T,S,topk", [("fp8", 70, 9000, 128), ("bf16", 29, 5000, 64)])
+@pytest.mark.parametrize("dtype,T,S,topk", [("fp8", 150, 9000, 128), ("bf16", 133, 5000, 64)])
 def test_pruning_64_heads_fires_and_changes_nothing(dtype, T, S, topk):
     c = wl.block_structured(seed=42, dtype=dtype, T=T, S=S, topk=topk, heads=64)
     idx, val, info, worst, overlaps = check_case(c)

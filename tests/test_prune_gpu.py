@@ -52,7 +52,7 @@ def _same(a, b):
     return np.array_equal(a[0], b[0]) and np.array_equal(a[1].view(np.int32), b[1].view(np.int32))
 
 
-@pytest.mark.parametrize("dtype,T,S,topk", [("fp8", 70, 9000, 128), ("bf16", 29, 5000, 64)])
+@pytest.mark.parametrize("dtype,T,S,topk", [("fp8", 150, 9000, 128), ("bf16", 133, 5000, 64)])
 def test_pruning_fires_on_block_structured_keys(dtype, T, S, topk):
     c = wl.block_structured(seed=53, dtype=dtype, T=T, S=S, topk=topk)
     idx, val, info, worst, overlaps = check_case(c)
@@ -80,7 +80,7 @@ def _expected_blocks_total(c, rt):
 
 @pytest.mark.parametrize("dtype", ["fp8", "bf16"])
 def test_pruning_declines_on_normal_keys(dtype):
-    c = wl.small_case(seed=54, dtype=dtype, T=45, S=6000, topk=100, windows="causal")
+    c = wl.small_case(seed=54, dtype=dtype, T=140, S=6000, topk=100, windows="causal")
     idx, val, info, worst, overlaps = check_case(c)
     assert info["prune_enabled"] == 0 and info["blocks_pruned"] == 0, info
     assert info["blocks_total"] == _expected_blocks_total(c, 16 if dtype == "fp8" else 8)
