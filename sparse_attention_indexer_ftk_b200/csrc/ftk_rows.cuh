@@ -243,7 +243,9 @@ __device__ __forceinline__ bool find_bin_top(RowsSmem &sm, const uint32_t *h, ui
 {
     constexpr int B = NB / kRowsThreads;
     static_assert(B >= 1 && B * kRowsThreads == NB, "bins per thread");
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // (the warp index through a shuffle: provably warp-uniform, so per-warp
+    // addresses stay in uniform registers)
+    const int tid = threadIdx.x, lane = tid & 31, warp = __shfl_sync(0xFFFFFFFFu, tid >> 5, 0);
     uint32_t c[B], sum = 0;
 #pragma unroll
     for (int i = 0; i < B; ++i) {
@@ -431,7 +433,9 @@ __device__ __noinline__ void rows_fallback(const RowsArgs &a, RowsSmem &sm, cg::
     using Tr = RowsTraits<DT>;
     using elem = typename Tr::elem;
     constexpr int VEC = Tr::kVec;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // (the warp index through a shuffle: provably warp-uniform, so per-warp
+    // addresses stay in uniform registers)
+    const int tid = threadIdx.x, lane = tid & 31, warp = __shfl_sync(0xFFFFFFFFu, tid >> 5, 0);
     const int k = a.k;
     const int nvec = n / VEC;
     const int per = (nvec + kRowsWarps - 1) / kRowsWarps;
@@ -660,7 +664,9 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
     using Tr = RowsTraits<DT>;
     using elem = typename Tr::elem;
     constexpr int VEC = Tr::kVec;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // (the warp index through a shuffle: provably warp-uniform, so per-warp
+    // addresses stay in uniform registers)
+    const int tid = threadIdx.x, lane = tid & 31, warp = __shfl_sync(0xFFFFFFFFu, tid >> 5, 0);
     const uint32_t lt_mask = (1u << lane) - 1u;
     const RowGeom<DT> gm(a, r, rank, warp);
     const int64_t orow = gm.orow, len = gm.len, base_index = gm.base_index, c0 = gm.c0;
@@ -765,6 +771,30 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
         const uint32_t fm1 = Tr::fm1_of(DT == FTK_BF16 ? (fraw & 0xFFFFu) : fraw);
         auto append = [&](uint32_t msk, const uint4 &x, int col0) {
             const uint32_t c = __popc(msk);
+            const uint32_t one = __ballot_sync(0xFFFFFFFFu, c == 1u);
+            if (__all_sync(0xFFFFFFFFu, c <= 1u)) {
+                // The common case: at most one element per lane, its slot
+                // from one ballot.
+                const uint32_t pos = wcnt + __popc(one & lt_mask);
+                if (c) {
+                    const int j = __ffs(msk) - 1;
+                    const uint32_t bits = Tr::element(x, j);
+                    const uint32_t key = Tr::key(bits);
+                    if (pos < static_cast<uint32_t>(kRowsCapWarp)) {
+                        cb[pos] = bits;
+                        cc[pos] = col0 + j;
+                        ngt += key > fkey ? 1u : 0u;
+                        neq += key == fkey ? 1u : 0u;
+                        kmx = max(kmx, key);
+                    } else if (key == fkey) {
+                        ++lost;
+                    } else {
+                        over = true;
+                    }
+                }
+                wcnt += __popc(one);
+                return;
+            }
             const uint32_t incl = warp_incl_scan(c);
             uint32_t pos = wcnt + incl - c;
             while (msk) {  // the set bits, in column order
@@ -944,13 +974,11 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
                         const uint32_t i = i0 + tid;
                         fn(i < total ? gath[i] : 0u, i < total);
                     }
-                } else {
-                    for (int w = 0; w < kRowsWarps; ++w) {
-                        const uint32_t cnt = sm.w_cnt[w];
-                        for (uint32_t i0 = 0; i0 < cnt; i0 += kRowsThreads) {
-                            const uint32_t i = i0 + tid;
-                            fn(i < cnt ? Tr::key(sm.cand_bits[w][i]) : 0u, i < cnt);
-                        }
+                } else {  // every warp its own list
+                    const uint32_t cnt = sm.w_cnt[warp];
+                    for (uint32_t i0 = 0; i0 < cnt; i0 += 32) {
+                        const uint32_t i = i0 + lane;
+                        fn(i < cnt ? Tr::key(sm.cand_bits[warp][i]) : 0u, i < cnt);
                     }
                 }
             };
@@ -1106,32 +1134,37 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
         const int L = static_cast<int>(rank) * kRowsWarps + warp;
         const uint32_t cnt = sm.w_cnt[warp], take = sm.l_take[L];
         uint32_t pos = sm.l_selb[L], eq_rank = 0;
-        for (uint32_t i0 = 0; i0 < cnt; i0 += 32) {
-            const uint32_t i = i0 + lane;
-            uint32_t bits = 0;
-            int col = 0;
-            bool gt = false, eq = false;
-            if (i < cnt) {
-                bits = sm.cand_bits[warp][i];
-                col = sm.cand_col[warp][i];
-                const uint32_t u = Tr::key(bits);
-                gt = u > ustar;
-                eq = u == ustar;
+        for (uint32_t i0 = 0; i0 < cnt; i0 += 4 * 32) {
+            // four rounds of the list's entries read first (loads overlap)
+            uint32_t bits[4];
+            int col[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const uint32_t i = i0 + 32 * u + lane;
+                bits[u] = i < cnt ? sm.cand_bits[warp][i] : 0u;
+                col[u] = i < cnt ? sm.cand_col[warp][i] : 0;
             }
-            const uint32_t eq_bal = __ballot_sync(0xFFFFFFFFu, eq);
-            const bool sel = gt || (eq && eq_rank + __popc(eq_bal & lt_mask) < take);
-            const uint32_t sel_bal = __ballot_sync(0xFFFFFFFFu, sel);
-            if (sel) {
-                const uint32_t p = pos + __popc(sel_bal & lt_mask);
-                if (p < static_cast<uint32_t>(k)) {
-                    oidx[p] = static_cast<IT>(static_cast<int32_t>(base_index + c0 + col));
-                    if (oval) oval[p] = static_cast<elem>(bits);
-                } else {
-                    set_status(a.status, FTK_STATUS_INTERNAL);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const uint32_t i = i0 + 32 * u + lane;
+                const uint32_t key = Tr::key(bits[u]);
+                const bool gt = i < cnt && key > ustar;
+                const bool eq = i < cnt && key == ustar;
+                const uint32_t eq_bal = __ballot_sync(0xFFFFFFFFu, eq);
+                const bool sel = gt || (eq && eq_rank + __popc(eq_bal & lt_mask) < take);
+                const uint32_t sel_bal = __ballot_sync(0xFFFFFFFFu, sel);
+                if (sel) {
+                    const uint32_t p = pos + __popc(sel_bal & lt_mask);
+                    if (p < static_cast<uint32_t>(k)) {
+                        oidx[p] = static_cast<IT>(static_cast<int32_t>(base_index + c0 + col[u]));
+                        if (oval) oval[p] = static_cast<elem>(bits[u]);
+                    } else {
+                        set_status(a.status, FTK_STATUS_INTERNAL);
+                    }
                 }
+                pos += __popc(sel_bal);
+                eq_rank += __popc(eq_bal);
             }
-            pos += __popc(sel_bal);
-            eq_rank += __popc(eq_bal);
         }
     }
     if (tid == 0 && sm.nan_seen) set_status(a.status, FTK_STATUS_NAN);

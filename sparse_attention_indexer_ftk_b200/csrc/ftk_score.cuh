@@ -417,7 +417,10 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     ScoreMisc &ms = *reinterpret_cast<ScoreMisc *>(smem + Lay::kOffMisc);
     volatile int *abort = &ms.abort;
 
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // The warp index through a shuffle from lane 0 is provably uniform over
+    // the warp, so the values derived from it (role branches, TMEM
+    // addresses) stay in uniform registers.
+    const int warp = __shfl_sync(0xFFFFFFFFu, static_cast<int>(threadIdx.x >> 5), 0), lane = threadIdx.x & 31;
     const int64_t nlist = list_rows(a);
     if (nlist <= 0) return;  // e.g. a recovery pass with no rows left: no TMEM, no barriers
     const Sched sc = make_sched<MODE, RT>(a, nlist);

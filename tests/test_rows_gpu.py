@@ -64,6 +64,26 @@ def test_random_rows(dtype, rows, cols, k):
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("rows,cols,k", [(3, 131072, 512), (4, 40000, 2048), (600, 5000, 100)])
+def test_structured_rows(dtype, rows, cols, k):
+    """Rows whose largest values crowd one part of the row (sorted
+    descending, sorted ascending, one hot block): the sampled threshold
+    misses the k-th value or a candidate list overflows, and the exact
+    fallback gives the oracle's result.  With 600 rows (one CTA per row,
+    the next row's stages already in flight) the fallback first drains
+    them."""
+    g = torch.Generator().manual_seed(rows + cols + k)
+    x = torch.randn((rows, cols), generator=g)
+    for r in range(0, rows, 3):
+        x[r] = torch.sort(x[r], descending=True).values
+    for r in range(1, rows, 3):
+        x[r] = torch.sort(x[r]).values
+    for r in range(2, rows, 3):
+        x[r, (r * 97) % (cols // 2): (r * 97) % (cols // 2) + cols // 8] += 6.0
+    assert run_and_compare(x.to(dtype), k) == 0
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 def test_heavy_ties_and_signed_zero(dtype):
     g = torch.Generator().manual_seed(5)
     x = torch.randint(-2, 3, (8, 20000), generator=g).float() * 0.5
