@@ -35,6 +35,7 @@
 #pragma once
 
 #include <cooperative_groups.h>
+#include <type_traits>
 
 #include "ftk_device.cuh"
 
@@ -47,8 +48,8 @@ constexpr int kRowsWarps = kRowsThreads / 32;
 constexpr int kRowsMaxCluster = 8;
 constexpr int kRowsLists = kRowsMaxCluster * kRowsWarps;  // candidate lists of a cluster
 constexpr int kRowsCapWarp = 512;      // candidates per warp list
-constexpr int kRowsStages = 4;         // ring stages per warp
-constexpr int kRowsStageVecs = 128;    // 16-byte vectors per stage (2 KB)
+constexpr int kRowsStages = 2;         // ring stages per warp
+constexpr int kRowsStageVecs = 256;    // 16-byte vectors per stage (4 KB)
 constexpr int kRowsGather = kRowsWarps * kRowsStages * kRowsStageVecs * 4;  // keys that fit the rings
 constexpr int kRowsBins = 2048;        // 11-bit digits
 constexpr int kRowsKeepAll = 4096;     // chunks of at most this many elements keep all of them
@@ -383,12 +384,24 @@ struct WarpStream {
                 const uint4 *buf = sm.ring[warp][s];
                 const int cnt = min(kRowsStageVecs, nv - j * kRowsStageVecs);
                 const int vb = wv0 + j * kRowsStageVecs;
+                // every vector of the stage read first (the loads overlap)
+                uint4 xs[kRowsStageVecs / 32];
+                if (cnt == kRowsStageVecs) {  // a full stage: every vector valid
 #pragma unroll
-                for (int it = 0; it < kRowsStageVecs / 32; ++it) {
-                    const int i = it * 32 + lane;
-                    const bool valid = i < cnt;
-                    const uint4 x = valid ? buf[i] : make_uint4(0u, 0u, 0u, 0u);
-                    visit(x, valid, vb + i);
+                    for (int it = 0; it < kRowsStageVecs / 32; ++it) xs[it] = buf[it * 32 + lane];
+#pragma unroll
+                    for (int it = 0; it < kRowsStageVecs / 32; ++it) visit(xs[it], true, vb + it * 32 + lane);
+                } else {  // the chunk's last, partial stage
+#pragma unroll
+                    for (int it = 0; it < kRowsStageVecs / 32; ++it) {
+                        const int i = it * 32 + lane;
+                        xs[it] = i < cnt ? buf[i] : make_uint4(0u, 0u, 0u, 0u);
+                    }
+#pragma unroll
+                    for (int it = 0; it < kRowsStageVecs / 32; ++it) {
+                        const int i = it * 32 + lane;
+                        visit(xs[it], i < cnt, vb + i);
+                    }
                 }
                 end(buf, vb);
             }
@@ -766,105 +779,126 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
         uint32_t *cb = sm.cand_bits[warp];
         int32_t *cc = sm.cand_col[warp];
         uint32_t wcnt = 0, lost = 0, smx = Tr::kSmaxInit, umx = 0u;
-        uint32_t ngt = 0, neq = 0, kmx = 0u;  // stored entries > F and == F, largest key
         bool over = false;
         const uint32_t fm1 = Tr::fm1_of(DT == FTK_BF16 ? (fraw & 0xFFFFu) : fraw);
-        auto append = [&](uint32_t msk, const uint4 &x, int col0) {
-            const uint32_t c = __popc(msk);
-            const uint32_t one = __ballot_sync(0xFFFFFFFFu, c == 1u);
-            if (__all_sync(0xFFFFFFFFu, c <= 1u)) {
-                // The common case: at most one element per lane, its slot
-                // from one ballot.
-                const uint32_t pos = wcnt + __popc(one & lt_mask);
-                if (c) {
-                    const int j = __ffs(msk) - 1;
-                    const uint32_t bits = Tr::element(x, j);
-                    const uint32_t key = Tr::key(bits);
-                    if (pos < static_cast<uint32_t>(kRowsCapWarp)) {
-                        cb[pos] = bits;
-                        cc[pos] = col0 + j;
-                        ngt += key > fkey ? 1u : 0u;
-                        neq += key == fkey ? 1u : 0u;
-                        kmx = max(kmx, key);
-                    } else if (key == fkey) {
-                        ++lost;
-                    } else {
-                        over = true;
-                    }
-                }
-                wcnt += __popc(one);
-                return;
+        // Element `bits` (column col) at list position pos; past the list's
+        // end a tie at F is only counted, anything else is an overflow.
+        auto put = [&](uint32_t pos, uint32_t bits, int col) {
+            if (pos < static_cast<uint32_t>(kRowsCapWarp)) {
+                cb[pos] = bits;
+                cc[pos] = col;
+            } else if (Tr::key(bits) == fkey) {
+                ++lost;
+            } else {
+                over = true;
             }
-            const uint32_t incl = warp_incl_scan(c);
-            uint32_t pos = wcnt + incl - c;
-            while (msk) {  // the set bits, in column order
-                const int j = __ffs(msk) - 1;
-                msk &= msk - 1u;
-                const uint32_t bits = Tr::element(x, j);
-                const uint32_t key = Tr::key(bits);
-                if (pos < static_cast<uint32_t>(kRowsCapWarp)) {
-                    cb[pos] = bits;
-                    cc[pos] = col0 + j;
-                    ngt += key > fkey ? 1u : 0u;
-                    neq += key == fkey ? 1u : 0u;
-                    kmx = max(kmx, key);
-                } else if (key == fkey) {
-                    ++lost;  // a tie at F past the list's end: counted only
-                } else {
-                    over = true;
+        };
+        // The warp-exclusive prefix and the total of the lanes' counts c <=
+        // VEC, from one ballot per bit of c (independent, not a shuffle
+        // chain); two ballots when every count is below 4.
+        auto offsets = [&](uint32_t c, uint32_t &pre, uint32_t &tot) {
+            pre = 0;
+            tot = 0;
+            const int nb = __all_sync(0xFFFFFFFFu, c < 4u) ? 2 : (VEC == 8 ? 4 : 3);
+#pragma unroll
+            for (int bt = 0; bt < 4; ++bt) {
+                if (bt < nb) {
+                    const uint32_t bb = __ballot_sync(0xFFFFFFFFu, (c >> bt) & 1u);
+                    pre += static_cast<uint32_t>(__popc(bb & lt_mask)) << bt;
+                    tot += static_cast<uint32_t>(__popc(bb)) << bt;
                 }
-                ++pos;
             }
-            wcnt += __shfl_sync(0xFFFFFFFFu, incl, 31);
+        };
+        // Elements >= F of a vector, as a bit mask.
+        auto ge_mask = [&](const uint4 &x) {
+            if (fpos) return Tr::ge_mask_pos(x, fm1);
+            uint32_t m = 0;
+#pragma unroll
+            for (int j = 0; j < VEC; ++j)
+                if (Tr::key(Tr::element(x, j)) >= fkey) m |= 1u << j;
+            return m;
         };
         // A vector with an element >= F is rare, but with 32 lanes some lane
         // has one in most iterations: the stage's hit vectors are noted (their
         // index in the stage, in column order) and appended once per stage,
-        // before the stage is refilled.  The notes use the histogram's space,
+        // 32 at a time, before the stage is refilled; each element is read
+        // from the stage where it lies.  The notes use the histogram's space,
         // idle while the row streams.
         uint32_t *note = sm.hist + warp * kRowsStageVecs;
         uint32_t nhit = 0;  // warp-uniform
-        ws.run(
-            [&](const uint4 &x, bool valid, int v) {
-                bool hit = false;
-                if (valid) {
-                    const uint32_t vs = Tr::vsmax(x);
-                    smx = Tr::smax(smx, vs);
-                    umx = Tr::umax(umx, Tr::vumax(x));
-                    if (fpos) {
-                        hit = Tr::ge_from_smax(vs, fm1);
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < VEC; ++j) hit |= Tr::key(Tr::element(x, j)) >= fkey;
-                    }
+        auto append_noted = [&](const uint4 *buf, int vb) {
+            __syncwarp();  // the notes are visible to every lane
+            for (uint32_t h0 = 0; h0 < nhit; h0 += 32) {
+                const uint32_t h = h0 + lane;
+                uint32_t msk = 0;
+                int i = 0;
+                if (h < nhit) {
+                    i = static_cast<int>(note[h]);
+                    msk = ge_mask(buf[i]);
                 }
-                const uint32_t bal = __ballot_sync(0xFFFFFFFFu, hit);
-                if (hit) note[nhit + __popc(bal & lt_mask)] = static_cast<uint32_t>(v - wv0) % kRowsStageVecs;
-                nhit += __popc(bal);
-            },
-            [&](const uint4 *buf, int vb) {
-                __syncwarp();  // the notes are visible to every lane
-                for (uint32_t h0 = 0; h0 < nhit; h0 += 32) {
-                    const uint32_t h = h0 + lane;
-                    uint32_t msk = 0;
-                    uint4 x = make_uint4(0u, 0u, 0u, 0u);
-                    int i = 0;
-                    if (h < nhit) {
-                        i = static_cast<int>(note[h]);
-                        x = buf[i];
-                        if (fpos) {
-                            msk = Tr::ge_mask_pos(x, fm1);
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < VEC; ++j)
-                                if (Tr::key(Tr::element(x, j)) >= fkey) msk |= 1u << j;
+                const elem *ev = reinterpret_cast<const elem *>(buf + i);
+                const int col0 = (vb + i) * VEC;
+                const uint32_t c = __popc(msk);
+                if (__all_sync(0xFFFFFFFFu, c <= 2u)) {
+                    // The common case: at most two elements per lane.  When
+                    // the list has room for all of them, they are stored
+                    // without a loop or a capacity check.
+                    const uint32_t b1 = __ballot_sync(0xFFFFFFFFu, c == 1u);
+                    const uint32_t b2 = __ballot_sync(0xFFFFFFFFu, c == 2u);
+                    const uint32_t tot = __popc(b1) + 2u * __popc(b2);
+                    if (wcnt + tot <= static_cast<uint32_t>(kRowsCapWarp)) {
+                        if (c) {
+                            const uint32_t pos = wcnt + __popc(b1 & lt_mask) + 2u * __popc(b2 & lt_mask);
+                            const int j1 = __ffs(msk) - 1, j2 = 31 - __clz(msk);
+                            cb[pos] = static_cast<uint32_t>(ev[j1]);
+                            cc[pos] = col0 + j1;
+                            if (c == 2u) {
+                                cb[pos + 1] = static_cast<uint32_t>(ev[j2]);
+                                cc[pos + 1] = col0 + j2;
+                            }
                         }
+                        wcnt += tot;
+                        continue;
                     }
-                    append(msk, x, (vb + i) * VEC);
                 }
-                nhit = 0;
-                __syncwarp();  // every note is read before the next stage writes them
-            });
+                uint32_t pre, tot;
+                offsets(c, pre, tot);
+                uint32_t pos = wcnt + pre;
+                while (msk) {  // the set bits, in column order
+                    const int j = __ffs(msk) - 1;
+                    msk &= msk - 1u;
+                    put(pos++, static_cast<uint32_t>(ev[j]), col0 + j);
+                }
+                wcnt += tot;
+            }
+            nhit = 0;
+            __syncwarp();  // every note is read before the next stage writes them
+        };
+        // One vector: running maxima (for the NaN check) and the hit note.
+        // FP: F is strictly positive (packed raw-bits test); VALID: the
+        // vector lies in the chunk.
+        auto visit = [&](auto fp, const uint4 &x, bool valid, int v) {
+            constexpr bool FP = decltype(fp)::value;
+            bool hit = false;
+            if (valid) {
+                const uint32_t vs = Tr::vsmax(x);
+                smx = Tr::smax(smx, vs);
+                umx = Tr::umax(umx, Tr::vumax(x));
+                if constexpr (FP) {
+                    hit = Tr::ge_from_smax(vs, fm1);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < VEC; ++j) hit |= Tr::key(Tr::element(x, j)) >= fkey;
+                }
+            }
+            const uint32_t bal = __ballot_sync(0xFFFFFFFFu, hit);
+            if (hit) note[nhit + __popc(bal & lt_mask)] = static_cast<uint32_t>(v - wv0) % kRowsStageVecs;
+            nhit += __popc(bal);
+        };
+        if (fpos)
+            ws.run([&](const uint4 &x, bool valid, int v) { visit(std::true_type{}, x, valid, v); }, append_noted);
+        else
+            ws.run([&](const uint4 &x, bool valid, int v) { visit(std::false_type{}, x, valid, v); }, append_noted);
         // ragged tail (n not a multiple of VEC): the last warp, in order
         bool tail_nan = false;
         if (warp == kRowsWarps - 1) {
@@ -877,10 +911,25 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
                     tail_nan |= Tr::isnan_bits(bits);
                     hit = Tr::key(bits) >= fkey;
                 }
-                append(hit ? 1u : 0u, make_uint4(bits, 0u, 0u, 0u), e - 0);
+                const uint32_t bal = __ballot_sync(0xFFFFFFFFu, hit);
+                if (hit) put(wcnt + __popc(bal & lt_mask), bits, e);
+                wcnt += __popc(bal);
             }
         }
         if (Tr::nan_from(smx, umx) || tail_nan) sm.nan_seen = 1;
+        // The stored entries > F and == F, and the largest key, from the list.
+        uint32_t ngt = 0, neq = 0, kmx = 0u;
+        const uint32_t stored = min(wcnt, static_cast<uint32_t>(kRowsCapWarp));
+        __syncwarp();  // the list is visible to every lane
+        for (uint32_t i0 = 0; i0 < stored; i0 += 32) {
+            const uint32_t i = i0 + lane;
+            if (i < stored) {
+                const uint32_t key = Tr::key(cb[i]);
+                ngt += key > fkey ? 1u : 0u;
+                neq += key == fkey ? 1u : 0u;
+                kmx = max(kmx, key);
+            }
+        }
         lost = __reduce_add_sync(0xFFFFFFFFu, lost);
         ngt = __reduce_add_sync(0xFFFFFFFFu, ngt);
         neq = __reduce_add_sync(0xFFFFFFFFu, neq);
