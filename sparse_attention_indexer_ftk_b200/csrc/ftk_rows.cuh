@@ -106,6 +106,10 @@ struct RowsSmem {
     uint32_t nan_seen, overflow;
 };
 
+// The warps' stage notes tile the histogram exactly (each warp clears its
+// part after its stream).
+static_assert(kRowsWarps * kRowsStageVecs == kRowsBins && kRowsStageVecs % 128 == 0, "notes tile the histogram");
+
 template <int DT>
 struct RowsTraits;
 
@@ -499,6 +503,8 @@ __device__ __noinline__ void rows_fallback(const RowsArgs &a, RowsSmem &sm, cg::
     }
     const uint32_t ustar = prefix;
     const uint32_t need = static_cast<uint32_t>(k) - above;  // ties at u* to take, >= 1
+    // (the histogram is all zero again for the next row's sample)
+    for (int b = tid; b < 512; b += kRowsThreads) sm.hist[b] = 0;
 
     // ---- counts of > u* and == u* per warp segment ----
     uint32_t g = 0, q = 0;
@@ -734,9 +740,7 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
         const float m = static_cast<float>(kRowsThreads * VEC);
         const float lam = static_cast<float>(k) * m / static_cast<float>(len);
         const float rf = ceilf(lam + 4.f * sqrtf(lam) + 4.f);
-        if (rf < m) {
-            for (int b = tid; b < kRowsBins; b += kRowsThreads) sm.hist[b] = 0;
-            __syncthreads();
+        if (rf < m) {  // (the histogram is all zero here)
             uint32_t keys[VEC];
 #pragma unroll
             for (int j = 0; j < VEC; ++j) {
@@ -899,6 +903,12 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
             ws.run([&](const uint4 &x, bool valid, int v) { visit(std::true_type{}, x, valid, v); }, append_noted);
         else
             ws.run([&](const uint4 &x, bool valid, int v) { visit(std::false_type{}, x, valid, v); }, append_noted);
+        // The notes are done with: the warp's part of the histogram is
+        // cleared for the radix select (ordered by the barrier that follows
+        // the stream).
+#pragma unroll
+        for (int q = 0; q < kRowsStageVecs / 128; ++q)
+            reinterpret_cast<uint4 *>(note)[q * 32 + lane] = make_uint4(0u, 0u, 0u, 0u);
         // ragged tail (n not a multiple of VEC): the last warp, in order
         bool tail_nan = false;
         if (warp == kRowsWarps - 1) {
@@ -1081,16 +1091,19 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
             uint32_t prefix = kmx & mask, krem = static_cast<uint32_t>(k);
             above = 0;
             bool found = true;
+            // The histogram is all zero on entry to each pass (cleared after
+            // the stream, then after each pass: it is all zero again for the
+            // next row's sample).
             for (int hi = top; hi >= lo_bit && found; hi -= 11) {
                 const int shift = hi - 10 >= lo_bit ? hi - 10 : lo_bit;
                 const uint32_t dmask = (2u << (hi - shift)) - 1u;
-                for (int b = tid; b < kRowsBins; b += kRowsThreads) sm.hist[b] = 0;
-                __syncthreads();
+                if (hi != top) __syncthreads();  // the previous pass cleared it
                 for_keys([&](uint32_t u, bool act) {
                     hist_add(sm.hist, (u >> shift) & dmask, act && u > fu && (u & mask) == prefix);
                 });
                 __syncthreads();
                 found = find_bin_top<kRowsBins>(sm, sm.hist, krem);
+                for (int b = tid; b < kRowsBins; b += kRowsThreads) sm.hist[b] = 0;
                 if (found) {
                     prefix |= sm.sel_bin << shift;
                     mask |= dmask << shift;
@@ -1100,7 +1113,39 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
             }
             ustar = prefix;
             exact_ok = found;
-            if (exact_ok) {
+            if (exact_ok && cs == 1) {
+                // Per list (my own): keys > u* and keys == u* (all stored:
+                // u* > Fu).  The list is compacted in place, in column order,
+                // to those entries: the ordered output walks only them.
+                uint32_t *cb = sm.cand_bits[warp];
+                int32_t *cc = sm.cand_col[warp];
+                const uint32_t cnt = sm.w_cnt[warp];
+                uint32_t g = 0, q = 0;
+                for (uint32_t i0 = 0; i0 < cnt; i0 += 32) {
+                    const uint32_t i = i0 + lane;
+                    const uint32_t bits = i < cnt ? cb[i] : 0u;
+                    const int32_t col = i < cnt ? cc[i] : 0;
+                    const uint32_t u = Tr::key(bits);
+                    const bool gt = i < cnt && u > ustar, eq = i < cnt && u == ustar;
+                    const uint32_t kb = __ballot_sync(0xFFFFFFFFu, gt || eq);
+                    // (entries kept so far <= i0: the writes reach only
+                    // entries this round has read)
+                    __syncwarp();
+                    if (gt || eq) {
+                        const uint32_t p = g + q + __popc(kb & lt_mask);
+                        cb[p] = bits;
+                        cc[p] = col;
+                    }
+                    g += __popc(__ballot_sync(0xFFFFFFFFu, gt));
+                    q += __popc(__ballot_sync(0xFFFFFFFFu, eq));
+                }
+                if (lane == 0) {
+                    sm.l_gt[warp] = g;
+                    sm.l_eq[warp] = q;
+                    sm.l_eqt[warp] = q;
+                    sm.w_cnt[warp] = g + q;
+                }
+            } else if (exact_ok) {
                 // Per list: keys > u* and keys == u* (all stored: u* > Fu).
                 for (int l = warp; l < nl; l += kRowsWarps) {
                     const uint32_t cnt = sm.l_cnt[l], off = sm.l_off[l];
@@ -1246,6 +1291,8 @@ __global__ void __launch_bounds__(kRowsThreads, 2) rows_topk_kernel(const RowsAr
             for (int s = 0; s < kRowsStages; ++s) mbar_init(&sm.full[w][s], 1);
         fence_barrier_init();
     }
+    // The histogram is all zero on entry to each row (each row leaves it so).
+    for (int b = threadIdx.x; b < kRowsBins; b += kRowsThreads) sm.hist[b] = 0;
     __syncthreads();
     uint32_t ph = 0;   // parity each stage barrier of my warp waits for next
     bool pre = false;  // the row's first stages and sample were issued already
