@@ -228,6 +228,13 @@ __device__ __forceinline__ void hist_add(uint32_t *hist, uint32_t bin, bool acti
     }
 }
 
+// One atomic per active lane, no warp vote first: independent calls can
+// overlap (colliding lanes are serialised by the shared-memory unit).
+__device__ __forceinline__ void hist_add_plain(uint32_t *hist, uint32_t bin, bool active)
+{
+    if (active) atomicAdd(&hist[bin], 1u);
+}
+
 __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v)
 {
     const int lane = threadIdx.x & 31;
@@ -745,7 +752,7 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
 #pragma unroll
             for (int j = 0; j < VEC; ++j) {
                 keys[j] = Tr::key(Tr::element(sx, j));
-                hist_add(sm.hist, keys[j] >> 21, true);
+                hist_add_plain(sm.hist, keys[j] >> 21, true);
             }
             __syncthreads();
             find_bin_top<kRowsBins>(sm, sm.hist, static_cast<uint32_t>(rf));
@@ -1033,11 +1040,17 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
                         const uint32_t i = i0 + tid;
                         fn(i < total ? gath[i] : 0u, i < total);
                     }
-                } else {  // every warp its own list
+                } else {  // every warp its own list, four rounds read at a time
                     const uint32_t cnt = sm.w_cnt[warp];
-                    for (uint32_t i0 = 0; i0 < cnt; i0 += 32) {
-                        const uint32_t i = i0 + lane;
-                        fn(i < cnt ? Tr::key(sm.cand_bits[warp][i]) : 0u, i < cnt);
+                    for (uint32_t i0 = 0; i0 < cnt; i0 += 4 * 32) {
+                        uint32_t kv[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const uint32_t i = i0 + 32 * u + lane;
+                            kv[u] = i < cnt ? Tr::key(sm.cand_bits[warp][i]) : 0u;
+                        }
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) fn(kv[u], i0 + 32 * u + lane < cnt);
                     }
                 }
             };
@@ -1099,7 +1112,7 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
                 const uint32_t dmask = (2u << (hi - shift)) - 1u;
                 if (hi != top) __syncthreads();  // the previous pass cleared it
                 for_keys([&](uint32_t u, bool act) {
-                    hist_add(sm.hist, (u >> shift) & dmask, act && u > fu && (u & mask) == prefix);
+                    hist_add_plain(sm.hist, (u >> shift) & dmask, act && u > fu && (u & mask) == prefix);
                 });
                 __syncthreads();
                 found = find_bin_top<kRowsBins>(sm, sm.hist, krem);
