@@ -748,6 +748,14 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
         const float lam = static_cast<float>(k) * m / static_cast<float>(len);
         const float rf = ceilf(lam + 4.f * sqrtf(lam) + 4.f);
         if (rf < m) {  // (the histogram is all zero here)
+            // Two levels of 11-bit bins: the top bits of the keys, then the
+            // next bits of the keys in the first level's bin (bf16: the
+            // whole key, so F is the r-th largest sample itself; a coarse F
+            // would let in up to a quarter octave more candidates).  The
+            // second level's bins use the candidate lists' space, idle until
+            // the stream.
+            uint32_t *h2 = sm.cand_bits[0];
+            for (int b = tid; b < kRowsBins; b += kRowsThreads) h2[b] = 0;
             uint32_t keys[VEC];
 #pragma unroll
             for (int j = 0; j < VEC; ++j) {
@@ -757,10 +765,16 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
             __syncthreads();
             find_bin_top<kRowsBins>(sm, sm.hist, static_cast<uint32_t>(rf));
             const uint32_t b = sm.sel_bin;  // found: the counts sum to m > r
+            const uint32_t r2 = static_cast<uint32_t>(rf) - sm.sel_above;  // rank within bin b, >= 1
+#pragma unroll
+            for (int j = 0; j < VEC; ++j) hist_add_plain(h2, (keys[j] >> 10) & 0x7FFu, (keys[j] >> 21) == b);
+            __syncthreads();  // (also: every thread has read b before it is overwritten)
+            find_bin_top<kRowsBins>(sm, h2, r2);
+            const uint32_t b2 = sm.sel_bin;  // found: bin b holds >= r2 samples
             uint32_t mn = 0xFFFFFFFFu;
 #pragma unroll
             for (int j = 0; j < VEC; ++j)
-                if ((keys[j] >> 21) == b) mn = min(mn, keys[j]);
+                if ((keys[j] >> 21) == b && ((keys[j] >> 10) & 0x7FFu) == b2) mn = min(mn, keys[j]);
             mn = __reduce_min_sync(0xFFFFFFFFu, mn);
             if (lane == 0) atomicMin(&sm.fmin, mn);
             __syncthreads();
