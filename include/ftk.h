@@ -72,7 +72,7 @@ typedef enum {
 typedef struct {
     int32_t sample_keys; /* target strided-sample size per row, m (default 4096) */
     float oversample;    /* beta: the threshold keeps ~beta*topk keys (default 1.5) */
-    int32_t capacity;    /* C: candidate slots per row (0: 2*topk) */
+    int32_t capacity;    /* C: candidate slots per row (0: 5*topk/2, at most 2*FTK_MAX_TOPK) */
     int32_t prune;       /* score-bound key pruning (FlashTopK README, "Highlights":
                           * adaptive key pruning by a score bound): 0 auto, the
                           * default (for calls of at least 128 query rows,

@@ -604,7 +604,10 @@ static SelectCfg resolve_cfg(int64_t T, int64_t S, int topk, const ftk_config *c
     r.heads = c && c->heads == 64 ? 64 : 32;
     r.m = c && c->sample_keys > 0 ? c->sample_keys : 4096;
     r.beta = c && c->oversample > 0.f ? c->oversample : 1.5f;
-    r.cap = c && c->capacity > 0 ? c->capacity : 2 * topk;
+    // Default capacity 2.5 * topk: the candidate count of a row is about
+    // 1.5 * topk with a spread of a few percent, and a row past the
+    // capacity costs a dense recovery pass.
+    r.cap = c && c->capacity > 0 ? c->capacity : topk * 5 / 2;
     if (r.cap > 2 * FTK_MAX_TOPK) r.cap = 2 * FTK_MAX_TOPK;
     const int pr = c ? c->prune : 0;
     r.prune = pr == 0 ? PRUNE_AUTO : pr > 0 ? PRUNE_ON : PRUNE_OFF;
