@@ -367,6 +367,20 @@ def bench_rows(name: str, dev, reps: int = 64):
             "inputs": f"{ncopy} rotating copies (> L2) so every call reads from HBM"}
 
 
+def stage_breakdown(ftk, step, flush, n):
+    """Per-stage times of n more calls, each with an event recorded at every
+    stage boundary.  Separate from the timed calls: recording the events
+    costs device time of its own."""
+    import torch
+    evs = [ftk.stage_events() for _ in range(n)]
+    for i in range(n):
+        flush.zero_()
+        with evs[i]:
+            step()
+    torch.cuda.synchronize()
+    return [e.times_ms() for e in evs]
+
+
 def bench_decode(c, dev, rows: int = 64, reps: int = 50):
     """A decode-shaped call: the first `rows` query rows of the batch (each
     with its long causal window) through the same ftk_select, inputs in
@@ -387,21 +401,19 @@ def bench_decode(c, dev, rows: int = 64, reps: int = 50):
     for _ in range(3):
         step()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
-    stage_evs = [ftk.stage_events() for _ in range(reps)]
     for i in range(reps):
         flush.zero_()
-        with stage_evs[i]:
-            ev[i][0].record()
-            step()
-            ev[i][1].record()
+        ev[i][0].record()
+        step()
+        ev[i][1].record()
     torch.cuda.synchronize()
     ms = sum(a.elapsed_time(b) for a, b in ev) / reps
-    stages = [s.times_ms() for s in stage_evs]
+    stages = stage_breakdown(ftk, step, flush, min(reps, 10))
     info = ftk.read_info(ws)
     pairs = d.pairs()
     return {"workload": d.name, "T": d.T, "S": d.S, "topk": d.topk, "ms_per_call": ms,
             "queries_per_s": d.T / (ms * 1e-3), "dense_eq_tflops": 2.0 * 32 * 128 * pairs / (ms * 1e-3) / 1e12,
-            "stage_ms": {name: sum(s[name] for s in stages) / reps for name in stages[0]},
+            "stage_ms": {name: sum(s[name] for s in stages) / len(stages) for name in stages[0]},
             "kernel_launches": int(info["kernel_launches"]), "prune_enabled": info["prune_enabled"],
             "rows_recovered": info["rows_overflow"] + info["rows_underflow"]}
 
@@ -632,23 +644,21 @@ def _run_ours(args, pg, world, rank, local):
 
     K = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    stage_evs = [ftk.stage_events() for _ in range(K)]
     with ClockSampler(gpu_index(local)) as clk:
         barrier()
         torch.cuda.synchronize()
         for i in range(K):
             flush.zero_()  # evict the L2 between timed steps (outside the events)
-            with stage_evs[i]:
-                ev[i][0].record(stream)
-                step()
-                ev[i][1].record(stream)
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
         torch.cuda.synchronize()
         barrier()
     clocks = clk.summary()
     step_ms = [a.elapsed_time(b) for a, b in ev]
     mean_ms = sum(step_ms) / K
-    stages = [s.times_ms() for s in stage_evs]
-    stage_mean = {name: sum(s[name] for s in stages) / K for name in stages[0]}
+    stages = stage_breakdown(ftk, step, flush, min(K, 10))
+    stage_mean = {name: sum(s[name] for s in stages) / len(stages) for name in stages[0]}
     mean_ms = shard.max_over_ranks(mean_ms, dev)  # the step time is the slowest rank's
 
     # end to end through the public API: inputs from pinned host memory,

@@ -83,7 +83,11 @@ typedef struct {
     int32_t heads;         /* indexer heads H: 32 (or 0, the default) or 64 (FlashTopK
                             * README, "Roadmap": other head counts such as 64); q is then
                             * [T, H, 128] and weights [T, H]. */
-    int32_t reserved[2];   /* must be 0 */
+    int32_t dense_rows;    /* calls of at most this many query rows (and at most 2^25
+                            * (row, key) pairs) score every key of every window and
+                            * select with the row top-k instead of the sampled
+                            * threshold (0: 128, the default; -1: never) */
+    int32_t reserved;      /* must be 0 */
 } ftk_config;
 
 /* Per-call information (FlashTopK README, "Usage": last_info), filled on

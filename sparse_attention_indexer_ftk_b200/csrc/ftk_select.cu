@@ -70,6 +70,13 @@ struct PlanArgs {
     int32_t *bad_count;
     DevInfo *info;
     int64_t launches;
+    // dense calls: every row with a valid window goes to rows_out (the
+    // dense pass's row list, count in *bad_count); the others are padded
+    int32_t dense;
+    int32_t topk;
+    int32_t *rows_out;
+    int32_t *out_idx;
+    float *out_val;
 };
 
 __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *sh, uint32_t &total)
@@ -120,8 +127,44 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanArgs p)
         p.info->work_next = 0;
     }
     __syncthreads();
-    unsigned long long nblocks = 0;  // (row tile, key block) pairs of the scan
     if (bad) atomicOr(&p.info->info.status, FTK_STATUS_BAD_WINDOW);
+    if (p.dense) {
+        // The row list of the dense pass (valid windows, in row order); every
+        // key of a window counts as a candidate.
+        uint32_t carry = 0;
+        unsigned long long ltot = 0, lmax = 0;
+        for (int64_t base = 0; base < p.T; base += blockDim.x) {
+            const int64_t t = base + tid;
+            bool ok = false;
+            if (t < p.T) {
+                const int64_t a = p.ks[t], b = p.ke[t];
+                ok = window_ok(a, b, p.S);
+                if (ok) {
+                    ltot += static_cast<unsigned long long>(b - a);
+                    lmax = max(lmax, static_cast<unsigned long long>(b - a));
+                }
+            }
+            uint32_t tot;
+            const uint32_t e = block_excl_scan(ok ? 1u : 0u, sh, tot);
+            if (ok) p.rows_out[carry + e] = static_cast<int32_t>(t);
+            carry += tot;
+        }
+        if (ltot) atomicAdd(reinterpret_cast<unsigned long long *>(&p.info->info.candidates_total), ltot);
+        if (lmax) atomicMax(reinterpret_cast<unsigned long long *>(&p.info->info.candidates_max), lmax);
+        if (tid == 0) *p.bad_count = static_cast<int32_t>(carry);
+        // rows with an invalid window: all (-1, -inf)
+        if (__syncthreads_or(bad ? 1 : 0)) {
+            for (int64_t t = 0; t < p.T; ++t) {
+                if (window_ok(p.ks[t], p.ke[t], p.S)) continue;
+                for (int j = tid; j < p.topk; j += blockDim.x) {
+                    p.out_idx[t * p.topk + j] = -1;
+                    if (p.out_val) p.out_val[t * p.topk + j] = -INFINITY;
+                }
+            }
+        }
+        return;
+    }
+    unsigned long long nblocks = 0;  // (row tile, key block) pairs of the scan
     uint32_t carry_s = 0, carry_c = 0;
     for (int32_t base = 0; base < p.ntiles; base += blockDim.x) {
         const int32_t tile = base + tid;
@@ -584,6 +627,11 @@ static int num_sms()
 
 enum PruneMode { PRUNE_AUTO = 0, PRUNE_ON = 1, PRUNE_OFF = 2 };
 constexpr int64_t kAutoPruneRows = 128;
+// Calls of at most this many query rows (and at most 2^25 (row, key) pairs,
+// one recovery pass) take the dense path: the threshold machinery's fixed
+// stages cost more than scoring and selecting every key of a few rows.
+constexpr int64_t kDenseRows = 128;
+constexpr int64_t kDensePairs = int64_t(1) << 25;
 
 struct SelectCfg {
     int heads;      // 32 or 64
@@ -593,6 +641,7 @@ struct SelectCfg {
     PruneMode prune;
     int rec_rows;
     int64_t scratch_floats;  // recovery scratch reserved, >= rec_rows * scratch row stride
+    bool dense;              // score every key and select with the row top-k
 };
 
 // Row stride of the recovery scratch (floats): S rounded up to 8.
@@ -637,6 +686,8 @@ static SelectCfg resolve_cfg(int64_t T, int64_t S, int topk, const ftk_config *c
     if (budget > tcap * ld) budget = tcap * ld;
     r.scratch_floats = budget;
     r.rec_rows = static_cast<int>(budget / ld / kMaxRowTile * kMaxRowTile);
+    const int64_t dense_rows = !c || c->dense_rows == 0 ? kDenseRows : c->dense_rows < 0 ? 0 : c->dense_rows;
+    r.dense = T <= dense_rows && T * S <= kDensePairs && T <= r.rec_rows;
     return r;
 }
 
@@ -760,7 +811,7 @@ ftk_status check_select_call(int dtype, const void *q, const void *kv, const flo
                              const int32_t *ke, int64_t T, int64_t S, int topk, const int32_t *out_idx,
                              const ftk_config *config)
 {
-    if (config && (config->reserved[0] || config->reserved[1] ||
+    if (config && (config->reserved ||
                    (config->heads != 0 && config->heads != 32 && config->heads != 64)))
         return FTK_ERR_INVALID_ARG;
     const int heads = config && config->heads == 64 ? 64 : 32;
@@ -851,6 +902,49 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
     const int sms = num_sms();
     uint32_t *status = &w.info->info.status;
 
+    // The dense pass over the listed rows [b0, b0 + nrows) of w.bad_rows
+    // (count on the device): dense_scores writes every key's score of their
+    // windows into the scratch, dense_select takes each row's top-k from
+    // them (the row top-k kernel).
+    auto dense_scores = [&](int64_t b0, int nrows) -> ftk_status {
+        ScoreArgs da = {};
+        da.T = T;
+        da.S = S;
+        da.kv_scales = kv_scales;
+        da.weights = weights;
+        da.ks = ks;
+        da.ke = ke;
+        da.rows = w.bad_rows + b0;
+        da.nrows = nrows;
+        da.count_dev = w.bad_count;
+        da.count_off = static_cast<int32_t>(b0);
+        da.out = w.scratch;
+        da.ld = w.scratch_ld;
+        da.status = status;
+        return launch_score_dt<MODE_DUMP>(dtype, heads, da, tq, kvm, sms, s);
+    };
+    auto dense_select = [&](int64_t b0, int nrows, int rcluster, int rchunk) -> ftk_status {
+        RowsArgs ra2 = {};
+        ra2.x = w.scratch;
+        ra2.ld = w.scratch_ld;
+        ra2.cols = S;
+        ra2.rows = nrows;
+        ra2.nrows_dev = w.bad_count;
+        ra2.nrows_off = static_cast<int32_t>(b0);
+        ra2.row_map = w.bad_rows + b0;
+        ra2.win_ks = ks;
+        ra2.win_ke = ke;
+        ra2.out_idx = out_idx;
+        ra2.out_val = out_val;
+        ra2.ldo = topk;
+        ra2.idx_fill = -1;
+        ra2.val_fill = 0xFF800000u;  // -inf
+        ra2.k = topk;
+        ra2.chunk = rchunk;
+        ra2.status = status;
+        return launch_rows_topk(FTK_F32, ra2, rcluster, s);
+    };
+
     stage_mark(0, s);
     PlanArgs pa;
     pa.T = T;
@@ -890,6 +984,29 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
     pa.bad_count = w.bad_count;
     pa.info = w.info;
     pa.launches = 5 + 2 * ((T + c.rec_rows - 1) / c.rec_rows) + (c.prune == PRUNE_OFF ? 0 : c.prune == PRUNE_AUTO ? 4 : 2);
+    pa.dense = c.dense ? 1 : 0;
+    pa.topk = topk;
+    pa.rows_out = w.bad_rows;
+    pa.out_idx = out_idx;
+    pa.out_val = out_val;
+    if (c.dense) {
+        // Few query rows: one dense pass over every row (plan, dump, row
+        // top-k); the sample, threshold, scan and refine stages are skipped.
+        pa.launches = 3;
+        // (Stage marks: the dense scores stand in the scan's place, the row
+        // top-k in the refine's; the skipped stages take no time.)
+        plan_kernel<<<1, kPlanThreads, 0, s>>>(pa);
+        if ((st = cuda_status(cudaGetLastError())) != FTK_OK) return st;
+        for (int i : {1, 2, 3, 7}) stage_mark(i, s);
+        int rcluster = 1, rchunk = 8;
+        rows_plan(T, S, topk, &rcluster, &rchunk);
+        if ((st = dense_scores(0, static_cast<int>(T))) != FTK_OK) return st;
+        stage_mark(4, s);
+        if ((st = dense_select(0, static_cast<int>(T), rcluster, rchunk)) != FTK_OK) return st;
+        stage_mark(5, s);
+        stage_mark(6, s);
+        return FTK_OK;
+    }
     plan_kernel<<<1, kPlanThreads, 0, s>>>(pa);
     if ((st = cuda_status(cudaGetLastError())) != FTK_OK) return st;
     stage_mark(1, s);
@@ -1043,42 +1160,8 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
     int rcluster = 1, rchunk = 8;
     rows_plan(c.rec_rows < 16 ? c.rec_rows : 16, S, topk, &rcluster, &rchunk);
     for (int64_t b0 = 0; b0 < T; b0 += c.rec_rows) {
-        ScoreArgs da = {};
-        da.T = T;
-        da.S = S;
-        da.kv_scales = kv_scales;
-        da.weights = weights;
-        da.ks = ks;
-        da.ke = ke;
-        da.rows = w.bad_rows + b0;
-        da.nrows = c.rec_rows;
-        da.count_dev = w.bad_count;
-        da.count_off = static_cast<int32_t>(b0);
-        da.out = w.scratch;
-        da.ld = w.scratch_ld;
-        da.status = status;
-        st = launch_score_dt<MODE_DUMP>(dtype, heads, da, tq, kvm, sms, s);
-        if (st != FTK_OK) return st;
-        RowsArgs ra2 = {};
-        ra2.x = w.scratch;
-        ra2.ld = w.scratch_ld;
-        ra2.cols = S;
-        ra2.rows = c.rec_rows;
-        ra2.nrows_dev = w.bad_count;
-        ra2.nrows_off = static_cast<int32_t>(b0);
-        ra2.row_map = w.bad_rows + b0;
-        ra2.win_ks = ks;
-        ra2.win_ke = ke;
-        ra2.out_idx = out_idx;
-        ra2.out_val = out_val;
-        ra2.ldo = topk;
-        ra2.idx_fill = -1;
-        ra2.val_fill = 0xFF800000u;  // -inf
-        ra2.k = topk;
-        ra2.chunk = rchunk;
-        ra2.status = status;
-        st = launch_rows_topk(FTK_F32, ra2, rcluster, s);
-        if (st != FTK_OK) return st;
+        if ((st = dense_scores(b0, c.rec_rows)) != FTK_OK) return st;
+        if ((st = dense_select(b0, c.rec_rows, rcluster, rchunk)) != FTK_OK) return st;
     }
     stage_mark(6, s);
     return FTK_OK;

@@ -55,7 +55,7 @@ class FtkConfig(ctypes.Structure):
     _fields_ = [("sample_keys", ctypes.c_int32), ("oversample", ctypes.c_float),
                 ("capacity", ctypes.c_int32), ("prune", ctypes.c_int32),
                 ("recovery_rows", ctypes.c_int32), ("heads", ctypes.c_int32),
-                ("reserved", ctypes.c_int32 * 2)]
+                ("dense_rows", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 class FtkRowsOptions(ctypes.Structure):

@@ -191,7 +191,7 @@ def test_select_host_validation(lib):
     assert call(ws=P(A + 16)) == -5
     assert call(wsb=1000) == -5
     bad = ftk.FtkConfig()
-    bad.reserved[0] = 1
+    bad.reserved = 1
     assert call(cfg=ctypes.byref(bad)) == -1
 
 

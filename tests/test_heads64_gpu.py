@@ -37,8 +37,8 @@ def test_small_cases_64_heads(spec):
     assert worst < 1e-4
 
 
-@pytest.mark.parametrize("config", [dict(capacity=64), dict(oversample=0.05), dict(recovery_rows=8, capacity=64),
-                                    dict(prune=1)])
+@pytest.mark.parametrize("config", [dict(dense_rows=-1, capacity=64), dict(dense_rows=-1, oversample=0.05),
+                                    dict(dense_rows=-1, recovery_rows=8, capacity=64), dict(dense_rows=-1, prune=1)])
 def test_config_does_not_change_the_result_64_heads(config):
     c = wl.small_case(seed=37, dtype="fp8", T=29, S=9000, topk=64, windows="random", heads=64)
     g = gpu_inputs(c)

@@ -152,14 +152,17 @@ def test_all_equal_workload_closed_form():
 
 
 @pytest.mark.parametrize("config", [
-    dict(capacity=64),                 # every long row overflows -> dense recovery
-    dict(oversample=0.05),             # thresholds too high -> underflow -> recovery
-    dict(sample_keys=64),              # coarse samples
-    dict(recovery_rows=8, capacity=64),  # many recovery passes
-    dict(prune=-1),
-    dict(prune=1),
+    dict(dense_rows=-1),               # the sampled-threshold path (29 rows would go dense)
+    dict(dense_rows=-1, capacity=64),  # every long row overflows -> dense recovery
+    dict(dense_rows=-1, oversample=0.05),  # thresholds too high -> underflow -> recovery
+    dict(dense_rows=-1, sample_keys=64),   # coarse samples
+    dict(dense_rows=-1, recovery_rows=8, capacity=64),  # many recovery passes
+    dict(dense_rows=-1, prune=-1),
+    dict(dense_rows=-1, prune=1),
 ])
 def test_config_does_not_change_the_result(config):
+    """The reference run takes the default (dense) path for these 29 rows;
+    every config forces the sampled-threshold path: identical bits."""
     c = wl.small_case(seed=11, dtype="fp8", T=29, S=9000, topk=64, windows="random")
     g = gpu_inputs(c)
     ref_idx, ref_val, _ = run_select(g)
@@ -171,6 +174,24 @@ def test_config_does_not_change_the_result(config):
     if "oversample" in config:
         assert info["rows_underflow"] > 0
     check_case(c, config=config)
+
+
+@pytest.mark.parametrize("dtype,T,S,topk", [("fp8", 64, 40000, 512), ("bf16", 100, 20000, 256),
+                                           ("fp8", 7, 60000, 2048)])
+def test_dense_path_matches_threshold_path(dtype, T, S, topk):
+    """Calls of few query rows score every key and select with the row
+    top-k (three launches); forcing the sampled-threshold path gives the
+    same bits, and both match the oracle."""
+    c = wl.small_case(seed=T + S, dtype=dtype, T=T, S=S, topk=topk, windows="causal")
+    g = gpu_inputs(c)
+    d_idx, d_val, d_info = run_select(g)
+    t_idx, t_val, t_info = run_select(g, dict(dense_rows=-1))
+    assert d_info["kernel_launches"] == 3 and t_info["kernel_launches"] > 3
+    assert np.array_equal(d_idx, t_idx)
+    assert np.array_equal(d_val.view(np.uint32), t_val.view(np.uint32))
+    lens = (c.ke - c.ks).numpy().astype(np.int64)
+    assert d_info["candidates_total"] == int(lens.sum()) and d_info["candidates_max"] == int(lens.max())
+    check_case(c)
 
 
 def test_determinism():
