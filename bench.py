@@ -17,7 +17,8 @@ bf16 / fp32 batches and a 1024-row bf16 batch with a warm-L2 time and a
 trivial read-reduce over the same bytes, and the CPU oracle's rate.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--no-rows] [--only-rows] [--no-decode] [--no-cpu-baseline]
+                    [--no-rows] [--only-rows [--rows-workload NAME]] [--no-decode]
+                    [--no-cpu-baseline]
 
 Multi-GPU (launched with torch.distributed.run): every rank runs its own
 independent batch of the same shape (weak scaling; no data-path collective);
@@ -57,6 +58,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-rows", action="store_true", help="skip the row top-k section")
     ap.add_argument("--only-rows", action="store_true", help="run only the row top-k section")
+    ap.add_argument("--rows-workload", default="",
+                    help="with --only-rows: only this row workload (rows_bf16, rows_f32, rows_bf16_1024)")
     ap.add_argument("--no-decode", action="store_true", help="skip the 64-query (decode-shaped) section")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the decode-shaped, packed-workload and FP8 GEMM reference sections")
@@ -786,8 +789,9 @@ def main():
     if args.only_rows:
         import torch
         dev = torch.device("cuda")
-        print(json.dumps({"row_topk": [bench_rows("rows_bf16", dev), bench_rows("rows_f32", dev),
-                                       bench_rows("rows_bf16_1024", dev, reps=16)]}), flush=True)
+        names = [args.rows_workload] if args.rows_workload else ["rows_bf16", "rows_f32", "rows_bf16_1024"]
+        print(json.dumps({"row_topk": [bench_rows(n, dev, reps=16 if n == "rows_bf16_1024" else 64)
+                                       for n in names]}), flush=True)
         return
     if args.impl == "reference":
         run_reference(args)
