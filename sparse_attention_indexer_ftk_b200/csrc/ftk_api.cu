@@ -2,6 +2,8 @@
 // causal windows.
 #include <cudaTypedefs.h>
 
+#include <stdlib.h>
+
 #include <atomic>
 #include <mutex>
 
@@ -9,6 +11,15 @@
 #include "ftk_host.h"
 
 namespace ftk {
+
+bool pdl_enabled()
+{
+    static const bool on = [] {
+        const char *e = getenv("FTK_NO_PDL");
+        return !(e && e[0] == '1');
+    }();
+    return on;
+}
 
 void *current_context()
 {

@@ -50,6 +50,43 @@ struct Carver {
 // The calling thread's current CUDA context (a driver handle), or NULL.
 void *current_context();
 
+// False when the environment variable FTK_NO_PDL is set to 1 (read once).
+bool pdl_enabled();
+
+// Launches kern with programmatic stream serialization (unless disabled):
+// the kernel may be scheduled while the kernel before it on the stream
+// finishes, which hides launch latency between the many short kernels of a
+// call; every kernel of the library starts with griddep_wait(), so it reads
+// nothing before its predecessor is complete.  cluster > 1 adds
+// thread-block clusters of that many CTAs.
+template <typename... KArgs, typename... Args>
+inline ftk_status launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                unsigned cluster, Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    unsigned n = 0;
+    if (cluster > 1) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = cluster;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    if (pdl_enabled()) {
+        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    return cuda_status(cudaLaunchKernelEx(&cfg, kern, static_cast<Args &&>(args)...));
+}
+
 // Raises the dynamic shared-memory limit of kernel `func` to at least
 // `bytes`, once per (kernel, context): later calls find it in a small table
 // instead of calling cudaFuncSetAttribute again.  A context that is

@@ -47,6 +47,7 @@ __device__ __forceinline__ void unpack4(uint2 x, float (&v)[4])
 template <int DT>
 __global__ void __launch_bounds__(kBoxThreads) box_kernel(const BoxArgs a)
 {
+    griddep_wait();  // the previous kernel on the stream is complete
     __shared__ float sh_hi[8][kDim], sh_lo[8][kDim];
     __shared__ float sh_m[8];
     __shared__ int sh_bad;
@@ -186,6 +187,7 @@ struct BoundSmem {
 template <int DT, int MODE, int H>
 __global__ void __launch_bounds__(kBoundWarps * 32, 1) bound_kernel(const BoundArgs a)
 {
+    griddep_wait();  // the previous kernel on the stream is complete
     __shared__ BoundSmem sm;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (MODE == BOUND_FULL) {
@@ -410,8 +412,7 @@ __global__ void __launch_bounds__(kBoundWarps * 32, 1) bound_kernel(const BoundA
 template <int DT>
 static ftk_status launch_box_dt(const BoxArgs &a, cudaStream_t s)
 {
-    box_kernel<DT><<<a.nblocks, kBoxThreads, 0, s>>>(a);
-    return cuda_status(cudaGetLastError());
+    return launch_kernel(box_kernel<DT>, dim3(a.nblocks), dim3(kBoxThreads), 0, s, 1, a);
 }
 
 ftk_status launch_box(int dtype, const BoxArgs &a, cudaStream_t s)
@@ -423,10 +424,9 @@ template <int DT, int H>
 static ftk_status launch_bound_dt(int mode, const BoundArgs &a, int grid, cudaStream_t s)
 {
     const int threads = kBoundWarps * 32;
-    if (mode == BOUND_EST) bound_kernel<DT, BOUND_EST, H><<<grid, threads, 0, s>>>(a);
-    else if (mode == BOUND_FULL) bound_kernel<DT, BOUND_FULL, H><<<grid, threads, 0, s>>>(a);
-    else bound_kernel<DT, BOUND_OUT, H><<<grid, threads, 0, s>>>(a);
-    return cuda_status(cudaGetLastError());
+    if (mode == BOUND_EST) return launch_kernel(bound_kernel<DT, BOUND_EST, H>, dim3(grid), dim3(threads), 0, s, 1, a);
+    if (mode == BOUND_FULL) return launch_kernel(bound_kernel<DT, BOUND_FULL, H>, dim3(grid), dim3(threads), 0, s, 1, a);
+    return launch_kernel(bound_kernel<DT, BOUND_OUT, H>, dim3(grid), dim3(threads), 0, s, 1, a);
 }
 
 ftk_status launch_bound(int dtype, int mode, const BoundArgs &a, int grid, cudaStream_t s, int heads)

@@ -68,19 +68,8 @@ static ftk_status launch_rows_dt(const RowsArgs &a, int cluster, bool idx64, cud
                       : (loop ? rows_topk_kernel<DT, true, int32_t> : rows_topk_kernel<DT, false, int32_t>);
     const ftk_status e = ensure_smem_limit(reinterpret_cast<const void *>(kern), static_cast<int>(smem));
     if (e != FTK_OK) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(nclusters * cluster), 1, 1);
-    cfg.blockDim = dim3(kRowsThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = cluster;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cuda_status(cudaLaunchKernelEx(&cfg, kern, a));
+    return launch_kernel(kern, dim3(static_cast<unsigned>(nclusters * cluster)), dim3(kRowsThreads), smem, stream,
+                         static_cast<unsigned>(cluster), a);
 }
 
 ftk_status launch_rows_topk(int dtype, const RowsArgs &a, int cluster, cudaStream_t stream, bool idx64)
@@ -113,6 +102,7 @@ __global__ void __launch_bounds__(kSortThreads) sort_rows_kernel(const void *x, 
                                                                  void *vals, IT *idx, int64_t ldo, int k,
                                                                  int kp)
 {
+    griddep_wait();  // the previous kernel on the stream is complete
     using Tr = RowsTraits<DT>;
     using elem = typename Tr::elem;
     extern __shared__ unsigned long long skey[];

@@ -110,6 +110,7 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *sh, ui
 
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanArgs p)
 {
+    griddep_wait();  // the previous kernel on the stream is complete
     __shared__ uint32_t sh[96];
     const int tid = threadIdx.x;
     bool bad = false;
@@ -325,6 +326,7 @@ struct ThreshArgs {
 
 __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const ThreshArgs p)
 {
+    griddep_wait();  // the previous kernel on the stream is complete
     extern __shared__ uint32_t tkeys[];
     __shared__ SelShared ss;
     const int64_t t = blockIdx.x;
@@ -400,6 +402,7 @@ __device__ __forceinline__ void pad_row(int32_t *oi, float *ov, int from, int k)
 // kernel is latency-bound per row.
 __global__ void __launch_bounds__(kSelThreads, 6) refine_kernel(const RefineArgs p)
 {
+    griddep_wait();  // the previous kernel on the stream is complete
     extern __shared__ __align__(16) uint32_t rsm[];
     __shared__ SelShared ss;
     __shared__ uint32_t bitmap[kBitmapWords];
@@ -758,8 +761,7 @@ static ftk_status launch_score(const ScoreArgs &a, const CUtensorMap &tq, const 
     auto kern = score_kernel<DT, MODE, PR, H64>;
     const ftk_status e = ensure_smem_limit(reinterpret_cast<const void *>(kern), smem);
     if (e != FTK_OK) return e;
-    kern<<<grid, kScoreThreads, smem, st>>>(a, tq, kvm);
-    return cuda_status(cudaGetLastError());
+    return launch_kernel(kern, dim3(grid), dim3(kScoreThreads), smem, st, 1, a, tq, kvm);
 }
 
 template <int MODE, bool PR = false>
@@ -995,8 +997,7 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
         pa.launches = 3;
         // (Stage marks: the dense scores stand in the scan's place, the row
         // top-k in the refine's; the skipped stages take no time.)
-        plan_kernel<<<1, kPlanThreads, 0, s>>>(pa);
-        if ((st = cuda_status(cudaGetLastError())) != FTK_OK) return st;
+        if ((st = launch_kernel(plan_kernel, dim3(1), dim3(kPlanThreads), 0, s, 1, pa)) != FTK_OK) return st;
         for (int i : {1, 2, 3, 7}) stage_mark(i, s);
         int rcluster = 1, rchunk = 8;
         rows_plan(T, S, topk, &rcluster, &rchunk);
@@ -1007,8 +1008,7 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
         stage_mark(6, s);
         return FTK_OK;
     }
-    plan_kernel<<<1, kPlanThreads, 0, s>>>(pa);
-    if ((st = cuda_status(cudaGetLastError())) != FTK_OK) return st;
+    if ((st = launch_kernel(plan_kernel, dim3(1), dim3(kPlanThreads), 0, s, 1, pa)) != FTK_OK) return st;
     stage_mark(1, s);
 
     ScoreArgs sa = {};
@@ -1054,8 +1054,8 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
         const size_t smem = static_cast<size_t>(w.sld) * 4;
         st = ensure_smem_limit(reinterpret_cast<const void *>(threshold_kernel), static_cast<int>(smem));
         if (st != FTK_OK) return st;
-        threshold_kernel<<<static_cast<unsigned>(T), kSelThreads, smem, s>>>(ta);
-        if ((st = cuda_status(cudaGetLastError())) != FTK_OK) return st;
+        st = launch_kernel(threshold_kernel, dim3(static_cast<unsigned>(T)), dim3(kSelThreads), smem, s, 1, ta);
+        if (st != FTK_OK) return st;
     }
     stage_mark(3, s);
 
@@ -1149,8 +1149,8 @@ extern "C" ftk_status ftk_select(ftk_dtype dtype, const void *q, const void *kv,
         const size_t smem = static_cast<size_t>(c.cap) * 4;
         st = ensure_smem_limit(reinterpret_cast<const void *>(refine_kernel), static_cast<int>(smem));
         if (st != FTK_OK) return st;
-        refine_kernel<<<static_cast<unsigned>(T), kSelThreads, smem, s>>>(ra);
-        if ((st = cuda_status(cudaGetLastError())) != FTK_OK) return st;
+        st = launch_kernel(refine_kernel, dim3(static_cast<unsigned>(T)), dim3(kSelThreads), smem, s, 1, ra);
+        if (st != FTK_OK) return st;
     }
     stage_mark(5, s);
 
