@@ -50,6 +50,10 @@ __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
 // each waits here, before its first read of global memory, until that kernel
 // has completed and its writes are visible (a no-op for an ordinary launch).
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the next kernel on the stream be scheduled as soon as every CTA of
+// this one has started (it still waits for this one's completion before it
+// reads anything): its CTAs take the SMs this kernel's last wave frees.
+__device__ __forceinline__ void griddep_launch_next() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 __device__ __forceinline__ void fence_barrier_init()
 {

@@ -48,6 +48,7 @@ template <int DT>
 __global__ void __launch_bounds__(kBoxThreads) box_kernel(const BoxArgs a)
 {
     griddep_wait();  // the previous kernel on the stream is complete
+    griddep_launch_next();
     __shared__ float sh_hi[8][kDim], sh_lo[8][kDim];
     __shared__ float sh_m[8];
     __shared__ int sh_bad;
@@ -188,6 +189,7 @@ template <int DT, int MODE, int H>
 __global__ void __launch_bounds__(kBoundWarps * 32, 1) bound_kernel(const BoundArgs a)
 {
     griddep_wait();  // the previous kernel on the stream is complete
+    griddep_launch_next();
     __shared__ BoundSmem sm;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (MODE == BOUND_FULL) {

@@ -103,6 +103,7 @@ __global__ void __launch_bounds__(kSortThreads) sort_rows_kernel(const void *x, 
                                                                  int kp)
 {
     griddep_wait();  // the previous kernel on the stream is complete
+    griddep_launch_next();
     using Tr = RowsTraits<DT>;
     using elem = typename Tr::elem;
     extern __shared__ unsigned long long skey[];

@@ -1303,6 +1303,7 @@ template <int DT, bool LOOP, typename IT>
 __global__ void __launch_bounds__(kRowsThreads, 2) rows_topk_kernel(const RowsArgs a)
 {
     griddep_wait();  // the previous kernel on the stream is complete
+    griddep_launch_next();
     extern __shared__ __align__(16) uint8_t smem_raw[];
     RowsSmem &sm = *reinterpret_cast<RowsSmem *>(smem_raw);
     cg::cluster_group cluster = cg::this_cluster();

@@ -396,6 +396,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                  const __grid_constant__ KvMaps kvm)
 {
     griddep_wait();  // the previous kernel on the stream is complete
+    griddep_launch_next();
     if (MODE == MODE_COLLECT && a.prune_bits != nullptr && ((*a.prune_on != 0) != PR)) return;
     using C = ScoreCfg<DT>;
     using Lay = ScoreSmemLayout<DT>;

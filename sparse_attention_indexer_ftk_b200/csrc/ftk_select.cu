@@ -111,6 +111,7 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t *sh, ui
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanArgs p)
 {
     griddep_wait();  // the previous kernel on the stream is complete
+    griddep_launch_next();
     __shared__ uint32_t sh[96];
     const int tid = threadIdx.x;
     bool bad = false;
@@ -327,6 +328,7 @@ struct ThreshArgs {
 __global__ void __launch_bounds__(kSelThreads) threshold_kernel(const ThreshArgs p)
 {
     griddep_wait();  // the previous kernel on the stream is complete
+    griddep_launch_next();
     extern __shared__ uint32_t tkeys[];
     __shared__ SelShared ss;
     const int64_t t = blockIdx.x;
@@ -403,6 +405,7 @@ __device__ __forceinline__ void pad_row(int32_t *oi, float *ov, int from, int k)
 __global__ void __launch_bounds__(kSelThreads, 6) refine_kernel(const RefineArgs p)
 {
     griddep_wait();  // the previous kernel on the stream is complete
+    griddep_launch_next();
     extern __shared__ __align__(16) uint32_t rsm[];
     __shared__ SelShared ss;
     __shared__ uint32_t bitmap[kBitmapWords];
