@@ -91,6 +91,7 @@ struct RowsSmem {
     uint32_t w_gtf[kRowsWarps];    // stored entries > F
     uint32_t w_eqs[kRowsWarps];    // stored entries == F
     uint32_t w_eqf[kRowsWarps];    // entries == F, stored or counted past the end of a full list
+    uint32_t w_all[kRowsWarps];    // entries >= F, stored or not
     uint32_t w_kmax[kRowsWarps];   // largest stored key
     uint32_t cta_fkey, cta_over, cta_gt, cta_eq;
     // every list of the cluster in column order (index rank * kRowsWarps + warp)
@@ -102,7 +103,7 @@ struct RowsSmem {
     uint32_t wsum[kRowsWarps];
     uint32_t red[2 * kRowsWarps];
     uint32_t sel_bin, sel_above, fmin, short_eq;
-    uint32_t g_gt, g_eqt, g_over, g_kmax;
+    uint32_t g_gt, g_eqt, g_over, g_kmax, g_all;
     uint32_t nan_seen, overflow;
 };
 
@@ -452,7 +453,7 @@ template <int DT, typename IT>
 __device__ __noinline__ void rows_fallback(const RowsArgs &a, RowsSmem &sm, cg::cluster_group &cluster,
                                            unsigned cs, unsigned rank, const typename RowsTraits<DT>::elem *row,
                                            int64_t c0, int n, int64_t base_index, IT *oidx,
-                                           typename RowsTraits<DT>::elem *oval, uint32_t &ph)
+                                           typename RowsTraits<DT>::elem *oval, uint32_t &ph, uint32_t lo)
 {
     using Tr = RowsTraits<DT>;
     using elem = typename Tr::elem;
@@ -469,6 +470,19 @@ __device__ __noinline__ void rows_fallback(const RowsArgs &a, RowsSmem &sm, cg::
                         warp, lane, ph, a.status};
     const bool tail_warp = warp == kRowsWarps - 1;
     uint32_t *tot = sm.hist + 256;
+    // A vector certainly holds no key >= t when t is strictly positive and
+    // the packed maximum of its raw elements is below t's raw bits; the
+    // passes skip such vectors whole (one test for the warp).
+    auto fm1_of_key = [&](uint32_t t) {
+        const uint32_t tb = f32_from_key(t);
+        return Tr::fm1_of(DT == FTK_BF16 ? (tb >> 16) : tb);
+    };
+    auto may_hold = [&](const uint4 &x, uint32_t t, uint32_t t_fm1) {
+        return t <= 0x80000000u || Tr::ge_from_smax(Tr::vsmax(x), t_fm1);
+    };
+    // Keys below lo cannot be the k-th largest (lo is 0 or a bound the row
+    // has >= topk keys at or above).
+    const uint32_t lo_fm1 = lo > 0x80000000u ? fm1_of_key(lo) : 0u;
 
     // ---- u*: radix select over the row, 8-bit digits ----
     const int passes = DT == FTK_BF16 ? 2 : 4;
@@ -479,17 +493,31 @@ __device__ __noinline__ void rows_fallback(const RowsArgs &a, RowsSmem &sm, cg::
         __syncthreads();
         ws.prologue();
         ws.run([&](const uint4 &x, bool valid, int) {
+            const bool cand = valid && may_hold(x, lo, lo_fm1);
+            if (lo != 0u) {
+                // Few keys reach the histogram: each lane adds its own, with
+                // no warp vote.
+                if (cand) {
+#pragma unroll
+                    for (int j = 0; j < VEC; ++j) {
+                        const uint32_t u = Tr::key(Tr::element(x, j));
+                        if (u >= lo && (u & mask) == prefix) atomicAdd(&sm.hist[(u >> shift) & 255u], 1u);
+                    }
+                }
+                return;
+            }
+            if (!__any_sync(0xFFFFFFFFu, cand)) return;  // (warp-uniform)
 #pragma unroll
             for (int j = 0; j < VEC; ++j) {
                 const uint32_t u = Tr::key(Tr::element(x, j));
-                hist_add(sm.hist, (u >> shift) & 255u, valid && (u & mask) == prefix);
+                hist_add(sm.hist, (u >> shift) & 255u, cand && (u & mask) == prefix);
             }
         });
         if (tail_warp) {
             for (int e0 = nvec * VEC; e0 < n; e0 += 32) {
                 const int e = e0 + lane;
                 const uint32_t u = e < n ? Tr::key(row[c0 + e]) : 0u;
-                hist_add(sm.hist, (u >> shift) & 255u, e < n && (u & mask) == prefix);
+                hist_add(sm.hist, (u >> shift) & 255u, e < n && u >= lo && (u & mask) == prefix);
             }
         }
         cluster.sync();
@@ -514,9 +542,11 @@ __device__ __noinline__ void rows_fallback(const RowsArgs &a, RowsSmem &sm, cg::
     for (int b = tid; b < 512; b += kRowsThreads) sm.hist[b] = 0;
 
     // ---- counts of > u* and == u* per warp segment ----
+    const uint32_t us_fm1 = ustar > 0x80000000u ? fm1_of_key(ustar) : 0u;
     uint32_t g = 0, q = 0;
     ws.prologue();
     ws.run([&](const uint4 &x, bool valid, int) {
+        if (!__any_sync(0xFFFFFFFFu, valid && may_hold(x, ustar, us_fm1))) return;  // (warp-uniform)
         uint32_t gt, eq;
         cmp_masks<DT>(x, ustar, gt, eq);
         if (valid) {
@@ -599,6 +629,7 @@ __device__ __noinline__ void rows_fallback(const RowsArgs &a, RowsSmem &sm, cg::
     };
     ws.prologue();
     ws.run([&](const uint4 &x, bool valid, int v) {
+        if (!__any_sync(0xFFFFFFFFu, valid && may_hold(x, ustar, us_fm1))) return;  // (warp-uniform)
         uint32_t gt = 0, eq = 0;
         if (valid) cmp_masks<DT>(x, ustar, gt, eq);
         if (__ballot_sync(0xFFFFFFFFu, (gt | eq) != 0u)) emit(gt, eq, x, v * VEC);
@@ -968,6 +999,7 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
         over = __any_sync(0xFFFFFFFFu, over);
         if (lane == 0) {
             sm.w_cnt[warp] = min(wcnt, static_cast<uint32_t>(kRowsCapWarp));
+            sm.w_all[warp] = wcnt;
             sm.w_gtf[warp] = ngt;
             sm.w_eqs[warp] = neq;
             sm.w_eqf[warp] = neq + lost;
@@ -992,7 +1024,7 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
     const int nl = static_cast<int>(cs) * kRowsWarps;
     const uint32_t fu = fkey;
     if (warp == 0) {
-        uint32_t cnt[2], ov = 0, gsum = 0, esum = 0, kmax = 0;
+        uint32_t cnt[2], ov = 0, gsum = 0, esum = 0, kmax = 0, asum = 0;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const int L = lane + 32 * h;
@@ -1008,6 +1040,7 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
                 sm.l_eqt[L] = et;
                 gsum += g;
                 esum += et;
+                asum += o->w_all[w];
                 kmax = max(kmax, o->w_kmax[w]);
                 ov |= o->cta_over;
             }
@@ -1024,12 +1057,14 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
         gsum = __reduce_add_sync(0xFFFFFFFFu, gsum);
         esum = __reduce_add_sync(0xFFFFFFFFu, esum);
         kmax = __reduce_max_sync(0xFFFFFFFFu, kmax);
+        asum = __reduce_add_sync(0xFFFFFFFFu, asum);
         if (lane == 31) sm.l_off[nl] = i1;
         if (lane == 0) {
             sm.g_over = ov;
             sm.g_gt = gsum;
             sm.g_eqt = esum;
             sm.g_kmax = kmax;
+            sm.g_all = asum;
         }
     }
     __syncthreads();
@@ -1247,7 +1282,10 @@ __device__ __forceinline__ void rows_topk_row(const RowsArgs &a, RowsSmem &sm, c
             pre_next = false;
         }
         __syncthreads();
-        rows_fallback<DT, IT>(a, sm, cluster, cs, rank, row, c0, n, base_index, oidx, oval, ph);
+        // At least topk elements >= F: the k-th largest is >= F, and the
+        // fallback's passes look at nothing below it.
+        const uint32_t lo = sm.g_all >= static_cast<uint32_t>(k) ? fkey : 0u;
+        rows_fallback<DT, IT>(a, sm, cluster, cs, rank, row, c0, n, base_index, oidx, oval, ph, lo);
     } else {
         __syncthreads();
         cluster_arrive();  // no more reads of other CTAs' shared memory

@@ -84,6 +84,18 @@ def test_structured_rows(dtype, rows, cols, k):
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_quantized_rows(dtype):
+    """Values on a grid of quarters (hundreds of equal values around the
+    k-th): some candidate lists overflow with values above the sample
+    threshold, and those rows take the exact fallback, whose passes skip
+    every key below the threshold once the row has topk keys at or above
+    it."""
+    g = torch.Generator().manual_seed(3)
+    x = (torch.randn((256, 131072), generator=g) * 4).round() / 4
+    assert run_and_compare(x.to(dtype), 512) == 0
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 def test_heavy_ties_and_signed_zero(dtype):
     g = torch.Generator().manual_seed(5)
     x = torch.randint(-2, 3, (8, 20000), generator=g).float() * 0.5
