@@ -39,7 +39,7 @@ constexpr float kPruneEps = 0.0009765625f;  // 2^-10
 constexpr float kPruneCutoff = 0.25f;  // auto mode: prune when >= 25% of pairs are skippable
 constexpr int kEstTiles = 8;           // sampled row tiles of the estimate
 constexpr int kEstBlocks = 32;         // sampled blocks per sampled tile
-constexpr int kEstChunk = 4;           // sampled blocks per estimate work item
+constexpr int kEstChunk = 2;           // sampled blocks per estimate work item
 
 enum { BOUND_EST = 0, BOUND_FULL = 1, BOUND_OUT = 2 };
 

@@ -194,6 +194,30 @@ def test_dense_path_matches_threshold_path(dtype, T, S, topk):
     check_case(c)
 
 
+def test_programmatic_launch_off_gives_the_same_bits(tmp_path):
+    """Launching without programmatic dependent launch (FTK_NO_PDL=1, read
+    once per process, so in a child process) gives the same bits as the
+    default launches, on the sampled-threshold path (11 launches)."""
+    import os
+    import subprocess
+    import sys
+    spec = dict(seed=41, dtype="fp8", T=200, S=20000, topk=256, windows="causal")
+    g = gpu_inputs(wl.small_case(**spec))
+    idx, val, _ = run_select(g)
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = (
+        "import sys, numpy as np\n"
+        f"sys.path.insert(0, {root!r})\n"
+        "from sparse_attention_indexer_ftk_b200 import ftk, workloads as wl\n"
+        f"c = wl.small_case(**{spec!r}).to('cuda')\n"
+        "i, v = ftk.select(c.q, c.kv, c.weights, c.ks, c.ke, c.kv_scales, c.topk, return_scores=True)\n"
+        f"np.save({str(tmp_path / 'i.npy')!r}, i.cpu().numpy())\n"
+        f"np.save({str(tmp_path / 'v.npy')!r}, v.cpu().numpy())\n")
+    subprocess.run([sys.executable, "-c", code], env=dict(os.environ, FTK_NO_PDL="1"), check=True, timeout=900)
+    assert np.array_equal(np.load(tmp_path / "i.npy"), idx)
+    assert np.array_equal(np.load(tmp_path / "v.npy").view(np.uint32), val.view(np.uint32))
+
+
 def test_determinism():
     c = wl.small_case(seed=12, dtype="fp8", T=64, S=30000, topk=512, windows="causal")
     g = gpu_inputs(c)
