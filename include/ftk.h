@@ -84,9 +84,12 @@ typedef struct {
                             * README, "Roadmap": other head counts such as 64); q is then
                             * [T, H, 128] and weights [T, H]. */
     int32_t dense_rows;    /* calls of at most this many query rows (and at most 2^25
-                            * (row, key) pairs) score every key of every window and
-                            * select with the row top-k instead of the sampled
-                            * threshold (0: 128, the default; -1: never) */
+                            * (row, key) pairs, and rows that fit one recovery pass)
+                            * score every key of every window and select with the
+                            * row top-k instead of the sampled threshold (0: 128, the
+                            * default; -1: never).  Such calls skip the sample,
+                            * threshold, pruning and refine stages (prune has no
+                            * effect); info counts every window key as a candidate. */
     int32_t reserved;      /* must be 0 */
 } ftk_config;
 
