@@ -115,6 +115,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanArgs p)
     __shared__ uint32_t sh[96];
     const int tid = threadIdx.x;
     bool bad = false;
+#pragma unroll 4
     for (int64_t t = tid; t < p.T; t += blockDim.x) {
         p.cnt[t] = 0;
         bad |= !window_ok(p.ks[t], p.ke[t], p.S);
@@ -172,12 +173,20 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanArgs p)
         const int32_t tile = base + tid;
         uint32_t ns = 0, nc = 0;
         if (tile < p.ntiles) {
-            int64_t lo = INT64_MAX, hi = -1;
-            for (int j = 0; j < p.rt; ++j) {
+            // The tile's windows: every load issued before any is used.
+            int32_t wa[kMaxRowTile], wb[kMaxRowTile];
+#pragma unroll
+            for (int j = 0; j < kMaxRowTile; ++j) {
                 const int64_t t = static_cast<int64_t>(tile) * p.rt + j;
-                if (t >= p.T) break;
-                const int64_t a = p.ks[t], b = p.ke[t];
-                if (!window_ok(a, b, p.S) || a == b) continue;
+                const bool in = j < p.rt && t < p.T;
+                wa[j] = in ? p.ks[t] : 0;
+                wb[j] = in ? p.ke[t] : 0;
+            }
+            int64_t lo = INT64_MAX, hi = -1;
+#pragma unroll
+            for (int j = 0; j < kMaxRowTile; ++j) {
+                const int64_t a = wa[j], b = wb[j];
+                if (!window_ok(a, b, p.S) || a == b) continue;  // (absent rows: 0 == 0)
                 lo = min(lo, a);
                 hi = max(hi, b);
             }
