@@ -9,13 +9,15 @@
 //      multicast; lane 0 issues them, an mbarrier per stage), so about 8 KB
 //      per warp are in flight without any thread issuing loads;
 //   2. threshold F, while the first stages are in flight: a spread sample of
-//      the chunk (one 16-byte vector per thread) and F = the smallest sampled
-//      key of the 11-bit bin that holds the r-th largest sample, r chosen so
-//      that the whole row very likely keeps >= topk elements >= F;
+//      the chunk (one 16-byte vector per thread) and F = the r-th largest
+//      sample (two levels of 11-bit bins; for bf16 exact, for fp32 to within
+//      the lowest 10 key bits), r chosen so that the whole row very likely
+//      keeps >= topk elements >= F;
 //   3. filter: each vector is tested against F with one packed compare; the
-//      rare elements >= F go, in column order, to the warp's candidate list
-//      in shared memory.  Elements equal to F that find the list full are
-//      only counted (heavy ties);
+//      rare vectors holding an element >= F are noted and, once per stage,
+//      their elements go in column order to the warp's candidate list in
+//      shared memory.  Elements equal to F that find the list full are only
+//      counted (heavy ties);
 //   4. exact k-th key u*: the cluster filters with one F (the largest of
 //      its CTAs' estimates, exchanged while the first stages load), so every
 //      list holds all of its chunk's elements > F and its elements == F are
@@ -31,7 +33,8 @@
 // many candidates) take an exact fallback: multi-pass radix select over the
 // chunk (8-bit digits, histograms summed over the cluster), a counting pass
 // and an ordered writing pass, each streaming the chunk through the same
-// rings.  No sort, no global scratch.
+// rings and skipping what lies below F once the row is known to hold topk
+// elements >= F.  No sort, no global scratch.
 #pragma once
 
 #include <cooperative_groups.h>
