@@ -247,12 +247,24 @@ __device__ __forceinline__ bool get_item(const ScoreArgs &a, const Sched &sc, in
         m.tile = it / sc.chunks;
         const int chunk = it - m.tile * sc.chunks;
         m.lg = 0;
-        int64_t lo = INT64_MAX, hi = -1;
+        // The tile's rows and windows, every load issued before any is used.
+        const int64_t p0 = static_cast<int64_t>(m.tile) * RT;
+        int32_t tq[RT], wa[RT], wb[RT];
+#pragma unroll
+        for (int j = 0; j < RT; ++j)
+            tq[j] = p0 + j < nlist ? (a.rows ? a.rows[p0 + j] : static_cast<int32_t>(p0 + j)) : -1;
+#pragma unroll
         for (int j = 0; j < RT; ++j) {
-            const int32_t t = list_query(a, static_cast<int64_t>(m.tile) * RT + j, nlist);
-            if (t < 0 || a.ks[t] == a.ke[t]) continue;
-            lo = min(lo, static_cast<int64_t>(a.ks[t]));
-            hi = max(hi, static_cast<int64_t>(a.ke[t]));
+            const bool in = tq[j] >= 0 && tq[j] < a.T;
+            wa[j] = in ? a.ks[tq[j]] : 0;
+            wb[j] = in ? a.ke[tq[j]] : -1;
+        }
+        int64_t lo = INT64_MAX, hi = -1;
+#pragma unroll
+        for (int j = 0; j < RT; ++j) {
+            if (!window_ok(wa[j], wb[j], a.S) || wa[j] == wb[j]) continue;
+            lo = min(lo, static_cast<int64_t>(wa[j]));
+            hi = max(hi, static_cast<int64_t>(wb[j]));
         }
         if (hi < 0) return false;
         lo &= ~static_cast<int64_t>(kKeyTile - 1);
@@ -379,6 +391,7 @@ struct ScoreMisc {
     uint32_t tmem_base;
     int32_t abort;
     int32_t item_q[2];                     // item index, -1: no more items
+    Item item_m[2];                        // the item itself (valid when item_q >= 0)
 };
 
 static_assert(sizeof(ScoreMisc) <= ScoreSmemLayout<FTK_F8E4M3>::kMiscBytes, "misc area");
@@ -489,17 +502,32 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                     if (dynamic) {
                         it = atomicAdd(a.work_next, 1);
                         if (it >= total) it = -1;
+                        else get_item<MODE, RT>(a, sc, it, nlist, m);
                     } else if (next_item<MODE, RT>(a, sc, it_s, nlist, m)) {
                         it = it_s;
                         it_s += gridDim.x;
                     }
                 }
+                // The item's query rows, every load issued before any is
+                // used (list position -> row -> window).
+                int32_t tq[RT];
+                if (it >= 0) {
+                    const int64_t p0 = static_cast<int64_t>(m.tile) * RT;
+#pragma unroll
+                    for (int j = 0; j < RT; ++j)
+                        tq[j] = p0 + j < nlist ? (a.rows ? a.rows[p0 + j] : static_cast<int32_t>(p0 + j)) : -1;
+#pragma unroll
+                    for (int j = 0; j < RT; ++j) {  // placeholder rows are masked in the epilogue
+                        const bool in = tq[j] >= 0 && tq[j] < a.T;
+                        if (!in || !window_ok(a.ks[tq[j]], a.ke[tq[j]], a.S)) tq[j] = 0;
+                    }
+                }
                 if (!mbar_wait(&ms.item_empty[islot], iph ^ 1u, abort, a.status)) break;
                 ms.item_q[islot] = it;
+                if (it >= 0) ms.item_m[islot] = m;  // the other roles read it, not recompute it
                 mbar_arrive(&ms.item_full[islot]);
                 if (++islot == 2) { islot = 0; iph ^= 1u; }
                 if (it < 0) break;
-                if (dynamic) get_item<MODE, RT>(a, sc, it, nlist, m);
                 // The query group: the 32 head rows of each of RT queries.
                 if (!mbar_wait(&ms.q_empty, qph ^ 1u, abort, a.status)) break;
                 mbar_arrive_expect_tx(&ms.q_full, Lay::kQBytes);
@@ -507,9 +535,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
                 q_armed_ph = qph;
                 for (int vt = 0; vt < QG; ++vt) {
                     for (int j = 0; j < kQTile; ++j) {  // MMA row j: half j % VPQ of query j / VPQ
-                        int32_t t = list_query(a, static_cast<int64_t>(m.tile) * RT + vt * QPT + j / VPQ,
-                                               nlist);
-                        if (t < 0) t = 0;  // placeholder rows are masked in the epilogue
+                        const int32_t t = tq[vt * QPT + j / VPQ];
                         for (int at = 0; at < C::kAtoms; ++at)
                             tma_load_2d(sq + vt * Lay::kQTileBytes + at * (Lay::kQTileBytes / C::kAtoms) +
                                             j * kHeads * 128,
@@ -550,10 +576,10 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             while (ok && !*abort) {
                 if (!mbar_wait(&ms.item_full[islot], iph, abort, a.status)) break;
                 const int it = *reinterpret_cast<volatile int32_t *>(&ms.item_q[islot]);
+                if (it >= 0) m = ms.item_m[islot];
                 mbar_arrive(&ms.item_empty[islot]);
                 if (++islot == 2) { islot = 0; iph ^= 1u; }
                 if (it < 0) break;
-                get_item<MODE, RT>(a, sc, it, nlist, m);
                 if (!mbar_wait(&ms.q_full, qph, abort, a.status)) break;
                 qph ^= 1u;
                 tc_fence_after();
@@ -626,11 +652,11 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
             const bool got_item = mbar_wait(&ms.item_full[islot], iph, abort, a.status);
             if (!__all_sync(0xFFFFFFFFu, got_item)) break;
             const int it = *reinterpret_cast<volatile int32_t *>(&ms.item_q[islot]);
-            __syncwarp();  // every lane has the index before the slot is released
+            if (it >= 0) m = ms.item_m[islot];
+            __syncwarp();  // every lane has the item before the slot is released
             if (lane == 0) mbar_arrive(&ms.item_empty[islot]);
             if (++islot == 2) { islot = 0; iph ^= 1u; }
             if (it < 0) break;
-            get_item<MODE, RT>(a, sc, it, nlist, m);
             // Per-item parameters of this warp's queries (warp-uniform).  Slot
             // qq = vt * NR + qi is query qg * NR + qi of query tile vt, whose
             // MMA rows are qg * NQ + qi * VPQ + (0 .. VPQ - 1).
