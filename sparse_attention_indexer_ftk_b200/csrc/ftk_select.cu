@@ -237,18 +237,20 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const PlanArgs p)
 
 struct SelShared {
     uint32_t hist[256];
-    uint32_t bin, above;
+    uint32_t bin, above, bin_count;
     uint32_t red[96];
 };
 
 // The k-th largest (1 <= k <= count of keys) of key(i), i < n, where key
-// is any functor.  *gt receives how many keys are strictly larger.
+// is any functor.  *gt receives how many keys are strictly larger and, if
+// given, *eq how many are equal to it (the last digit's bin count).
 // kmin / kmax, if given, bound every key: the bits above the highest bit
 // where they differ are common to all keys, and the radix passes (8-bit
 // digits) start below them.  Block-wide; every thread of the block calls it.
 template <class KeyFn>
 __device__ uint32_t block_kth_largest(int n, uint32_t k, KeyFn key, SelShared &ss, uint32_t *gt,
-                                      uint32_t kmin = 0u, uint32_t kmax = 0xFFFFFFFFu)
+                                      uint32_t kmin = 0u, uint32_t kmax = 0xFFFFFFFFu,
+                                      uint32_t *eq = nullptr)
 {
     const uint32_t diff = kmin ^ kmax;
     const int top = diff ? 31 - __clz(diff) : -1;  // highest bit where keys may differ
@@ -286,6 +288,7 @@ __device__ uint32_t block_kth_largest(int n, uint32_t k, KeyFn key, SelShared &s
                     if (above + c[i] >= k) {
                         ss.bin = 255 - 8 * lane - i;
                         ss.above = above;
+                        ss.bin_count = c[i];
                         break;
                     }
                     above += c[i];
@@ -298,23 +301,14 @@ __device__ uint32_t block_kth_largest(int n, uint32_t k, KeyFn key, SelShared &s
         mask |= dmask << shift;
         k -= ss.above;
         above_total += ss.above;
+        // The last pass has digit shift 0: its bin holds exactly the keys
+        // equal to the result.
+        if (eq) *eq = ss.bin_count;
         __syncthreads();
     }
     *gt = above_total;
+    if (eq && top < 0) *eq = static_cast<uint32_t>(n);  // every key is kmax
     return prefix;
-}
-
-__device__ __forceinline__ uint32_t block_sum(uint32_t v, SelShared &ss)
-{
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
-    if (lane == 0) ss.red[warp] = v;
-    __syncthreads();
-    uint32_t s = 0;
-    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) s += ss.red[w];
-    __syncthreads();
-    return s;
 }
 
 // ---------------------------------------------------------------------------
@@ -498,13 +492,10 @@ __global__ void __launch_bounds__(kSelThreads, 6) refine_kernel(const RefineArgs
     // key == u* and index <= idx* (the smallest indices among the ties).
     uint32_t ustar = 0, idxcut = 0xFFFFFFFFu;
     if (n > k) {
-        uint32_t gt;
+        uint32_t gt, eq;
         ustar = block_kth_largest(n, static_cast<uint32_t>(k), [&](int i) { return keys[i]; }, ss, &gt,
-                                  kmin, kmax);
+                                  kmin, kmax, &eq);
         const uint32_t need = static_cast<uint32_t>(k) - gt;
-        uint32_t eq = 0;
-        for (int i = threadIdx.x; i < n; i += blockDim.x) eq += keys[i] == ustar;
-        eq = block_sum(eq, ss);
         if (eq > need) {
             // need-th smallest index among the ties = need-th largest of ~index.
             uint32_t g2;
