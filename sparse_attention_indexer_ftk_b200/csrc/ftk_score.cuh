@@ -191,8 +191,9 @@ __device__ __forceinline__ bool tile_pruned(const ScoreArgs &a, const Item &m, i
 }
 
 // Static schedules: a few rows (dense recovery of the rows a threshold
-// missed) must still spread over every SM, so the key chunk of an item
-// shrinks until the row tiles in use give about two items per CTA.
+// missed, the dense path) must still spread over every SM, so the key chunk
+// of an item shrinks until the row tiles in use give about one item per CTA
+// (one query-tile load and one pipeline fill per CTA).
 constexpr int kMinChunkTiles = 8;
 
 struct Sched {
@@ -210,8 +211,9 @@ __device__ __forceinline__ Sched make_sched(const ScoreArgs &a, int64_t nlist)
     sc.chunks = 0;
     if (MODE == MODE_DUMP) {  // the one static-schedule mode
         const int64_t kt = (a.S + kKeyTile - 1) / kKeyTile + 1;  // + 1: the aligned start
-        const int64_t want = 2 * static_cast<int64_t>(gridDim.x);
-        int64_t ct = (sc.tiles * kt + want - 1) / want;
+        // Row tiles split into as many chunks as give every CTA one item.
+        const int64_t per = sc.tiles < gridDim.x ? gridDim.x / sc.tiles : 1;
+        int64_t ct = (kt + per - 1) / per;
         ct = ct < kMinChunkTiles ? kMinChunkTiles : (ct > kChunkTiles ? kChunkTiles : ct);
         sc.chunk_keys = static_cast<int32_t>(ct * kKeyTile);
         sc.chunks = static_cast<int32_t>((kt + ct - 1) / ct);
